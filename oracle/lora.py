@@ -1,0 +1,83 @@
+"""Oracle: the LoRA / QLoRA linear layer in float64.
+
+TEST INFRASTRUCTURE ONLY (see ``oracle/__init__``).
+
+Equations followed:
+  * [P1] "How it works / The update LoRA is allowed to learn": h = W0 x + B A x
+    with W0 d x k frozen, B d x r, A r x k; the product scaled by alpha / r;
+    "W0 gets no gradient. A and B do."
+  * [P2] "The LoRA hypothesis" figure: h = W0 x + (alpha/r) B A x.
+  * [P1] "What QLoRA freezes, and in how many bits", forward equation:
+    Y = X doubleDequant(c1, c2, W) + X L1 L2 (row-vector form, so L1 = A^T,
+    L2 = B^T with the alpha/r scale s folded in), and "the backward pass still
+    dequantises W to BF16 to form the activation gradient".
+  * [P1] deploy paragraph and [P2] "fold it back in": W = W0 + (alpha/r) B A;
+    switching tasks subtracts B A.  [P2] "What actually goes wrong": merge into
+    the 16-bit base, keep the adapter separate (so the merged output is bf16
+    and the NF4 base is kept).
+
+Tokens are rows: X is T x k, Y is T x d.  All products are plain numpy
+float64 matmuls of exactly-converted bf16 inputs; no blocking or fusion.
+"""
+from __future__ import annotations
+
+from typing import Dict
+
+import numpy as np
+
+from .nf4 import bf16_to_f64, to_bf16_bits
+
+
+def forward(X: np.ndarray, Wp: np.ndarray, A: np.ndarray, B: np.ndarray, s: float) -> Dict[str, np.ndarray]:
+    """U = X A^T;  Y = X W'^T + s U B^T   (all float64 inputs)."""
+    U = X @ A.T
+    Y = X @ Wp.T + s * (U @ B.T)
+    return {"U": U, "Y": Y}
+
+
+def backward(X: np.ndarray, Wp: np.ndarray, A: np.ndarray, B: np.ndarray, s: float,
+             dY: np.ndarray, U: np.ndarray = None) -> Dict[str, np.ndarray]:
+    """Gradients of <dY, Y> w.r.t. X, A and B; none for W (frozen).
+
+    G = dY B;  dX = dY W' + s G A;  dA = s G^T X;  dB = s dY^T U,  U = X A^T.
+    """
+    if U is None:
+        U = X @ A.T
+    G = dY @ B
+    dX = dY @ Wp + s * (G @ A)
+    dA = s * (G.T @ X)
+    dB = s * (dY.T @ U)
+    return {"G": G, "dX": dX, "dA": dA, "dB": dB}
+
+
+def merge(Wp: np.ndarray, A: np.ndarray, B: np.ndarray, s: float) -> np.ndarray:
+    """W = bf16(W' + s B A), computed in float64 and rounded once."""
+    return to_bf16_bits(Wp + s * (B @ A))
+
+
+def unmerge(W: np.ndarray, A: np.ndarray, B: np.ndarray, s: float) -> np.ndarray:
+    """W0'' = bf16(W - s B A)."""
+    return to_bf16_bits(W - s * (B @ A))
+
+
+def as_f64(bits: np.ndarray) -> np.ndarray:
+    return bf16_to_f64(bits)
+
+
+# --------------------------------------------------------------------------
+# Parameter-count arithmetic ([P1] "The update LoRA is allowed to learn";
+# [P2] "The LoRA hypothesis")
+# --------------------------------------------------------------------------
+def adapter_params(d: int, k: int, r: int) -> int:
+    """Trainable parameters of one adapted d x k matrix: B (d x r) + A (r x k)."""
+    return d * r + r * k
+
+
+def model_adapter_params(n_adapted: int, d_model: int, r: int) -> int:
+    """2 * L_LoRA * d_model * r, attention projections treated as d_model x d_model."""
+    return 2 * n_adapted * d_model * r
+
+
+def algorithmic_flops(T: int, d: int, k: int, r: int) -> int:
+    """fwd + bwd flops without any weight gradient: 4Tdk + 6Tr(d+k)."""
+    return 4 * T * d * k + 6 * T * r * (d + k)
