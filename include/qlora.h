@@ -1,0 +1,229 @@
+/*
+ * libqlora — the QLoRA linear layer on NVIDIA B200 (sm_100a).
+ *
+ * C ABI.  Every pointer argument is a plain pointer; unless stated otherwise
+ * it is a DEVICE pointer to memory owned by the caller (for example a PyTorch
+ * tensor's data pointer).  The library never allocates or frees device
+ * memory: scratch space is passed in as a workspace whose size the matching
+ * *_workspace_bytes() query returns.  Every compute call is asynchronous on
+ * the given stream and returns a qlora_status_t after validating its
+ * arguments on the host (nothing is launched when validation fails).
+ *
+ * Layouts: row-major and contiguous.  bf16 tensors are passed as uint16_t
+ * bit patterns.  Notation follows the layer h = W0 x + (alpha/r) B A x with
+ * W0 d x k (frozen), A r x k, B d x r, tokens as rows: X is T x k, Y is T x d.
+ * s = alpha / r.
+ *
+ * Sources, cited by page title and section:
+ *   [P1] "LoRA and QLoRA fine-tuning: mechanics, and when not to fine-tune"
+ *   [P2] "Fine-Tuning on a Budget: LoRA and QLoRA"
+ *
+ * Inputs must be finite; results for NaN/Inf inputs are unspecified.
+ */
+#ifndef QLORA_H_
+#define QLORA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define QLORA_API __attribute__((visibility("default")))
+#else
+#define QLORA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  QLORA_OK = 0,
+  QLORA_ERR_INVALID_ARG = 1,       /* null pointer, negative size, bad alpha */
+  QLORA_ERR_UNSUPPORTED_SHAPE = 2, /* k % 64 != 0, r outside [1, 256], too large */
+  QLORA_ERR_MISALIGNED = 3,        /* a pointer is not 16-byte aligned */
+  QLORA_ERR_WORKSPACE_TOO_SMALL = 4,
+  QLORA_ERR_CUDA = 5,              /* a CUDA runtime/driver call or launch failed */
+  QLORA_ERR_TIMEOUT = 6,           /* a device-side wait gave up (device status) */
+  QLORA_ERR_NO_DEVICE = 7          /* no sm_100 device is current */
+} qlora_status_t;
+
+/* A cudaStream_t passed as an opaque pointer (NULL = legacy default stream). */
+typedef void* qlora_stream_t;
+
+/*
+ * NF4 storage of a frozen d x k weight with double-quantised block constants
+ * ([P1] "What QLoRA freezes, and in how many bits": NF4, first-level block
+ * 64, second-level FP8 constants in blocks of 256 after subtracting their
+ * mean; [P1] "What to choose and why": keep NF4/64/256 with the bundle).
+ * All buffers are device memory owned by the caller:
+ *   codes     d*k/2 bytes; byte m holds element 2m (row-major order) in bits
+ *             0-3 and element 2m+1 in bits 4-7
+ *   absmax_q  n_b = d*k/64 bytes: E4M3 code of (absmax_b - mean)/scale2_j
+ *   scale2    n_g = ceil(n_b/256) floats: second-level scale of group j
+ *   mean      1 float: mean of the first-level absmax constants
+ * block and block2 must be 64 and 256.
+ */
+typedef struct {
+  uint8_t* codes;
+  uint8_t* absmax_q;
+  float* scale2;
+  float* mean;
+  int64_t d;
+  int64_t k;
+  int32_t block;
+  int32_t block2;
+} qlora_nf4_t;
+
+/* Per-kernel timing collected while profiling is on (see qlora_profile_*). */
+typedef struct {
+  char name[48];
+  int64_t launches;
+  double total_ms;       /* sum of CUDA-event durations on the launch stream */
+  double flops;          /* algorithmic flops of all launches (0 if not a GEMM) */
+  double bytes;          /* algorithmic DRAM bytes of all launches */
+} qlora_kernel_stat_t;
+
+/* Human-readable text for a status code (static storage, never NULL). */
+QLORA_API const char* qlora_strerror(int status);
+
+/* Library version as 10000*major + 100*minor + patch. */
+QLORA_API int qlora_version(void);
+
+/*
+ * The library's own NF4 table (host call, no GPU needed): the 16 fp32 levels
+ * in ascending order and the 15 encoder thresholds t_i = the smallest fp32
+ * strictly above the exact midpoint of levels i and i+1, so that
+ * code(x) = #{i : x >= t_i} is the nearest level with ties to the lower code.
+ * Either pointer may be NULL.  Always returns QLORA_OK.
+ */
+QLORA_API int qlora_nf4_levels(float* levels16, float* thresholds15);
+
+/* ---------------------------------------------------------------- quantise */
+
+/* Workspace for qlora_nf4_quantize: fp32 absmax per block + fp64 per group. */
+QLORA_API size_t qlora_quantize_workspace_bytes(int64_t d, int64_t k);
+
+/*
+ * nf4_quantize(W0, block=64) ([P1] 4-bit NormalFloat and Double
+ * quantisation paragraphs).  W0: fp32 d x k, device.  `out` is a HOST struct
+ * whose four device pointers the caller has set; the call writes d, k, block
+ * and block2 into it and fills the device buffers:
+ *   a_b  = max |w| over each 64-block,
+ *   code = nearest NF4 level of fp32(w / a_b) (ties to the lower code; an
+ *          all-zero block gives the zero level),
+ *   mean = fp32(S / n_b), S the float64 pairwise sum of all a_b,
+ *   scale2_j = fp32(max_b |fp32(a_b - mean)| / 448) per group of 256,
+ *   absmax_q_b = E4M3_RN_satfinite(fp32(fp32(a_b - mean) / scale2_j))
+ *               (0 when scale2_j == 0).
+ * Requires block == 64, k % 64 == 0, d >= 1, d*k < 2^34.  W0 and the output
+ * buffers must be 16-byte aligned.
+ */
+QLORA_API int qlora_nf4_quantize(const float* W0, int64_t d, int64_t k, int block, qlora_nf4_t* out,
+                       void* workspace, size_t workspace_bytes, qlora_stream_t stream);
+
+/*
+ * doubleDequant ([P1] forward equation): W' (bf16, d x k, device) with
+ *   a'_b = fp32(fp32(E4M3(absmax_q_b) * scale2_j) + mean),
+ *   w'   = bf16_RN(fp32(level[code] * a'_b)).
+ * This is the exact bf16 weight every GEMM of this library multiplies by.
+ */
+QLORA_API int qlora_nf4_dequantize(const qlora_nf4_t* q, uint16_t* W_out, qlora_stream_t stream);
+
+/* ---------------------------------------------------------------- forward */
+
+QLORA_API size_t qlora_fwd_workspace_bytes(int64_t d, int64_t k, int r, int64_t T);
+
+/*
+ * Forward ([P1] forward equation; [P2] "The LoRA hypothesis" figure):
+ *   U = X A^T                  (fp32, T x r, written to U_save for backward)
+ *   Y = X W'^T + s U B^T       (bf16, T x d)
+ * W' is doubleDequant(q) in bf16; the rank-r term is accumulated in the same
+ * fp32 tile as the base product (its operand s*U is rounded to bf16).
+ * X: bf16 T x k; A: bf16 r x k; B: bf16 d x r; alpha > 0 (s = alpha / r).
+ * T may be 0 (no work).  Requires 1 <= r <= 256.
+ */
+QLORA_API int qlora_fwd(const qlora_nf4_t* q, const uint16_t* A, const uint16_t* B, int r, float alpha,
+              const uint16_t* X, int64_t T, uint16_t* Y, float* U_save, void* workspace,
+              size_t workspace_bytes, qlora_stream_t stream);
+
+/* ---------------------------------------------------------------- backward */
+
+QLORA_API size_t qlora_bwd_workspace_bytes(int64_t d, int64_t k, int r, int64_t T);
+
+/*
+ * Backward of L with dL/dY = dY ([P1] "The update LoRA is allowed to learn":
+ * only the adapter factors are trained; [P1] "What QLoRA freezes": the
+ * activation gradient is formed through W dequantised to bf16):
+ *   G  = dY B                  (fp32 accumulate, used as bf16 s*G)
+ *   dX = dY W' + s G A         (bf16, T x k)
+ *   dA = s G^T X               (fp32, r x k, overwritten)
+ *   dB = s dY^T U              (fp32, d x r, overwritten; U = U_saved)
+ * No weight gradient is formed.  dA and dB are reduced in a fixed order, so
+ * repeated calls give identical bits.
+ */
+QLORA_API int qlora_bwd(const qlora_nf4_t* q, const uint16_t* A, const uint16_t* B, int r, float alpha,
+              const uint16_t* X, const float* U_saved, const uint16_t* dY, int64_t T,
+              uint16_t* dX, float* dA, float* dB, void* workspace, size_t workspace_bytes,
+              qlora_stream_t stream);
+
+/* ---------------------------------------------------------------- deploy */
+
+QLORA_API size_t lora_merge_workspace_bytes(int64_t d, int64_t k, int r);
+
+/*
+ * Merge ([P1] deploy paragraph; [P2] "The LoRA hypothesis": the scaled
+ * product is added to the base weight; [P2] "What actually goes wrong": the
+ * merge goes into a 16-bit base while the adapter is kept separately):
+ *   W = bf16_RN(fp32(w' + s (B A)_fp32))   (bf16 d x k, out of place)
+ * The NF4 storage is left untouched so the merge can be undone.
+ */
+QLORA_API int lora_merge(const qlora_nf4_t* q, const uint16_t* A, const uint16_t* B, int r, float alpha,
+               uint16_t* W_out, void* workspace, size_t workspace_bytes, qlora_stream_t stream);
+
+/*
+ * Unmerge / task switch ([P1] deploy paragraph: a task is removed by
+ * subtracting its scaled product again):
+ *   W0'' = bf16_RN(fp32(W - s (B A)_fp32))   (bf16 d x k, out of place)
+ */
+QLORA_API int lora_unmerge(const uint16_t* W, const uint16_t* A, const uint16_t* B, int r, float alpha,
+                 int64_t d, int64_t k, uint16_t* W0_out, void* workspace,
+                 size_t workspace_bytes, qlora_stream_t stream);
+
+/* ---------------------------------------------------------------- status */
+
+/*
+ * Synchronises `stream`, then returns (in *status) and clears the device
+ * status word of the current device: QLORA_OK, or the first error a kernel
+ * recorded (QLORA_ERR_TIMEOUT when a bounded device wait gave up).  The
+ * return value reports failures of this call itself.
+ */
+QLORA_API int qlora_get_device_status(qlora_stream_t stream, int* status);
+
+/*
+ * Self-test of the bounded wait: launches one block that waits on a barrier
+ * nothing will complete, with a limit of `limit_us` microseconds (1..2e6).
+ * The kernel gives up, records QLORA_ERR_TIMEOUT and exits; read it with
+ * qlora_get_device_status.  The wait limit of other kernels is unchanged.
+ */
+QLORA_API int qlora_selftest_wait_timeout(int limit_us, qlora_stream_t stream);
+
+/* ---------------------------------------------------------------- profiling */
+
+/*
+ * Profiling: while on, every kernel launch of this library is bracketed by
+ * CUDA events recorded on its launch stream.  qlora_profile_begin clears the
+ * counters; qlora_profile_end synchronises the recorded events, writes up to
+ * `capacity` per-kernel-class sums to `out` (host array) and the number of
+ * classes to *n_out, and turns profiling off.
+ */
+QLORA_API int qlora_profile_begin(void);
+QLORA_API int qlora_profile_end(qlora_kernel_stat_t* out, int capacity, int* n_out);
+
+/* Number of kernels this library has launched in this process (all devices). */
+QLORA_API int64_t qlora_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QLORA_H_ */

@@ -5,13 +5,13 @@ TEST INFRASTRUCTURE ONLY (see ``oracle/__init__``).
 Equations followed:
   * [P1] "How it works / The update LoRA is allowed to learn": h = W0 x + B A x
     with W0 d x k frozen, B d x r, A r x k; the product scaled by alpha / r;
-    "W0 gets no gradient. A and B do."
+    only A and B receive gradients.
   * [P2] "The LoRA hypothesis" figure: h = W0 x + (alpha/r) B A x.
   * [P1] "What QLoRA freezes, and in how many bits", forward equation:
     Y = X doubleDequant(c1, c2, W) + X L1 L2 (row-vector form, so L1 = A^T,
-    L2 = B^T with the alpha/r scale s folded in), and "the backward pass still
-    dequantises W to BF16 to form the activation gradient".
-  * [P1] deploy paragraph and [P2] "fold it back in": W = W0 + (alpha/r) B A;
+    L2 = B^T with the alpha/r scale s folded in); the activation gradient is
+    also formed through the bf16-dequantised W.
+  * [P1] deploy paragraph and [P2] "The LoRA hypothesis": W = W0 + (alpha/r) B A;
     switching tasks subtracts B A.  [P2] "What actually goes wrong": merge into
     the 16-bit base, keep the adapter separate (so the merged output is bf16
     and the NF4 base is kept).
@@ -41,13 +41,24 @@ def backward(X: np.ndarray, Wp: np.ndarray, A: np.ndarray, B: np.ndarray, s: flo
 
     G = dY B;  dX = dY W' + s G A;  dA = s G^T X;  dB = s dY^T U,  U = X A^T.
     """
+    out = grad_input(Wp, A, B, s, dY)
+    out.update(grad_adapters(X, A, B, s, dY, U))
+    return out
+
+
+def grad_input(Wp: np.ndarray, A: np.ndarray, B: np.ndarray, s: float, dY: np.ndarray) -> Dict[str, np.ndarray]:
+    """dX = dY W' + s (dY B) A  (rows of dX depend only on the same rows of dY)."""
+    G = dY @ B
+    return {"G": G, "dX": dY @ Wp + s * (G @ A)}
+
+
+def grad_adapters(X: np.ndarray, A: np.ndarray, B: np.ndarray, s: float, dY: np.ndarray,
+                  U: np.ndarray = None) -> Dict[str, np.ndarray]:
+    """dA = s (dY B)^T X;  dB = s dY^T (X A^T)."""
     if U is None:
         U = X @ A.T
     G = dY @ B
-    dX = dY @ Wp + s * (G @ A)
-    dA = s * (G.T @ X)
-    dB = s * (dY.T @ U)
-    return {"G": G, "dX": dX, "dA": dA, "dB": dB}
+    return {"dA": s * (G.T @ X), "dB": s * (dY.T @ U)}
 
 
 def merge(Wp: np.ndarray, A: np.ndarray, B: np.ndarray, s: float) -> np.ndarray:

@@ -1,0 +1,313 @@
+"""Python binding of libqlora (the QLoRA linear layer on B200).
+
+Argument marshalling only: every step runs in the CUDA kernels of
+``libqlora.so``, reached through its C ABI (``include/qlora.h``).  PyTorch
+provides device memory and the current stream.  If the shared library is
+missing the import of any call raises; there is no CPU fallback.
+
+Names mirror the C entry points.  bf16 tensors are ``torch.bfloat16``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libqlora.so")
+
+QLORA_OK = 0
+QLORA_ERR_TIMEOUT = 6
+BLOCK = 64
+BLOCK2 = 256
+
+
+class QloraError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {strerror(status)} (status {status})")
+
+
+class _NF4(ctypes.Structure):
+    _fields_ = [("codes", ctypes.c_void_p), ("absmax_q", ctypes.c_void_p),
+                ("scale2", ctypes.c_void_p), ("mean", ctypes.c_void_p),
+                ("d", ctypes.c_int64), ("k", ctypes.c_int64),
+                ("block", ctypes.c_int32), ("block2", ctypes.c_int32)]
+
+
+class KernelStat(ctypes.Structure):
+    _fields_ = [("name", ctypes.c_char * 48), ("launches", ctypes.c_int64),
+                ("total_ms", ctypes.c_double), ("flops", ctypes.c_double),
+                ("bytes", ctypes.c_double)]
+
+
+_lib = None
+
+_VP = ctypes.c_void_p
+_I64 = ctypes.c_int64
+_SIZE = ctypes.c_size_t
+_INT = ctypes.c_int
+_F = ctypes.c_float
+_NF4P = ctypes.POINTER(_NF4)
+
+_SIGNATURES = {
+    "qlora_strerror": (ctypes.c_char_p, [_INT]),
+    "qlora_version": (_INT, []),
+    "qlora_nf4_levels": (_INT, [_VP, _VP]),
+    "qlora_quantize_workspace_bytes": (_SIZE, [_I64, _I64]),
+    "qlora_nf4_quantize": (_INT, [_VP, _I64, _I64, _INT, _NF4P, _VP, _SIZE, _VP]),
+    "qlora_nf4_dequantize": (_INT, [_NF4P, _VP, _VP]),
+    "qlora_fwd_workspace_bytes": (_SIZE, [_I64, _I64, _INT, _I64]),
+    "qlora_fwd": (_INT, [_NF4P, _VP, _VP, _INT, _F, _VP, _I64, _VP, _VP, _VP, _SIZE, _VP]),
+    "qlora_bwd_workspace_bytes": (_SIZE, [_I64, _I64, _INT, _I64]),
+    "qlora_bwd": (_INT, [_NF4P, _VP, _VP, _INT, _F, _VP, _VP, _VP, _I64, _VP, _VP, _VP, _VP,
+                         _SIZE, _VP]),
+    "lora_merge_workspace_bytes": (_SIZE, [_I64, _I64, _INT]),
+    "lora_merge": (_INT, [_NF4P, _VP, _VP, _INT, _F, _VP, _VP, _SIZE, _VP]),
+    "lora_unmerge": (_INT, [_VP, _VP, _VP, _INT, _F, _I64, _I64, _VP, _VP, _SIZE, _VP]),
+    "qlora_get_device_status": (_INT, [_VP, ctypes.POINTER(_INT)]),
+    "qlora_selftest_wait_timeout": (_INT, [_INT, _VP]),
+    "qlora_profile_begin": (_INT, []),
+    "qlora_profile_end": (_INT, [ctypes.POINTER(KernelStat), _INT, ctypes.POINTER(_INT)]),
+    "qlora_launch_count": (_I64, []),
+}
+
+EXPORTED = tuple(_SIGNATURES)
+
+
+def lib() -> ctypes.CDLL:
+    """Load libqlora.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"libqlora.so not found at {LIB_PATH}; build it with "
+                "`python -m parameter_efficient_fine_nf4_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGNATURES.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def strerror(status: int) -> str:
+    return lib().qlora_strerror(int(status)).decode()
+
+
+def _check(status: int, what: str):
+    if status != QLORA_OK:
+        raise QloraError(status, what)
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(int(stream.cuda_stream))
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to libqlora must be contiguous")
+    return t.data_ptr()
+
+
+def _need(t: torch.Tensor, dtype, shape, name):
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_cuda:
+        raise ValueError(f"{name}: must be a CUDA tensor")
+
+
+class NF4Weight:
+    """Device buffers of one NF4 + double-quant weight (the qlora_nf4_t)."""
+
+    def __init__(self, d: int, k: int, device=None):
+        device = torch.device("cuda") if device is None else torch.device(device)
+        n_b = d * k // BLOCK
+        n_g = (n_b + BLOCK2 - 1) // BLOCK2
+        self.d, self.k = d, k
+        self.codes = torch.empty(d * k // 2, dtype=torch.uint8, device=device)
+        self.absmax_q = torch.empty(n_b, dtype=torch.uint8, device=device)
+        self.scale2 = torch.empty(n_g, dtype=torch.float32, device=device)
+        self.mean = torch.empty(1, dtype=torch.float32, device=device)
+        self._c = _NF4(self.codes.data_ptr(), self.absmax_q.data_ptr(), self.scale2.data_ptr(),
+                       self.mean.data_ptr(), d, k, BLOCK, BLOCK2)
+
+    @property
+    def cstruct(self) -> _NF4:
+        return self._c
+
+    def nbytes(self) -> int:
+        return sum(t.numel() * t.element_size() for t in (self.codes, self.absmax_q, self.scale2, self.mean))
+
+
+def workspace(nbytes: int, device=None) -> torch.Tensor:
+    device = torch.device("cuda") if device is None else torch.device(device)
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+# ------------------------------------------------------------------- host-only
+def qlora_version() -> int:
+    return lib().qlora_version()
+
+
+def qlora_nf4_levels():
+    lv = (ctypes.c_float * 16)()
+    th = (ctypes.c_float * 15)()
+    _check(lib().qlora_nf4_levels(ctypes.addressof(lv), ctypes.addressof(th)), "qlora_nf4_levels")
+    return list(lv), list(th)
+
+
+def qlora_quantize_workspace_bytes(d: int, k: int) -> int:
+    return lib().qlora_quantize_workspace_bytes(d, k)
+
+
+def qlora_fwd_workspace_bytes(d: int, k: int, r: int, T: int) -> int:
+    return lib().qlora_fwd_workspace_bytes(d, k, r, T)
+
+
+def qlora_bwd_workspace_bytes(d: int, k: int, r: int, T: int) -> int:
+    return lib().qlora_bwd_workspace_bytes(d, k, r, T)
+
+
+def lora_merge_workspace_bytes(d: int, k: int, r: int) -> int:
+    return lib().lora_merge_workspace_bytes(d, k, r)
+
+
+def qlora_launch_count() -> int:
+    return lib().qlora_launch_count()
+
+
+# ------------------------------------------------------------------- device calls
+def qlora_nf4_quantize(W0: torch.Tensor, out: Optional[NF4Weight] = None,
+                       ws: Optional[torch.Tensor] = None, stream=None) -> NF4Weight:
+    d, k = W0.shape
+    _need(W0, torch.float32, (d, k), "W0")
+    out = NF4Weight(d, k, W0.device) if out is None else out
+    nbytes = qlora_quantize_workspace_bytes(d, k)
+    ws = workspace(nbytes, W0.device) if ws is None else ws
+    st = lib().qlora_nf4_quantize(_ptr(W0), d, k, BLOCK, ctypes.byref(out.cstruct), _ptr(ws),
+                                  ws.numel(), _stream(stream))
+    _check(st, "qlora_nf4_quantize")
+    return out
+
+
+def qlora_nf4_dequantize(q: NF4Weight, W_out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    W_out = torch.empty(q.d, q.k, dtype=torch.bfloat16, device=q.codes.device) if W_out is None else W_out
+    _need(W_out, torch.bfloat16, (q.d, q.k), "W_out")
+    _check(lib().qlora_nf4_dequantize(ctypes.byref(q.cstruct), _ptr(W_out), _stream(stream)),
+           "qlora_nf4_dequantize")
+    return W_out
+
+
+def qlora_fwd(q: NF4Weight, A: torch.Tensor, B: torch.Tensor, alpha: float, X: torch.Tensor,
+              Y: Optional[torch.Tensor] = None, U_save: Optional[torch.Tensor] = None,
+              ws: Optional[torch.Tensor] = None, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    r = A.shape[0]
+    T = X.shape[0]
+    _need(A, torch.bfloat16, (r, q.k), "A")
+    _need(B, torch.bfloat16, (q.d, r), "B")
+    _need(X, torch.bfloat16, (T, q.k), "X")
+    dev = X.device
+    Y = torch.empty(T, q.d, dtype=torch.bfloat16, device=dev) if Y is None else Y
+    U_save = torch.empty(T, r, dtype=torch.float32, device=dev) if U_save is None else U_save
+    _need(Y, torch.bfloat16, (T, q.d), "Y")
+    _need(U_save, torch.float32, (T, r), "U_save")
+    nbytes = qlora_fwd_workspace_bytes(q.d, q.k, r, T)
+    ws = workspace(nbytes, dev) if ws is None else ws
+    st = lib().qlora_fwd(ctypes.byref(q.cstruct), _ptr(A), _ptr(B), r, float(alpha), _ptr(X), T,
+                         _ptr(Y), _ptr(U_save), _ptr(ws), ws.numel(), _stream(stream))
+    _check(st, "qlora_fwd")
+    return Y, U_save
+
+
+def qlora_bwd(q: NF4Weight, A: torch.Tensor, B: torch.Tensor, alpha: float, X: torch.Tensor,
+              U_saved: torch.Tensor, dY: torch.Tensor, dX: Optional[torch.Tensor] = None,
+              dA: Optional[torch.Tensor] = None, dB: Optional[torch.Tensor] = None,
+              ws: Optional[torch.Tensor] = None, stream=None):
+    r = A.shape[0]
+    T = X.shape[0]
+    _need(A, torch.bfloat16, (r, q.k), "A")
+    _need(B, torch.bfloat16, (q.d, r), "B")
+    _need(X, torch.bfloat16, (T, q.k), "X")
+    _need(U_saved, torch.float32, (T, r), "U_saved")
+    _need(dY, torch.bfloat16, (T, q.d), "dY")
+    dev = X.device
+    dX = torch.empty(T, q.k, dtype=torch.bfloat16, device=dev) if dX is None else dX
+    dA = torch.empty(r, q.k, dtype=torch.float32, device=dev) if dA is None else dA
+    dB = torch.empty(q.d, r, dtype=torch.float32, device=dev) if dB is None else dB
+    _need(dX, torch.bfloat16, (T, q.k), "dX")
+    _need(dA, torch.float32, (r, q.k), "dA")
+    _need(dB, torch.float32, (q.d, r), "dB")
+    nbytes = qlora_bwd_workspace_bytes(q.d, q.k, r, T)
+    ws = workspace(nbytes, dev) if ws is None else ws
+    st = lib().qlora_bwd(ctypes.byref(q.cstruct), _ptr(A), _ptr(B), r, float(alpha), _ptr(X),
+                         _ptr(U_saved), _ptr(dY), T, _ptr(dX), _ptr(dA), _ptr(dB), _ptr(ws),
+                         ws.numel(), _stream(stream))
+    _check(st, "qlora_bwd")
+    return dX, dA, dB
+
+
+def lora_merge(q: NF4Weight, A: torch.Tensor, B: torch.Tensor, alpha: float,
+               W_out: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
+               stream=None) -> torch.Tensor:
+    r = A.shape[0]
+    _need(A, torch.bfloat16, (r, q.k), "A")
+    _need(B, torch.bfloat16, (q.d, r), "B")
+    W_out = torch.empty(q.d, q.k, dtype=torch.bfloat16, device=A.device) if W_out is None else W_out
+    _need(W_out, torch.bfloat16, (q.d, q.k), "W_out")
+    nbytes = lora_merge_workspace_bytes(q.d, q.k, r)
+    ws = workspace(nbytes, A.device) if ws is None else ws
+    st = lib().lora_merge(ctypes.byref(q.cstruct), _ptr(A), _ptr(B), r, float(alpha), _ptr(W_out),
+                          _ptr(ws), ws.numel(), _stream(stream))
+    _check(st, "lora_merge")
+    return W_out
+
+
+def lora_unmerge(W: torch.Tensor, A: torch.Tensor, B: torch.Tensor, alpha: float,
+                 W0_out: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
+                 stream=None) -> torch.Tensor:
+    d, k = W.shape
+    r = A.shape[0]
+    _need(W, torch.bfloat16, (d, k), "W")
+    _need(A, torch.bfloat16, (r, k), "A")
+    _need(B, torch.bfloat16, (d, r), "B")
+    W0_out = torch.empty(d, k, dtype=torch.bfloat16, device=W.device) if W0_out is None else W0_out
+    _need(W0_out, torch.bfloat16, (d, k), "W0_out")
+    nbytes = lora_merge_workspace_bytes(d, k, r)
+    ws = workspace(nbytes, W.device) if ws is None else ws
+    st = lib().lora_unmerge(_ptr(W), _ptr(A), _ptr(B), r, float(alpha), d, k, _ptr(W0_out),
+                            _ptr(ws), ws.numel(), _stream(stream))
+    _check(st, "lora_unmerge")
+    return W0_out
+
+
+def qlora_get_device_status(stream=None) -> int:
+    v = ctypes.c_int(0)
+    _check(lib().qlora_get_device_status(_stream(stream), ctypes.byref(v)), "qlora_get_device_status")
+    return v.value
+
+
+def qlora_selftest_wait_timeout(limit_us: int, stream=None) -> None:
+    _check(lib().qlora_selftest_wait_timeout(int(limit_us), _stream(stream)), "qlora_selftest_wait_timeout")
+
+
+def qlora_profile_begin() -> None:
+    _check(lib().qlora_profile_begin(), "qlora_profile_begin")
+
+
+def qlora_profile_end():
+    cap = 64
+    arr = (KernelStat * cap)()
+    n = ctypes.c_int(0)
+    _check(lib().qlora_profile_end(arr, cap, ctypes.byref(n)), "qlora_profile_end")
+    return [{"name": arr[i].name.decode(), "launches": arr[i].launches, "total_ms": arr[i].total_ms,
+             "flops": arr[i].flops, "bytes": arr[i].bytes} for i in range(min(n.value, cap))]

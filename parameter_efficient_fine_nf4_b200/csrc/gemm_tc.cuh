@@ -1,0 +1,342 @@
+// Tensor-core GEMM engine for sm_100a (tcgen05 + TMEM + TMA).
+//
+//   C[M x N] (fp32, TMEM) = sum over K-steps of  A_tile * B_tile^T
+//
+// over two K segments: the main product (K0) followed by an optional
+// extension (K1 = r) whose operands are the rank-r factors.  This is how the
+// LoRA term joins the base product in one accumulator:
+//   Y  = [X | sU] [W' | B]^T      (forward, [P1] forward equation)
+//   dX = [dY | sG] [W' ; A]       (backward)
+// Each operand of each segment is K-major or MN-major in global memory; TMA
+// moves 64-wide (128-byte, 128B-swizzled) boxes into shared memory, so the
+// same tile serves as a K-major or MN-major UMMA operand by descriptor alone.
+//
+// Roles (192 threads): warp 0 issues TMA, warp 1 owns TMEM and issues UMMA
+// (one thread), warps 2-5 drain TMEM in the epilogue.  A STAGES-deep ring of
+// full/empty mbarriers couples producer and MMA; tcgen05.commit frees a stage
+// when the MMAs reading it finish.  All waits are bounded (see ptx.cuh).
+#pragma once
+#include "ptx.cuh"
+#include "nf4_kernels.cuh"
+
+namespace qlora {
+
+constexpr int kBM = 128;
+constexpr int kBK = 64;
+constexpr int kGemmThreads = 192;
+
+enum EpiKind : int {
+  EPI_BF16 = 0,      // out bf16 [M][ldo] = acc
+  EPI_F32 = 1,       // out fp32 [M][ldo] = alpha*acc ; out2 bf16 = alpha2*acc
+  EPI_F32_T = 2,     // out fp32 [N][ldo] = alpha*acc (transposed store)
+  EPI_MERGE = 3,     // out bf16 = bf16(alpha*acc + dequant(codes))
+  EPI_UNMERGE = 4    // out bf16 = bf16(alpha*acc + w_in)
+};
+
+struct GemmArgs {
+  int M, N;
+  int K0, K1;
+  int a0_mn, b0_mn, a1_mn, b1_mn;
+  int k_per_split;            // K0 columns per blockIdx.y (multiple of 64)
+  int tiles_m, tiles_n, group_m;
+  int epi;
+  void* out;
+  int64_t ldo;
+  int64_t split_stride;       // elements between split-K partial outputs
+  float alpha;
+  int n_store;
+  uint16_t* out2;
+  int64_t ldo2;
+  float alpha2;
+  int n_store2;
+  const uint8_t* codes;
+  const uint8_t* absmax_q;
+  const float* scale2;
+  const float* mean;
+  const uint16_t* w_in;
+  int64_t ldw;
+  float levels[16];
+};
+
+template <int BN>
+struct GemmCfg {
+  static constexpr int kStages = (BN >= 256) ? 4 : (BN >= 128 ? 5 : 6);
+  static constexpr int kABytes = kBM * kBK * 2;                 // 16 KB
+  static constexpr int kBBytes = BN * kBK * 2;
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kTmemCols = BN;                           // power of two >= 64
+  static constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 512 /*bars*/;
+};
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  const __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&p);
+}
+
+__device__ __forceinline__ float bf16_bits_to_f32(uint32_t b16) { return __uint_as_float(b16 << 16); }
+
+template <int BN>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmB0,
+                   const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
+                   const __grid_constant__ GemmArgs p) {
+  using Cfg = GemmCfg<BN>;
+  constexpr int S = Cfg::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  // 1024-byte alignment for the 128B-swizzle atoms
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  const uint32_t pad = (1024u - (raw_addr & 1023u)) & 1023u;
+  uint8_t* smem = smem_raw + pad;
+  const uint32_t sbase = raw_addr + pad;
+  uint8_t* ctrl = smem + S * Cfg::kStageBytes;
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(ctrl);
+  uint64_t* empty_bar = full_bar + S;
+  uint64_t* accum_bar = empty_bar + S;
+  uint64_t* drain_bar = accum_bar + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_bar + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* s_lut = reinterpret_cast<float*>(tmem_slot + 4);        // 16 floats
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // tile coordinates (grouped rasterisation along M)
+  const int tile = blockIdx.x;
+  const int per_group = p.group_m * p.tiles_n;
+  const int gidx = tile / per_group;
+  const int first_m = gidx * p.group_m;
+  const int gsize = min(p.group_m, p.tiles_m - first_m);
+  const int in_group = tile - gidx * per_group;
+  const int tm = first_m + in_group % gsize;
+  const int tn = in_group / gsize;
+  const int m0 = tm * kBM;
+  const int n0 = tn * BN;
+  const int split = blockIdx.y;
+  const int k_begin = split * p.k_per_split;
+  const int k_len0 = min(p.K0 - k_begin, p.k_per_split);
+  const int steps0 = (k_len0 + kBK - 1) / kBK;
+  const int steps1 = (p.K1 + kBK - 1) / kBK;
+  const int steps = steps0 + steps1;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < S; ++i) {
+      mbar_init(smem_u32(&full_bar[i]), 1);
+      mbar_init(smem_u32(&empty_bar[i]), 1);
+    }
+    mbar_init(smem_u32(accum_bar), 1);
+    mbar_init(smem_u32(drain_bar), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (threadIdx.x < 16) s_lut[threadIdx.x] = p.levels[threadIdx.x];
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), Cfg::kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA0);
+    tma_prefetch_desc(&tmB0);
+    if (steps1 > 0) {
+      tma_prefetch_desc(&tmA1);
+      tma_prefetch_desc(&tmB1);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int issued[S];
+#pragma unroll
+      for (int i = 0; i < S; ++i) issued[i] = 0;
+      for (int step = 0; step < steps; ++step) {
+        const int st = step % S;
+        const uint32_t ph = (uint32_t)((step / S) & 1);
+        if (!mbar_wait_bounded(smem_u32(&empty_bar[st]), ph ^ 1u, abort_flag)) break;
+        const uint32_t fb = smem_u32(&full_bar[st]);
+        mbar_arrive_expect_tx(fb, Cfg::kStageBytes);
+        const uint32_t sa = sbase + st * Cfg::kStageBytes;
+        const uint32_t sb = sa + Cfg::kABytes;
+        const bool ext = step >= steps0;
+        const int kk = ext ? (step - steps0) * kBK : k_begin + step * kBK;
+        const CUtensorMap* ma = ext ? &tmA1 : &tmA0;
+        const CUtensorMap* mb = ext ? &tmB1 : &tmB0;
+        const int a_mn = ext ? p.a1_mn : p.a0_mn;
+        const int b_mn = ext ? p.b1_mn : p.b0_mn;
+        if (a_mn) {
+          tma_load_2d(sa, ma, fb, m0, kk);
+          tma_load_2d(sa + 8192, ma, fb, m0 + 64, kk);
+        } else {
+          tma_load_2d(sa, ma, fb, kk, m0);
+        }
+        if (b_mn) {
+#pragma unroll
+          for (int i = 0; i < BN / 64; ++i) tma_load_2d(sb + i * 8192, mb, fb, n0 + 64 * i, kk);
+        } else {
+          tma_load_2d(sb, mb, fb, kk, n0);
+        }
+        issued[st] += 1;
+      }
+      if (*abort_flag) {
+        // let copies already in flight land before the CTA exits
+        for (int i = 0; i < S; ++i)
+          if (issued[i] > 0) mbar_wait_bounded(smem_u32(&full_bar[i]), (uint32_t)((issued[i] - 1) & 1), nullptr);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc0 = idesc_bf16_f32(kBM, BN, p.a0_mn, p.b0_mn);
+      const uint32_t idesc1 = idesc_bf16_f32(kBM, BN, p.a1_mn, p.b1_mn);
+      bool ok = true;
+      int issued_any = 0;
+      for (int step = 0; step < steps; ++step) {
+        const int st = step % S;
+        const uint32_t ph = (uint32_t)((step / S) & 1);
+        if (!mbar_wait_bounded(smem_u32(&full_bar[st]), ph, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const bool ext = step >= steps0;
+        const int a_mn = ext ? p.a1_mn : p.a0_mn;
+        const int b_mn = ext ? p.b1_mn : p.b0_mn;
+        const uint32_t idesc = ext ? idesc1 : idesc0;
+        int nsub = 4;
+        if (ext) {
+          const int rem = p.K1 - (step - steps0) * kBK;
+          nsub = min(4, (rem + 15) / 16);
+        }
+        const uint32_t sa = sbase + st * Cfg::kStageBytes;
+        const uint32_t sb = sa + Cfg::kABytes;
+        for (int j = 0; j < nsub; ++j) {
+          // K-major: 16 elements = 32 bytes along the swizzled row;
+          // MN-major: 16 K-rows of 128 bytes.
+          const uint32_t ao = a_mn ? (uint32_t)j * 2048u : (uint32_t)j * 32u;
+          const uint32_t bo = b_mn ? (uint32_t)j * 2048u : (uint32_t)j * 32u;
+          const uint64_t adesc = a_mn ? smem_desc_sw128(sa + ao, 8192, 1024) : smem_desc_sw128(sa + ao, 16, 1024);
+          const uint64_t bdesc = b_mn ? smem_desc_sw128(sb + bo, 8192, 1024) : smem_desc_sw128(sb + bo, 16, 1024);
+          umma_bf16(tmem_base, adesc, bdesc, idesc, (step > 0 || j > 0) ? 1u : 0u);
+          issued_any = 1;
+        }
+        umma_commit(smem_u32(&empty_bar[st]));
+      }
+      if (ok) {
+        umma_commit(smem_u32(accum_bar));
+      } else if (issued_any) {
+        // wait for MMAs already issued before TMEM is released
+        umma_commit(smem_u32(drain_bar));
+        mbar_wait_bounded(smem_u32(drain_bar), 0, nullptr);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int quarter = warp & 3;             // TMEM lane quarter of this warp
+    const int row = quarter * 32 + lane;
+    const int m = m0 + row;
+    const bool row_ok = m < p.M;
+    const bool have = mbar_wait_bounded(smem_u32(accum_bar), 0, abort_flag);
+    tc_fence_after();
+    if (have) {
+      const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16);
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(taddr + (uint32_t)(c * 32), v);
+        tmem_ld_wait();
+        const int n = n0 + c * 32;
+        if (!row_ok || n >= p.N) continue;
+        if (p.epi == EPI_BF16) {
+          uint16_t* out = reinterpret_cast<uint16_t*>(p.out) + (int64_t)m * p.ldo + n;
+          if (n + 32 <= p.n_store && (p.ldo & 7) == 0) {
+            uint4* o4 = reinterpret_cast<uint4*>(out);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              uint4 w;
+              w.x = pack_bf16x2(__uint_as_float(v[8 * i + 0]), __uint_as_float(v[8 * i + 1]));
+              w.y = pack_bf16x2(__uint_as_float(v[8 * i + 2]), __uint_as_float(v[8 * i + 3]));
+              w.z = pack_bf16x2(__uint_as_float(v[8 * i + 4]), __uint_as_float(v[8 * i + 5]));
+              w.w = pack_bf16x2(__uint_as_float(v[8 * i + 6]), __uint_as_float(v[8 * i + 7]));
+              o4[i] = w;
+            }
+          } else {
+            for (int i = 0; i < 32 && n + i < p.n_store; ++i) {
+              __nv_bfloat16 h = __float2bfloat16_rn(__uint_as_float(v[i]));
+              out[i] = *reinterpret_cast<uint16_t*>(&h);
+            }
+          }
+        } else if (p.epi == EPI_F32) {
+          float* out = reinterpret_cast<float*>(p.out) + (int64_t)split * p.split_stride + (int64_t)m * p.ldo + n;
+          if (p.out != nullptr) {
+            if (n + 32 <= p.n_store && (p.ldo & 3) == 0) {
+              float4* o4 = reinterpret_cast<float4*>(out);
+#pragma unroll
+              for (int i = 0; i < 8; ++i)
+                o4[i] = make_float4(p.alpha * __uint_as_float(v[4 * i]), p.alpha * __uint_as_float(v[4 * i + 1]),
+                                    p.alpha * __uint_as_float(v[4 * i + 2]), p.alpha * __uint_as_float(v[4 * i + 3]));
+            } else {
+              for (int i = 0; i < 32 && n + i < p.n_store; ++i) out[i] = p.alpha * __uint_as_float(v[i]);
+            }
+          }
+          if (p.out2 != nullptr) {
+            uint16_t* o2 = p.out2 + (int64_t)m * p.ldo2 + n;
+            for (int i = 0; i < 32 && n + i < p.n_store2; ++i) {
+              __nv_bfloat16 h = __float2bfloat16_rn(__fmul_rn(p.alpha2, __uint_as_float(v[i])));
+              o2[i] = *reinterpret_cast<uint16_t*>(&h);
+            }
+          }
+        } else if (p.epi == EPI_F32_T) {
+          float* out = reinterpret_cast<float*>(p.out) + (int64_t)split * p.split_stride + m;
+          for (int i = 0; i < 32 && n + i < p.n_store; ++i)
+            out[(int64_t)(n + i) * p.ldo] = p.alpha * __uint_as_float(v[i]);
+        } else if (p.epi == EPI_MERGE) {
+          // w' for row m, columns n..n+31: one 16-byte word of codes, one block
+          const int64_t e0 = (int64_t)m * p.N + n;
+          const uint4 cw = *reinterpret_cast<const uint4*>(p.codes + e0 / 2);
+          const float a_scale = block_scale(p.absmax_q, p.scale2, p.mean[0], e0 / kBlock);
+          uint32_t wq[16];
+          dequant32(cw, a_scale, s_lut, wq);
+          uint16_t* out = reinterpret_cast<uint16_t*>(p.out) + (int64_t)m * p.ldo + n;
+          uint4* o4 = reinterpret_cast<uint4*>(out);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            uint32_t r4[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const uint32_t wp = wq[4 * i + j];
+              const float lo = __fmaf_rn(p.alpha, __uint_as_float(v[8 * i + 2 * j]), bf16_bits_to_f32(wp & 0xFFFFu));
+              const float hi = __fmaf_rn(p.alpha, __uint_as_float(v[8 * i + 2 * j + 1]), bf16_bits_to_f32(wp >> 16));
+              r4[j] = pack_bf16x2(lo, hi);
+            }
+            o4[i] = make_uint4(r4[0], r4[1], r4[2], r4[3]);
+          }
+        } else if (p.epi == EPI_UNMERGE) {
+          const uint4* w4 = reinterpret_cast<const uint4*>(p.w_in + (int64_t)m * p.ldw + n);
+          uint16_t* out = reinterpret_cast<uint16_t*>(p.out) + (int64_t)m * p.ldo + n;
+          uint4* o4 = reinterpret_cast<uint4*>(out);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const uint4 wv = w4[i];
+            const uint32_t wr[4] = {wv.x, wv.y, wv.z, wv.w};
+            uint32_t r4[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const float lo = __fmaf_rn(p.alpha, __uint_as_float(v[8 * i + 2 * j]), bf16_bits_to_f32(wr[j] & 0xFFFFu));
+              const float hi = __fmaf_rn(p.alpha, __uint_as_float(v[8 * i + 2 * j + 1]), bf16_bits_to_f32(wr[j] >> 16));
+              r4[j] = pack_bf16x2(lo, hi);
+            }
+            o4[i] = make_uint4(r4[0], r4[1], r4[2], r4[3]);
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) tmem_dealloc(tmem_base, Cfg::kTmemCols);
+}
+
+}  // namespace qlora

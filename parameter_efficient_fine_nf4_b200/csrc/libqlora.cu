@@ -1,0 +1,761 @@
+// libqlora: C ABI of the QLoRA linear layer on sm_100a.
+//
+// One translation unit: the kernels (nf4_kernels.cuh, gemm_tc.cuh) and the
+// host entry points declared in include/qlora.h.  The host code validates
+// arguments, carves the caller's workspace, builds TMA tensor maps and
+// launches kernels on the caller's stream.  It never allocates device memory.
+#include <atomic>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "../../include/qlora.h"
+#include "gemm_tc.cuh"
+#include "nf4_kernels.cuh"
+#include "ptx.cuh"
+
+namespace qlora {
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr int kSMs = 148;
+
+std::atomic<int64_t> g_launches{0};
+
+// --------------------------------------------------------------- NF4 table
+// [P1] 4-bit NormalFloat paragraph: levels at N(0,1) quantiles, 2^(k-1)
+// negative and 2^(k-1)+1 positive points with one shared zero dropped, and
+// an exact zero; normalised so the ends are -1 and +1.  The outermost
+// probability is not printed on the pages; this library uses
+// p_max = 1 - (1/2)(1/32 + 1/30) and spaces each side's probabilities evenly
+// from p_max down to 1/2.  Quantiles by Newton's method on the normal CDF in
+// long double (monotone convergence from 0 because the CDF is concave on
+// the positive half-line).
+long double normal_cdf(long double x) { return 0.5L * erfcl(-x / sqrtl(2.0L)); }
+
+long double normal_quantile(long double p) {
+  if (p == 0.5L) return 0.0L;
+  const long double inv_sqrt_2pi = 0.398942280401432677939946059934381868L;
+  long double x = 0.0L;
+  for (int it = 0; it < 200; ++it) {
+    const long double f = normal_cdf(x) - p;
+    const long double dfdx = inv_sqrt_2pi * expl(-0.5L * x * x);
+    const long double dx = f / dfdx;
+    x -= dx;
+    if (fabsl(dx) <= 1e-19L * (1.0L + fabsl(x))) break;
+  }
+  return x;
+}
+
+struct HostTables {
+  float levels[16];
+  float thresholds[15];
+  EncTable enc;
+};
+
+HostTables build_tables() {
+  HostTables t;
+  const long double pmax = 1.0L - 0.5L * (1.0L / 32.0L + 1.0L / 30.0L);
+  long double v[16];
+  int n = 0;
+  for (int i = 0; i < 7; ++i) v[n++] = -normal_quantile(pmax - i * (pmax - 0.5L) / 7.0L);
+  v[n++] = 0.0L;
+  for (int i = 7; i >= 0; --i) v[n++] = normal_quantile(pmax - i * (pmax - 0.5L) / 8.0L);
+  const long double top = normal_quantile(pmax);
+  for (int i = 0; i < 16; ++i) t.levels[i] = (float)(v[i] / top);
+  t.levels[0] = -1.0f;
+  t.levels[15] = 1.0f;
+  for (int i = 0; i < 15; ++i) {
+    const double mid = 0.5 * ((double)t.levels[i] + (double)t.levels[i + 1]);  // exact
+    float f = (float)mid;
+    if ((double)f <= mid) f = nextafterf(f, 2.0f);
+    t.thresholds[i] = f;
+  }
+  for (int j = 0; j < kEncBins; ++j) {
+    const double lo = (double)(j - 64) / 64.0;
+    const double hi = (double)(j - 63) / 64.0;
+    int base = 0;
+    float inside = INFINITY;
+    for (int i = 0; i < 15; ++i) {
+      const double th = (double)t.thresholds[i];
+      if (th <= lo) ++base;
+      else if (th < hi) inside = t.thresholds[i];
+    }
+    t.enc.base[j] = base;
+    t.enc.thr[j] = inside;
+  }
+  return t;
+}
+
+const HostTables& tables() {
+  static const HostTables t = build_tables();
+  return t;
+}
+
+// --------------------------------------------------------------- device setup
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return (EncodeTiledFn) nullptr;
+    return reinterpret_cast<EncodeTiledFn>(p);
+  }();
+  return fn;
+}
+
+std::mutex g_init_mu;
+bool g_dev_ready[kMaxDevices] = {false};
+
+template <int BN>
+cudaError_t set_gemm_attrs() {
+  return cudaFuncSetAttribute(gemm_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              GemmCfg<BN>::kSmemBytes);
+}
+
+int ensure_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return QLORA_ERR_NO_DEVICE;
+  if (dev < 0 || dev >= kMaxDevices) return QLORA_ERR_NO_DEVICE;
+  std::lock_guard<std::mutex> lk(g_init_mu);
+  if (g_dev_ready[dev]) return QLORA_OK;
+  int major = 0, minor = 0;
+  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+  if (major != 10 || minor != 0) return QLORA_ERR_NO_DEVICE;
+  if (encode_fn() == nullptr) return QLORA_ERR_CUDA;
+  if (set_gemm_attrs<64>() != cudaSuccess || set_gemm_attrs<128>() != cudaSuccess ||
+      set_gemm_attrs<256>() != cudaSuccess)
+    return QLORA_ERR_CUDA;
+  g_dev_ready[dev] = true;
+  return QLORA_OK;
+}
+
+// --------------------------------------------------------------- profiling
+struct ProfRec {
+  std::string name;
+  double flops, bytes;
+  cudaEvent_t start, stop;
+};
+std::mutex g_prof_mu;
+bool g_prof_on = false;
+std::vector<ProfRec> g_prof;
+std::vector<cudaEvent_t> g_event_pool;
+
+cudaEvent_t take_event() {
+  if (!g_event_pool.empty()) {
+    cudaEvent_t e = g_event_pool.back();
+    g_event_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  cudaEventCreate(&e);
+  return e;
+}
+
+// Launch wrapper: counts the launch, checks the launch error and, when
+// profiling, brackets it with events on the launch stream.
+template <typename F>
+int launch(const char* name, double flops, double bytes, cudaStream_t stream, F&& fn) {
+  cudaEvent_t a = nullptr, b = nullptr;
+  bool prof = false;
+  {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    prof = g_prof_on;
+    if (prof) {
+      a = take_event();
+      b = take_event();
+    }
+  }
+  if (prof) cudaEventRecord(a, stream);
+  fn();
+  cudaError_t err = cudaGetLastError();
+  g_launches.fetch_add(1);
+  if (prof) {
+    cudaEventRecord(b, stream);
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    g_prof.push_back(ProfRec{name, flops, bytes, a, b});
+  }
+  return err == cudaSuccess ? QLORA_OK : QLORA_ERR_CUDA;
+}
+
+// --------------------------------------------------------------- helpers
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline int64_t round_up(int64_t a, int64_t b) { return (a + b - 1) / b * b; }
+inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+inline int grid_for(int64_t n, int threads) {
+  int64_t g = cdiv(n, threads);
+  const int64_t cap = (int64_t)kSMs * 16;
+  if (g > cap) g = cap;
+  if (g < 1) g = 1;
+  return (int)g;
+}
+
+// bf16 2-D tensor map: `inner` contiguous elements per row, `outer` rows,
+// `ld` elements between rows; box = 64 (inner, 128 bytes) x box_outer.
+bool make_map(CUtensorMap* map, const void* base, int64_t inner, int64_t outer, int64_t ld,
+              int box_outer) {
+  cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)outer};
+  cuuint64_t strides[1] = {(cuuint64_t)(ld * 2)};
+  cuuint32_t box[2] = {64u, (cuuint32_t)box_outer};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = encode_fn()(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                           strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// One GEMM operand as stored in global memory.
+struct Operand {
+  const void* ptr = nullptr;
+  int64_t inner = 0, outer = 0, ld = 0;   // bf16 elements
+  int mn_major = 0;                       // 1: the M (or N) index is the contiguous one
+};
+
+inline Operand kmajor(const void* p, int64_t K, int64_t rows, int64_t ld) {
+  Operand o; o.ptr = p; o.inner = K; o.outer = rows; o.ld = ld; o.mn_major = 0; return o;
+}
+inline Operand mnmajor(const void* p, int64_t MN, int64_t K, int64_t ld) {
+  Operand o; o.ptr = p; o.inner = MN; o.outer = K; o.ld = ld; o.mn_major = 1; return o;
+}
+
+struct GemmPlan {
+  int M, N, K0, K1 = 0;
+  Operand a0, b0, a1, b1;
+  int splits = 1;
+  int bn = 256;
+};
+
+template <int BN>
+int launch_gemm_bn(const char* name, const GemmPlan& g, GemmArgs args, cudaStream_t st) {
+  CUtensorMap m[4];
+  memset(m, 0, sizeof(m));
+  const Operand* ops[4] = {&g.a0, &g.b0, &g.a1, &g.b1};
+  const int nops = g.K1 > 0 ? 4 : 2;
+  for (int i = 0; i < nops; ++i) {
+    const Operand& o = *ops[i];
+    const bool is_a = (i % 2) == 0;
+    const int box_outer = o.mn_major ? 64 : (is_a ? kBM : BN);
+    if (!make_map(&m[i], o.ptr, o.inner, o.outer, o.ld, box_outer)) return QLORA_ERR_CUDA;
+  }
+  if (nops == 2) { m[2] = m[0]; m[3] = m[1]; }
+  args.M = g.M; args.N = g.N; args.K0 = g.K0; args.K1 = g.K1;
+  args.a0_mn = g.a0.mn_major; args.b0_mn = g.b0.mn_major;
+  args.a1_mn = g.K1 > 0 ? g.a1.mn_major : 0; args.b1_mn = g.K1 > 0 ? g.b1.mn_major : 0;
+  args.tiles_m = (int)cdiv(g.M, kBM);
+  args.tiles_n = (int)cdiv(g.N, BN);
+  args.group_m = 16;
+  args.k_per_split = (int)round_up(cdiv(g.K0, g.splits), kBK);
+  const int splits = (int)cdiv(g.K0, args.k_per_split);
+  const auto& T = tables();
+  memcpy(args.levels, T.levels, sizeof(args.levels));
+  dim3 grid((unsigned)(args.tiles_m * args.tiles_n), (unsigned)splits, 1);
+  const double flops = 2.0 * g.M * (double)g.N * (g.K0 + g.K1);
+  return launch(name, flops, 0.0, st, [&] {
+    gemm_tc_kernel<BN><<<grid, kGemmThreads, GemmCfg<BN>::kSmemBytes, st>>>(m[0], m[1], m[2], m[3], args);
+  });
+}
+
+int launch_gemm(const char* name, const GemmPlan& g, const GemmArgs& args, cudaStream_t st) {
+  for (const Operand* o : {&g.a0, &g.b0}) {
+    if (!aligned16(o->ptr) || (o->ld * 2) % 16 != 0) return QLORA_ERR_MISALIGNED;
+  }
+  if (g.K1 > 0) {
+    for (const Operand* o : {&g.a1, &g.b1})
+      if (!aligned16(o->ptr) || (o->ld * 2) % 16 != 0) return QLORA_ERR_MISALIGNED;
+  }
+  switch (g.bn) {
+    case 64: return launch_gemm_bn<64>(name, g, args, st);
+    case 128: return launch_gemm_bn<128>(name, g, args, st);
+    default: return launch_gemm_bn<256>(name, g, args, st);
+  }
+}
+
+inline int bn_for_rank(int r) { return r <= 64 ? 64 : (r <= 128 ? 128 : 256); }
+
+GemmArgs blank_args() {
+  GemmArgs a;
+  memset(&a, 0, sizeof(a));
+  a.alpha = 1.0f;
+  a.alpha2 = 1.0f;
+  return a;
+}
+
+// Workspace carving (256-byte aligned pieces).
+struct Carver {
+  uint8_t* base;
+  size_t off = 0;
+  void* take(size_t bytes) {
+    void* p = base ? base + off : nullptr;
+    off += (size_t)round_up((int64_t)bytes, 256);
+    return p;
+  }
+};
+
+int check_nf4(const qlora_nf4_t* q) {
+  if (!q || !q->codes || !q->absmax_q || !q->scale2 || !q->mean) return QLORA_ERR_INVALID_ARG;
+  if (q->block != kBlock || q->block2 != kBlock2) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (q->d < 1 || q->k < 64 || q->k % 64 != 0) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (q->d > (int64_t)1 << 31 || q->k > (int64_t)1 << 31 || q->d * q->k >= ((int64_t)1 << 34))
+    return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(q->codes)) return QLORA_ERR_MISALIGNED;
+  return QLORA_OK;
+}
+
+int check_rank(int r, float alpha) {
+  if (r < 1 || r > 256) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (!(alpha > 0.0f) || !std::isfinite(alpha)) return QLORA_ERR_INVALID_ARG;
+  return QLORA_OK;
+}
+
+#define QLORA_TRY(x)            \
+  do {                          \
+    int _s = (x);               \
+    if (_s != QLORA_OK) return _s; \
+  } while (0)
+
+int dequantize_into(const qlora_nf4_t* q, uint16_t* W, cudaStream_t st) {
+  const int64_t n_chunks = q->d * q->k / 32;
+  const auto& T = tables();
+  NF4Levels lv;
+  memcpy(lv.q, T.levels, sizeof(lv.q));
+  const int grid = grid_for(n_chunks, 256);
+  const double bytes = (double)q->d * q->k * 2.5;
+  return launch("nf4_dequantize", 0.0, bytes, st, [&] {
+    nf4_dequantize_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const uint4*>(q->codes), q->absmax_q,
+                                                q->scale2, q->mean, n_chunks,
+                                                reinterpret_cast<uint4*>(W), lv);
+  });
+}
+
+// B (d x r) with rows padded to r8 columns, when r is not a multiple of 8.
+const uint16_t* padded_B(const uint16_t* B, int64_t d, int r, int r8, uint16_t* ws, cudaStream_t st,
+                         int* status) {
+  if (r == r8) return B;
+  *status = launch("pad_cols_bf16", 0.0, 0.0, st, [&] {
+    pad_cols_bf16<<<grid_for(d * r8, 256), 256, 0, st>>>(B, d, r, ws, r8);
+  });
+  return ws;
+}
+
+struct FwdWs {
+  uint16_t* Wdq; uint16_t* sU; uint16_t* Bp; size_t bytes;
+};
+FwdWs carve_fwd(void* ws, int64_t d, int64_t k, int r, int64_t T) {
+  Carver c{reinterpret_cast<uint8_t*>(ws)};
+  const int64_t r8 = round_up(r, 8);
+  FwdWs w;
+  w.Wdq = (uint16_t*)c.take((size_t)(d * k * 2));
+  w.sU = (uint16_t*)c.take((size_t)(std::max<int64_t>(T, 1) * r8 * 2));
+  w.Bp = (uint16_t*)c.take((size_t)(d * r8 * 2));
+  w.bytes = c.off;
+  return w;
+}
+
+int splits_for(int64_t tiles, int64_t K) {
+  int s = 1;
+  while (tiles * s < 2 * kSMs && (K / (s * 2)) >= 1024 && s < 32) s *= 2;
+  return s;
+}
+
+struct BwdWs {
+  uint16_t* Wdq; uint16_t* Us; uint16_t* Gs; uint16_t* Bp; float* partA; float* partB;
+  int splitsA, splitsB; size_t bytes;
+};
+BwdWs carve_bwd(void* ws, int64_t d, int64_t k, int r, int64_t T) {
+  Carver c{reinterpret_cast<uint8_t*>(ws)};
+  const int64_t r8 = round_up(r, 8);
+  const int64_t Tm = std::max<int64_t>(T, 1);
+  BwdWs w;
+  w.Wdq = (uint16_t*)c.take((size_t)(d * k * 2));
+  w.Us = (uint16_t*)c.take((size_t)(Tm * r8 * 2));
+  w.Gs = (uint16_t*)c.take((size_t)(Tm * r8 * 2));
+  w.Bp = (uint16_t*)c.take((size_t)(d * r8 * 2));
+  w.splitsA = splits_for(cdiv(k, kBM), Tm);
+  w.splitsB = splits_for(cdiv(d, kBM), Tm);
+  w.partA = (float*)c.take((size_t)(w.splitsA > 1 ? w.splitsA * r * k * 4 : 0));
+  w.partB = (float*)c.take((size_t)(w.splitsB > 1 ? w.splitsB * d * r * 4 : 0));
+  w.bytes = c.off;
+  return w;
+}
+
+}  // namespace
+}  // namespace qlora
+
+using namespace qlora;
+
+// =====================================================================
+// C ABI
+// =====================================================================
+extern "C" {
+
+const char* qlora_strerror(int s) {
+  switch (s) {
+    case QLORA_OK: return "ok";
+    case QLORA_ERR_INVALID_ARG: return "invalid argument";
+    case QLORA_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+    case QLORA_ERR_MISALIGNED: return "pointer or leading dimension not 16-byte aligned";
+    case QLORA_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case QLORA_ERR_CUDA: return "CUDA error";
+    case QLORA_ERR_TIMEOUT: return "device wait timed out";
+    case QLORA_ERR_NO_DEVICE: return "no sm_100 device is current";
+    default: return "unknown status";
+  }
+}
+
+int qlora_version(void) { return 100; }
+
+int qlora_nf4_levels(float* levels16, float* thresholds15) {
+  const auto& T = tables();
+  if (levels16) memcpy(levels16, T.levels, sizeof(T.levels));
+  if (thresholds15) memcpy(thresholds15, T.thresholds, sizeof(T.thresholds));
+  return QLORA_OK;
+}
+
+int64_t qlora_launch_count(void) { return g_launches.load(); }
+
+size_t qlora_quantize_workspace_bytes(int64_t d, int64_t k) {
+  if (d < 1 || k < 1) return 0;
+  const int64_t n_b = d * k / kBlock;
+  const int64_t n_g = cdiv(n_b, kBlock2);
+  return (size_t)(round_up(n_b * 4, 256) + round_up(n_g * 8, 256));
+}
+
+int qlora_nf4_quantize(const float* W0, int64_t d, int64_t k, int block, qlora_nf4_t* out,
+                       void* ws, size_t ws_bytes, qlora_stream_t stream) {
+  if (!W0 || !out || !out->codes || !out->absmax_q || !out->scale2 || !out->mean)
+    return QLORA_ERR_INVALID_ARG;
+  if (block != kBlock) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (d < 1 || k < 64 || k % 64 != 0 || d * k >= ((int64_t)1 << 34)) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(W0) || !aligned16(out->codes)) return QLORA_ERR_MISALIGNED;
+  if (!ws || ws_bytes < qlora_quantize_workspace_bytes(d, k)) return QLORA_ERR_WORKSPACE_TOO_SMALL;
+  QLORA_TRY(ensure_device());
+  out->d = d; out->k = k; out->block = kBlock; out->block2 = kBlock2;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t n_b = d * k / kBlock;
+  const int64_t n_g = cdiv(n_b, kBlock2);
+  Carver c{reinterpret_cast<uint8_t*>(ws)};
+  float* absmax = (float*)c.take((size_t)(n_b * 4));
+  double* gsum = (double*)c.take((size_t)(n_g * 8));
+  const auto& T = tables();
+  const double bytes1 = (double)d * k * 4.5 + (double)n_b * 4;
+  QLORA_TRY(launch("nf4_quantize_phase1", 0.0, bytes1, st, [&] {
+    nf4_quantize_phase1<<<(unsigned)n_g, 256, 0, st>>>(W0, n_b, reinterpret_cast<uint32_t*>(out->codes),
+                                                       absmax, gsum, T.enc);
+  }));
+  QLORA_TRY(launch("nf4_quantize_mean", 0.0, (double)n_g * 8, st, [&] {
+    nf4_quantize_mean<<<1, 1024, 0, st>>>(gsum, n_g, n_b, out->mean);
+  }));
+  QLORA_TRY(launch("nf4_quantize_dq", 0.0, (double)n_b * 5 + n_g * 4, st, [&] {
+    nf4_quantize_dq<<<(unsigned)n_g, 256, 0, st>>>(absmax, n_b, out->mean, out->absmax_q, out->scale2);
+  }));
+  return QLORA_OK;
+}
+
+int qlora_nf4_dequantize(const qlora_nf4_t* q, uint16_t* W_out, qlora_stream_t stream) {
+  QLORA_TRY(check_nf4(q));
+  if (!W_out) return QLORA_ERR_INVALID_ARG;
+  if (!aligned16(W_out)) return QLORA_ERR_MISALIGNED;
+  QLORA_TRY(ensure_device());
+  return dequantize_into(q, W_out, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t qlora_fwd_workspace_bytes(int64_t d, int64_t k, int r, int64_t T) {
+  if (d < 1 || k < 1 || r < 1 || T < 0) return 0;
+  return carve_fwd(nullptr, d, k, r, T).bytes;
+}
+
+int qlora_fwd(const qlora_nf4_t* q, const uint16_t* A, const uint16_t* B, int r, float alpha,
+              const uint16_t* X, int64_t T, uint16_t* Y, float* U_save, void* ws, size_t ws_bytes,
+              qlora_stream_t stream) {
+  QLORA_TRY(check_nf4(q));
+  QLORA_TRY(check_rank(r, alpha));
+  if (T < 0) return QLORA_ERR_INVALID_ARG;
+  if (T == 0) return QLORA_OK;
+  if (!A || !B || !X || !Y || !U_save || !ws) return QLORA_ERR_INVALID_ARG;
+  if (!aligned16(A) || !aligned16(X) || !aligned16(Y) || !aligned16(U_save) || !aligned16(ws))
+    return QLORA_ERR_MISALIGNED;
+  const int64_t d = q->d, k = q->k;
+  if (T > ((int64_t)1 << 31)) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  FwdWs w = carve_fwd(ws, d, k, r, T);
+  if (ws_bytes < w.bytes) return QLORA_ERR_WORKSPACE_TOO_SMALL;
+  QLORA_TRY(ensure_device());
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const float s = alpha / (float)r;
+  const int r8 = (int)round_up(r, 8);
+
+  QLORA_TRY(dequantize_into(q, w.Wdq, st));
+  int pst = QLORA_OK;
+  const uint16_t* Bp = padded_B(B, d, r, r8, w.Bp, st, &pst);
+  QLORA_TRY(pst);
+
+  // U = X A^T (fp32 to U_save), sU = bf16(s U) (operand of the extension)
+  {
+    GemmPlan g;
+    g.M = (int)T; g.N = r; g.K0 = (int)k; g.bn = bn_for_rank(r);
+    g.a0 = kmajor(X, k, T, k);
+    g.b0 = kmajor(A, k, r, k);
+    GemmArgs a = blank_args();
+    a.epi = EPI_F32; a.out = U_save; a.ldo = r; a.alpha = 1.0f; a.n_store = r;
+    a.out2 = w.sU; a.ldo2 = r8; a.alpha2 = s; a.n_store2 = r8;
+    QLORA_TRY(launch_gemm("gemm_lora_down", g, a, st));
+  }
+  // Y = [X | sU] [W' | B]^T
+  {
+    GemmPlan g;
+    g.M = (int)T; g.N = (int)d; g.K0 = (int)k; g.K1 = r; g.bn = 256;
+    g.a0 = kmajor(X, k, T, k);
+    g.b0 = kmajor(w.Wdq, k, d, k);
+    g.a1 = kmajor(w.sU, r8, T, r8);
+    g.b1 = kmajor(Bp, r8, d, r8);
+    GemmArgs a = blank_args();
+    a.epi = EPI_BF16; a.out = Y; a.ldo = d; a.n_store = (int)d;
+    QLORA_TRY(launch_gemm("gemm_fwd_main", g, a, st));
+  }
+  return QLORA_OK;
+}
+
+size_t qlora_bwd_workspace_bytes(int64_t d, int64_t k, int r, int64_t T) {
+  if (d < 1 || k < 1 || r < 1 || T < 0) return 0;
+  return carve_bwd(nullptr, d, k, r, T).bytes;
+}
+
+int qlora_bwd(const qlora_nf4_t* q, const uint16_t* A, const uint16_t* B, int r, float alpha,
+              const uint16_t* X, const float* U_saved, const uint16_t* dY, int64_t T, uint16_t* dX,
+              float* dA, float* dB, void* ws, size_t ws_bytes, qlora_stream_t stream) {
+  QLORA_TRY(check_nf4(q));
+  QLORA_TRY(check_rank(r, alpha));
+  if (T < 0) return QLORA_ERR_INVALID_ARG;
+  if (!A || !B || !dA || !dB) return QLORA_ERR_INVALID_ARG;
+  const int64_t d = q->d, k = q->k;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (T == 0) {
+    QLORA_TRY(ensure_device());
+    if (cudaMemsetAsync(dA, 0, (size_t)r * k * 4, st) != cudaSuccess) return QLORA_ERR_CUDA;
+    if (cudaMemsetAsync(dB, 0, (size_t)d * r * 4, st) != cudaSuccess) return QLORA_ERR_CUDA;
+    return QLORA_OK;
+  }
+  if (!X || !U_saved || !dY || !dX || !ws) return QLORA_ERR_INVALID_ARG;
+  if (!aligned16(A) || !aligned16(X) || !aligned16(dY) || !aligned16(dX) || !aligned16(dA) ||
+      !aligned16(dB) || !aligned16(U_saved) || !aligned16(ws))
+    return QLORA_ERR_MISALIGNED;
+  if (T > ((int64_t)1 << 31)) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  BwdWs w = carve_bwd(ws, d, k, r, T);
+  if (ws_bytes < w.bytes) return QLORA_ERR_WORKSPACE_TOO_SMALL;
+  QLORA_TRY(ensure_device());
+  const float s = alpha / (float)r;
+  const int r8 = (int)round_up(r, 8);
+  const int bnr = bn_for_rank(r);
+
+  QLORA_TRY(dequantize_into(q, w.Wdq, st));
+  int pst = QLORA_OK;
+  const uint16_t* Bp = padded_B(B, d, r, r8, w.Bp, st, &pst);
+  QLORA_TRY(pst);
+  // Us = bf16(s U)
+  QLORA_TRY(launch("scale_f32_to_bf16", 0.0, (double)T * r * 6, st, [&] {
+    scale_f32_to_bf16<<<grid_for(T * r8, 256), 256, 0, st>>>(U_saved, T, r, s, w.Us, r8);
+  }));
+  // G = dY B  ->  Gs = bf16(s G)
+  {
+    GemmPlan g;
+    g.M = (int)T; g.N = r; g.K0 = (int)d; g.bn = bnr;
+    g.a0 = kmajor(dY, d, T, d);
+    g.b0 = mnmajor(Bp, r8, d, r8);
+    GemmArgs a = blank_args();
+    a.epi = EPI_F32; a.out = nullptr; a.n_store = 0;
+    a.out2 = w.Gs; a.ldo2 = r8; a.alpha2 = s; a.n_store2 = r8;
+    QLORA_TRY(launch_gemm("gemm_lora_g", g, a, st));
+  }
+  // dB = dY^T (sU)   (M = d, N = r, K = T)
+  {
+    GemmPlan g;
+    g.M = (int)d; g.N = r; g.K0 = (int)T; g.bn = bnr; g.splits = w.splitsB;
+    g.a0 = mnmajor(dY, d, T, d);
+    g.b0 = mnmajor(w.Us, r8, T, r8);
+    GemmArgs a = blank_args();
+    a.epi = EPI_F32; a.alpha = 1.0f; a.n_store = r;
+    if (w.splitsB > 1) {
+      a.out = w.partB; a.ldo = r; a.split_stride = d * r;
+    } else {
+      a.out = dB; a.ldo = r;
+    }
+    QLORA_TRY(launch_gemm("gemm_lora_dB", g, a, st));
+    if (w.splitsB > 1) {
+      const int splits = (int)cdiv(T, round_up(cdiv(T, w.splitsB), kBK));
+      QLORA_TRY(launch("splitk_reduce_f32", 0.0, (double)d * r * 4 * (splits + 1), st, [&] {
+        splitk_reduce_f32<<<grid_for(d * r, 256), 256, 0, st>>>(w.partB, splits, d * r, dB);
+      }));
+    }
+  }
+  // dA^T = X^T (sG)  (M = k, N = r, K = T), stored transposed into dA (r x k)
+  {
+    GemmPlan g;
+    g.M = (int)k; g.N = r; g.K0 = (int)T; g.bn = bnr; g.splits = w.splitsA;
+    g.a0 = mnmajor(X, k, T, k);
+    g.b0 = mnmajor(w.Gs, r8, T, r8);
+    GemmArgs a = blank_args();
+    a.epi = EPI_F32_T; a.alpha = 1.0f; a.n_store = r; a.ldo = k;
+    if (w.splitsA > 1) {
+      a.out = w.partA; a.split_stride = (int64_t)r * k;
+    } else {
+      a.out = dA;
+    }
+    QLORA_TRY(launch_gemm("gemm_lora_dA", g, a, st));
+    if (w.splitsA > 1) {
+      const int splits = (int)cdiv(T, round_up(cdiv(T, w.splitsA), kBK));
+      QLORA_TRY(launch("splitk_reduce_f32", 0.0, (double)r * k * 4 * (splits + 1), st, [&] {
+        splitk_reduce_f32<<<grid_for((int64_t)r * k, 256), 256, 0, st>>>(w.partA, splits, (int64_t)r * k, dA);
+      }));
+    }
+  }
+  // dX = [dY | sG] [W' ; A]   (M = T, N = k, K = d + r)
+  {
+    GemmPlan g;
+    g.M = (int)T; g.N = (int)k; g.K0 = (int)d; g.K1 = r; g.bn = 256;
+    g.a0 = kmajor(dY, d, T, d);
+    g.b0 = mnmajor(w.Wdq, k, d, k);
+    g.a1 = kmajor(w.Gs, r8, T, r8);
+    g.b1 = mnmajor(A, k, r, k);
+    GemmArgs a = blank_args();
+    a.epi = EPI_BF16; a.out = dX; a.ldo = k; a.n_store = (int)k;
+    QLORA_TRY(launch_gemm("gemm_bwd_dx", g, a, st));
+  }
+  return QLORA_OK;
+}
+
+size_t lora_merge_workspace_bytes(int64_t d, int64_t k, int r) {
+  if (d < 1 || k < 1 || r < 1) return 0;
+  return (size_t)round_up(d * round_up(r, 8) * 2, 256);
+}
+
+static int merge_common(const qlora_nf4_t* q, const uint16_t* W, const uint16_t* A, const uint16_t* B,
+                        int r, float alpha, int64_t d, int64_t k, uint16_t* out, void* ws,
+                        size_t ws_bytes, cudaStream_t st, bool merge) {
+  if (!A || !B || !out) return QLORA_ERR_INVALID_ARG;
+  if (!aligned16(A) || !aligned16(out) || (W && !aligned16(W))) return QLORA_ERR_MISALIGNED;
+  const int r8 = (int)round_up(r, 8);
+  if (r8 != r && (!ws || ws_bytes < lora_merge_workspace_bytes(d, k, r)))
+    return QLORA_ERR_WORKSPACE_TOO_SMALL;
+  if (r8 != r && !aligned16(ws)) return QLORA_ERR_MISALIGNED;
+  QLORA_TRY(ensure_device());
+  const float s = alpha / (float)r;
+  int pst = QLORA_OK;
+  const uint16_t* Bp = padded_B(B, d, r, r8, reinterpret_cast<uint16_t*>(ws), st, &pst);
+  QLORA_TRY(pst);
+  GemmPlan g;
+  g.M = (int)d; g.N = (int)k; g.K0 = r; g.bn = 256;
+  g.a0 = kmajor(Bp, r8, d, r8);
+  g.b0 = mnmajor(A, k, r, k);
+  GemmArgs a = blank_args();
+  a.out = out; a.ldo = k; a.n_store = (int)k;
+  if (merge) {
+    a.epi = EPI_MERGE; a.alpha = s;
+    a.codes = q->codes; a.absmax_q = q->absmax_q; a.scale2 = q->scale2; a.mean = q->mean;
+  } else {
+    a.epi = EPI_UNMERGE; a.alpha = -s; a.w_in = W; a.ldw = k;
+  }
+  return launch_gemm(merge ? "lora_merge" : "lora_unmerge", g, a, st);
+}
+
+int lora_merge(const qlora_nf4_t* q, const uint16_t* A, const uint16_t* B, int r, float alpha,
+               uint16_t* W_out, void* ws, size_t ws_bytes, qlora_stream_t stream) {
+  QLORA_TRY(check_nf4(q));
+  QLORA_TRY(check_rank(r, alpha));
+  return merge_common(q, nullptr, A, B, r, alpha, q->d, q->k, W_out, ws, ws_bytes,
+                      reinterpret_cast<cudaStream_t>(stream), true);
+}
+
+int lora_unmerge(const uint16_t* W, const uint16_t* A, const uint16_t* B, int r, float alpha,
+                 int64_t d, int64_t k, uint16_t* W0_out, void* ws, size_t ws_bytes,
+                 qlora_stream_t stream) {
+  QLORA_TRY(check_rank(r, alpha));
+  if (!W) return QLORA_ERR_INVALID_ARG;
+  if (d < 1 || k < 64 || k % 64 != 0 || d > ((int64_t)1 << 31) || k > ((int64_t)1 << 31))
+    return QLORA_ERR_UNSUPPORTED_SHAPE;
+  return merge_common(nullptr, W, A, B, r, alpha, d, k, W0_out, ws, ws_bytes,
+                      reinterpret_cast<cudaStream_t>(stream), false);
+}
+
+int qlora_get_device_status(qlora_stream_t stream, int* status) {
+  if (!status) return QLORA_ERR_INVALID_ARG;
+  QLORA_TRY(ensure_device());
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return QLORA_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_status, sizeof(int)) != cudaSuccess) return QLORA_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(g_status, &zero, sizeof(int)) != cudaSuccess) return QLORA_ERR_CUDA;
+  *status = v;
+  return QLORA_OK;
+}
+
+int qlora_selftest_wait_timeout(int limit_us, qlora_stream_t stream) {
+  if (limit_us < 1 || limit_us > 2000000) return QLORA_ERR_INVALID_ARG;
+  QLORA_TRY(ensure_device());
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  return launch("selftest_wait", 0.0, 0.0, st, [&] {
+    selftest_wait_kernel<<<1, 32, 0, st>>>((unsigned long long)limit_us * 1000ull);
+  });
+}
+
+int qlora_profile_begin(void) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  for (auto& r : g_prof) {
+    g_event_pool.push_back(r.start);
+    g_event_pool.push_back(r.stop);
+  }
+  g_prof.clear();
+  g_prof_on = true;
+  return QLORA_OK;
+}
+
+int qlora_profile_end(qlora_kernel_stat_t* out, int capacity, int* n_out) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  g_prof_on = false;
+  std::vector<qlora_kernel_stat_t> agg;
+  int status = QLORA_OK;
+  for (auto& r : g_prof) {
+    if (cudaEventSynchronize(r.stop) != cudaSuccess) { status = QLORA_ERR_CUDA; continue; }
+    float ms = 0.f;
+    if (cudaEventElapsedTime(&ms, r.start, r.stop) != cudaSuccess) { status = QLORA_ERR_CUDA; continue; }
+    qlora_kernel_stat_t* slot = nullptr;
+    for (auto& a : agg)
+      if (strncmp(a.name, r.name.c_str(), sizeof(a.name)) == 0) slot = &a;
+    if (!slot) {
+      qlora_kernel_stat_t z;
+      memset(&z, 0, sizeof(z));
+      strncpy(z.name, r.name.c_str(), sizeof(z.name) - 1);
+      agg.push_back(z);
+      slot = &agg.back();
+    }
+    slot->launches += 1;
+    slot->total_ms += ms;
+    slot->flops += r.flops;
+    slot->bytes += r.bytes;
+  }
+  for (auto& r : g_prof) {
+    g_event_pool.push_back(r.start);
+    g_event_pool.push_back(r.stop);
+  }
+  g_prof.clear();
+  const int n = (int)agg.size();
+  if (n_out) *n_out = n;
+  if (out)
+    for (int i = 0; i < n && i < capacity; ++i) out[i] = agg[i];
+  return status;
+}
+
+}  // extern "C"

@@ -1,0 +1,315 @@
+// NF4 + double-quant storage kernels (HBM-streaming, CUDA cores).
+//
+// [P1] "LoRA and QLoRA fine-tuning: mechanics, and when not to fine-tune",
+// section "What QLoRA freezes, and in how many bits": blockwise 4-bit
+// NormalFloat with block 64; block constants quantised again to FP8 in
+// blocks of 256 after subtracting their mean; doubleDequant in the forward
+// equation.
+//
+// Arithmetic is pinned to fp32/fp64 round-to-nearest operations written out
+// explicitly (__fmul_rn, __fadd_rn, ...) so that no contraction changes a
+// rounding; the CPU oracle states the same steps.
+#pragma once
+#include <cuda_fp8.h>
+#include "ptx.cuh"
+
+namespace qlora {
+
+constexpr int kBlock = 64;
+constexpr int kBlock2 = 256;
+constexpr int kEncBins = 129;     // x*64 floored, x in [-1, 1]
+
+// Encoder table: for bin j (x in [(j-64)/64, (j-63)/64)) the number of
+// thresholds <= the bin's lower edge, and the single threshold (if any)
+// strictly inside the bin (+inf otherwise).  Built on the host from the
+// library's own level table; at most one threshold falls in a bin because the
+// smallest level gap (~0.08) exceeds the bin width 1/64.
+struct EncTable {
+  float thr[kEncBins];
+  int base[kEncBins];
+};
+
+struct NF4Levels {
+  float q[16];
+};
+
+// Correctly rounded fp32 quotient w / a given y = RN(1/a) (Markstein 1990,
+// "Computation of elementary functions on the IBM RISC System/6000 processor":
+// if q0 is within one ulp of w/a and y = RN(1/a), then RN(q0 + r*y) with the
+// exact remainder r = w - a*q0 is the correctly rounded quotient).  Valid for
+// the ranges used here (|w| <= a, normal a); checked against IEEE division on
+// the device by the test suite.
+__device__ __forceinline__ float div_markstein(float w, float a, float y) {
+  const float q0 = __fmul_rn(w, y);
+  const float r = __fmaf_rn(-a, q0, w);
+  return __fmaf_rn(r, y, q0);
+}
+
+__device__ __forceinline__ uint32_t enc_code(float x, const float* s_thr, const int* s_base) {
+  int j = __float2int_rd(x * 64.0f) + 64;          // x*64 is exact
+  j = min(max(j, 0), kEncBins - 1);
+  return (uint32_t)(s_base[j] + (x >= s_thr[j] ? 1 : 0));
+}
+
+// ---------------------------------------------------------------------------
+// Phase 1: one CTA per group of 256 blocks (16384 weights).  8 threads per
+// block, 8 consecutive weights per thread.  Writes packed codes, the fp32
+// block absmax (scratch) and the fp64 pairwise sum of the group's absmax.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) nf4_quantize_phase1(
+    const float* __restrict__ W0, int64_t n_b, uint32_t* __restrict__ codes_u32,
+    float* __restrict__ absmax, double* __restrict__ group_sum, const __grid_constant__ EncTable tab) {
+  __shared__ float s_thr[kEncBins];
+  __shared__ int s_base[kEncBins];
+  __shared__ float s_abs[kBlock2];
+  const int tid = threadIdx.x;
+  for (int i = tid; i < kEncBins; i += blockDim.x) {
+    s_thr[i] = tab.thr[i];
+    s_base[i] = tab.base[i];
+  }
+  __syncthreads();
+
+  const int64_t g = blockIdx.x;
+  const int sub = tid & 7;          // 8 threads per block
+  const int lb0 = tid >> 3;         // 32 blocks per pass
+#pragma unroll 1
+  for (int half = 0; half < 2; ++half) {
+    float4 v[4][2];
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+      const int lb = (half * 4 + p) * 32 + lb0;
+      const int64_t b = g * kBlock2 + lb;
+      if (b < n_b) {
+        const float4* src = reinterpret_cast<const float4*>(W0 + b * kBlock + sub * 8);
+        v[p][0] = __ldcs(src);
+        v[p][1] = __ldcs(src + 1);
+      } else {
+        v[p][0] = make_float4(0.f, 0.f, 0.f, 0.f);
+        v[p][1] = v[p][0];
+      }
+    }
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+      const int lb = (half * 4 + p) * 32 + lb0;
+      const int64_t b = g * kBlock2 + lb;
+      float w[8] = {v[p][0].x, v[p][0].y, v[p][0].z, v[p][0].w,
+                    v[p][1].x, v[p][1].y, v[p][1].z, v[p][1].w};
+      float m = 0.f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(w[i]));
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
+      uint32_t packed = 0x77777777u;             // all-zero block: zero level (code 7)
+      if (m > 0.f) {
+        const float y = __frcp_rn(m);
+        packed = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float x = div_markstein(w[i], m, y);
+          packed |= enc_code(x, s_thr, s_base) << (4 * i);
+        }
+      }
+      if (b < n_b) {
+        codes_u32[b * 8 + sub] = packed;
+        if (sub == 0) absmax[b] = m;
+      }
+      if (sub == 0) s_abs[lb] = (b < n_b) ? m : 0.f;
+    }
+  }
+  __syncthreads();
+  if (tid < 32) {
+    // pairwise tree over the 256 constants: lane l sums leaves 8l..8l+7, then
+    // the lanes are combined in halves (shfl_down by 1, 2, 4, 8, 16)
+    double a[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) a[i] = (double)s_abs[tid * 8 + i];
+    double s = ((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]));
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) s = s + __shfl_down_sync(0xffffffffu, s, off);
+    if (tid == 0) group_sum[g] = s;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Phase 2: single CTA; pairwise tree over the group sums (padded with zeros
+// to a power of two), mean = fp32(S / n_b).
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(1024) nf4_quantize_mean(const double* __restrict__ group_sum,
+                                                          int64_t n_g, int64_t n_b,
+                                                          float* __restrict__ mean_out) {
+  __shared__ double s_v[1024];
+  const int tid = threadIdx.x;
+  int64_t P = 1;
+  while (P < n_g) P <<= 1;
+  const int64_t C = (P > 1024) ? (P / 1024) : 1;     // leaves per thread (power of two)
+  double stack[24];
+  int level[24];
+  int sp = 0;
+  for (int64_t j = 0; j < C; ++j) {
+    const int64_t idx = (int64_t)tid * C + j;
+    double v = (idx < n_g) ? group_sum[idx] : 0.0;
+    int l = 0;
+    while (sp > 0 && level[sp - 1] == l) {
+      v = stack[sp - 1] + v;
+      --sp;
+      ++l;
+    }
+    stack[sp] = v;
+    level[sp] = l;
+    ++sp;
+  }
+  s_v[tid] = stack[0];
+  __syncthreads();
+  for (int s = 1; s < 1024; s <<= 1) {
+    if ((tid % (2 * s)) == 0) s_v[tid] = s_v[tid] + s_v[tid + s];
+    __syncthreads();
+  }
+  if (tid == 0) mean_out[0] = __double2float_rn(__ddiv_rn(s_v[0], (double)n_b));
+}
+
+// ---------------------------------------------------------------------------
+// Phase 3: one CTA per group; second-level scale and E4M3 codes.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) nf4_quantize_dq(const float* __restrict__ absmax,
+                                                       int64_t n_b, const float* __restrict__ mean,
+                                                       uint8_t* __restrict__ absmax_q,
+                                                       float* __restrict__ scale2) {
+  __shared__ float s_max[8];
+  const int64_t g = blockIdx.x;
+  const int tid = threadIdx.x;
+  const int64_t b = g * kBlock2 + tid;
+  const float mu = mean[0];
+  float cen = 0.f;
+  if (b < n_b) cen = __fsub_rn(absmax[b], mu);
+  float m = fabsf(cen);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+  if ((tid & 31) == 0) s_max[tid >> 5] = m;
+  __syncthreads();
+  float c1 = s_max[0];
+#pragma unroll
+  for (int i = 1; i < 8; ++i) c1 = fmaxf(c1, s_max[i]);
+  const float s1 = (c1 > 0.f) ? __fdiv_rn(c1, 448.0f) : 0.f;
+  if (tid == 0) scale2[g] = s1;
+  if (b < n_b) {
+    uint8_t code = 0;
+    if (s1 > 0.f) {
+      const float x = __fdiv_rn(cen, s1);
+      code = (uint8_t)__nv_cvt_float_to_fp8(x, __NV_SATFINITE, __NV_E4M3);
+    }
+    absmax_q[b] = code;
+  }
+}
+
+__device__ __forceinline__ float e4m3_to_f32(uint8_t c) {
+  __half_raw h = __nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)c, __NV_E4M3);
+  return __half2float(__half(h));
+}
+
+// a'_b = fp32(fp32(E4M3(c2_b) * s1_j) + mean)
+__device__ __forceinline__ float block_scale(const uint8_t* absmax_q, const float* scale2,
+                                             float mu, int64_t b) {
+  return __fadd_rn(__fmul_rn(e4m3_to_f32(absmax_q[b]), scale2[b / kBlock2]), mu);
+}
+
+// 32 codes (one 16-byte word) -> 32 bf16 values of level[code] * a'.
+__device__ __forceinline__ void dequant32(const uint4 c, float a, const float* s_q, uint32_t (&o)[16]) {
+  const uint32_t w[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t lo = (w[i] >> (8 * j)) & 0xFu;
+      const uint32_t hi = (w[i] >> (8 * j + 4)) & 0xFu;
+      const __nv_bfloat162 p = __floats2bfloat162_rn(__fmul_rn(s_q[lo], a), __fmul_rn(s_q[hi], a));
+      o[i * 4 + j] = *reinterpret_cast<const uint32_t*>(&p);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Dequantise to a bf16 d x k matrix.  One thread per 32 consecutive weights
+// (a 16-byte load of codes, a 64-byte store of bf16).
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) nf4_dequantize_kernel(
+    const uint4* __restrict__ codes, const uint8_t* __restrict__ absmax_q,
+    const float* __restrict__ scale2, const float* __restrict__ mean, int64_t n_chunks,
+    uint4* __restrict__ W_out, const __grid_constant__ NF4Levels lv) {
+  __shared__ float s_q[16];
+  if (threadIdx.x < 16) s_q[threadIdx.x] = lv.q[threadIdx.x];
+  __syncthreads();
+  const float mu = mean[0];
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; t < n_chunks; t += stride) {
+    const uint4 c = __ldcs(codes + t);
+    const float a = block_scale(absmax_q, scale2, mu, t >> 1);
+    uint32_t o[16];
+    dequant32(c, a, s_q, o);
+    uint4* dst = W_out + t * 4;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) dst[i] = make_uint4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Small helpers for the rank-r operands.
+// ---------------------------------------------------------------------------
+// dst (rows x ld_dst, bf16) = src (rows x cols, bf16) with zero columns
+// [cols, ld_dst).
+__global__ void pad_cols_bf16(const uint16_t* __restrict__ src, int64_t rows, int cols,
+                              uint16_t* __restrict__ dst, int ld_dst) {
+  const int64_t n = rows * ld_dst;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride) {
+    const int64_t rrow = i / ld_dst;
+    const int c = (int)(i - rrow * ld_dst);
+    dst[i] = (c < cols) ? src[rrow * cols + c] : (uint16_t)0;
+  }
+}
+
+// dst (rows x ld_dst, bf16) = bf16(scale * src) with zero padding columns.
+__global__ void scale_f32_to_bf16(const float* __restrict__ src, int64_t rows, int cols,
+                                  float scale, uint16_t* __restrict__ dst, int ld_dst) {
+  const int64_t n = rows * ld_dst;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride) {
+    const int64_t rrow = i / ld_dst;
+    const int c = (int)(i - rrow * ld_dst);
+    float v = (c < cols) ? __fmul_rn(scale, src[rrow * cols + c]) : 0.f;
+    __nv_bfloat16 h = __float2bfloat16_rn(v);
+    dst[i] = *reinterpret_cast<uint16_t*>(&h);
+  }
+}
+
+// out[i] = sum_z part[z * stride + i], z = 0, 1, ... in order (deterministic).
+__global__ void splitk_reduce_f32(const float* __restrict__ part, int splits, int64_t n,
+                                  float* __restrict__ out) {
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride) {
+    float s = part[i];
+    for (int z = 1; z < splits; ++z) s = __fadd_rn(s, part[(int64_t)z * n + i]);
+    out[i] = s;
+  }
+}
+
+// Bounded-wait self test: waits on a barrier that nothing completes.
+__global__ void selftest_wait_kernel(unsigned long long limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const uint64_t start = globaltimer_ns();
+    while (!mbar_try_wait(smem_u32(&bar), 0)) {
+      if (globaltimer_ns() - start > limit_ns) {
+        record_status(QLORA_ERR_TIMEOUT);
+        break;
+      }
+    }
+  }
+}
+
+}  // namespace qlora

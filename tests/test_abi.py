@@ -1,0 +1,91 @@
+"""The C-ABI library loads, exports every symbol include/qlora.h declares, and
+its host-only parts agree with the oracle.  No kernel is launched here."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import parameter_efficient_fine_nf4_b200 as q4
+from oracle import nf4
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from parameter_efficient_fine_nf4_b200 import build
+    build.build()
+    return q4.lib()
+
+
+def declared_symbols():
+    text = open(os.path.join(ROOT, "include", "qlora.h")).read()
+    return sorted(set(re.findall(r"^QLORA_API\s+[\w\s\*]+?\b((?:qlora|lora)_\w+)\s*\(", text, re.M)))
+
+
+def test_header_declares_the_path():
+    names = declared_symbols()
+    for required in ("qlora_nf4_quantize", "qlora_nf4_dequantize", "qlora_fwd", "qlora_bwd",
+                     "lora_merge", "lora_unmerge"):
+        assert required in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_symbols()
+    assert len(names) >= 18
+    for n in names:
+        assert hasattr(lib, n), n
+    # the binding wraps exactly the declared set
+    assert set(q4.EXPORTED) == set(names)
+
+
+def test_library_levels_equal_oracle_bit_for_bit(lib):
+    levels, thr = q4.qlora_nf4_levels()
+    lv = np.array(levels, np.float32)
+    assert np.array_equal(lv.view(np.uint32), nf4.nf4_levels().view(np.uint32))
+    # thresholds: counting thresholds <= x equals the oracle's nearest level
+    # (ties low) for every fp32 x within 2048 ulps of each threshold
+    t = np.array(thr, np.float32)
+    xs = []
+    for ti in t:
+        bits = ti.view(np.uint32).astype(np.int64)
+        if ti > 0:
+            rng_bits = np.arange(bits - 2048, bits + 2048)
+        else:
+            rng_bits = np.arange(bits - 2048, bits + 2048)   # negative: bit order reversed, same set
+        xs.append(rng_bits.astype(np.uint32).view(np.float32))
+    x = np.concatenate(xs)
+    x = x[np.abs(x) <= 1]
+    x = x[: (x.size // 64) * 64]
+    oracle_codes = nf4.encode_blocks(x.reshape(-1, 64), np.ones(x.size // 64, np.float32)).ravel()
+    lib_codes = (x[:, None] >= t[None, :]).sum(axis=1)
+    assert np.array_equal(oracle_codes, lib_codes)
+
+
+def test_workspace_queries(lib):
+    assert q4.qlora_quantize_workspace_bytes(256, 256) >= (256 * 256 // 64) * 4
+    assert q4.qlora_fwd_workspace_bytes(22016, 8192, 64, 16384) >= 22016 * 8192 * 2
+    assert q4.qlora_bwd_workspace_bytes(22016, 8192, 64, 16384) >= 22016 * 8192 * 2
+    assert q4.lora_merge_workspace_bytes(256, 256, 8) >= 256 * 8 * 2
+    assert q4.qlora_fwd_workspace_bytes(0, 256, 8, 16) == 0
+
+
+def test_argument_validation_without_device(lib):
+    L = lib
+    # unsupported shapes and bad arguments are rejected on the host before any launch
+    nf = q4._NF4(16, 16, 16, 16, 256, 100, 64, 256)              # k % 64 != 0
+    st = L.qlora_fwd(ctypes.byref(nf), 16, 16, 8, 16.0, 16, 16, 16, 16, 16, 1 << 20, None)
+    assert st == 2
+    nf = q4._NF4(16, 16, 16, 16, 256, 256, 64, 256)
+    assert L.qlora_fwd(ctypes.byref(nf), 16, 16, 0, 16.0, 16, 16, 16, 16, 16, 1 << 20, None) == 2   # r = 0
+    assert L.qlora_fwd(ctypes.byref(nf), 16, 16, 8, -1.0, 16, 16, 16, 16, 16, 1 << 20, None) == 1   # alpha
+    assert L.qlora_fwd(ctypes.byref(nf), None, 16, 8, 16.0, 16, 16, 16, 16, 16, 1 << 20, None) == 1  # null A
+    assert L.qlora_fwd(ctypes.byref(nf), 16, 16, 8, 16.0, 17, 16, 16, 16, 16, 1 << 20, None) == 3   # misaligned X
+    assert L.qlora_fwd(ctypes.byref(nf), 16, 16, 8, 16.0, 16, 16, 16, 16, 16, 64, None) == 4        # workspace
+    assert L.qlora_nf4_quantize(16, 256, 100, 64, ctypes.byref(nf), 16, 1 << 20, None) == 2
+    assert L.qlora_nf4_quantize(16, 256, 256, 32, ctypes.byref(nf), 16, 1 << 20, None) == 2
+    nf_bad = q4._NF4(16, 16, 16, 16, 256, 256, 32, 256)           # block != 64
+    assert L.qlora_nf4_dequantize(ctypes.byref(nf_bad), 16, None) == 2
+    assert q4.strerror(6) == "device wait timed out"

@@ -1,0 +1,183 @@
+"""GPU parity of the QLoRA layer: forward, backward, merge and unmerge against
+the float64 oracle on the same seeded inputs."""
+import numpy as np
+import pytest
+import torch
+
+import synthetic
+from oracle import lora, nf4
+from tests.gpu_helpers import (bf16_dev, bf16_host_bits, bf16_host_f64, f32_dev, f32_host_f64,
+                               rows_within, within_one_bf16_ulp)
+
+pytestmark = pytest.mark.gpu
+
+q4 = pytest.importorskip("parameter_efficient_fine_nf4_b200")
+
+
+_WP_CACHE = {}
+
+
+def oracle_Wp(W0: np.ndarray) -> np.ndarray:
+    """Oracle dequantised weight (float64), cached per seeded weight."""
+    key = (W0.shape, W0[0, :16].tobytes(), W0[-1, -16:].tobytes())
+    if key not in _WP_CACHE:
+        if len(_WP_CACHE) > 3:
+            _WP_CACHE.clear()
+        qt = nf4.quantize(W0)
+        _WP_CACHE[key] = nf4.bf16_to_f64(nf4.dequantize(qt))
+    return _WP_CACHE[key]
+
+
+class Case:
+    """GPU run + oracle pieces for one layer."""
+
+    def __init__(self, lay: synthetic.LayerInputs, alpha: float):
+        self.lay = lay
+        self.alpha = alpha
+        self.s = alpha / lay.r
+        self.qw = q4.qlora_nf4_quantize(f32_dev(lay.W0))
+        self.A = bf16_dev(lay.A)
+        self.B = bf16_dev(lay.B)
+        self.X = bf16_dev(lay.X)
+        self.dY = bf16_dev(lay.dY)
+        self.Y, self.U = q4.qlora_fwd(self.qw, self.A, self.B, alpha, self.X)
+        self.dX, self.dA, self.dB = q4.qlora_bwd(self.qw, self.A, self.B, alpha, self.X, self.U, self.dY)
+        torch.cuda.synchronize()
+        assert q4.qlora_get_device_status() == 0
+
+    def oracle_Wp(self):
+        return oracle_Wp(self.lay.W0)
+
+    def check(self, rows=None, full_adapter_grads=True):
+        lay = self.lay
+        Wp = self.oracle_Wp()
+        X = nf4.bf16_to_f64(lay.X)
+        A = nf4.bf16_to_f64(lay.A)
+        B = nf4.bf16_to_f64(lay.B)
+        dY = nf4.bf16_to_f64(lay.dY)
+        if rows is None:
+            rows = np.arange(lay.T)
+        fw = lora.forward(X[rows], Wp, A, B, self.s)
+        rows_within(bf16_host_f64(self.Y)[rows], fw["Y"], what="Y")
+        rows_within(f32_host_f64(self.U)[rows], fw["U"], what="U")
+        gi = lora.grad_input(Wp, A, B, self.s, dY[rows])
+        rows_within(bf16_host_f64(self.dX)[rows], gi["dX"], what="dX")
+        if full_adapter_grads:
+            ga = lora.grad_adapters(X, A, B, self.s, dY)
+            rows_within(f32_host_f64(self.dA), ga["dA"], what="dA")
+            rows_within(f32_host_f64(self.dB), ga["dB"], what="dB")
+        return Wp
+
+
+def test_config1_full():
+    cfg = synthetic.config(1)
+    Case(synthetic.make_layer(cfg), cfg.alpha).check()
+
+
+def test_config1_b_zero_init():
+    # B = 0 at initialisation: the adapter adds nothing, dA is exactly zero
+    cfg = synthetic.config(1)
+    c = Case(synthetic.make_layer(cfg, zero_b=True), cfg.alpha)
+    Wp = c.check()
+    assert torch.count_nonzero(c.dA).item() == 0
+    X = nf4.bf16_to_f64(c.lay.X)
+    rows_within(bf16_host_f64(c.Y), X @ Wp.T, what="Y base")
+
+
+@pytest.mark.parametrize("d,k,r,T", [
+    (320, 192, 5, 200),      # ragged M and N tiles, r not a multiple of 8
+    (64, 64, 1, 1),          # one token, rank 1
+    (130, 128, 3, 129),      # d one past a tile in the extension operand rows
+    (256, 512, 100, 300),    # r > 64: two extension steps on a 128-wide N tile
+    (384, 256, 256, 64),     # maximum rank
+    (200, 64, 16, 1000),     # K = 64: one main step
+])
+def test_ragged_shapes(d, k, r, T):
+    lay = synthetic.custom_layer(seed=d * 131 + k * 7 + r + T, d=d, k=k, r=r, T=T, alpha=2.0 * r)
+    Case(lay, 2.0 * r).check()
+
+
+@pytest.mark.parametrize("ci", [2, 3])
+def test_configs_sampled_rows(ci):
+    cfg = synthetic.config(ci)
+    lay = synthetic.make_layer(cfg)
+    rows = synthetic.sample_rows(77 + ci, lay.T, 192)
+    Case(lay, cfg.alpha).check(rows=rows)
+
+
+@pytest.mark.parametrize("li", [0, 1])
+def test_config4_sampled_rows(li):
+    cfg = synthetic.config(4)
+    lay = synthetic.make_layer(cfg, li)
+    rows = synthetic.sample_rows(401 + li, lay.T, 64)
+    Case(lay, cfg.alpha).check(rows=rows)
+
+
+@pytest.mark.parametrize("li", range(7))
+@pytest.mark.parametrize("T", [16, 4096])
+def test_config5_linears(li, T):
+    cfg = synthetic.config(5)
+    lay = synthetic.make_layer(cfg, li, T=T)
+    rows = None if T == 16 else synthetic.sample_rows(500 + li, T, 64)
+    Case(lay, cfg.alpha).check(rows=rows, full_adapter_grads=(li in (0, 4, 6)))
+
+
+def test_bwd_deterministic_and_zero_tokens():
+    cfg = synthetic.config(2)
+    lay = synthetic.make_layer(cfg)
+    c = Case(lay, cfg.alpha)
+    dX2, dA2, dB2 = q4.qlora_bwd(c.qw, c.A, c.B, cfg.alpha, c.X, c.U, c.dY)
+    torch.cuda.synchronize()
+    assert torch.equal(dA2, c.dA) and torch.equal(dB2, c.dB) and torch.equal(dX2, c.dX)
+    # T = 0: nothing to do, adapter gradients are overwritten with zeros
+    X0 = c.X[:0]
+    dA = torch.full_like(c.dA, 7.0)
+    dB = torch.full_like(c.dB, 7.0)
+    q4.qlora_bwd(c.qw, c.A, c.B, cfg.alpha, X0, c.U[:0], c.dY[:0], dA=dA, dB=dB)
+    torch.cuda.synchronize()
+    assert torch.count_nonzero(dA).item() == 0 and torch.count_nonzero(dB).item() == 0
+
+
+@pytest.mark.parametrize("ci", [1, 3])
+def test_merge_unmerge(ci):
+    cfg = synthetic.config(ci)
+    lay = synthetic.make_layer(cfg, with_acts=False)
+    s = cfg.s
+    qw = q4.qlora_nf4_quantize(f32_dev(lay.W0))
+    A, B = bf16_dev(lay.A), bf16_dev(lay.B)
+    W = q4.lora_merge(qw, A, B, cfg.alpha)
+    torch.cuda.synchronize()
+    qt = nf4.quantize(lay.W0)
+    Wp = nf4.bf16_to_f64(nf4.dequantize(qt))
+    Af, Bf = nf4.bf16_to_f64(lay.A), nf4.bf16_to_f64(lay.B)
+    ref_W = lora.merge(Wp, Af, Bf, s)
+    within_one_bf16_ulp(bf16_host_bits(W), ref_W, "merge")
+    # unmerge of the oracle's merged weight
+    W_in = bf16_dev(ref_W)
+    W0pp = q4.lora_unmerge(W_in, A, B, cfg.alpha)
+    torch.cuda.synchronize()
+    ref_W0pp = lora.unmerge(nf4.bf16_to_f64(ref_W), Af, Bf, s)
+    within_one_bf16_ulp(bf16_host_bits(W0pp), ref_W0pp, "unmerge")
+    # merge then unmerge on the GPU gives back the dequantised base (1 ulp),
+    # and with B = 0 both are exactly the dequantised base
+    back = q4.lora_unmerge(W, A, B, cfg.alpha)
+    Wdq = q4.qlora_nf4_dequantize(qw)
+    Z = torch.zeros_like(B)
+    Wz = q4.lora_merge(qw, A, Z, cfg.alpha)
+    Wz2 = q4.lora_unmerge(Wdq, A, Z, cfg.alpha)
+    torch.cuda.synchronize()
+    # two roundings (merge, then unmerge), each at most half an ulp of the
+    # larger of W and W'
+    within_one_bf16_ulp(bf16_host_bits(back), nf4.dequantize(qt), "merge-unmerge", ulps=2)
+    assert torch.equal(Wz, Wdq) and torch.equal(Wz2, Wdq)
+    assert q4.qlora_get_device_status() == 0
+
+
+def test_merged_layer_matches_unmerged_forward():
+    cfg = synthetic.config(1)
+    lay = synthetic.make_layer(cfg)
+    c = Case(lay, cfg.alpha)
+    W = q4.lora_merge(c.qw, c.A, c.B, cfg.alpha)
+    Y_merged = (c.X.float() @ W.float().T)
+    torch.cuda.synchronize()
+    rows_within(Y_merged.double().cpu().numpy(), bf16_host_f64(c.Y).astype(np.float64), what="merged")
