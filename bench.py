@@ -1,0 +1,424 @@
+#!/usr/bin/env python
+"""Throughput of the QLoRA linear layer hot path on B200.
+
+One step = the whole hot path over one batch, for each linear of the
+workload (default: the large MLP pair k=8192 -> d=22016 and 22016 -> 8192,
+r = 64, alpha = 16, 16384 tokens per GPU):
+    nf4_quantize(W0) -> qlora_fwd -> qlora_bwd -> lora_merge -> lora_unmerge
+and, with more than one GPU, the data-parallel sum of dA and dB over ranks.
+
+Metric: algorithmic fwd+bwd TFLOP/s, F = 4Tdk + 6Tr(d+k) per linear (no
+weight gradient), summed over linears and ranks, divided by the step time.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line (rank 0).  ``--impl reference`` times the CPU oracle on a
+bounded sample of the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import synthetic  # noqa: E402
+
+METRIC = "QLoRA linear fwd+bwd TFLOP/s and tokens/s at 1 B200; % of bf16 tensor peak"
+L2_BYTES = 126 * 1024 * 1024
+
+
+def algorithmic_flops(T, d, k, r):
+    return 4 * T * d * k + 6 * T * r * (d + k)
+
+
+def workload(config_index: int):
+    cfg = synthetic.config(config_index)
+    T = cfg.tokens[0]
+    return cfg, T
+
+
+def workload_name(cfg, T):
+    lin = ", ".join(f"{l.name} k={l.k}->d={l.d}" for l in cfg.linears)
+    return f"QLoRA linear layer: {lin}; r={cfg.r}, alpha={cfg.alpha:g}, T={T} tokens per GPU"
+
+
+def read_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return json.load(f), "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+# --------------------------------------------------------------------------- clocks
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for ln in self.proc.stdout:
+            self.lines.append(ln.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.t.join(timeout=2)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        top = max(sm)
+        loaded = [v for v in sm if v >= 0.5 * top] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(smax),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------- CPU oracle sample
+def oracle_sample_step(cfg, rows_d=512, tokens=1024):
+    """The oracle on a bounded slice of the first linear: W0 cut to `rows_d`
+    output rows, `tokens` tokens; quantise, fwd, bwd, merge, unmerge.
+    Returns (algorithmic fwd+bwd flops of the slice, seconds)."""
+    from oracle import lora, nf4
+    lin = cfg.linears[0]
+    lay = synthetic.make_layer(cfg, 0, shape_override=(rows_d, lin.k, tokens))
+    t0 = time.perf_counter()
+    qt = nf4.quantize(lay.W0)
+    Wp = nf4.bf16_to_f64(nf4.dequantize(qt))
+    X, A, B, dY = (nf4.bf16_to_f64(a) for a in (lay.X, lay.A, lay.B, lay.dY))
+    fw = lora.forward(X, Wp, A, B, cfg.s)
+    lora.backward(X, Wp, A, B, cfg.s, dY, fw["U"])
+    Wm = lora.merge(Wp, A, B, cfg.s)
+    lora.unmerge(nf4.bf16_to_f64(Wm), A, B, cfg.s)
+    dt = time.perf_counter() - t0
+    return algorithmic_flops(tokens, rows_d, lin.k, cfg.r), dt
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+def cpu_baseline(cfg, budget_s=15.0):
+    flops, dt = oracle_sample_step(cfg)
+    reps = 1
+    total_f, total_t = flops, dt
+    while total_t < budget_s and reps < 8:
+        f, t = oracle_sample_step(cfg)
+        total_f += f
+        total_t += t
+        reps += 1
+    lin = cfg.linears[0]
+    return {"value": total_f / total_t / 1e12, "unit": "TFLOP/s", "cores": blas_threads(),
+            "kind": "oracle",
+            "sample": (f"{reps} x oracle quantise+fwd+bwd+merge+unmerge of linear '{lin.name}' cut to "
+                       f"d=512 rows (k={lin.k}), r={cfg.r}, 1024 tokens; float64 numpy, "
+                       f"{total_t:.1f} s")}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    cfg, T = workload(args.config)
+    flops_step = 0.0
+    times = []
+    for i in range(args.warmup + args.steps):
+        f, t = oracle_sample_step(cfg)
+        if i >= args.warmup:
+            times.append(t)
+            flops_step = f
+    ms = 1e3 * statistics.mean(times)
+    value = flops_step / (ms / 1e3) / 1e12
+    cores = blas_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": workload_name(cfg, T) + " (oracle: bounded slice per step)",
+                   "l2": "n/a (CPU)"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": "one step = oracle quantise+fwd+bwd+merge+unmerge of the first "
+                                   "linear cut to d=512 rows and 1024 tokens"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------------------- GPU arm
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "parameter_efficient_fine_nf4_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def read_traffic(kernel: str):
+    """ncu DRAM bytes per launch for `kernel`, if captured on the current sources."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        with open(p) as f:
+            t = json.load(f)
+        if t.get("source_hash") != kernel_source_hash():
+            return None
+        return t.get("kernels", {}).get(kernel)
+    except Exception:
+        return None
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    import parameter_efficient_fine_nf4_b200 as q4
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        args.gpus = world
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    q4.lib()
+    cfg, T = workload(args.config)
+
+    # ---- resident inputs (per rank: its own tokens, the same frozen weights)
+    layers = []
+    for li, lin in enumerate(cfg.linears):
+        lay = synthetic.make_layer(cfg, li, T=T, with_acts=False)
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(synthetic.seed_for(cfg.index, "X", li) + 1000 * rank)
+        X = torch.randn(T, lin.k, generator=gen, device=dev, dtype=torch.float32).to(torch.bfloat16)
+        dY = torch.randn(T, lin.d, generator=gen, device=dev, dtype=torch.float32).to(torch.bfloat16)
+        L = {
+            "lin": lin,
+            "W0": torch.from_numpy(lay.W0).to(dev),
+            "A": torch.from_numpy(lay.A.view(np.int16)).view(torch.bfloat16).to(dev),
+            "B": torch.from_numpy(lay.B.view(np.int16)).view(torch.bfloat16).to(dev),
+            "X": X, "dY": dY,
+            "qw": q4.NF4Weight(lin.d, lin.k, dev),
+            "Y": torch.empty(T, lin.d, dtype=torch.bfloat16, device=dev),
+            "U": torch.empty(T, cfg.r, dtype=torch.float32, device=dev),
+            "dX": torch.empty(T, lin.k, dtype=torch.bfloat16, device=dev),
+            "dA": torch.empty(cfg.r, lin.k, dtype=torch.float32, device=dev),
+            "dB": torch.empty(lin.d, cfg.r, dtype=torch.float32, device=dev),
+            "Wm": torch.empty(lin.d, lin.k, dtype=torch.bfloat16, device=dev),
+            "W0u": torch.empty(lin.d, lin.k, dtype=torch.bfloat16, device=dev),
+        }
+        nbytes = max(q4.qlora_quantize_workspace_bytes(lin.d, lin.k),
+                     q4.qlora_fwd_workspace_bytes(lin.d, lin.k, cfg.r, T),
+                     q4.qlora_bwd_workspace_bytes(lin.d, lin.k, cfg.r, T),
+                     q4.lora_merge_workspace_bytes(lin.d, lin.k, cfg.r))
+        L["ws"] = q4.workspace(nbytes, dev)
+        layers.append(L)
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        for L in layers:
+            q4.qlora_nf4_quantize(L["W0"], out=L["qw"], ws=L["ws"])
+            q4.qlora_fwd(L["qw"], L["A"], L["B"], cfg.alpha, L["X"], Y=L["Y"], U_save=L["U"], ws=L["ws"])
+            q4.qlora_bwd(L["qw"], L["A"], L["B"], cfg.alpha, L["X"], L["U"], L["dY"], dX=L["dX"],
+                         dA=L["dA"], dB=L["dB"], ws=L["ws"])
+            if world > 1:
+                dist.all_reduce(L["dA"])
+                dist.all_reduce(L["dB"])
+            q4.lora_merge(L["qw"], L["A"], L["B"], cfg.alpha, W_out=L["Wm"], ws=L["ws"])
+            q4.lora_unmerge(L["Wm"], L["A"], L["B"], cfg.alpha, W0_out=L["W0u"], ws=L["ws"])
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[local])
+        torch.cuda.synchronize(dev)
+
+    for _ in range(args.warmup):
+        step()
+    assert q4.qlora_get_device_status() == 0
+
+    # ---- timed region (device time per step with CUDA events; L2 flushed
+    # between steps outside the events)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    clocks.start()
+    barrier()
+    n0 = q4.qlora_launch_count()
+    q4.qlora_profile_begin()
+    for i in range(args.steps):
+        flush.zero_()
+        evs[i][0].record(stream)
+        step()
+        evs[i][1].record(stream)
+    barrier()
+    stats = q4.qlora_profile_end()
+    launches = q4.qlora_launch_count() - n0
+    clk = clocks.stop()
+    ms_steps = [a.elapsed_time(b) for a, b in evs]
+    ms = statistics.mean(ms_steps)
+    t = torch.tensor([ms], device=dev, dtype=torch.float64)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms = float(t.item())
+    flops_rank = sum(algorithmic_flops(T, L["lin"].d, L["lin"].k, cfg.r) for L in layers)
+    value = flops_rank * world / (ms / 1e3) / 1e12
+    tokens_s = T * world / (ms / 1e3)
+
+    # ---- e2e through the public API with host buffers: per step, copy X and
+    # dY of every linear in from pinned memory, run the step, read dA and dB back
+    host_in = [(L["X"].cpu().pin_memory(), L["dY"].cpu().pin_memory()) for L in layers]
+    host_out = [(torch.empty_like(L["dA"], device="cpu").pin_memory(),
+                 torch.empty_like(L["dB"], device="cpu").pin_memory()) for L in layers]
+    h2d = sum(x.numel() * x.element_size() + y.numel() * y.element_size() for x, y in host_in)
+    d2h = sum(a.numel() * a.element_size() + b.numel() * b.element_size() for a, b in host_out)
+    e2e_ms = []
+    e2e_steps = max(3, min(args.steps, 5))
+    barrier()
+    for i in range(e2e_steps + 1):
+        flush.zero_()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for L, (hx, hdy) in zip(layers, host_in):
+            L["X"].copy_(hx, non_blocking=True)
+            L["dY"].copy_(hdy, non_blocking=True)
+        step()
+        for L, (ha, hb) in zip(layers, host_out):
+            ha.copy_(L["dA"], non_blocking=True)
+            hb.copy_(L["dB"], non_blocking=True)
+        b.record(stream)
+        b.synchronize()
+        if i > 0:
+            e2e_ms.append(a.elapsed_time(b))
+    barrier()
+    te = torch.tensor([statistics.mean(e2e_ms)], device=dev, dtype=torch.float64)
+    if world > 1:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+    e2e_value = flops_rank * world / (float(te.item()) / 1e3) / 1e12
+    assert q4.qlora_get_device_status() == 0
+
+    # ---- roofline of the dominant kernel (the tcgen05 GEMM: forward main and dX)
+    peaks, peak_src = read_peaks()
+    gemm = [s for s in stats if s["name"] in ("gemm_fwd_main", "gemm_bwd_dx")]
+    g_ms = sum(s["total_ms"] for s in gemm)
+    g_launches = sum(s["launches"] for s in gemm)
+    g_flops = sum(s["flops"] for s in gemm)
+    achieved = g_flops / (g_ms / 1e3) / 1e12 if g_ms > 0 else 0.0
+    peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
+    traffic = read_traffic("gemm_tc_kernel")
+    rows = {s["name"]: {"launches": s["launches"], "ms_per_step": s["total_ms"] / args.steps,
+                        "share": s["total_ms"] / max(1e-9, sum(x["total_ms"] for x in stats))}
+            for s in stats}
+
+    if world > 1:
+        dist.barrier(device_ids=[local])
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded W0/A/B from the config recipe, X and dY ~ N(0,1) drawn on device)",
+            "config": {"workload": workload_name(cfg, T), "tokens_per_gpu": T,
+                       "global_tokens": T * world, "r": cfg.r, "alpha": cfg.alpha,
+                       "step": "per linear: nf4_quantize, qlora_fwd, qlora_bwd, lora_merge, lora_unmerge"
+                               + (" + all-reduce(dA, dB)" if world > 1 else ""),
+                       "l2": "inputs larger than L2; L2 flushed (256 MB write) between timed steps",
+                       "parallelism": f"dp{world}"},
+            "tokens_per_s": tokens_s,
+            "roofline": {"kernel": "gemm_tc_kernel<256> (fwd main + dX)", "bound": "tensor",
+                         "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak if peak else None, "traffic": traffic,
+                         "peak_source": f"{peak_src} bf16_tflops_sustained",
+                         "launches": g_launches, "ms_per_launch": g_ms / max(1, g_launches)},
+            "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "ms_per_step": float(te.item())},
+            "gpu_launches": launches // args.steps * args.steps,
+            "gpu_launches_per_step": launches / args.steps,
+            "clocks": clk,
+            "rows": rows,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(cfg)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier(device_ids=[local])
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", type=int, default=4)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

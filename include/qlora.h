@@ -158,7 +158,8 @@ QLORA_API size_t qlora_bwd_workspace_bytes(int64_t d, int64_t k, int r, int64_t 
  *   dX = dY W' + s G A         (bf16, T x k)
  *   dA = s G^T X               (fp32, r x k, overwritten)
  *   dB = s dY^T U              (fp32, d x r, overwritten; U = U_saved)
- * No weight gradient is formed.  dA and dB are reduced in a fixed order, so
+ * Requires d % 8 == 0 (rows of dY 16-byte aligned).  No weight gradient is
+ * formed.  dA and dB are reduced in a fixed order, so
  * repeated calls give identical bits.
  */
 QLORA_API int qlora_bwd(const qlora_nf4_t* q, const uint16_t* A, const uint16_t* B, int r, float alpha,

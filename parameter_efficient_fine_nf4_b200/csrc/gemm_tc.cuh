@@ -49,6 +49,8 @@ struct GemmArgs {
   int64_t ldo2;
   float alpha2;
   int n_store2;
+  int lo_offset;              // > 0: out2 also gets lo = bf16(v - bf16(v)) at this column offset
+  int pair_offset;            // > 0: the result is acc[j] + acc[j + pair_offset] (hi/lo operand pair)
   const uint8_t* codes;
   const uint8_t* absmax_q;
   const float* scale2;
@@ -244,9 +246,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16);
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
+        if (p.pair_offset > 0 && c * 32 >= p.pair_offset) break;   // lo columns: consumed below
         uint32_t v[32];
         tmem_ld_32x32b_x32(taddr + (uint32_t)(c * 32), v);
         tmem_ld_wait();
+        if (p.pair_offset > 0) {
+          uint32_t lo[32];
+          tmem_ld_32x32b_x32(taddr + (uint32_t)(c * 32 + p.pair_offset), lo);
+          tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            v[i] = __float_as_uint(__fadd_rn(__uint_as_float(v[i]), __uint_as_float(lo[i])));
+        }
         const int n = n0 + c * 32;
         if (!row_ok || n >= p.N) continue;
         if (p.epi == EPI_BF16) {
@@ -284,8 +295,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           if (p.out2 != nullptr) {
             uint16_t* o2 = p.out2 + (int64_t)m * p.ldo2 + n;
             for (int i = 0; i < 32 && n + i < p.n_store2; ++i) {
-              __nv_bfloat16 h = __float2bfloat16_rn(__fmul_rn(p.alpha2, __uint_as_float(v[i])));
-              o2[i] = *reinterpret_cast<uint16_t*>(&h);
+              const float x = __fmul_rn(p.alpha2, __uint_as_float(v[i]));
+              const __nv_bfloat16 h = __float2bfloat16_rn(x);
+              o2[i] = *reinterpret_cast<const uint16_t*>(&h);
+              if (p.lo_offset > 0) {
+                const __nv_bfloat16 l = __float2bfloat16_rn(__fsub_rn(x, __bfloat162float(h)));
+                o2[i + p.lo_offset] = *reinterpret_cast<const uint16_t*>(&l);
+              }
             }
           }
         } else if (p.epi == EPI_F32_T) {

@@ -371,25 +371,81 @@ int splits_for(int64_t tiles, int64_t K) {
   return s;
 }
 
+// Effective split count of a K range cut into 64-aligned pieces (the kernel
+// derives the same value from k_per_split).
+int eff_splits(int64_t K, int splits) {
+  const int64_t per = round_up(cdiv(K, splits), kBK);
+  return (int)cdiv(K, per);
+}
+
 struct BwdWs {
-  uint16_t* Wdq; uint16_t* Us; uint16_t* Gs; uint16_t* Bp; float* partA; float* partB;
-  int splitsA, splitsB; size_t bytes;
+  uint16_t* Wdq; uint16_t* Us2; uint16_t* Gs2; uint16_t* Bp; float* partA; float* partB;
+  int rp, halves, splitsA, splitsB; size_t bytes;
 };
+// Backward workspace.  U and G enter the T-reductions (dB, dA) as two bf16
+// terms, hi = bf16(v) and lo = bf16(v - hi), stored side by side in rows of
+// 2*rp columns (rp = r rounded up to 32); with rp <= 128 one GEMM with N = 2*rp
+// multiplies both and the epilogue adds the paired columns, otherwise the two
+// halves run as two GEMMs whose partial outputs are summed.
 BwdWs carve_bwd(void* ws, int64_t d, int64_t k, int r, int64_t T) {
   Carver c{reinterpret_cast<uint8_t*>(ws)};
   const int64_t r8 = round_up(r, 8);
   const int64_t Tm = std::max<int64_t>(T, 1);
   BwdWs w;
+  w.rp = (int)round_up(r, 32);
+  w.halves = w.rp > 128 ? 2 : 1;
   w.Wdq = (uint16_t*)c.take((size_t)(d * k * 2));
-  w.Us = (uint16_t*)c.take((size_t)(Tm * r8 * 2));
-  w.Gs = (uint16_t*)c.take((size_t)(Tm * r8 * 2));
+  w.Us2 = (uint16_t*)c.take((size_t)(Tm * 2 * w.rp * 2));
+  w.Gs2 = (uint16_t*)c.take((size_t)(Tm * 2 * w.rp * 2));
   w.Bp = (uint16_t*)c.take((size_t)(d * r8 * 2));
-  w.splitsA = splits_for(cdiv(k, kBM), Tm);
-  w.splitsB = splits_for(cdiv(d, kBM), Tm);
-  w.partA = (float*)c.take((size_t)(w.splitsA > 1 ? w.splitsA * r * k * 4 : 0));
-  w.partB = (float*)c.take((size_t)(w.splitsB > 1 ? w.splitsB * d * r * 4 : 0));
+  w.splitsA = eff_splits(Tm, splits_for(cdiv(k, kBM), Tm));
+  w.splitsB = eff_splits(Tm, splits_for(cdiv(d, kBM), Tm));
+  const int64_t pa = (int64_t)w.splitsA * w.halves, pb = (int64_t)w.splitsB * w.halves;
+  w.partA = (float*)c.take((size_t)(pa > 1 ? pa * r * k * 4 : 0));
+  w.partB = (float*)c.take((size_t)(pb > 1 ? pb * d * r * 4 : 0));
   w.bytes = c.off;
   return w;
+}
+
+// One T-reduction GEMM of the adapter gradients: out (M x r, or r x M when
+// transposed) = big^T hilo, big an MN-major T x M bf16 matrix, hilo the
+// T x 2rp hi/lo operand.  Deterministic: partials are reduced in fixed order.
+int adapter_grad_gemm(const char* name, const uint16_t* big, int64_t M, int64_t T, const uint16_t* hilo,
+                      int r, int rp, int halves, int splits, bool transposed, float* out,
+                      float* part, cudaStream_t st) {
+  const int nparts = splits * halves;
+  const int64_t plane = M * r;
+  for (int h = 0; h < halves; ++h) {
+    GemmPlan g;
+    g.M = (int)M; g.K0 = (int)T; g.splits = splits;
+    g.a0 = mnmajor(big, M, T, M);
+    GemmArgs a = blank_args();
+    a.epi = transposed ? EPI_F32_T : EPI_F32;
+    a.alpha = 1.0f;
+    a.n_store = r;
+    a.ldo = transposed ? M : r;
+    if (halves == 1) {
+      g.N = 2 * rp; g.bn = 2 * rp;
+      g.b0 = mnmajor(hilo, 2 * rp, T, 2 * rp);
+      a.pair_offset = rp;
+    } else {
+      g.N = r; g.bn = 256;
+      g.b0 = mnmajor(hilo + (size_t)h * rp, r, T, 2 * rp);
+    }
+    if (nparts > 1) {
+      a.out = part + (size_t)h * splits * plane;
+      a.split_stride = plane;
+    } else {
+      a.out = out;
+    }
+    QLORA_TRY(launch_gemm(name, g, a, st));
+  }
+  if (nparts > 1) {
+    QLORA_TRY(launch("splitk_reduce_f32", 0.0, (double)plane * 4 * (nparts + 1), st, [&] {
+      splitk_reduce_f32<<<grid_for(plane, 256), 256, 0, st>>>(part, nparts, plane, out);
+    }));
+  }
+  return QLORA_OK;
 }
 
 }  // namespace
@@ -553,6 +609,7 @@ int qlora_bwd(const qlora_nf4_t* q, const uint16_t* A, const uint16_t* B, int r,
       !aligned16(dB) || !aligned16(U_saved) || !aligned16(ws))
     return QLORA_ERR_MISALIGNED;
   if (T > ((int64_t)1 << 31)) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (d % 8 != 0) return QLORA_ERR_UNSUPPORTED_SHAPE;   // dY rows must be 16-byte aligned for TMA
   BwdWs w = carve_bwd(ws, d, k, r, T);
   if (ws_bytes < w.bytes) return QLORA_ERR_WORKSPACE_TOO_SMALL;
   QLORA_TRY(ensure_device());
@@ -564,11 +621,12 @@ int qlora_bwd(const qlora_nf4_t* q, const uint16_t* A, const uint16_t* B, int r,
   int pst = QLORA_OK;
   const uint16_t* Bp = padded_B(B, d, r, r8, w.Bp, st, &pst);
   QLORA_TRY(pst);
-  // Us = bf16(s U)
-  QLORA_TRY(launch("scale_f32_to_bf16", 0.0, (double)T * r * 6, st, [&] {
-    scale_f32_to_bf16<<<grid_for(T * r8, 256), 256, 0, st>>>(U_saved, T, r, s, w.Us, r8);
+  const int rp = w.rp;
+  // Us2 = hi/lo of bf16(s U)
+  QLORA_TRY(launch("scale_f32_to_bf16_hilo", 0.0, (double)T * r * 8, st, [&] {
+    scale_f32_to_bf16_hilo<<<grid_for(T * rp, 256), 256, 0, st>>>(U_saved, T, r, s, w.Us2, rp);
   }));
-  // G = dY B  ->  Gs = bf16(s G)
+  // G = dY B  ->  Gs2 = hi/lo of bf16(s G)
   {
     GemmPlan g;
     g.M = (int)T; g.N = r; g.K0 = (int)d; g.bn = bnr;
@@ -576,58 +634,22 @@ int qlora_bwd(const qlora_nf4_t* q, const uint16_t* A, const uint16_t* B, int r,
     g.b0 = mnmajor(Bp, r8, d, r8);
     GemmArgs a = blank_args();
     a.epi = EPI_F32; a.out = nullptr; a.n_store = 0;
-    a.out2 = w.Gs; a.ldo2 = r8; a.alpha2 = s; a.n_store2 = r8;
+    a.out2 = w.Gs2; a.ldo2 = 2 * rp; a.alpha2 = s; a.n_store2 = rp; a.lo_offset = rp;
     QLORA_TRY(launch_gemm("gemm_lora_g", g, a, st));
   }
-  // dB = dY^T (sU)   (M = d, N = r, K = T)
-  {
-    GemmPlan g;
-    g.M = (int)d; g.N = r; g.K0 = (int)T; g.bn = bnr; g.splits = w.splitsB;
-    g.a0 = mnmajor(dY, d, T, d);
-    g.b0 = mnmajor(w.Us, r8, T, r8);
-    GemmArgs a = blank_args();
-    a.epi = EPI_F32; a.alpha = 1.0f; a.n_store = r;
-    if (w.splitsB > 1) {
-      a.out = w.partB; a.ldo = r; a.split_stride = d * r;
-    } else {
-      a.out = dB; a.ldo = r;
-    }
-    QLORA_TRY(launch_gemm("gemm_lora_dB", g, a, st));
-    if (w.splitsB > 1) {
-      const int splits = (int)cdiv(T, round_up(cdiv(T, w.splitsB), kBK));
-      QLORA_TRY(launch("splitk_reduce_f32", 0.0, (double)d * r * 4 * (splits + 1), st, [&] {
-        splitk_reduce_f32<<<grid_for(d * r, 256), 256, 0, st>>>(w.partB, splits, d * r, dB);
-      }));
-    }
-  }
-  // dA^T = X^T (sG)  (M = k, N = r, K = T), stored transposed into dA (r x k)
-  {
-    GemmPlan g;
-    g.M = (int)k; g.N = r; g.K0 = (int)T; g.bn = bnr; g.splits = w.splitsA;
-    g.a0 = mnmajor(X, k, T, k);
-    g.b0 = mnmajor(w.Gs, r8, T, r8);
-    GemmArgs a = blank_args();
-    a.epi = EPI_F32_T; a.alpha = 1.0f; a.n_store = r; a.ldo = k;
-    if (w.splitsA > 1) {
-      a.out = w.partA; a.split_stride = (int64_t)r * k;
-    } else {
-      a.out = dA;
-    }
-    QLORA_TRY(launch_gemm("gemm_lora_dA", g, a, st));
-    if (w.splitsA > 1) {
-      const int splits = (int)cdiv(T, round_up(cdiv(T, w.splitsA), kBK));
-      QLORA_TRY(launch("splitk_reduce_f32", 0.0, (double)r * k * 4 * (splits + 1), st, [&] {
-        splitk_reduce_f32<<<grid_for((int64_t)r * k, 256), 256, 0, st>>>(w.partA, splits, (int64_t)r * k, dA);
-      }));
-    }
-  }
+  // dB = dY^T (s U)   (M = d, N = r, K = T)
+  QLORA_TRY(adapter_grad_gemm("gemm_lora_dB", dY, d, T, w.Us2, r, rp, w.halves, w.splitsB,
+                              false, dB, w.partB, st));
+  // dA^T = X^T (s G)  (M = k, N = r, K = T), stored transposed into dA (r x k)
+  QLORA_TRY(adapter_grad_gemm("gemm_lora_dA", X, k, T, w.Gs2, r, rp, w.halves, w.splitsA,
+                              true, dA, w.partA, st));
   // dX = [dY | sG] [W' ; A]   (M = T, N = k, K = d + r)
   {
     GemmPlan g;
     g.M = (int)T; g.N = (int)k; g.K0 = (int)d; g.K1 = r; g.bn = 256;
     g.a0 = kmajor(dY, d, T, d);
     g.b0 = mnmajor(w.Wdq, k, d, k);
-    g.a1 = kmajor(w.Gs, r8, T, r8);
+    g.a1 = kmajor(w.Gs2, r, T, 2 * rp);          // hi part of s G
     g.b1 = mnmajor(A, k, r, k);
     GemmArgs a = blank_args();
     a.epi = EPI_BF16; a.out = dX; a.ldo = k; a.n_store = (int)k;

@@ -268,17 +268,23 @@ __global__ void pad_cols_bf16(const uint16_t* __restrict__ src, int64_t rows, in
   }
 }
 
-// dst (rows x ld_dst, bf16) = bf16(scale * src) with zero padding columns.
-__global__ void scale_f32_to_bf16(const float* __restrict__ src, int64_t rows, int cols,
-                                  float scale, uint16_t* __restrict__ dst, int ld_dst) {
-  const int64_t n = rows * ld_dst;
+// Two-term bf16 split of v = fp32(scale * src): hi = bf16(v), lo = bf16(v - hi)
+// (v - hi is exact in fp32), so hi + lo carries about 16 significant bits.
+// dst row t: columns [0, half) hold hi, [half, 2*half) hold lo; columns at or
+// beyond `cols` within each half are zero.
+__global__ void scale_f32_to_bf16_hilo(const float* __restrict__ src, int64_t rows, int cols,
+                                       float scale, uint16_t* __restrict__ dst, int half) {
+  const int ld = 2 * half;
+  const int64_t n = rows * half;
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride) {
-    const int64_t rrow = i / ld_dst;
-    const int c = (int)(i - rrow * ld_dst);
-    float v = (c < cols) ? __fmul_rn(scale, src[rrow * cols + c]) : 0.f;
-    __nv_bfloat16 h = __float2bfloat16_rn(v);
-    dst[i] = *reinterpret_cast<uint16_t*>(&h);
+    const int64_t rrow = i / half;
+    const int c = (int)(i - rrow * half);
+    const float v = (c < cols) ? __fmul_rn(scale, src[rrow * cols + c]) : 0.f;
+    const __nv_bfloat16 h = __float2bfloat16_rn(v);
+    const __nv_bfloat16 l = __float2bfloat16_rn(__fsub_rn(v, __bfloat162float(h)));
+    dst[rrow * ld + c] = *reinterpret_cast<const uint16_t*>(&h);
+    dst[rrow * ld + half + c] = *reinterpret_cast<const uint16_t*>(&l);
   }
 }
 

@@ -49,12 +49,20 @@ def rows_within(gpu: np.ndarray, ref: np.ndarray, tol: float = TOL, what: str = 
     return worst
 
 
-def within_one_bf16_ulp(gpu_bits: np.ndarray, ref_bits: np.ndarray, what: str = "", ulps: int = 1):
-    """|gpu - ref| <= ulps * (bf16 spacing at the larger of the two magnitudes)."""
+def within_one_bf16_ulp(gpu_bits: np.ndarray, ref_bits: np.ndarray, what: str = "", ulps: int = 1,
+                        abs_extra=0.0, mag_extra=None):
+    """|gpu - ref| <= ulps * (bf16 spacing at the larger of the two magnitudes) + abs_extra.
+
+    abs_extra carries the fp32 error of the GPU's rank-r product before the one
+    rounding to bf16 (it matters only where W' + s B A cancels to a value far
+    smaller than its terms)."""
     g = (gpu_bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
     r = (ref_bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
-    mag = np.maximum(np.abs(r), np.abs(g)).astype(np.float32)
+    mag = np.maximum(np.abs(r), np.abs(g))
+    if mag_extra is not None:
+        mag = np.maximum(mag, np.abs(mag_extra))
+    mag = mag.astype(np.float32)
     ulp = np.spacing(mag).astype(np.float64) * 65536.0
-    ulp = np.maximum(ulp, 2.0 ** -133) * ulps
+    ulp = np.maximum(ulp, 2.0 ** -133) * ulps + abs_extra
     bad = np.abs(g - r) > ulp
     assert not bad.any(), f"{what}: {int(bad.sum())} elements beyond 1 bf16 ulp"

@@ -87,7 +87,7 @@ def test_config1_b_zero_init():
 @pytest.mark.parametrize("d,k,r,T", [
     (320, 192, 5, 200),      # ragged M and N tiles, r not a multiple of 8
     (64, 64, 1, 1),          # one token, rank 1
-    (130, 128, 3, 129),      # d one past a tile in the extension operand rows
+    (136, 128, 3, 129),      # d just past a tile, T just past a tile
     (256, 512, 100, 300),    # r > 64: two extension steps on a 128-wide N tile
     (384, 256, 256, 64),     # maximum rank
     (200, 64, 16, 1000),     # K = 64: one main step
@@ -95,6 +95,21 @@ def test_config1_b_zero_init():
 def test_ragged_shapes(d, k, r, T):
     lay = synthetic.custom_layer(seed=d * 131 + k * 7 + r + T, d=d, k=k, r=r, T=T, alpha=2.0 * r)
     Case(lay, 2.0 * r).check()
+
+
+def test_forward_any_d_backward_needs_d_multiple_of_8():
+    # forward accepts any d; backward needs 16-byte aligned rows of dY
+    lay = synthetic.custom_layer(seed=9, d=130, k=128, r=3, T=40, alpha=6.0)
+    qw = q4.qlora_nf4_quantize(f32_dev(lay.W0))
+    A, B, X, dY = bf16_dev(lay.A), bf16_dev(lay.B), bf16_dev(lay.X), bf16_dev(lay.dY)
+    Y, U = q4.qlora_fwd(qw, A, B, 6.0, X)
+    torch.cuda.synchronize()
+    Wp = oracle_Wp(lay.W0)
+    fw = lora.forward(nf4.bf16_to_f64(lay.X), Wp, nf4.bf16_to_f64(lay.A), nf4.bf16_to_f64(lay.B), 2.0)
+    rows_within(bf16_host_f64(Y), fw["Y"], what="Y")
+    with pytest.raises(q4.QloraError) as e:
+        q4.qlora_bwd(qw, A, B, 6.0, X, U, dY)
+    assert e.value.status == 2
 
 
 @pytest.mark.parametrize("ci", [2, 3])
@@ -151,13 +166,17 @@ def test_merge_unmerge(ci):
     Wp = nf4.bf16_to_f64(nf4.dequantize(qt))
     Af, Bf = nf4.bf16_to_f64(lay.A), nf4.bf16_to_f64(lay.B)
     ref_W = lora.merge(Wp, Af, Bf, s)
-    within_one_bf16_ulp(bf16_host_bits(W), ref_W, "merge")
+    # fp32 error bound of the GPU's r-term product (accumulated on the tensor
+    # core) and of the fused multiply-add, before the single bf16 rounding:
+    # r * 2^-22 * s * sum_q |B_iq A_qj|  +  2^-23 * |W'_ij|
+    extra = cfg.r * 2.0 ** -22 * s * (np.abs(Bf) @ np.abs(Af)) + 2.0 ** -23 * np.abs(Wp)
+    within_one_bf16_ulp(bf16_host_bits(W), ref_W, "merge", abs_extra=extra)
     # unmerge of the oracle's merged weight
     W_in = bf16_dev(ref_W)
     W0pp = q4.lora_unmerge(W_in, A, B, cfg.alpha)
     torch.cuda.synchronize()
     ref_W0pp = lora.unmerge(nf4.bf16_to_f64(ref_W), Af, Bf, s)
-    within_one_bf16_ulp(bf16_host_bits(W0pp), ref_W0pp, "unmerge")
+    within_one_bf16_ulp(bf16_host_bits(W0pp), ref_W0pp, "unmerge", abs_extra=extra)
     # merge then unmerge on the GPU gives back the dequantised base (1 ulp),
     # and with B = 0 both are exactly the dequantised base
     back = q4.lora_unmerge(W, A, B, cfg.alpha)
@@ -167,8 +186,16 @@ def test_merge_unmerge(ci):
     Wz2 = q4.lora_unmerge(Wdq, A, Z, cfg.alpha)
     torch.cuda.synchronize()
     # two roundings (merge, then unmerge), each at most half an ulp of the
-    # larger of W and W'
-    within_one_bf16_ulp(bf16_host_bits(back), nf4.dequantize(qt), "merge-unmerge", ulps=2)
+    # larger of the merged W and the result
+    W_mag = bf16_host_f64(W)
+    within_one_bf16_ulp(bf16_host_bits(back), nf4.dequantize(qt), "merge-unmerge", ulps=1,
+                        abs_extra=2 * extra, mag_extra=W_mag)
+    # the round trip re-encodes to the stored codes with the stored block scales
+    a2 = nf4.block_scale(qt["absmax_q"], qt["scale2"], qt["mean"]).astype(np.float64)
+    q = nf4.nf4_levels().astype(np.float64)
+    x = bf16_host_f64(back).reshape(-1, 64) / a2[:, None]
+    codes = np.abs(x[..., None] - q).argmin(-1).ravel().astype(np.uint8)
+    assert np.array_equal(codes, nf4.unpack_codes(qt["codes"]))
     assert torch.equal(Wz, Wdq) and torch.equal(Wz2, Wdq)
     assert q4.qlora_get_device_status() == 0
 
