@@ -44,7 +44,8 @@ typedef enum {
   QLORA_ERR_WORKSPACE_TOO_SMALL = 4,
   QLORA_ERR_CUDA = 5,              /* a CUDA runtime/driver call or launch failed */
   QLORA_ERR_TIMEOUT = 6,           /* a device-side wait gave up (device status) */
-  QLORA_ERR_NO_DEVICE = 7          /* no sm_100 device is current */
+  QLORA_ERR_NO_DEVICE = 7,         /* no sm_100 device is current */
+  QLORA_ERR_EXCEEDS_STATIC_SCRATCH = 8 /* too large for qlora_nf4_quantize_noalloc */
 } qlora_status_t;
 
 /* A cudaStream_t passed as an opaque pointer (NULL = legacy default stream). */
@@ -128,6 +129,38 @@ QLORA_API int qlora_nf4_quantize(const float* W0, int64_t d, int64_t k, int bloc
  * This is the exact bf16 weight every GEMM of this library multiplies by.
  */
 QLORA_API int qlora_nf4_dequantize(const qlora_nf4_t* q, uint16_t* W_out, qlora_stream_t stream);
+
+/*
+ * Quantise without any allocation and without a caller workspace.
+ *
+ * (This entry point has no counterpart on the source pages; it exists for
+ * callers that cannot allocate device memory at all.)  Some callers hold only
+ * the device buffers they were handed: a plugin whose host framework owns
+ * every byte of device memory through its own pool and forbids allocations
+ * outside it, or a recovery path that re-quantises weights after the device
+ * has run out of memory, where any new cudaMalloc would fail.  They can call
+ * this instead of qlora_nf4_quantize.
+ *
+ * Same arguments and results as qlora_nf4_quantize, minus the workspace.  The
+ * scratch space (fp32 block constants and fp64 group sums) lives in a
+ * file-scope __device__ array of QLORA_NOALLOC_MAX_WEIGHTS/16 +
+ * QLORA_NOALLOC_MAX_WEIGHTS/2048 bytes (16.1 MiB) that every GPU which loads
+ * this library holds until the process exits.  d*k above
+ * QLORA_NOALLOC_MAX_WEIGHTS (2^28 weights) is rejected with
+ * QLORA_ERR_EXCEEDS_STATIC_SCRATCH before anything is launched.
+ *
+ * The first call on a device looks up the array's device address (with that
+ * device current) and caches it; make that first call before any stream
+ * capture begins.  All calls share the one array, which keeps the contents
+ * of the last call; every byte a call reads from it is first written by the
+ * same call, so nothing needs clearing.  Calls that overlap on the GPU (on
+ * different streams, or from different threads) race on the array and must
+ * be serialised by the caller.  No cudaMalloc, cudaFree or allocating library
+ * routine is called.
+ */
+#define QLORA_NOALLOC_MAX_WEIGHTS ((int64_t)1 << 28)
+QLORA_API int qlora_nf4_quantize_noalloc(const float* W0, int64_t d, int64_t k, int block,
+                                         qlora_nf4_t* out, qlora_stream_t stream);
 
 /* ---------------------------------------------------------------- forward */
 

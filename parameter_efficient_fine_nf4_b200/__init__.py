@@ -59,6 +59,7 @@ _SIGNATURES = {
     "qlora_quantize_workspace_bytes": (_SIZE, [_I64, _I64]),
     "qlora_nf4_quantize": (_INT, [_VP, _I64, _I64, _INT, _NF4P, _VP, _SIZE, _VP]),
     "qlora_nf4_dequantize": (_INT, [_NF4P, _VP, _VP]),
+    "qlora_nf4_quantize_noalloc": (_INT, [_VP, _I64, _I64, _INT, _NF4P, _VP]),
     "qlora_fwd_workspace_bytes": (_SIZE, [_I64, _I64, _INT, _I64]),
     "qlora_fwd": (_INT, [_NF4P, _VP, _VP, _INT, _F, _VP, _I64, _VP, _VP, _VP, _SIZE, _VP]),
     "qlora_bwd_workspace_bytes": (_SIZE, [_I64, _I64, _INT, _I64]),
@@ -197,6 +198,24 @@ def qlora_nf4_quantize(W0: torch.Tensor, out: Optional[NF4Weight] = None,
     st = lib().qlora_nf4_quantize(_ptr(W0), d, k, BLOCK, ctypes.byref(out.cstruct), _ptr(ws),
                                   ws.numel(), _stream(stream))
     _check(st, "qlora_nf4_quantize")
+    return out
+
+
+NOALLOC_MAX_WEIGHTS = 1 << 28
+
+
+def qlora_nf4_quantize_noalloc(W0: torch.Tensor, out: NF4Weight, stream=None) -> NF4Weight:
+    """Quantise using the library's static device scratch (no workspace).
+
+    For callers that cannot allocate device memory: pass preallocated output
+    buffers in ``out``; nothing else is allocated.  d*k is limited to 2^28.
+    Calls share one scratch array, so calls that overlap on the GPU race.
+    """
+    d, k = W0.shape
+    _need(W0, torch.float32, (d, k), "W0")
+    st = lib().qlora_nf4_quantize_noalloc(_ptr(W0), d, k, BLOCK, ctypes.byref(out.cstruct),
+                                          _stream(stream))
+    _check(st, "qlora_nf4_quantize_noalloc")
     return out
 
 

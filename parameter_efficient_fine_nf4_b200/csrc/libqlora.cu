@@ -453,6 +453,34 @@ int adapter_grad_gemm(const char* name, const uint16_t* big, int64_t M, int64_t 
 
 using namespace qlora;
 
+// Scratch of qlora_nf4_quantize_noalloc: room for the fp32 block constants and
+// fp64 group sums of QLORA_NOALLOC_MAX_WEIGHTS weights.  In host code this
+// name is only a stand-in for the device array; its device address comes from
+// cudaGetSymbolAddress, once per device.
+static constexpr size_t kNoallocScratchBytes =
+    (size_t)(QLORA_NOALLOC_MAX_WEIGHTS / 16) + (size_t)(QLORA_NOALLOC_MAX_WEIGHTS / 2048);
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratchBytes];
+
+namespace {
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[64] = {nullptr};
+
+// Device address of g_noalloc_scratch on the current device (looked up on the
+// first call per device, with that device current, then cached).
+int noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return QLORA_ERR_NO_DEVICE;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return QLORA_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return QLORA_OK;
+}
+}  // namespace
+
 // =====================================================================
 // C ABI
 // =====================================================================
@@ -468,6 +496,8 @@ const char* qlora_strerror(int s) {
     case QLORA_ERR_CUDA: return "CUDA error";
     case QLORA_ERR_TIMEOUT: return "device wait timed out";
     case QLORA_ERR_NO_DEVICE: return "no sm_100 device is current";
+    case QLORA_ERR_EXCEEDS_STATIC_SCRATCH:
+      return "d*k exceeds the static scratch of qlora_nf4_quantize_noalloc (2^28 weights)";
     default: return "unknown status";
   }
 }
@@ -519,6 +549,15 @@ int qlora_nf4_quantize(const float* W0, int64_t d, int64_t k, int block, qlora_n
     nf4_quantize_dq<<<(unsigned)n_g, 256, 0, st>>>(absmax, n_b, out->mean, out->absmax_q, out->scale2);
   }));
   return QLORA_OK;
+}
+
+int qlora_nf4_quantize_noalloc(const float* W0, int64_t d, int64_t k, int block, qlora_nf4_t* out,
+                               qlora_stream_t stream) {
+  if (d >= 1 && k >= 1 && d * k > QLORA_NOALLOC_MAX_WEIGHTS) return QLORA_ERR_EXCEEDS_STATIC_SCRATCH;
+  QLORA_TRY(ensure_device());
+  void* scratch = nullptr;
+  QLORA_TRY(noalloc_scratch(&scratch));
+  return qlora_nf4_quantize(W0, d, k, block, out, scratch, kNoallocScratchBytes, stream);
 }
 
 int qlora_nf4_dequantize(const qlora_nf4_t* q, uint16_t* W_out, qlora_stream_t stream) {
