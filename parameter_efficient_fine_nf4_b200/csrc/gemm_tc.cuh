@@ -66,7 +66,7 @@ struct GemmCfg {
   static constexpr int kABytes = kBM * kBK * 2;                 // 16 KB
   static constexpr int kBBytes = BN * kBK * 2;
   static constexpr int kStageBytes = kABytes + kBBytes;
-  static constexpr int kTmemCols = BN;                           // power of two >= 64
+  static constexpr int kTmemCols = 2 * BN;                       // two accumulators
   static constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 512 /*bars*/;
 };
 
@@ -77,6 +77,212 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 
 __device__ __forceinline__ float bf16_bits_to_f32(uint32_t b16) { return __uint_as_float(b16 << 16); }
 
+// Work unit u -> (tile row, tile column, K split), tiles rasterised in groups
+// of `group_m` tile rows so that concurrently running CTAs share A and B tiles
+// in L2.
+struct Unit {
+  int m0, n0, split;
+};
+__device__ __forceinline__ Unit unit_coords(const GemmArgs& p, int u, int bn) {
+  const int tiles = p.tiles_m * p.tiles_n;
+  Unit r;
+  r.split = u / tiles;
+  const int t = u - r.split * tiles;
+  const int per_group = p.group_m * p.tiles_n;
+  const int gidx = t / per_group;
+  const int first_m = gidx * p.group_m;
+  const int gsize = min(p.group_m, p.tiles_m - first_m);
+  const int in_group = t - gidx * per_group;
+  r.m0 = (first_m + in_group % gsize) * kBM;
+  r.n0 = (in_group / gsize) * bn;
+  return r;
+}
+
+// Store one 32-column chunk of one accumulator row (row m, columns n..n+31).
+__device__ __forceinline__ void epilogue_chunk(const GemmArgs& p, uint32_t (&v)[32], int m, int n,
+                                               int split, const float* s_lut) {
+  if (p.epi == EPI_BF16) {
+    uint16_t* out = reinterpret_cast<uint16_t*>(p.out) + (int64_t)m * p.ldo + n;
+    if (n + 32 <= p.n_store && (p.ldo & 7) == 0) {
+      uint4* o4 = reinterpret_cast<uint4*>(out);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        uint4 w;
+        w.x = pack_bf16x2(__uint_as_float(v[8 * i + 0]), __uint_as_float(v[8 * i + 1]));
+        w.y = pack_bf16x2(__uint_as_float(v[8 * i + 2]), __uint_as_float(v[8 * i + 3]));
+        w.z = pack_bf16x2(__uint_as_float(v[8 * i + 4]), __uint_as_float(v[8 * i + 5]));
+        w.w = pack_bf16x2(__uint_as_float(v[8 * i + 6]), __uint_as_float(v[8 * i + 7]));
+        o4[i] = w;
+      }
+    } else {
+      for (int i = 0; i < 32 && n + i < p.n_store; ++i) {
+        __nv_bfloat16 h = __float2bfloat16_rn(__uint_as_float(v[i]));
+        out[i] = *reinterpret_cast<uint16_t*>(&h);
+      }
+    }
+  } else if (p.epi == EPI_F32) {
+    if (p.out != nullptr) {
+      float* out = reinterpret_cast<float*>(p.out) + (int64_t)split * p.split_stride + (int64_t)m * p.ldo + n;
+      if (n + 32 <= p.n_store && (p.ldo & 3) == 0) {
+        float4* o4 = reinterpret_cast<float4*>(out);
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          o4[i] = make_float4(p.alpha * __uint_as_float(v[4 * i]), p.alpha * __uint_as_float(v[4 * i + 1]),
+                              p.alpha * __uint_as_float(v[4 * i + 2]), p.alpha * __uint_as_float(v[4 * i + 3]));
+      } else {
+        for (int i = 0; i < 32 && n + i < p.n_store; ++i) out[i] = p.alpha * __uint_as_float(v[i]);
+      }
+    }
+    if (p.out2 != nullptr) {
+      uint16_t* o2 = p.out2 + (int64_t)m * p.ldo2 + n;
+      for (int i = 0; i < 32 && n + i < p.n_store2; ++i) {
+        const float x = __fmul_rn(p.alpha2, __uint_as_float(v[i]));
+        const __nv_bfloat16 h = __float2bfloat16_rn(x);
+        o2[i] = *reinterpret_cast<const uint16_t*>(&h);
+        if (p.lo_offset > 0) {
+          const __nv_bfloat16 l = __float2bfloat16_rn(__fsub_rn(x, __bfloat162float(h)));
+          o2[i + p.lo_offset] = *reinterpret_cast<const uint16_t*>(&l);
+        }
+      }
+    }
+  } else if (p.epi == EPI_F32_T) {
+    float* out = reinterpret_cast<float*>(p.out) + (int64_t)split * p.split_stride + m;
+    for (int i = 0; i < 32 && n + i < p.n_store; ++i) out[(int64_t)(n + i) * p.ldo] = p.alpha * __uint_as_float(v[i]);
+  } else if (p.epi == EPI_MERGE) {
+    // w' for row m, columns n..n+31: one 16-byte word of codes, one block
+    const int64_t e0 = (int64_t)m * p.N + n;
+    const uint4 cw = *reinterpret_cast<const uint4*>(p.codes + e0 / 2);
+    const float a_scale = block_scale(p.absmax_q, p.scale2, p.mean[0], e0 / kBlock);
+    uint32_t wq[16];
+    dequant32(cw, a_scale, s_lut, wq);
+    uint4* o4 = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(p.out) + (int64_t)m * p.ldo + n);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      uint32_t r4[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t wp = wq[4 * i + j];
+        const float lo = __fmaf_rn(p.alpha, __uint_as_float(v[8 * i + 2 * j]), bf16_bits_to_f32(wp & 0xFFFFu));
+        const float hi = __fmaf_rn(p.alpha, __uint_as_float(v[8 * i + 2 * j + 1]), bf16_bits_to_f32(wp >> 16));
+        r4[j] = pack_bf16x2(lo, hi);
+      }
+      o4[i] = make_uint4(r4[0], r4[1], r4[2], r4[3]);
+    }
+  } else if (p.epi == EPI_UNMERGE) {
+    const uint4* w4 = reinterpret_cast<const uint4*>(p.w_in + (int64_t)m * p.ldw + n);
+    uint4 wv[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) wv[i] = w4[i];
+    uint4* o4 = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(p.out) + (int64_t)m * p.ldo + n);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint32_t wr[4] = {wv[i].x, wv[i].y, wv[i].z, wv[i].w};
+      uint32_t r4[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float lo = __fmaf_rn(p.alpha, __uint_as_float(v[8 * i + 2 * j]), bf16_bits_to_f32(wr[j] & 0xFFFFu));
+        const float hi = __fmaf_rn(p.alpha, __uint_as_float(v[8 * i + 2 * j + 1]), bf16_bits_to_f32(wr[j] >> 16));
+        r4[j] = pack_bf16x2(lo, hi);
+      }
+      o4[i] = make_uint4(r4[0], r4[1], r4[2], r4[3]);
+    }
+  }
+}
+
+// Merge / unmerge epilogue of one accumulator row: these kernels are bound by
+// the epilogue's global traffic (one K-step of MMA per tile), so the loads of
+// the codes (merge) or of W (unmerge) are issued ahead of the TMEM reads that
+// consume them: all of a row's code words at once, W one chunk ahead.
+template <int BN>
+__device__ __forceinline__ void epilogue_merge_row(const GemmArgs& p, uint32_t taddr, int m, bool row_ok,
+                                                   int n0, const float* s_lut) {
+  constexpr int NC = BN / 32;
+  if (p.epi == EPI_MERGE) {
+    uint4 cw[NC];
+    float asc[NC];
+    const float mu = p.mean[0];
+#pragma unroll
+    for (int ch = 0; ch < NC; ++ch) {
+      const int n = n0 + ch * 32;
+      cw[ch] = make_uint4(0u, 0u, 0u, 0u);
+      asc[ch] = 0.f;
+      if (row_ok && n < p.N) {
+        const int64_t e0 = (int64_t)m * p.N + n;
+        cw[ch] = __ldg(reinterpret_cast<const uint4*>(p.codes + e0 / 2));
+        asc[ch] = block_scale(p.absmax_q, p.scale2, mu, e0 / kBlock);
+      }
+    }
+#pragma unroll
+    for (int ch = 0; ch < NC; ++ch) {
+      uint32_t v[32];
+      tmem_ld_32x32b_x32(taddr + (uint32_t)(ch * 32), v);
+      tmem_ld_wait();
+      const int n = n0 + ch * 32;
+      if (!row_ok || n >= p.N) continue;
+      uint32_t wq[16];
+      dequant32(cw[ch], asc[ch], s_lut, wq);
+      uint4* o4 = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(p.out) + (int64_t)m * p.ldo + n);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        uint32_t r4[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint32_t wp = wq[4 * i + j];
+          const float lo = __fmaf_rn(p.alpha, __uint_as_float(v[8 * i + 2 * j]), bf16_bits_to_f32(wp & 0xFFFFu));
+          const float hi = __fmaf_rn(p.alpha, __uint_as_float(v[8 * i + 2 * j + 1]), bf16_bits_to_f32(wp >> 16));
+          r4[j] = pack_bf16x2(lo, hi);
+        }
+        o4[i] = make_uint4(r4[0], r4[1], r4[2], r4[3]);
+      }
+    }
+  } else {
+    uint4 wv[2][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) wv[0][i] = make_uint4(0u, 0u, 0u, 0u);
+    if (row_ok && n0 < p.N) {
+      const uint4* w4 = reinterpret_cast<const uint4*>(p.w_in + (int64_t)m * p.ldw + n0);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) wv[0][i] = __ldg(w4 + i);
+    }
+#pragma unroll
+    for (int ch = 0; ch < NC; ++ch) {
+      const int n = n0 + ch * 32;
+      if (ch + 1 < NC) {
+        const int nn = n + 32;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) wv[(ch + 1) & 1][i] = make_uint4(0u, 0u, 0u, 0u);
+        if (row_ok && nn < p.N) {
+          const uint4* w4 = reinterpret_cast<const uint4*>(p.w_in + (int64_t)m * p.ldw + nn);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) wv[(ch + 1) & 1][i] = __ldg(w4 + i);
+        }
+      }
+      uint32_t v[32];
+      tmem_ld_32x32b_x32(taddr + (uint32_t)(ch * 32), v);
+      tmem_ld_wait();
+      if (!row_ok || n >= p.N) continue;
+      uint4* o4 = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(p.out) + (int64_t)m * p.ldo + n);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const uint4 w = wv[ch & 1][i];
+        const uint32_t wr[4] = {w.x, w.y, w.z, w.w};
+        uint32_t r4[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float lo = __fmaf_rn(p.alpha, __uint_as_float(v[8 * i + 2 * j]), bf16_bits_to_f32(wr[j] & 0xFFFFu));
+          const float hi = __fmaf_rn(p.alpha, __uint_as_float(v[8 * i + 2 * j + 1]), bf16_bits_to_f32(wr[j] >> 16));
+          r4[j] = pack_bf16x2(lo, hi);
+        }
+        o4[i] = make_uint4(r4[0], r4[1], r4[2], r4[3]);
+      }
+    }
+  }
+}
+
+// Persistent kernel: CTA b processes work units b, b + gridDim.x, ...  The
+// shared-memory ring runs continuously across units; two TMEM accumulators
+// (columns [0, BN) and [BN, 2 BN)) let the epilogue of one unit overlap the
+// mainloop of the next (acc_full / acc_empty barriers per accumulator).
 template <int BN>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmB0,
@@ -93,39 +299,27 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint8_t* ctrl = smem + S * Cfg::kStageBytes;
   uint64_t* full_bar = reinterpret_cast<uint64_t*>(ctrl);
   uint64_t* empty_bar = full_bar + S;
-  uint64_t* accum_bar = empty_bar + S;
-  uint64_t* drain_bar = accum_bar + 1;
+  uint64_t* acc_full = empty_bar + S;       // [2]
+  uint64_t* acc_empty = acc_full + 2;       // [2]
+  uint64_t* drain_bar = acc_empty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_bar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* s_lut = reinterpret_cast<float*>(tmem_slot + 4);        // 16 floats
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-
-  // tile coordinates (grouped rasterisation along M)
-  const int tile = blockIdx.x;
-  const int per_group = p.group_m * p.tiles_n;
-  const int gidx = tile / per_group;
-  const int first_m = gidx * p.group_m;
-  const int gsize = min(p.group_m, p.tiles_m - first_m);
-  const int in_group = tile - gidx * per_group;
-  const int tm = first_m + in_group % gsize;
-  const int tn = in_group / gsize;
-  const int m0 = tm * kBM;
-  const int n0 = tn * BN;
-  const int split = blockIdx.y;
-  const int k_begin = split * p.k_per_split;
-  const int k_len0 = min(p.K0 - k_begin, p.k_per_split);
-  const int steps0 = (k_len0 + kBK - 1) / kBK;
+  const int units = p.tiles_m * p.tiles_n * (int)((p.K0 + p.k_per_split - 1) / p.k_per_split);
   const int steps1 = (p.K1 + kBK - 1) / kBK;
-  const int steps = steps0 + steps1;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < S; ++i) {
       mbar_init(smem_u32(&full_bar[i]), 1);
       mbar_init(smem_u32(&empty_bar[i]), 1);
     }
-    mbar_init(smem_u32(accum_bar), 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&acc_full[i]), 1);
+      mbar_init(smem_u32(&acc_empty[i]), 4);    // one arrive per epilogue warp
+    }
     mbar_init(smem_u32(drain_bar), 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -154,33 +348,42 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       int issued[S];
 #pragma unroll
       for (int i = 0; i < S; ++i) issued[i] = 0;
-      for (int step = 0; step < steps; ++step) {
-        const int st = step % S;
-        const uint32_t ph = (uint32_t)((step / S) & 1);
-        if (!mbar_wait_bounded(smem_u32(&empty_bar[st]), ph ^ 1u, abort_flag)) break;
-        const uint32_t fb = smem_u32(&full_bar[st]);
-        mbar_arrive_expect_tx(fb, Cfg::kStageBytes);
-        const uint32_t sa = sbase + st * Cfg::kStageBytes;
-        const uint32_t sb = sa + Cfg::kABytes;
-        const bool ext = step >= steps0;
-        const int kk = ext ? (step - steps0) * kBK : k_begin + step * kBK;
-        const CUtensorMap* ma = ext ? &tmA1 : &tmA0;
-        const CUtensorMap* mb = ext ? &tmB1 : &tmB0;
-        const int a_mn = ext ? p.a1_mn : p.a0_mn;
-        const int b_mn = ext ? p.b1_mn : p.b0_mn;
-        if (a_mn) {
-          tma_load_2d(sa, ma, fb, m0, kk);
-          tma_load_2d(sa + 8192, ma, fb, m0 + 64, kk);
-        } else {
-          tma_load_2d(sa, ma, fb, kk, m0);
-        }
-        if (b_mn) {
+      int g = 0;                                     // global step counter (ring position)
+      for (int u = blockIdx.x; u < units && !*abort_flag; u += gridDim.x) {
+        const Unit c = unit_coords(p, u, BN);
+        const int k_begin = c.split * p.k_per_split;
+        const int steps0 = (min(p.K0 - k_begin, p.k_per_split) + kBK - 1) / kBK;
+        const int steps = steps0 + (c.split == 0 ? steps1 : 0);
+        bool ok = true;
+        for (int step = 0; step < steps; ++step, ++g) {
+          const int st = g % S;
+          const uint32_t ph = (uint32_t)((g / S) & 1);
+          if (!mbar_wait_bounded(smem_u32(&empty_bar[st]), ph ^ 1u, abort_flag)) { ok = false; break; }
+          const uint32_t fb = smem_u32(&full_bar[st]);
+          mbar_arrive_expect_tx(fb, Cfg::kStageBytes);
+          const uint32_t sa = sbase + st * Cfg::kStageBytes;
+          const uint32_t sb = sa + Cfg::kABytes;
+          const bool ext = step >= steps0;
+          const int kk = ext ? (step - steps0) * kBK : k_begin + step * kBK;
+          const CUtensorMap* ma = ext ? &tmA1 : &tmA0;
+          const CUtensorMap* mb = ext ? &tmB1 : &tmB0;
+          const int a_mn = ext ? p.a1_mn : p.a0_mn;
+          const int b_mn = ext ? p.b1_mn : p.b0_mn;
+          if (a_mn) {
+            tma_load_2d(sa, ma, fb, c.m0, kk);
+            tma_load_2d(sa + 8192, ma, fb, c.m0 + 64, kk);
+          } else {
+            tma_load_2d(sa, ma, fb, kk, c.m0);
+          }
+          if (b_mn) {
 #pragma unroll
-          for (int i = 0; i < BN / 64; ++i) tma_load_2d(sb + i * 8192, mb, fb, n0 + 64 * i, kk);
-        } else {
-          tma_load_2d(sb, mb, fb, kk, n0);
+            for (int i = 0; i < BN / 64; ++i) tma_load_2d(sb + i * 8192, mb, fb, c.n0 + 64 * i, kk);
+          } else {
+            tma_load_2d(sb, mb, fb, kk, c.n0);
+          }
+          issued[st] += 1;
         }
-        issued[st] += 1;
+        if (!ok) break;
       }
       if (*abort_flag) {
         // let copies already in flight land before the CTA exits
@@ -195,40 +398,51 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const uint32_t idesc1 = idesc_bf16_f32(kBM, BN, p.a1_mn, p.b1_mn);
       bool ok = true;
       int issued_any = 0;
-      for (int step = 0; step < steps; ++step) {
-        const int st = step % S;
-        const uint32_t ph = (uint32_t)((step / S) & 1);
-        if (!mbar_wait_bounded(smem_u32(&full_bar[st]), ph, abort_flag)) {
+      int g = 0, it = 0;
+      for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++it) {
+        const Unit c = unit_coords(p, u, BN);
+        const int k_begin = c.split * p.k_per_split;
+        const int steps0 = (min(p.K0 - k_begin, p.k_per_split) + kBK - 1) / kBK;
+        const int steps = steps0 + (c.split == 0 ? steps1 : 0);
+        const int buf = it & 1;
+        // the epilogue must have drained this accumulator (two units ago)
+        if (!mbar_wait_bounded(smem_u32(&acc_empty[buf]), (uint32_t)(((it >> 1) & 1) ^ 1), abort_flag)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const bool ext = step >= steps0;
-        const int a_mn = ext ? p.a1_mn : p.a0_mn;
-        const int b_mn = ext ? p.b1_mn : p.b0_mn;
-        const uint32_t idesc = ext ? idesc1 : idesc0;
-        int nsub = 4;
-        if (ext) {
-          const int rem = p.K1 - (step - steps0) * kBK;
-          nsub = min(4, (rem + 15) / 16);
+        const uint32_t d_tmem = tmem_base + (uint32_t)(buf * BN);
+        for (int step = 0; step < steps; ++step, ++g) {
+          const int st = g % S;
+          const uint32_t ph = (uint32_t)((g / S) & 1);
+          if (!mbar_wait_bounded(smem_u32(&full_bar[st]), ph, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const bool ext = step >= steps0;
+          const int a_mn = ext ? p.a1_mn : p.a0_mn;
+          const int b_mn = ext ? p.b1_mn : p.b0_mn;
+          const uint32_t idesc = ext ? idesc1 : idesc0;
+          int nsub = 4;
+          if (ext) {
+            const int rem = p.K1 - (step - steps0) * kBK;
+            nsub = min(4, (rem + 15) / 16);
+          }
+          const uint32_t sa = sbase + st * Cfg::kStageBytes;
+          const uint32_t sb = sa + Cfg::kABytes;
+          for (int j = 0; j < nsub; ++j) {
+            // K-major: 16 elements = 32 bytes along the swizzled row;
+            // MN-major: 16 K-rows of 128 bytes.
+            const uint32_t ao = a_mn ? (uint32_t)j * 2048u : (uint32_t)j * 32u;
+            const uint32_t bo = b_mn ? (uint32_t)j * 2048u : (uint32_t)j * 32u;
+            const uint64_t adesc = a_mn ? smem_desc_sw128(sa + ao, 8192, 1024) : smem_desc_sw128(sa + ao, 16, 1024);
+            const uint64_t bdesc = b_mn ? smem_desc_sw128(sb + bo, 8192, 1024) : smem_desc_sw128(sb + bo, 16, 1024);
+            umma_bf16(d_tmem, adesc, bdesc, idesc, (step > 0 || j > 0) ? 1u : 0u);
+            issued_any = 1;
+          }
+          umma_commit(smem_u32(&empty_bar[st]));
         }
-        const uint32_t sa = sbase + st * Cfg::kStageBytes;
-        const uint32_t sb = sa + Cfg::kABytes;
-        for (int j = 0; j < nsub; ++j) {
-          // K-major: 16 elements = 32 bytes along the swizzled row;
-          // MN-major: 16 K-rows of 128 bytes.
-          const uint32_t ao = a_mn ? (uint32_t)j * 2048u : (uint32_t)j * 32u;
-          const uint32_t bo = b_mn ? (uint32_t)j * 2048u : (uint32_t)j * 32u;
-          const uint64_t adesc = a_mn ? smem_desc_sw128(sa + ao, 8192, 1024) : smem_desc_sw128(sa + ao, 16, 1024);
-          const uint64_t bdesc = b_mn ? smem_desc_sw128(sb + bo, 8192, 1024) : smem_desc_sw128(sb + bo, 16, 1024);
-          umma_bf16(tmem_base, adesc, bdesc, idesc, (step > 0 || j > 0) ? 1u : 0u);
-          issued_any = 1;
-        }
-        umma_commit(smem_u32(&empty_bar[st]));
+        if (ok) umma_commit(smem_u32(&acc_full[buf]));
       }
-      if (ok) {
-        umma_commit(smem_u32(accum_bar));
-      } else if (issued_any) {
+      if (!ok && issued_any) {
         // wait for MMAs already issued before TMEM is released
         umma_commit(smem_u32(drain_bar));
         mbar_wait_bounded(smem_u32(drain_bar), 0, nullptr);
@@ -238,116 +452,39 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // ------------------------------------------------------------ epilogue
     const int quarter = warp & 3;             // TMEM lane quarter of this warp
     const int row = quarter * 32 + lane;
-    const int m = m0 + row;
-    const bool row_ok = m < p.M;
-    const bool have = mbar_wait_bounded(smem_u32(accum_bar), 0, abort_flag);
-    tc_fence_after();
-    if (have) {
-      const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16);
+    int it = 0;
+    for (int u = blockIdx.x; u < units; u += gridDim.x, ++it) {
+      const Unit c = unit_coords(p, u, BN);
+      const int buf = it & 1;
+      if (!mbar_wait_bounded(smem_u32(&acc_full[buf]), (uint32_t)((it >> 1) & 1), abort_flag)) break;
+      tc_fence_after();
+      const int m = c.m0 + row;
+      const bool row_ok = m < p.M;
+      const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * BN);
+      if (p.epi == EPI_MERGE || p.epi == EPI_UNMERGE) {
+        epilogue_merge_row<BN>(p, taddr, m, row_ok, c.n0, s_lut);
+      } else
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        if (p.pair_offset > 0 && c * 32 >= p.pair_offset) break;   // lo columns: consumed below
+      for (int ch = 0; ch < BN / 32; ++ch) {
+        if (p.pair_offset > 0 && ch * 32 >= p.pair_offset) break;   // lo columns: consumed below
         uint32_t v[32];
-        tmem_ld_32x32b_x32(taddr + (uint32_t)(c * 32), v);
+        tmem_ld_32x32b_x32(taddr + (uint32_t)(ch * 32), v);
         tmem_ld_wait();
         if (p.pair_offset > 0) {
           uint32_t lo[32];
-          tmem_ld_32x32b_x32(taddr + (uint32_t)(c * 32 + p.pair_offset), lo);
+          tmem_ld_32x32b_x32(taddr + (uint32_t)(ch * 32 + p.pair_offset), lo);
           tmem_ld_wait();
 #pragma unroll
           for (int i = 0; i < 32; ++i)
             v[i] = __float_as_uint(__fadd_rn(__uint_as_float(v[i]), __uint_as_float(lo[i])));
         }
-        const int n = n0 + c * 32;
-        if (!row_ok || n >= p.N) continue;
-        if (p.epi == EPI_BF16) {
-          uint16_t* out = reinterpret_cast<uint16_t*>(p.out) + (int64_t)m * p.ldo + n;
-          if (n + 32 <= p.n_store && (p.ldo & 7) == 0) {
-            uint4* o4 = reinterpret_cast<uint4*>(out);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              uint4 w;
-              w.x = pack_bf16x2(__uint_as_float(v[8 * i + 0]), __uint_as_float(v[8 * i + 1]));
-              w.y = pack_bf16x2(__uint_as_float(v[8 * i + 2]), __uint_as_float(v[8 * i + 3]));
-              w.z = pack_bf16x2(__uint_as_float(v[8 * i + 4]), __uint_as_float(v[8 * i + 5]));
-              w.w = pack_bf16x2(__uint_as_float(v[8 * i + 6]), __uint_as_float(v[8 * i + 7]));
-              o4[i] = w;
-            }
-          } else {
-            for (int i = 0; i < 32 && n + i < p.n_store; ++i) {
-              __nv_bfloat16 h = __float2bfloat16_rn(__uint_as_float(v[i]));
-              out[i] = *reinterpret_cast<uint16_t*>(&h);
-            }
-          }
-        } else if (p.epi == EPI_F32) {
-          float* out = reinterpret_cast<float*>(p.out) + (int64_t)split * p.split_stride + (int64_t)m * p.ldo + n;
-          if (p.out != nullptr) {
-            if (n + 32 <= p.n_store && (p.ldo & 3) == 0) {
-              float4* o4 = reinterpret_cast<float4*>(out);
-#pragma unroll
-              for (int i = 0; i < 8; ++i)
-                o4[i] = make_float4(p.alpha * __uint_as_float(v[4 * i]), p.alpha * __uint_as_float(v[4 * i + 1]),
-                                    p.alpha * __uint_as_float(v[4 * i + 2]), p.alpha * __uint_as_float(v[4 * i + 3]));
-            } else {
-              for (int i = 0; i < 32 && n + i < p.n_store; ++i) out[i] = p.alpha * __uint_as_float(v[i]);
-            }
-          }
-          if (p.out2 != nullptr) {
-            uint16_t* o2 = p.out2 + (int64_t)m * p.ldo2 + n;
-            for (int i = 0; i < 32 && n + i < p.n_store2; ++i) {
-              const float x = __fmul_rn(p.alpha2, __uint_as_float(v[i]));
-              const __nv_bfloat16 h = __float2bfloat16_rn(x);
-              o2[i] = *reinterpret_cast<const uint16_t*>(&h);
-              if (p.lo_offset > 0) {
-                const __nv_bfloat16 l = __float2bfloat16_rn(__fsub_rn(x, __bfloat162float(h)));
-                o2[i + p.lo_offset] = *reinterpret_cast<const uint16_t*>(&l);
-              }
-            }
-          }
-        } else if (p.epi == EPI_F32_T) {
-          float* out = reinterpret_cast<float*>(p.out) + (int64_t)split * p.split_stride + m;
-          for (int i = 0; i < 32 && n + i < p.n_store; ++i)
-            out[(int64_t)(n + i) * p.ldo] = p.alpha * __uint_as_float(v[i]);
-        } else if (p.epi == EPI_MERGE) {
-          // w' for row m, columns n..n+31: one 16-byte word of codes, one block
-          const int64_t e0 = (int64_t)m * p.N + n;
-          const uint4 cw = *reinterpret_cast<const uint4*>(p.codes + e0 / 2);
-          const float a_scale = block_scale(p.absmax_q, p.scale2, p.mean[0], e0 / kBlock);
-          uint32_t wq[16];
-          dequant32(cw, a_scale, s_lut, wq);
-          uint16_t* out = reinterpret_cast<uint16_t*>(p.out) + (int64_t)m * p.ldo + n;
-          uint4* o4 = reinterpret_cast<uint4*>(out);
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            uint32_t r4[4];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const uint32_t wp = wq[4 * i + j];
-              const float lo = __fmaf_rn(p.alpha, __uint_as_float(v[8 * i + 2 * j]), bf16_bits_to_f32(wp & 0xFFFFu));
-              const float hi = __fmaf_rn(p.alpha, __uint_as_float(v[8 * i + 2 * j + 1]), bf16_bits_to_f32(wp >> 16));
-              r4[j] = pack_bf16x2(lo, hi);
-            }
-            o4[i] = make_uint4(r4[0], r4[1], r4[2], r4[3]);
-          }
-        } else if (p.epi == EPI_UNMERGE) {
-          const uint4* w4 = reinterpret_cast<const uint4*>(p.w_in + (int64_t)m * p.ldw + n);
-          uint16_t* out = reinterpret_cast<uint16_t*>(p.out) + (int64_t)m * p.ldo + n;
-          uint4* o4 = reinterpret_cast<uint4*>(out);
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const uint4 wv = w4[i];
-            const uint32_t wr[4] = {wv.x, wv.y, wv.z, wv.w};
-            uint32_t r4[4];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const float lo = __fmaf_rn(p.alpha, __uint_as_float(v[8 * i + 2 * j]), bf16_bits_to_f32(wr[j] & 0xFFFFu));
-              const float hi = __fmaf_rn(p.alpha, __uint_as_float(v[8 * i + 2 * j + 1]), bf16_bits_to_f32(wr[j] >> 16));
-              r4[j] = pack_bf16x2(lo, hi);
-            }
-            o4[i] = make_uint4(r4[0], r4[1], r4[2], r4[3]);
-          }
-        }
+        const int n = c.n0 + ch * 32;
+        if (row_ok && n < p.N) epilogue_chunk(p, v, m, n, c.split, s_lut);
       }
+      // this accumulator may be overwritten once all four warps are done
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&acc_empty[buf]));
     }
   }
   tc_fence_before();

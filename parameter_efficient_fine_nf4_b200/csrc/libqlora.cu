@@ -57,6 +57,7 @@ struct HostTables {
   float levels[16];
   float thresholds[15];
   EncTable enc;
+  bool enc_ok;
 };
 
 HostTables build_tables() {
@@ -77,18 +78,24 @@ HostTables build_tables() {
     if ((double)f <= mid) f = nextafterf(f, 2.0f);
     t.thresholds[i] = f;
   }
+  t.enc_ok = true;
   for (int j = 0; j < kEncBins; ++j) {
-    const double lo = (double)(j - 64) / 64.0;
-    const double hi = (double)(j - 63) / 64.0;
-    int base = 0;
-    float inside = INFINITY;
+    const double lo = ((double)j - 64.5) / 64.0;
+    const double hi = ((double)j - 63.5) / 64.0;
+    int base = 0, inside = 0;
+    float thr = INFINITY;
     for (int i = 0; i < 15; ++i) {
       const double th = (double)t.thresholds[i];
-      if (th <= lo) ++base;
-      else if (th < hi) inside = t.thresholds[i];
+      if (th <= lo) {
+        ++base;
+      } else if (th <= hi) {
+        thr = t.thresholds[i];
+        ++inside;
+      }
     }
-    t.enc.base[j] = base;
-    t.enc.thr[j] = inside;
+    if (inside > 1) t.enc_ok = false;
+    t.enc.e[j].base = base;
+    t.enc.e[j].thr = thr;
   }
   return t;
 }
@@ -118,6 +125,15 @@ EncodeTiledFn encode_fn() {
 
 std::mutex g_init_mu;
 bool g_dev_ready[kMaxDevices] = {false};
+int g_dev_sms[kMaxDevices] = {0};
+
+// SM count of the current device (persistent grids are sized to it).
+int current_sms() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices || g_dev_sms[dev] <= 0)
+    return kSMs;
+  return g_dev_sms[dev];
+}
 
 template <int BN>
 cudaError_t set_gemm_attrs() {
@@ -135,7 +151,9 @@ int ensure_device() {
   cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
   cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
   if (major != 10 || minor != 0) return QLORA_ERR_NO_DEVICE;
+  cudaDeviceGetAttribute(&g_dev_sms[dev], cudaDevAttrMultiProcessorCount, dev);
   if (encode_fn() == nullptr) return QLORA_ERR_CUDA;
+  if (!tables().enc_ok) return QLORA_ERR_CUDA;
   if (set_gemm_attrs<64>() != cudaSuccess || set_gemm_attrs<128>() != cudaSuccess ||
       set_gemm_attrs<256>() != cudaSuccess)
     return QLORA_ERR_CUDA;
@@ -262,7 +280,9 @@ int launch_gemm_bn(const char* name, const GemmPlan& g, GemmArgs args, cudaStrea
   const int splits = (int)cdiv(g.K0, args.k_per_split);
   const auto& T = tables();
   memcpy(args.levels, T.levels, sizeof(args.levels));
-  dim3 grid((unsigned)(args.tiles_m * args.tiles_n), (unsigned)splits, 1);
+  // persistent: one CTA per SM (or per unit when there are fewer units)
+  const int64_t units = (int64_t)args.tiles_m * args.tiles_n * splits;
+  dim3 grid((unsigned)std::min<int64_t>(units, current_sms()), 1, 1);
   const double flops = 2.0 * g.M * (double)g.N * (g.K0 + g.K1);
   return launch(name, flops, 0.0, st, [&] {
     gemm_tc_kernel<BN><<<grid, kGemmThreads, GemmCfg<BN>::kSmemBytes, st>>>(m[0], m[1], m[2], m[3], args);
@@ -328,15 +348,15 @@ int check_rank(int r, float alpha) {
   } while (0)
 
 int dequantize_into(const qlora_nf4_t* q, uint16_t* W, cudaStream_t st) {
-  const int64_t n_chunks = q->d * q->k / 32;
+  const int64_t n_units = q->d * q->k / 8;
   const auto& T = tables();
   NF4Levels lv;
   memcpy(lv.q, T.levels, sizeof(lv.q));
-  const int grid = grid_for(n_chunks, 256);
+  const int grid = std::max(1, std::min<int>((int)cdiv(n_units, 256 * 4), current_sms() * 8));
   const double bytes = (double)q->d * q->k * 2.5;
   return launch("nf4_dequantize", 0.0, bytes, st, [&] {
-    nf4_dequantize_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const uint4*>(q->codes), q->absmax_q,
-                                                q->scale2, q->mean, n_chunks,
+    nf4_dequantize_kernel<<<grid, 256, 0, st>>>(reinterpret_cast<const uint32_t*>(q->codes), q->absmax_q,
+                                                q->scale2, q->mean, n_units,
                                                 reinterpret_cast<uint4*>(W), lv);
   });
 }

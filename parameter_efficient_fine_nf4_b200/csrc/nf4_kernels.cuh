@@ -17,18 +17,22 @@ namespace qlora {
 
 constexpr int kBlock = 64;
 constexpr int kBlock2 = 256;
-constexpr int kEncBins = 129;     // x*64 floored, x in [-1, 1]
+constexpr int kEncBins = 129;     // rint(64 x) + 64, x in [-1, 1]
 
-// Encoder table: for bin j (x in [(j-64)/64, (j-63)/64)) the number of
-// thresholds <= the bin's lower edge, and the single threshold (if any)
-// strictly inside the bin (+inf otherwise).  Built on the host from the
-// library's own level table; at most one threshold falls in a bin because the
-// smallest level gap (~0.08) exceeds the bin width 1/64.
-struct EncTable {
-  float thr[kEncBins];
-  int base[kEncBins];
+// Encoder table.  Bin j holds every x with rint(64 x) = j - 64, i.e. the
+// closed interval [(j - 64.5)/64, (j - 63.5)/64] (closed because a tie may
+// round either way).  Entry: the number of thresholds at or below the lower
+// edge, and the single threshold inside the bin (+inf if none), so that
+// code(x) = base + (x >= thr).  At most one threshold falls in a bin because
+// the smallest gap between thresholds (~0.08) exceeds the bin width 1/64; the
+// host builder checks it.
+struct __align__(8) EncEntry {
+  float thr;
+  int base;
 };
-
+struct EncTable {
+  EncEntry e[kEncBins];
+};
 struct NF4Levels {
   float q[16];
 };
@@ -45,10 +49,13 @@ __device__ __forceinline__ float div_markstein(float w, float a, float y) {
   return __fmaf_rn(r, y, q0);
 }
 
-__device__ __forceinline__ uint32_t enc_code(float x, const float* s_thr, const int* s_base) {
-  int j = __float2int_rd(x * 64.0f) + 64;          // x*64 is exact
-  j = min(max(j, 0), kEncBins - 1);
-  return (uint32_t)(s_base[j] + (x >= s_thr[j] ? 1 : 0));
+// rint(64 x) for |x| <= 1 without a float-to-int conversion: adding 1.5 * 2^23
+// leaves the rounded integer in the low mantissa bits (round to nearest even).
+__device__ __forceinline__ uint32_t enc_code(float x, const EncEntry* s_tab) {
+  const float t = __fadd_rn(__fmul_rn(x, 64.0f), 12582912.0f);
+  const uint32_t j = min((uint32_t)(__float_as_int(t) - 0x4B400000 + 64), (uint32_t)(kEncBins - 1));
+  const EncEntry e = s_tab[j];
+  return (uint32_t)(e.base + (x >= e.thr ? 1 : 0));
 }
 
 // ---------------------------------------------------------------------------
@@ -59,14 +66,10 @@ __device__ __forceinline__ uint32_t enc_code(float x, const float* s_thr, const 
 __global__ void __launch_bounds__(256) nf4_quantize_phase1(
     const float* __restrict__ W0, int64_t n_b, uint32_t* __restrict__ codes_u32,
     float* __restrict__ absmax, double* __restrict__ group_sum, const __grid_constant__ EncTable tab) {
-  __shared__ float s_thr[kEncBins];
-  __shared__ int s_base[kEncBins];
+  __shared__ EncEntry s_tab[kEncBins];
   __shared__ float s_abs[kBlock2];
   const int tid = threadIdx.x;
-  for (int i = tid; i < kEncBins; i += blockDim.x) {
-    s_thr[i] = tab.thr[i];
-    s_base[i] = tab.base[i];
-  }
+  for (int i = tid; i < kEncBins; i += blockDim.x) s_tab[i] = tab.e[i];
   __syncthreads();
 
   const int64_t g = blockIdx.x;
@@ -107,7 +110,7 @@ __global__ void __launch_bounds__(256) nf4_quantize_phase1(
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           const float x = div_markstein(w[i], m, y);
-          packed |= enc_code(x, s_thr, s_base) << (4 * i);
+          packed |= enc_code(x, s_tab) << (4 * i);
         }
       }
       if (b < n_b) {
@@ -228,27 +231,51 @@ __device__ __forceinline__ void dequant32(const uint4 c, float a, const float* s
   }
 }
 
+// 8 codes (one 32-bit word) -> 8 bf16 values of level[code] * a (one 16-byte word).
+__device__ __forceinline__ uint4 dequant8(uint32_t w, float a, const float* s_q) {
+  uint32_t o[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint32_t lo = (w >> (8 * j)) & 0xFu;
+    const uint32_t hi = (w >> (8 * j + 4)) & 0xFu;
+    const __nv_bfloat162 p = __floats2bfloat162_rn(__fmul_rn(s_q[lo], a), __fmul_rn(s_q[hi], a));
+    o[j] = *reinterpret_cast<const uint32_t*>(&p);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
 // ---------------------------------------------------------------------------
-// Dequantise to a bf16 d x k matrix.  One thread per 32 consecutive weights
-// (a 16-byte load of codes, a 64-byte store of bf16).
+// Dequantise to a bf16 d x k matrix.  Unit = 8 consecutive weights: a 4-byte
+// code load and a 16-byte store, consecutive threads on consecutive units so
+// both streams are fully coalesced; 4 independent units per thread in flight.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) nf4_dequantize_kernel(
-    const uint4* __restrict__ codes, const uint8_t* __restrict__ absmax_q,
-    const float* __restrict__ scale2, const float* __restrict__ mean, int64_t n_chunks,
+    const uint32_t* __restrict__ codes, const uint8_t* __restrict__ absmax_q,
+    const float* __restrict__ scale2, const float* __restrict__ mean, int64_t n_units,
     uint4* __restrict__ W_out, const __grid_constant__ NF4Levels lv) {
   __shared__ float s_q[16];
   if (threadIdx.x < 16) s_q[threadIdx.x] = lv.q[threadIdx.x];
   __syncthreads();
   const float mu = mean[0];
   const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-  for (int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; t < n_chunks; t += stride) {
-    const uint4 c = __ldcs(codes + t);
-    const float a = block_scale(absmax_q, scale2, mu, t >> 1);
-    uint32_t o[16];
-    dequant32(c, a, s_q, o);
-    uint4* dst = W_out + t * 4;
+  for (int64_t base = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; base < n_units; base += 4 * stride) {
+    uint32_t c[4];
+    float a[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) dst[i] = make_uint4(o[4 * i], o[4 * i + 1], o[4 * i + 2], o[4 * i + 3]);
+    for (int j = 0; j < 4; ++j) {
+      const int64_t u = base + j * stride;
+      c[j] = 0u;
+      a[j] = 0.f;
+      if (u < n_units) {
+        c[j] = __ldcs(codes + u);
+        a[j] = block_scale(absmax_q, scale2, mu, u >> 3);
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int64_t u = base + j * stride;
+      if (u < n_units) __stcs(W_out + u, dequant8(c[j], a[j], s_q));
+    }
   }
 }
 
