@@ -279,6 +279,44 @@ __device__ __forceinline__ void epilogue_merge_row(const GemmArgs& p, uint32_t t
   }
 }
 
+// Shared-memory descriptors of stage 0 for both segments; a stage or a K
+// sub-step only adds a byte offset / 16 to the start-address field (the
+// field never carries: shared addresses stay below 2^18).  K-major: 16
+// elements = 32 bytes along the swizzled row; MN-major: 16 K-rows of 128 B.
+struct StageDescs {
+  uint64_t a[2], b[2];
+  uint32_t astep[2], bstep[2];
+  uint32_t idesc[2];
+};
+__device__ __forceinline__ StageDescs make_stage_descs(const GemmArgs& p, uint32_t sa0, uint32_t sb0, int M, int N) {
+  StageDescs d;
+  const int amn[2] = {p.a0_mn, p.a1_mn};
+  const int bmn[2] = {p.b0_mn, p.b1_mn};
+#pragma unroll
+  for (int s = 0; s < 2; ++s) {
+    d.a[s] = amn[s] ? smem_desc_sw128(sa0, 8192, 1024) : smem_desc_sw128(sa0, 16, 1024);
+    d.b[s] = bmn[s] ? smem_desc_sw128(sb0, 8192, 1024) : smem_desc_sw128(sb0, 16, 1024);
+    d.astep[s] = amn[s] ? 128u : 2u;
+    d.bstep[s] = bmn[s] ? 128u : 2u;
+    d.idesc[s] = idesc_bf16_f32(M, N, amn[s], bmn[s]);
+  }
+  return d;
+}
+
+__device__ __forceinline__ void issue_kstep(uint32_t d_tmem, const StageDescs& d, int seg, uint32_t stage_off16,
+                                            int nsub, bool first) {
+  const uint64_t a = d.a[seg] + stage_off16;
+  const uint64_t b = d.b[seg] + stage_off16;
+  const uint32_t as = d.astep[seg], bs = d.bstep[seg], id = d.idesc[seg];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    if (j < nsub) {
+      const uint32_t acc = (first && j == 0) ? 0u : 1u;
+      umma_bf16(d_tmem, a + (uint64_t)(j * as), b + (uint64_t)(j * bs), id, acc);
+    }
+  }
+}
+
 // Persistent kernel: CTA b processes work units b, b + gridDim.x, ...  The
 // shared-memory ring runs continuously across units; two TMEM accumulators
 // (columns [0, BN) and [BN, 2 BN)) let the epilogue of one unit overlap the
@@ -394,8 +432,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t idesc0 = idesc_bf16_f32(kBM, BN, p.a0_mn, p.b0_mn);
-      const uint32_t idesc1 = idesc_bf16_f32(kBM, BN, p.a1_mn, p.b1_mn);
+      const StageDescs dsc = make_stage_descs(p, sbase, sbase + Cfg::kABytes, kBM, BN);
       bool ok = true;
       int issued_any = 0;
       int g = 0, it = 0;
@@ -418,26 +455,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           if (!mbar_wait_bounded(smem_u32(&full_bar[st]), ph, abort_flag)) { ok = false; break; }
           tc_fence_after();
           const bool ext = step >= steps0;
-          const int a_mn = ext ? p.a1_mn : p.a0_mn;
-          const int b_mn = ext ? p.b1_mn : p.b0_mn;
-          const uint32_t idesc = ext ? idesc1 : idesc0;
           int nsub = 4;
-          if (ext) {
-            const int rem = p.K1 - (step - steps0) * kBK;
-            nsub = min(4, (rem + 15) / 16);
-          }
-          const uint32_t sa = sbase + st * Cfg::kStageBytes;
-          const uint32_t sb = sa + Cfg::kABytes;
-          for (int j = 0; j < nsub; ++j) {
-            // K-major: 16 elements = 32 bytes along the swizzled row;
-            // MN-major: 16 K-rows of 128 bytes.
-            const uint32_t ao = a_mn ? (uint32_t)j * 2048u : (uint32_t)j * 32u;
-            const uint32_t bo = b_mn ? (uint32_t)j * 2048u : (uint32_t)j * 32u;
-            const uint64_t adesc = a_mn ? smem_desc_sw128(sa + ao, 8192, 1024) : smem_desc_sw128(sa + ao, 16, 1024);
-            const uint64_t bdesc = b_mn ? smem_desc_sw128(sb + bo, 8192, 1024) : smem_desc_sw128(sb + bo, 16, 1024);
-            umma_bf16(d_tmem, adesc, bdesc, idesc, (step > 0 || j > 0) ? 1u : 0u);
-            issued_any = 1;
-          }
+          if (ext) nsub = min(4, (p.K1 - (step - steps0) * kBK + 15) / 16);
+          issue_kstep(d_tmem, dsc, ext ? 1 : 0, (uint32_t)(st * Cfg::kStageBytes) >> 4, nsub, step == 0);
+          issued_any = 1;
           umma_commit(smem_u32(&empty_bar[st]));
         }
         if (ok) umma_commit(smem_u32(&acc_full[buf]));
