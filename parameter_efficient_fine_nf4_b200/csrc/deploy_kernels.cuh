@@ -1,0 +1,281 @@
+// Deploy-time merge and unmerge ([P1] deploy paragraph; [P2] "The LoRA
+// hypothesis": W = W0 + (alpha/r) B A; a task is removed by subtracting its
+// scaled product again):
+//   merge   W    = bf16(fp32(w' + s (B A)_fp32)),  w' = doubleDequant(codes)
+//   unmerge W0'' = bf16(fp32(W  - s (B A)_fp32))
+//
+// Both are HBM-bound (2.5 and 4 bytes per weight) with a small rank-r
+// product per tile, so the kernel is built around moving bytes in bulk:
+//   * a persistent CTA walks 128 x 256 tiles of W;
+//   * warp 0 brings, by TMA, the tile's rank-r operands (B rows, A columns)
+//     and the tile's input (the 16 KB of NF4 codes, or the 64 KB of W) in
+//     128-byte-swizzled form, double-buffered;
+//   * warp 1 computes (B A) for the tile with tcgen05 into one of two TMEM
+//     accumulators;
+//   * warps 2-5 combine accumulator and input row by row, write the bf16
+//     result into a swizzled shared tile (in place over W for unmerge), and
+//     one thread stores it with TMA.
+// Rows or columns beyond d or k are zero-filled by the loads and clipped by
+// the stores, so no element masks are needed.
+#pragma once
+#include "gemm_tc.cuh"
+#include "nf4_kernels.cuh"
+#include "ptx.cuh"
+
+namespace qlora {
+
+struct DeployArgs {
+  int d, k, r;
+  int tiles_m, tiles_n;
+  float alpha;                 // +s for merge, -s for unmerge
+  const uint8_t* absmax_q;
+  const float* scale2;
+  const float* mean;
+  float levels[16];
+};
+
+template <bool kMerge, int KS>
+struct DeployCfg {
+  static constexpr int kOpA = KS * 16384;               // B rows: 128 x 64 bf16 per K-step
+  static constexpr int kOpB = KS * 32768;               // A columns: 4 atoms of 64 x 64 bf16 per K-step
+  static constexpr int kIo = kMerge ? 16384 : 65536;    // codes tile (128 x 128 B) or W tile
+  static constexpr int kOut = kMerge ? 65536 : 0;       // merge output tile (unmerge: in place)
+  static constexpr int kBytes = kOpA + kOpB + 2 * kIo + kOut;
+  static constexpr int kSmemBytes = kBytes + 1024 + 512;
+};
+
+// Byte offset of 16-byte chunk `chunk` (0..7) of row `row` in a 128-byte-row,
+// 128B-swizzled tile.
+__device__ __forceinline__ uint32_t sw128(int row, int chunk) {
+  return (uint32_t)(row * 128 + ((chunk ^ (row & 7)) << 4));
+}
+
+template <bool kMerge, int KS>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    lora_deploy_kernel(const __grid_constant__ CUtensorMap tmOpA, const __grid_constant__ CUtensorMap tmOpB,
+                       const __grid_constant__ CUtensorMap tmIo, const __grid_constant__ CUtensorMap tmOut,
+                       const __grid_constant__ DeployArgs p) {
+  using Cfg = DeployCfg<kMerge, KS>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  const uint32_t pad = (1024u - (raw_addr & 1023u)) & 1023u;
+  uint8_t* smem = smem_raw + pad;
+  const uint32_t sbase = raw_addr + pad;
+  const uint32_t sA = sbase;
+  const uint32_t sB = sA + Cfg::kOpA;
+  const uint32_t sIo = sB + Cfg::kOpB;
+  const uint32_t sOut = sIo + 2 * Cfg::kIo;
+  uint8_t* gIo = smem + Cfg::kOpA + Cfg::kOpB;
+  uint8_t* gOut = gIo + 2 * Cfg::kIo;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::kBytes);
+  uint64_t* op_full = bars + 0;
+  uint64_t* op_empty = bars + 1;
+  uint64_t* io_full = bars + 2;      // [2]
+  uint64_t* io_empty = bars + 4;     // [2]
+  uint64_t* acc_full = bars + 6;     // [2]
+  uint64_t* acc_empty = bars + 8;    // [2]
+  uint64_t* drain_bar = bars + 10;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 11);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* s_lut = reinterpret_cast<float*>(tmem_slot + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int units = p.tiles_m * p.tiles_n;
+
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(op_full), 1);
+    mbar_init(smem_u32(op_empty), 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&io_full[i]), 1);
+      mbar_init(smem_u32(&io_empty[i]), 1);
+      mbar_init(smem_u32(&acc_full[i]), 1);
+      mbar_init(smem_u32(&acc_empty[i]), 4);
+    }
+    mbar_init(smem_u32(drain_bar), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (threadIdx.x < 16) s_lut[threadIdx.x] = p.levels[threadIdx.x];
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmOpA);
+    tma_prefetch_desc(&tmOpB);
+    tma_prefetch_desc(&tmIo);
+    tma_prefetch_desc(&tmOut);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int it = 0;
+      int io_issued[2] = {0, 0};
+      int op_issued = 0;
+      for (int u = blockIdx.x; u < units; u += gridDim.x, ++it) {
+        const int m0 = (u / p.tiles_n) * 128;
+        const int n0 = (u % p.tiles_n) * 256;
+        const int s = it & 1;
+        // rank-r operands (single buffer, freed by the MMA commit)
+        if (!mbar_wait_bounded(smem_u32(op_empty), (uint32_t)((it & 1) ^ 1), abort_flag)) break;
+        const uint32_t fo = smem_u32(op_full);
+        mbar_arrive_expect_tx(fo, (uint32_t)(Cfg::kOpA + Cfg::kOpB));
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+          tma_load_2d(sA + ks * 16384, &tmOpA, fo, ks * 64, m0);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) tma_load_2d(sB + ks * 32768 + i * 8192, &tmOpB, fo, n0 + 64 * i, ks * 64);
+        }
+        op_issued = 1;
+        // input tile (double buffer, freed by the epilogue)
+        if (!mbar_wait_bounded(smem_u32(&io_empty[s]), (uint32_t)(((it >> 1) & 1) ^ 1), abort_flag)) break;
+        const uint32_t fi = smem_u32(&io_full[s]);
+        mbar_arrive_expect_tx(fi, (uint32_t)Cfg::kIo);
+        if (kMerge) {
+          tma_load_2d(sIo + s * Cfg::kIo, &tmIo, fi, n0 / 2, m0);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) tma_load_2d(sIo + s * Cfg::kIo + i * 16384, &tmIo, fi, n0 + 64 * i, m0);
+        }
+        io_issued[s] = it + 1;
+      }
+      if (*abort_flag) {
+        if (op_issued) mbar_wait_bounded(smem_u32(op_full), (uint32_t)((it - 1) & 1), nullptr);
+        for (int s = 0; s < 2; ++s)
+          if (io_issued[s] > 0)
+            mbar_wait_bounded(smem_u32(&io_full[s]), (uint32_t)(((io_issued[s] - 1) >> 1) & 1), nullptr);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(128, 256, 0, 1);
+      const uint64_t da = smem_desc_sw128(sA, 16, 1024);
+      const uint64_t db = smem_desc_sw128(sB, 8192, 1024);
+      bool ok = true;
+      int issued_any = 0;
+      int it = 0;
+      for (int u = blockIdx.x; u < units; u += gridDim.x, ++it) {
+        const int s = it & 1;
+        if (!mbar_wait_bounded(smem_u32(&acc_empty[s]), (uint32_t)(((it >> 1) & 1) ^ 1), abort_flag)) { ok = false; break; }
+        if (!mbar_wait_bounded(smem_u32(op_full), (uint32_t)(it & 1), abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(s * 256);
+#pragma unroll
+        for (int ks = 0; ks < KS; ++ks) {
+          const int nsub = min(4, (p.r - ks * 64 + 15) / 16);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            if (j < nsub) {
+              umma_bf16(d_tmem, da + (uint64_t)((ks * 16384 + j * 32) >> 4), db + (uint64_t)((ks * 32768 + j * 2048) >> 4),
+                        idesc, (ks > 0 || j > 0) ? 1u : 0u);
+              issued_any = 1;
+            }
+          }
+        }
+        umma_commit(smem_u32(op_empty));
+        umma_commit(smem_u32(&acc_full[s]));
+      }
+      if (!ok && issued_any) {
+        umma_commit(smem_u32(drain_bar));
+        mbar_wait_bounded(smem_u32(drain_bar), 0, nullptr);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const bool elected = threadIdx.x == 64;       // warp 2, lane 0 issues the stores
+    const float mu = kMerge ? p.mean[0] : 0.f;
+    const int kb = p.k / kBlock;                  // blocks per row of W
+    int it = 0;
+    for (int u = blockIdx.x; u < units; u += gridDim.x, ++it) {
+      const int m0 = (u / p.tiles_n) * 128;
+      const int n0 = (u % p.tiles_n) * 256;
+      const int s = it & 1;
+      const int m = m0 + row;
+      // block scales of this row's four 64-blocks: global loads issued before
+      // waiting for the tile so their latency overlaps the wait
+      float asc[4] = {0.f, 0.f, 0.f, 0.f};
+      if (kMerge && m < p.d) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if (n0 + 64 * j < p.k) asc[j] = block_scale(p.absmax_q, p.scale2, mu, (int64_t)m * kb + n0 / 64 + j);
+      }
+      bool ok = mbar_wait_bounded(smem_u32(&io_full[s]), (uint32_t)((it >> 1) & 1), abort_flag);
+      ok = ok && mbar_wait_bounded(smem_u32(&acc_full[s]), (uint32_t)((it >> 1) & 1), abort_flag);
+      // every epilogue thread leaves together (the tile below uses named barriers)
+      if (named_bar_any(3, 128, !ok)) break;
+      tc_fence_after();
+      // the previous tile's store must have read its shared tile before this
+      // tile's results are written (merge: the one output tile; unmerge: the
+      // other input buffer, which the producer then refills)
+      if (it > 0) {
+        if (elected) {
+          bulk_wait_group_read0();
+          if (!kMerge) mbar_arrive(smem_u32(&io_empty[s ^ 1]));
+        }
+        named_bar_sync(2, 128);
+      }
+      const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(s * 256);
+      uint8_t* io = gIo + s * Cfg::kIo;
+      uint8_t* outt = kMerge ? gOut : io;
+#pragma unroll 1
+      for (int c = 0; c < 8; ++c) {
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(taddr + (uint32_t)(c * 32), v);
+        tmem_ld_wait();
+        uint32_t w[16];                       // 32 bf16 inputs w' (merge) or W (unmerge)
+        if (kMerge) {
+          const uint4 cw = *reinterpret_cast<const uint4*>(io + sw128(row, c));
+          dequant32(cw, asc[c >> 1], s_lut, w);
+        } else {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const uint4 x = *reinterpret_cast<const uint4*>(io + (c >> 1) * 16384 + sw128(row, (c & 1) * 4 + q));
+            w[4 * q + 0] = x.x; w[4 * q + 1] = x.y; w[4 * q + 2] = x.z; w[4 * q + 3] = x.w;
+          }
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint32_t r4[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const uint32_t wp = w[4 * q + j];
+            const float lo = __fmaf_rn(p.alpha, __uint_as_float(v[8 * q + 2 * j]), bf16_bits_to_f32(wp & 0xFFFFu));
+            const float hi = __fmaf_rn(p.alpha, __uint_as_float(v[8 * q + 2 * j + 1]), bf16_bits_to_f32(wp >> 16));
+            r4[j] = pack_bf16x2(lo, hi);
+          }
+          *reinterpret_cast<uint4*>(outt + (c >> 1) * 16384 + sw128(row, (c & 1) * 4 + q)) =
+              make_uint4(r4[0], r4[1], r4[2], r4[3]);
+        }
+      }
+      // accumulator drained
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&acc_empty[s]));
+      // all rows written: one thread stores the tile
+      fence_proxy_async_smem();
+      named_bar_sync(1, 128);
+      if (elected) {
+        const uint32_t src = kMerge ? sOut : sIo + s * Cfg::kIo;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) tma_store_2d(&tmOut, src + i * 16384, n0 + 64 * i, m0);
+        bulk_commit_group();
+        if (kMerge) mbar_arrive(smem_u32(&io_empty[s]));      // codes tile fully read
+      }
+    }
+    if (elected) bulk_wait_group0();
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) tmem_dealloc(tmem_base, 512);
+}
+
+}  // namespace qlora

@@ -16,6 +16,7 @@
 #include <cuda_runtime.h>
 
 #include "../../include/qlora.h"
+#include "deploy_kernels.cuh"
 #include "gemm_tc.cuh"
 #include "nf4_kernels.cuh"
 #include "ptx.cuh"
@@ -141,6 +142,12 @@ cudaError_t set_gemm_attrs() {
                               GemmCfg<BN>::kSmemBytes);
 }
 
+template <bool kMerge, int KS>
+cudaError_t set_deploy_attrs() {
+  return cudaFuncSetAttribute(lora_deploy_kernel<kMerge, KS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              DeployCfg<kMerge, KS>::kSmemBytes);
+}
+
 int ensure_device() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return QLORA_ERR_NO_DEVICE;
@@ -155,7 +162,9 @@ int ensure_device() {
   if (encode_fn() == nullptr) return QLORA_ERR_CUDA;
   if (!tables().enc_ok) return QLORA_ERR_CUDA;
   if (set_gemm_attrs<64>() != cudaSuccess || set_gemm_attrs<128>() != cudaSuccess ||
-      set_gemm_attrs<256>() != cudaSuccess)
+      set_gemm_attrs<256>() != cudaSuccess || set_deploy_attrs<true, 1>() != cudaSuccess ||
+      set_deploy_attrs<true, 2>() != cudaSuccess || set_deploy_attrs<false, 1>() != cudaSuccess ||
+      set_deploy_attrs<false, 2>() != cudaSuccess)
     return QLORA_ERR_CUDA;
   g_dev_ready[dev] = true;
   return QLORA_OK;
@@ -234,6 +243,58 @@ bool make_map(CUtensorMap* map, const void* base, int64_t inner, int64_t outer, 
                            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+// uint8 2-D tensor map (for the NF4 codes): `inner` bytes per row, `outer`
+// rows, `ld` bytes between rows, 128-byte swizzle.
+bool make_map_u8(CUtensorMap* map, const void* base, int64_t inner, int64_t outer, int64_t ld,
+                 int box_inner, int box_outer) {
+  cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)outer};
+  cuuint64_t strides[1] = {(cuuint64_t)ld};
+  cuuint32_t box[2] = {(cuuint32_t)box_inner, (cuuint32_t)box_outer};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = encode_fn()(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides,
+                           box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// Merge / unmerge through the bulk-copy deploy kernel (r <= 128).
+template <bool kMerge, int KS>
+int launch_deploy_t(const qlora_nf4_t* q, const uint16_t* W, const uint16_t* A, const uint16_t* Bp,
+                    int r, int r8, int64_t d, int64_t k, float s, uint16_t* out, cudaStream_t st) {
+  CUtensorMap mA, mB, mIo, mOut;
+  if (!make_map(&mA, Bp, r8, d, r8, 128)) return QLORA_ERR_CUDA;     // B rows, K-major
+  if (!make_map(&mB, A, k, r, k, 64)) return QLORA_ERR_CUDA;         // A columns, MN-major
+  if (!make_map(&mOut, out, k, d, k, 128)) return QLORA_ERR_CUDA;
+  if (kMerge) {
+    if (!make_map_u8(&mIo, q->codes, k / 2, d, k / 2, 128, 128)) return QLORA_ERR_CUDA;
+  } else {
+    if (!make_map(&mIo, W, k, d, k, 128)) return QLORA_ERR_CUDA;
+  }
+  DeployArgs a;
+  memset(&a, 0, sizeof(a));
+  a.d = (int)d; a.k = (int)k; a.r = r;
+  a.tiles_m = (int)cdiv(d, 128);
+  a.tiles_n = (int)cdiv(k, 256);
+  a.alpha = kMerge ? s : -s;
+  if (kMerge) { a.absmax_q = q->absmax_q; a.scale2 = q->scale2; a.mean = q->mean; }
+  memcpy(a.levels, tables().levels, sizeof(a.levels));
+  const int64_t units = (int64_t)a.tiles_m * a.tiles_n;
+  const dim3 grid((unsigned)std::min<int64_t>(units, current_sms()));
+  const double bytes = (double)d * k * (kMerge ? 2.5 : 4.0);
+  return launch(kMerge ? "lora_merge" : "lora_unmerge", 2.0 * d * (double)k * r, bytes, st, [&] {
+    lora_deploy_kernel<kMerge, KS><<<grid, kGemmThreads, DeployCfg<kMerge, KS>::kSmemBytes, st>>>(mA, mB, mIo, mOut, a);
+  });
+}
+
+int launch_deploy(bool merge, const qlora_nf4_t* q, const uint16_t* W, const uint16_t* A,
+                  const uint16_t* Bp, int r, int r8, int64_t d, int64_t k, float s, uint16_t* out,
+                  cudaStream_t st) {
+  if (merge) return r <= 64 ? launch_deploy_t<true, 1>(q, W, A, Bp, r, r8, d, k, s, out, st)
+                            : launch_deploy_t<true, 2>(q, W, A, Bp, r, r8, d, k, s, out, st);
+  return r <= 64 ? launch_deploy_t<false, 1>(q, W, A, Bp, r, r8, d, k, s, out, st)
+                 : launch_deploy_t<false, 2>(q, W, A, Bp, r, r8, d, k, s, out, st);
 }
 
 // One GEMM operand as stored in global memory.
@@ -736,6 +797,7 @@ static int merge_common(const qlora_nf4_t* q, const uint16_t* W, const uint16_t*
   int pst = QLORA_OK;
   const uint16_t* Bp = padded_B(B, d, r, r8, reinterpret_cast<uint16_t*>(ws), st, &pst);
   QLORA_TRY(pst);
+  if (r <= 128) return launch_deploy(merge, q, W, A, Bp, r, r8, d, k, s, out, st);
   GemmPlan g;
   g.M = (int)d; g.N = (int)k; g.K0 = r; g.bn = 256;
   g.a0 = kmajor(Bp, r8, d, r8);

@@ -200,6 +200,33 @@ def test_merge_unmerge(ci):
     assert q4.qlora_get_device_status() == 0
 
 
+@pytest.mark.parametrize("d,k,r", [
+    (300, 320, 5),       # ragged tiles in both directions, r not a multiple of 8
+    (128, 256, 64),      # exactly one tile
+    (200, 576, 100),     # two K-steps of the rank-r product
+    (136, 192, 200),     # r > 128
+    (1, 64, 1),          # one row
+])
+def test_merge_unmerge_ragged(d, k, r):
+    lay = synthetic.custom_layer(seed=d * 7 + k + r, d=d, k=k, r=r, T=1, alpha=2.0 * r)
+    alpha = 2.0 * r
+    s = alpha / r
+    qw = q4.qlora_nf4_quantize(f32_dev(lay.W0))
+    A, B = bf16_dev(lay.A), bf16_dev(lay.B)
+    W = q4.lora_merge(qw, A, B, alpha)
+    torch.cuda.synchronize()
+    Wp = oracle_Wp(lay.W0)
+    Af, Bf = nf4.bf16_to_f64(lay.A), nf4.bf16_to_f64(lay.B)
+    ref_W = lora.merge(Wp, Af, Bf, s)
+    extra = r * 2.0 ** -22 * s * (np.abs(Bf) @ np.abs(Af)) + 2.0 ** -23 * np.abs(Wp)
+    within_one_bf16_ulp(bf16_host_bits(W), ref_W, "merge", abs_extra=extra)
+    W0pp = q4.lora_unmerge(bf16_dev(ref_W), A, B, alpha)
+    torch.cuda.synchronize()
+    ref_W0pp = lora.unmerge(nf4.bf16_to_f64(ref_W), Af, Bf, s)
+    within_one_bf16_ulp(bf16_host_bits(W0pp), ref_W0pp, "unmerge", abs_extra=extra)
+    assert q4.qlora_get_device_status() == 0
+
+
 def test_merged_layer_matches_unmerged_forward():
     cfg = synthetic.config(1)
     lay = synthetic.make_layer(cfg)
