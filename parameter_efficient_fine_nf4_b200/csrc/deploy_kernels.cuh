@@ -12,7 +12,7 @@
 //     128-byte-swizzled form, double-buffered;
 //   * warp 1 computes (B A) for the tile with tcgen05 into one of two TMEM
 //     accumulators;
-//   * warps 2-5 combine accumulator and input row by row, write the bf16
+//   * warps 2-9 combine accumulator and input row by row, write the bf16
 //     result into a swizzled shared tile (in place over W for unmerge), and
 //     one thread stores it with TMA.
 // Rows or columns beyond d or k are zero-filled by the loads and clipped by
@@ -38,11 +38,22 @@ template <bool kMerge, int KS>
 struct DeployCfg {
   static constexpr int kOpA = KS * 16384;               // B rows: 128 x 64 bf16 per K-step
   static constexpr int kOpB = KS * 32768;               // A columns: 4 atoms of 64 x 64 bf16 per K-step
+  static constexpr int kOpBytes = kOpA + kOpB;
+  // the operands of the next tile load while this tile's MMA runs (two
+  // buffers); with two K-steps only one fits beside the input tiles
+  static constexpr int kOpBufs = KS == 1 ? 2 : 1;
   static constexpr int kIo = kMerge ? 16384 : 65536;    // codes tile (128 x 128 B) or W tile
-  static constexpr int kOut = kMerge ? 65536 : 0;       // merge output tile (unmerge: in place)
-  static constexpr int kBytes = kOpA + kOpB + 2 * kIo + kOut;
+  static constexpr int kOutBufs = kMerge ? 1 : 0;       // merge output tile (unmerge: in place)
+  static constexpr int kOut = kOutBufs * 65536;
+  static constexpr int kBytes = kOpBufs * kOpBytes + 2 * kIo + kOut;
   static constexpr int kSmemBytes = kBytes + 1024 + 512;
 };
+
+// Warps: 0 producer, 1 MMA, 2-9 epilogue (two per TMEM lane quarter, each
+// taking one half of the tile's 256 columns).
+constexpr int kEpiWarps = 8;
+constexpr int kEpiThreads = kEpiWarps * 32;
+constexpr int kDeployThreads = 64 + kEpiThreads;
 
 // Byte offset of 16-byte chunk `chunk` (0..7) of row `row` in a 128-byte-row,
 // 128B-swizzled tile.
@@ -51,7 +62,7 @@ __device__ __forceinline__ uint32_t sw128(int row, int chunk) {
 }
 
 template <bool kMerge, int KS>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+__global__ void __launch_bounds__(kDeployThreads, 1)
     lora_deploy_kernel(const __grid_constant__ CUtensorMap tmOpA, const __grid_constant__ CUtensorMap tmOpB,
                        const __grid_constant__ CUtensorMap tmIo, const __grid_constant__ CUtensorMap tmOut,
                        const __grid_constant__ DeployArgs p) {
@@ -61,36 +72,35 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const uint32_t pad = (1024u - (raw_addr & 1023u)) & 1023u;
   uint8_t* smem = smem_raw + pad;
   const uint32_t sbase = raw_addr + pad;
-  const uint32_t sA = sbase;
-  const uint32_t sB = sA + Cfg::kOpA;
-  const uint32_t sIo = sB + Cfg::kOpB;
+  const uint32_t sOp = sbase;                           // kOpBufs x {A part, B part}
+  const uint32_t sIo = sOp + Cfg::kOpBufs * Cfg::kOpBytes;
   const uint32_t sOut = sIo + 2 * Cfg::kIo;
-  uint8_t* gIo = smem + Cfg::kOpA + Cfg::kOpB;
+  uint8_t* gIo = smem + Cfg::kOpBufs * Cfg::kOpBytes;
   uint8_t* gOut = gIo + 2 * Cfg::kIo;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::kBytes);
-  uint64_t* op_full = bars + 0;
-  uint64_t* op_empty = bars + 1;
-  uint64_t* io_full = bars + 2;      // [2]
-  uint64_t* io_empty = bars + 4;     // [2]
-  uint64_t* acc_full = bars + 6;     // [2]
-  uint64_t* acc_empty = bars + 8;    // [2]
-  uint64_t* drain_bar = bars + 10;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 11);
+  uint64_t* op_full = bars + 0;      // [2]
+  uint64_t* op_empty = bars + 2;     // [2]
+  uint64_t* io_full = bars + 4;      // [2]
+  uint64_t* io_empty = bars + 6;     // [2]
+  uint64_t* acc_full = bars + 8;     // [2]
+  uint64_t* acc_empty = bars + 10;   // [2]
+  uint64_t* drain_bar = bars + 12;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  float* s_lut = reinterpret_cast<float*>(tmem_slot + 4);
+  __shared__ float s_lut[16];                           // static: register + offset addressing
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int units = p.tiles_m * p.tiles_n;
 
   if (threadIdx.x == 0) {
-    mbar_init(smem_u32(op_full), 1);
-    mbar_init(smem_u32(op_empty), 1);
     for (int i = 0; i < 2; ++i) {
+      mbar_init(smem_u32(&op_full[i]), 1);
+      mbar_init(smem_u32(&op_empty[i]), 1);
       mbar_init(smem_u32(&io_full[i]), 1);
       mbar_init(smem_u32(&io_empty[i]), 1);
       mbar_init(smem_u32(&acc_full[i]), 1);
-      mbar_init(smem_u32(&acc_empty[i]), 4);
+      mbar_init(smem_u32(&acc_empty[i]), kEpiWarps);
     }
     mbar_init(smem_u32(drain_bar), 1);
     *abort_flag = 0;
@@ -117,22 +127,26 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     if (lane == 0) {
       int it = 0;
       int io_issued[2] = {0, 0};
-      int op_issued = 0;
+      int op_issued[2] = {0, 0};
       for (int u = blockIdx.x; u < units; u += gridDim.x, ++it) {
         const int m0 = (u / p.tiles_n) * 128;
         const int n0 = (u % p.tiles_n) * 256;
         const int s = it & 1;
-        // rank-r operands (single buffer, freed by the MMA commit)
-        if (!mbar_wait_bounded(smem_u32(op_empty), (uint32_t)((it & 1) ^ 1), abort_flag)) break;
-        const uint32_t fo = smem_u32(op_full);
-        mbar_arrive_expect_tx(fo, (uint32_t)(Cfg::kOpA + Cfg::kOpB));
+        // rank-r operands, freed by the MMA commit of the tile that used them
+        const int ob = it % Cfg::kOpBufs;
+        const int oq = it / Cfg::kOpBufs;
+        if (!mbar_wait_bounded(smem_u32(&op_empty[ob]), (uint32_t)((oq & 1) ^ 1), abort_flag)) break;
+        const uint32_t fo = smem_u32(&op_full[ob]);
+        const uint32_t sA = sOp + ob * Cfg::kOpBytes;
+        const uint32_t sB = sA + Cfg::kOpA;
+        mbar_arrive_expect_tx(fo, (uint32_t)Cfg::kOpBytes);
 #pragma unroll
         for (int ks = 0; ks < KS; ++ks) {
           tma_load_2d(sA + ks * 16384, &tmOpA, fo, ks * 64, m0);
 #pragma unroll
           for (int i = 0; i < 4; ++i) tma_load_2d(sB + ks * 32768 + i * 8192, &tmOpB, fo, n0 + 64 * i, ks * 64);
         }
-        op_issued = 1;
+        op_issued[ob] = oq + 1;
         // input tile (double buffer, freed by the epilogue)
         if (!mbar_wait_bounded(smem_u32(&io_empty[s]), (uint32_t)(((it >> 1) & 1) ^ 1), abort_flag)) break;
         const uint32_t fi = smem_u32(&io_full[s]);
@@ -146,26 +160,32 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         io_issued[s] = it + 1;
       }
       if (*abort_flag) {
-        if (op_issued) mbar_wait_bounded(smem_u32(op_full), (uint32_t)((it - 1) & 1), nullptr);
-        for (int s = 0; s < 2; ++s)
-          if (io_issued[s] > 0)
-            mbar_wait_bounded(smem_u32(&io_full[s]), (uint32_t)(((io_issued[s] - 1) >> 1) & 1), nullptr);
+        // let copies already in flight land before the CTA exits
+        for (int b = 0; b < 2; ++b) {
+          if (op_issued[b] > 0)
+            mbar_wait_bounded(smem_u32(&op_full[b]), (uint32_t)((op_issued[b] - 1) & 1), nullptr);
+          if (io_issued[b] > 0)
+            mbar_wait_bounded(smem_u32(&io_full[b]), (uint32_t)(((io_issued[b] - 1) >> 1) & 1), nullptr);
+        }
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t idesc = idesc_bf16_f32(128, 256, 0, 1);
-      const uint64_t da = smem_desc_sw128(sA, 16, 1024);
-      const uint64_t db = smem_desc_sw128(sB, 8192, 1024);
       bool ok = true;
       int issued_any = 0;
       int it = 0;
       for (int u = blockIdx.x; u < units; u += gridDim.x, ++it) {
         const int s = it & 1;
+        const int ob = it % Cfg::kOpBufs;
+        const int oq = it / Cfg::kOpBufs;
         if (!mbar_wait_bounded(smem_u32(&acc_empty[s]), (uint32_t)(((it >> 1) & 1) ^ 1), abort_flag)) { ok = false; break; }
-        if (!mbar_wait_bounded(smem_u32(op_full), (uint32_t)(it & 1), abort_flag)) { ok = false; break; }
+        if (!mbar_wait_bounded(smem_u32(&op_full[ob]), (uint32_t)(oq & 1), abort_flag)) { ok = false; break; }
         tc_fence_after();
+        const uint32_t sA = sOp + ob * Cfg::kOpBytes;
+        const uint64_t da = smem_desc_sw128(sA, 16, 1024);
+        const uint64_t db = smem_desc_sw128(sA + Cfg::kOpA, 8192, 1024);
         const uint32_t d_tmem = tmem_base + (uint32_t)(s * 256);
 #pragma unroll
         for (int ks = 0; ks < KS; ++ks) {
@@ -179,7 +199,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             }
           }
         }
-        umma_commit(smem_u32(op_empty));
+        umma_commit(smem_u32(&op_empty[ob]));
         umma_commit(smem_u32(&acc_full[s]));
       }
       if (!ok && issued_any) {
@@ -190,6 +210,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   } else {
     // ------------------------------------------------------------ epilogue
     const int quarter = warp & 3;
+    const int c0 = ((warp - 2) >> 2) * 4;         // first of this warp's four 32-column chunks
     const int row = quarter * 32 + lane;
     const bool elected = threadIdx.x == 64;       // warp 2, lane 0 issues the stores
     const float mu = kMerge ? p.mean[0] : 0.f;
@@ -200,18 +221,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const int n0 = (u % p.tiles_n) * 256;
       const int s = it & 1;
       const int m = m0 + row;
-      // block scales of this row's four 64-blocks: global loads issued before
-      // waiting for the tile so their latency overlaps the wait
-      float asc[4] = {0.f, 0.f, 0.f, 0.f};
+      // scales of the two 64-blocks this warp covers in its row: global loads
+      // issued before waiting for the tile so their latency overlaps the wait
+      float asc[2] = {0.f, 0.f};
       if (kMerge && m < p.d) {
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
-          if (n0 + 64 * j < p.k) asc[j] = block_scale(p.absmax_q, p.scale2, mu, (int64_t)m * kb + n0 / 64 + j);
+        for (int j = 0; j < 2; ++j) {
+          const int nb = n0 + 32 * c0 + 64 * j;
+          if (nb < p.k) asc[j] = block_scale(p.absmax_q, p.scale2, mu, (int64_t)m * kb + nb / 64);
+        }
       }
       bool ok = mbar_wait_bounded(smem_u32(&io_full[s]), (uint32_t)((it >> 1) & 1), abort_flag);
       ok = ok && mbar_wait_bounded(smem_u32(&acc_full[s]), (uint32_t)((it >> 1) & 1), abort_flag);
       // every epilogue thread leaves together (the tile below uses named barriers)
-      if (named_bar_any(3, 128, !ok)) break;
+      if (named_bar_any(3, kEpiThreads, !ok)) break;
       tc_fence_after();
       // the previous tile's store must have read its shared tile before this
       // tile's results are written (merge: the one output tile; unmerge: the
@@ -221,20 +244,27 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           bulk_wait_group_read0();
           if (!kMerge) mbar_arrive(smem_u32(&io_empty[s ^ 1]));
         }
-        named_bar_sync(2, 128);
+        named_bar_sync(2, kEpiThreads);
       }
       const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(s * 256);
       uint8_t* io = gIo + s * Cfg::kIo;
       uint8_t* outt = kMerge ? gOut : io;
-#pragma unroll 1
-      for (int c = 0; c < 8; ++c) {
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(taddr + (uint32_t)(c * 32), v);
+      // two chunks per TMEM round trip: both loads are in flight before the wait
+#pragma unroll
+      for (int cp = 0; cp < 4; cp += 2) {
+        uint32_t vv[2][32];
+        tmem_ld_32x32b_x32(taddr + (uint32_t)((c0 + cp) * 32), vv[0]);
+        tmem_ld_32x32b_x32(taddr + (uint32_t)((c0 + cp + 1) * 32), vv[1]);
         tmem_ld_wait();
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int cc = cp + h;
+        const int c = c0 + cc;
+        const uint32_t (&v)[32] = vv[h];
         uint32_t w[16];                       // 32 bf16 inputs w' (merge) or W (unmerge)
         if (kMerge) {
           const uint4 cw = *reinterpret_cast<const uint4*>(io + sw128(row, c));
-          dequant32(cw, asc[c >> 1], s_lut, w);
+          dequant32(cw, asc[cc >> 1], s_lut, w);
         } else {
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
@@ -256,13 +286,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               make_uint4(r4[0], r4[1], r4[2], r4[3]);
         }
       }
+      }
       // accumulator drained
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&acc_empty[s]));
       // all rows written: one thread stores the tile
       fence_proxy_async_smem();
-      named_bar_sync(1, 128);
+      named_bar_sync(1, kEpiThreads);
       if (elected) {
         const uint32_t src = kMerge ? sOut : sIo + s * Cfg::kIo;
 #pragma unroll

@@ -51,6 +51,7 @@ struct GemmArgs {
   int n_store2;
   int lo_offset;              // > 0: out2 also gets lo = bf16(v - bf16(v)) at this column offset
   int pair_offset;            // > 0: the result is acc[j] + acc[j + pair_offset] (hi/lo operand pair)
+  int tma_store;              // EPI_BF16 through shared staging and TMA stores (tmOut)
   const uint8_t* codes;
   const uint8_t* absmax_q;
   const float* scale2;
@@ -67,7 +68,9 @@ struct GemmCfg {
   static constexpr int kBBytes = BN * kBK * 2;
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kTmemCols = 2 * BN;                       // two accumulators
-  static constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*align*/ + 512 /*bars*/;
+  // bf16 output staging for TMA stores: 2 boxes of 32 x 64 per epilogue warp
+  static constexpr int kStoreStage = (BN == 256) ? 4 * 2 * 4096 : 0;
+  static constexpr int kSmemBytes = kStages * kStageBytes + kStoreStage + 1024 /*align*/ + 512 /*bars*/;
 };
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -325,7 +328,7 @@ template <int BN>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmB0,
                    const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
-                   const __grid_constant__ GemmArgs p) {
+                   const __grid_constant__ CUtensorMap tmOut, const __grid_constant__ GemmArgs p) {
   using Cfg = GemmCfg<BN>;
   constexpr int S = Cfg::kStages;
   extern __shared__ uint8_t smem_raw[];
@@ -334,7 +337,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const uint32_t pad = (1024u - (raw_addr & 1023u)) & 1023u;
   uint8_t* smem = smem_raw + pad;
   const uint32_t sbase = raw_addr + pad;
-  uint8_t* ctrl = smem + S * Cfg::kStageBytes;
+  uint8_t* ctrl = smem + S * Cfg::kStageBytes + Cfg::kStoreStage;
   uint64_t* full_bar = reinterpret_cast<uint64_t*>(ctrl);
   uint64_t* empty_bar = full_bar + S;
   uint64_t* acc_full = empty_bar + S;       // [2]
@@ -482,7 +485,44 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const int m = c.m0 + row;
       const bool row_ok = m < p.M;
       const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * BN);
-      if (p.epi == EPI_MERGE || p.epi == EPI_UNMERGE) {
+      if (Cfg::kStoreStage > 0 && p.tma_store) {
+        // bf16 output through shared memory: this warp's 32 rows x 64 columns
+        // per box, 128B-swizzled (conflict-free 16-byte writes), stored by TMA
+        // (coalesced, clipped at the matrix edge); two boxes in flight per warp
+        uint8_t* stg = smem + S * Cfg::kStageBytes + (warp - 2) * 8192;
+        const uint32_t stg_s = sbase + S * Cfg::kStageBytes + (uint32_t)((warp - 2) * 8192);
+#pragma unroll 1
+        for (int b = 0; b < BN / 64; ++b) {
+          uint32_t v0[32], v1[32];
+          tmem_ld_32x32b_x32(taddr + (uint32_t)(b * 64), v0);
+          tmem_ld_32x32b_x32(taddr + (uint32_t)(b * 64 + 32), v1);
+          tmem_ld_wait();
+          if (b >= 2) {
+            if (lane == 0) bulk_wait_group_read1();       // the store that used this buffer
+            __syncwarp();
+          }
+          uint8_t* box = stg + (b & 1) * 4096;
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            const uint32_t (&v)[32] = q < 4 ? v0 : v1;
+            const int o = (q & 3) * 8;
+            uint4 w;
+            w.x = pack_bf16x2(__uint_as_float(v[o + 0]), __uint_as_float(v[o + 1]));
+            w.y = pack_bf16x2(__uint_as_float(v[o + 2]), __uint_as_float(v[o + 3]));
+            w.z = pack_bf16x2(__uint_as_float(v[o + 4]), __uint_as_float(v[o + 5]));
+            w.w = pack_bf16x2(__uint_as_float(v[o + 6]), __uint_as_float(v[o + 7]));
+            *reinterpret_cast<uint4*>(box + lane * 128 + ((q ^ (lane & 7)) << 4)) = w;
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tmOut, stg_s + (uint32_t)((b & 1) * 4096), c.n0 + 64 * b, c.m0 + quarter * 32);
+            bulk_commit_group();
+          }
+        }
+        if (lane == 0) bulk_wait_group_read0();            // staging reusable by the next unit
+        __syncwarp();
+      } else if (p.epi == EPI_MERGE || p.epi == EPI_UNMERGE) {
         epilogue_merge_row<BN>(p, taddr, m, row_ok, c.n0, s_lut);
       } else
 #pragma unroll 1
@@ -507,6 +547,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&acc_empty[buf]));
     }
+    if (Cfg::kStoreStage > 0 && p.tma_store && lane == 0) bulk_wait_group0();   // stores complete
   }
   tc_fence_before();
   __syncthreads();

@@ -80,23 +80,20 @@ HostTables build_tables() {
     t.thresholds[i] = f;
   }
   t.enc_ok = true;
+  memset(&t.enc, 0, sizeof(t.enc));
+  for (int i = 0; i < 15; ++i) t.enc.thr[i] = t.thresholds[i];
+  t.enc.thr[15] = INFINITY;
   for (int j = 0; j < kEncBins; ++j) {
     const double lo = ((double)j - 64.5) / 64.0;
     const double hi = ((double)j - 63.5) / 64.0;
     int base = 0, inside = 0;
-    float thr = INFINITY;
     for (int i = 0; i < 15; ++i) {
       const double th = (double)t.thresholds[i];
-      if (th <= lo) {
-        ++base;
-      } else if (th <= hi) {
-        thr = t.thresholds[i];
-        ++inside;
-      }
+      if (th <= lo) ++base;
+      else if (th <= hi) ++inside;
     }
-    if (inside > 1) t.enc_ok = false;
-    t.enc.e[j].base = base;
-    t.enc.e[j].thr = thr;
+    if (inside > 1) t.enc_ok = false;      // the table form needs at most one per bin
+    t.enc.base[j] = (uint8_t)base;
   }
   return t;
 }
@@ -284,7 +281,7 @@ int launch_deploy_t(const qlora_nf4_t* q, const uint16_t* W, const uint16_t* A, 
   const dim3 grid((unsigned)std::min<int64_t>(units, current_sms()));
   const double bytes = (double)d * k * (kMerge ? 2.5 : 4.0);
   return launch(kMerge ? "lora_merge" : "lora_unmerge", 2.0 * d * (double)k * r, bytes, st, [&] {
-    lora_deploy_kernel<kMerge, KS><<<grid, kGemmThreads, DeployCfg<kMerge, KS>::kSmemBytes, st>>>(mA, mB, mIo, mOut, a);
+    lora_deploy_kernel<kMerge, KS><<<grid, kDeployThreads, DeployCfg<kMerge, KS>::kSmemBytes, st>>>(mA, mB, mIo, mOut, a);
   });
 }
 
@@ -341,12 +338,21 @@ int launch_gemm_bn(const char* name, const GemmPlan& g, GemmArgs args, cudaStrea
   const int splits = (int)cdiv(g.K0, args.k_per_split);
   const auto& T = tables();
   memcpy(args.levels, T.levels, sizeof(args.levels));
+  // bf16 outputs of the 256-wide kernel leave through shared staging and TMA
+  // stores when the rows are 16-byte aligned
+  CUtensorMap mo = m[0];
+  args.tma_store = 0;
+  if (BN == 256 && args.epi == EPI_BF16 && aligned16(args.out) && (args.ldo % 8) == 0 &&
+      args.n_store == g.N) {
+    if (!make_map(&mo, args.out, g.N, g.M, args.ldo, 32)) return QLORA_ERR_CUDA;
+    args.tma_store = 1;
+  }
   // persistent: one CTA per SM (or per unit when there are fewer units)
   const int64_t units = (int64_t)args.tiles_m * args.tiles_n * splits;
   dim3 grid((unsigned)std::min<int64_t>(units, current_sms()), 1, 1);
   const double flops = 2.0 * g.M * (double)g.N * (g.K0 + g.K1);
   return launch(name, flops, 0.0, st, [&] {
-    gemm_tc_kernel<BN><<<grid, kGemmThreads, GemmCfg<BN>::kSmemBytes, st>>>(m[0], m[1], m[2], m[3], args);
+    gemm_tc_kernel<BN><<<grid, kGemmThreads, GemmCfg<BN>::kSmemBytes, st>>>(m[0], m[1], m[2], m[3], mo, args);
   });
 }
 

@@ -19,19 +19,18 @@ constexpr int kBlock = 64;
 constexpr int kBlock2 = 256;
 constexpr int kEncBins = 129;     // rint(64 x) + 64, x in [-1, 1]
 
-// Encoder table.  Bin j holds every x with rint(64 x) = j - 64, i.e. the
+// Encoder tables.  Bin j holds every x with rint(64 x) = j - 64, i.e. the
 // closed interval [(j - 64.5)/64, (j - 63.5)/64] (closed because a tie may
-// round either way).  Entry: the number of thresholds at or below the lower
-// edge, and the single threshold inside the bin (+inf if none), so that
-// code(x) = base + (x >= thr).  At most one threshold falls in a bin because
-// the smallest gap between thresholds (~0.08) exceeds the bin width 1/64; the
-// host builder checks it.
-struct __align__(8) EncEntry {
-  float thr;
-  int base;
-};
+// round either way).  base[j] = the number of thresholds at or below the
+// bin's lower edge; the only threshold that can lie inside the bin is then
+// thr[base[j]] (the first one above the edge; thr[15] = +inf), because the
+// smallest gap between thresholds (~0.08) exceeds the bin width 1/64 (the
+// host builder checks it).  So code(x) = base[j] + (x >= thr[base[j]]): a
+// threshold above the bin never satisfies the comparison.  Both tables are
+// read with 1- and 4-byte shared loads that do not conflict across banks.
 struct EncTable {
-  EncEntry e[kEncBins];
+  uint8_t base[kEncBins + 3];
+  float thr[16];
 };
 struct NF4Levels {
   float q[16];
@@ -51,11 +50,13 @@ __device__ __forceinline__ float div_markstein(float w, float a, float y) {
 
 // rint(64 x) for |x| <= 1 without a float-to-int conversion: adding 1.5 * 2^23
 // leaves the rounded integer in the low mantissa bits (round to nearest even).
-__device__ __forceinline__ uint32_t enc_code(float x, const EncEntry* s_tab) {
-  const float t = __fadd_rn(__fmul_rn(x, 64.0f), 12582912.0f);
-  const uint32_t j = min((uint32_t)(__float_as_int(t) - 0x4B400000 + 64), (uint32_t)(kEncBins - 1));
-  const EncEntry e = s_tab[j];
-  return (uint32_t)(e.base + (x >= e.thr ? 1 : 0));
+// (x * 64 is exact, so one fused multiply-add rounds exactly like the add.)
+// The unsigned clamp keeps non-finite inputs inside the table.
+__device__ __forceinline__ uint32_t enc_code(float x, const uint8_t* s_base, const float* s_thr) {
+  const float t = __fmaf_rn(x, 64.0f, 12582912.0f);
+  const uint32_t j = min((uint32_t)__float_as_int(t) - (uint32_t)(0x4B400000 - 64), (uint32_t)(kEncBins - 1));
+  const uint32_t b = s_base[j];
+  return b + (x >= s_thr[b] ? 1u : 0u);
 }
 
 // ---------------------------------------------------------------------------
@@ -66,10 +67,12 @@ __device__ __forceinline__ uint32_t enc_code(float x, const EncEntry* s_tab) {
 __global__ void __launch_bounds__(256) nf4_quantize_phase1(
     const float* __restrict__ W0, int64_t n_b, uint32_t* __restrict__ codes_u32,
     float* __restrict__ absmax, double* __restrict__ group_sum, const __grid_constant__ EncTable tab) {
-  __shared__ EncEntry s_tab[kEncBins];
+  __shared__ uint8_t s_base[kEncBins + 3];
+  __shared__ float s_thr[16];
   __shared__ float s_abs[kBlock2];
   const int tid = threadIdx.x;
-  for (int i = tid; i < kEncBins; i += blockDim.x) s_tab[i] = tab.e[i];
+  for (int i = tid; i < kEncBins + 3; i += blockDim.x) s_base[i] = tab.base[i];
+  if (tid < 16) s_thr[tid] = tab.thr[tid];
   __syncthreads();
 
   const int64_t g = blockIdx.x;
@@ -110,7 +113,7 @@ __global__ void __launch_bounds__(256) nf4_quantize_phase1(
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
           const float x = div_markstein(w[i], m, y);
-          packed |= enc_code(x, s_tab) << (4 * i);
+          packed |= enc_code(x, s_base, s_thr) << (4 * i);
         }
       }
       if (b < n_b) {
@@ -217,31 +220,32 @@ __device__ __forceinline__ float block_scale(const uint8_t* absmax_q, const floa
 }
 
 // 32 codes (one 16-byte word) -> 32 bf16 values of level[code] * a'.
-__device__ __forceinline__ void dequant32(const uint4 c, float a, const float* s_q, uint32_t (&o)[16]) {
-  const uint32_t w[4] = {c.x, c.y, c.z, c.w};
+// 8 codes (one 32-bit word, element 2j in the low nibble of byte j) -> 8 bf16
+// values of level[code] * a, packed in pairs.  Both nibbles of every byte are
+// turned into byte offsets into the 16-entry level table with two logic ops,
+// then each offset is taken out with one byte permute; `s_q` must be a
+// shared-memory table so the load is a register-plus-offset address.
+__device__ __forceinline__ void dequant8(uint32_t w, float a, const float* s_q, uint32_t* o) {
+  const uint32_t lo = (w & 0x0F0F0F0Fu) << 2;      // byte j = 4 * code(2j)
+  const uint32_t hi = (w >> 2) & 0x3C3C3C3Cu;      // byte j = 4 * code(2j + 1)
+  const char* base = reinterpret_cast<const char*>(s_q);
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const uint32_t lo = (w[i] >> (8 * j)) & 0xFu;
-      const uint32_t hi = (w[i] >> (8 * j + 4)) & 0xFu;
-      const __nv_bfloat162 p = __floats2bfloat162_rn(__fmul_rn(s_q[lo], a), __fmul_rn(s_q[hi], a));
-      o[i * 4 + j] = *reinterpret_cast<const uint32_t*>(&p);
-    }
+  for (int j = 0; j < 4; ++j) {
+    const uint32_t ol = __byte_perm(lo, 0u, 0x4440u + j);
+    const uint32_t oh = __byte_perm(hi, 0u, 0x4440u + j);
+    const float ql = *reinterpret_cast<const float*>(base + ol);
+    const float qh = *reinterpret_cast<const float*>(base + oh);
+    const __nv_bfloat162 p = __floats2bfloat162_rn(__fmul_rn(ql, a), __fmul_rn(qh, a));
+    o[j] = *reinterpret_cast<const uint32_t*>(&p);
   }
 }
 
-// 8 codes (one 32-bit word) -> 8 bf16 values of level[code] * a (one 16-byte word).
-__device__ __forceinline__ uint4 dequant8(uint32_t w, float a, const float* s_q) {
-  uint32_t o[4];
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const uint32_t lo = (w >> (8 * j)) & 0xFu;
-    const uint32_t hi = (w >> (8 * j + 4)) & 0xFu;
-    const __nv_bfloat162 p = __floats2bfloat162_rn(__fmul_rn(s_q[lo], a), __fmul_rn(s_q[hi], a));
-    o[j] = *reinterpret_cast<const uint32_t*>(&p);
-  }
-  return make_uint4(o[0], o[1], o[2], o[3]);
+// 32 codes (one 16-byte word) -> 32 bf16 values of level[code] * a.
+__device__ __forceinline__ void dequant32(const uint4 c, float a, const float* s_q, uint32_t (&o)[16]) {
+  dequant8(c.x, a, s_q, o + 0);
+  dequant8(c.y, a, s_q, o + 4);
+  dequant8(c.z, a, s_q, o + 8);
+  dequant8(c.w, a, s_q, o + 12);
 }
 
 // ---------------------------------------------------------------------------
@@ -274,7 +278,11 @@ __global__ void __launch_bounds__(256) nf4_dequantize_kernel(
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const int64_t u = base + j * stride;
-      if (u < n_units) __stcs(W_out + u, dequant8(c[j], a[j], s_q));
+      if (u < n_units) {
+        uint32_t o[4];
+        dequant8(c[j], a[j], s_q, o);
+        __stcs(W_out + u, make_uint4(o[0], o[1], o[2], o[3]));
+      }
     }
   }
 }
