@@ -73,7 +73,9 @@ class ClockSampler:
         self.proc = None
         self.lines = []
 
-    def start(self):
+    def start(self, wait_first=5.0):
+        """Start sampling every 100 ms; returns once the first sample arrived
+        (nvidia-smi takes a moment to start) or after `wait_first` seconds."""
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}",
@@ -83,10 +85,17 @@ class ClockSampler:
             self.t.start()
         except Exception:
             self.proc = None
+            return
+        t_end = time.time() + wait_first
+        while not self.lines and time.time() < t_end:
+            time.sleep(0.02)
 
     def _read(self):
         for ln in self.proc.stdout:
-            self.lines.append(ln.strip())
+            self.lines.append((time.time(), ln.strip()))
+
+    def mark(self, which):
+        setattr(self, which, time.time())
 
     def stop(self):
         if self.proc is None:
@@ -99,7 +108,11 @@ class ClockSampler:
         self.t.join(timeout=2)
         sm, smax, reasons = [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        t0 = getattr(self, "t_begin", None)
+        t1 = getattr(self, "t_end", None)
+        window = [(t, ln) for t, ln in self.lines
+                  if t0 is None or t1 is None or t0 <= t <= t1]
+        for _, ln in window:
             parts = [p.strip() for p in ln.split(",")]
             if len(parts) < 9:
                 continue
@@ -113,9 +126,7 @@ class ClockSampler:
                     reasons.add(n)
         if not sm:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
-        top = max(sm)
-        loaded = [v for v in sm if v >= 0.5 * top] or sm
-        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(smax),
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
@@ -290,6 +301,10 @@ def run_ours(args):
             dist.barrier(device_ids=[local])
         torch.cuda.synchronize(dev)
 
+    # clock samples are taken from before the warm-up on, and only those that
+    # fall inside the timed region are kept
+    clocks = ClockSampler(local)
+    clocks.start()
     for _ in range(args.warmup):
         step()
     assert q4.qlora_get_device_status() == 0
@@ -298,9 +313,8 @@ def run_ours(args):
     # between steps outside the events)
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(args.steps)]
-    clocks = ClockSampler(local)
-    clocks.start()
     barrier()
+    clocks.mark("t_begin")
     n0 = q4.qlora_launch_count()
     q4.qlora_profile_begin()
     for i in range(args.steps):
@@ -309,6 +323,7 @@ def run_ours(args):
         step()
         evs[i][1].record(stream)
     barrier()
+    clocks.mark("t_end")
     stats = q4.qlora_profile_end()
     launches = q4.qlora_launch_count() - n0
     clk = clocks.stop()
@@ -355,8 +370,46 @@ def run_ours(args):
     e2e_value = flops_rank * world / (float(te.item()) / 1e3) / 1e12
     assert q4.qlora_get_device_status() == 0
 
+    # ---- the HBM-bound rows, in the step and alone.  Algorithmic bytes per
+    # weight: quantise 4 (W0) + 0.5 (codes) + 1/64 (E4M3 constants); merge and
+    # doubleDequant 0.5 + 1/64 + 2 (bf16 out); unmerge 2 + 2.
+    weights = sum(L["lin"].d * L["lin"].k for L in layers)
+    bpw = {"quantise": 4.5 + 1 / 64, "merge": 2.5 + 1 / 64, "unmerge": 4.0, "dequantise": 2.5 + 1 / 64}
+    kernels = {"quantise": ("nf4_quantize_phase1", "nf4_quantize_dq"), "merge": ("lora_merge",),
+               "unmerge": ("lora_unmerge",), "dequantise": ("nf4_dequantize",)}
+
+    def per_call_ms(st, names, calls):
+        return sum(x["total_ms"] for x in st if x["name"] in names) / calls
+
+    alone = {}
+    for name, fn in (("quantise", lambda L: q4.qlora_nf4_quantize(L["W0"], out=L["qw"], ws=L["ws"])),
+                     ("merge", lambda L: q4.lora_merge(L["qw"], L["A"], L["B"], cfg.alpha, W_out=L["Wm"],
+                                                       ws=L["ws"])),
+                     ("unmerge", lambda L: q4.lora_unmerge(L["Wm"], L["A"], L["B"], cfg.alpha,
+                                                           W0_out=L["W0u"], ws=L["ws"])),
+                     ("dequantise", lambda L: q4.qlora_nf4_dequantize(L["qw"], W_out=L["W0u"]))):
+        for L in layers:
+            fn(L)
+        torch.cuda.synchronize(dev)
+        q4.qlora_profile_begin()
+        for _ in range(5):
+            for L in layers:
+                fn(L)
+        st_alone = q4.qlora_profile_end()
+        alone[name] = per_call_ms(st_alone, kernels[name], 5)
+    assert q4.qlora_get_device_status() == 0
+
     # ---- roofline of the dominant kernel (the tcgen05 GEMM: forward main and dX)
     peaks, peak_src = read_peaks()
+    hbm = float(peaks.get("hbm_gbs"))
+    hbm_rows = {}
+    for name in bpw:
+        calls = args.steps * (2 if name == "dequantise" else 1)
+        ms_step = per_call_ms(stats, kernels[name], calls)
+        gb = weights * bpw[name] / 1e9
+        hbm_rows[name] = {"bytes_per_weight": round(bpw[name], 4),
+                          "in_step_gbs": gb / (ms_step / 1e3), "in_step_frac": gb / (ms_step / 1e3) / hbm,
+                          "alone_gbs": gb / (alone[name] / 1e3), "alone_frac": gb / (alone[name] / 1e3) / hbm}
     gemm = [s for s in stats if s["name"] in ("gemm_fwd_main", "gemm_bwd_dx")]
     g_ms = sum(s["total_ms"] for s in gemm)
     g_launches = sum(s["launches"] for s in gemm)
@@ -394,6 +447,9 @@ def run_ours(args):
             "gpu_launches_per_step": launches / args.steps,
             "clocks": clk,
             "rows": rows,
+            "hbm_rows": {"peak_gbs": hbm, "peak_source": f"{peak_src} hbm_gbs",
+                         "note": "in the step (clocks held down by the power-capped GEMMs) and alone "
+                                 "(5 calls back to back after the timed region)", **hbm_rows},
         }
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(cfg)
@@ -407,7 +463,7 @@ def run_ours(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=40)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", type=int, default=4)

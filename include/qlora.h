@@ -101,7 +101,8 @@ QLORA_API int qlora_nf4_levels(float* levels16, float* thresholds15);
 
 /* ---------------------------------------------------------------- quantise */
 
-/* Workspace for qlora_nf4_quantize: fp32 absmax per block + fp64 per group. */
+/* Workspace for qlora_nf4_quantize: fp32 absmax per block, fp64 sum per
+ * group and a 4-byte completion counter (each part 256-byte aligned). */
 QLORA_API size_t qlora_quantize_workspace_bytes(int64_t d, int64_t k);
 
 /*
@@ -117,7 +118,10 @@ QLORA_API size_t qlora_quantize_workspace_bytes(int64_t d, int64_t k);
  *   absmax_q_b = E4M3_RN_satfinite(fp32(fp32(a_b - mean) / scale2_j))
  *               (0 when scale2_j == 0).
  * Requires block == 64, k % 64 == 0, d >= 1, d*k < 2^34.  W0 and the output
- * buffers must be 16-byte aligned.
+ * buffers must be 16-byte aligned.  Every weight must be finite: a NaN or
+ * infinity makes the results unspecified (the call still completes and
+ * returns QLORA_OK; nothing is read or written out of bounds).  Subnormal
+ * weights and block maxima are handled exactly.
  */
 QLORA_API int qlora_nf4_quantize(const float* W0, int64_t d, int64_t k, int block, qlora_nf4_t* out,
                        void* workspace, size_t workspace_bytes, qlora_stream_t stream);
@@ -144,7 +148,7 @@ QLORA_API int qlora_nf4_dequantize(const qlora_nf4_t* q, uint16_t* W_out, qlora_
  * Same arguments and results as qlora_nf4_quantize, minus the workspace.  The
  * scratch space (fp32 block constants and fp64 group sums) lives in a
  * file-scope __device__ array of QLORA_NOALLOC_MAX_WEIGHTS/16 +
- * QLORA_NOALLOC_MAX_WEIGHTS/2048 bytes (16.1 MiB) that every GPU which loads
+ * QLORA_NOALLOC_MAX_WEIGHTS/2048 + 256 bytes (16.1 MiB) that every GPU which loads
  * this library holds until the process exits.  d*k above
  * QLORA_NOALLOC_MAX_WEIGHTS (2^28 weights) is rejected with
  * QLORA_ERR_EXCEEDS_STATIC_SCRATCH before anything is launched.

@@ -12,9 +12,10 @@
 //     128-byte-swizzled form, double-buffered;
 //   * warp 1 computes (B A) for the tile with tcgen05 into one of two TMEM
 //     accumulators;
-//   * warps 2-9 combine accumulator and input row by row, write the bf16
-//     result into a swizzled shared tile (in place over W for unmerge), and
-//     one thread stores it with TMA.
+//   * warps 2-9 combine accumulator and input row by row; each warp writes
+//     its 32 x 128 part of the bf16 result into swizzled shared boxes of its
+//     own (in place over W for unmerge) and stores them with TMA itself, so
+//     the eight warps never wait for one another.
 // Rows or columns beyond d or k are zero-filled by the loads and clipped by
 // the stores, so no element masks are needed.
 #pragma once
@@ -43,15 +44,17 @@ struct DeployCfg {
   // buffers); with two K-steps only one fits beside the input tiles
   static constexpr int kOpBufs = KS == 1 ? 2 : 1;
   static constexpr int kIo = kMerge ? 16384 : 65536;    // codes tile (128 x 128 B) or W tile
-  static constexpr int kOutBufs = kMerge ? 1 : 0;       // merge output tile (unmerge: in place)
-  static constexpr int kOut = kOutBufs * 65536;
+  // merge: one 32 x 64 bf16 staging box per epilogue warp (unmerge: in
+  // place), and per warp a 16 x 32 table of the block's dequantised levels
+  // (the per-warp level tables of merge are a static shared array)
+  static constexpr int kOut = kMerge ? 16 * 4096 : 0;
   static constexpr int kBytes = kOpBufs * kOpBytes + 2 * kIo + kOut;
   static constexpr int kSmemBytes = kBytes + 1024 + 512;
 };
 
-// Warps: 0 producer, 1 MMA, 2-9 epilogue (two per TMEM lane quarter, each
-// taking one half of the tile's 256 columns).
-constexpr int kEpiWarps = 8;
+// Warps: 0 producer, 1 MMA, 2-17 epilogue (four per TMEM lane quarter, each
+// taking one 64-column box of the tile's 256 columns).
+constexpr int kEpiWarps = 16;
 constexpr int kEpiThreads = kEpiWarps * 32;
 constexpr int kDeployThreads = 64 + kEpiThreads;
 
@@ -87,7 +90,11 @@ __global__ void __launch_bounds__(kDeployThreads, 1)
   uint64_t* drain_bar = bars + 12;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 13);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  __shared__ float s_lut[16];                           // static: register + offset addressing
+  // static, so that table reads are a register plus a constant offset
+  __shared__ float s_lut[16];
+  // merge: s_wlut[warp][c][lane] = float(bf16(level[c] * a')) for the block of
+  // that lane's row, so a code costs one conflict-free shared load
+  __shared__ float s_wlut[kMerge ? kEpiWarps : 1][16][32];
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -98,7 +105,7 @@ __global__ void __launch_bounds__(kDeployThreads, 1)
       mbar_init(smem_u32(&op_full[i]), 1);
       mbar_init(smem_u32(&op_empty[i]), 1);
       mbar_init(smem_u32(&io_full[i]), 1);
-      mbar_init(smem_u32(&io_empty[i]), 1);
+      mbar_init(smem_u32(&io_empty[i]), kEpiWarps);
       mbar_init(smem_u32(&acc_full[i]), 1);
       mbar_init(smem_u32(&acc_empty[i]), kEpiWarps);
     }
@@ -209,67 +216,100 @@ __global__ void __launch_bounds__(kDeployThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
+    // Every warp works alone on one 32-row x 64-column box of the tile (the
+    // box is one quantisation block wide) and stores it with TMA from its
+    // lane 0, so no barrier spans the epilogue warps.  Merge stages the box
+    // in a 4 KB buffer of the warp's own; unmerge writes in place over its
+    // part of the W tile.
+    const int ew = warp - 2;
     const int quarter = warp & 3;
-    const int c0 = ((warp - 2) >> 2) * 4;         // first of this warp's four 32-column chunks
+    const int bxi = ew >> 2;                      // box 0..3: columns 64 bxi .. 64 bxi + 63
+    const int cA = 2 * bxi;                       // its two 32-column chunks: cA, cA + 1
     const int row = quarter * 32 + lane;
-    const bool elected = threadIdx.x == 64;       // warp 2, lane 0 issues the stores
-    const float mu = kMerge ? p.mean[0] : 0.f;
     const int kb = p.k / kBlock;                  // blocks per row of W
+    const float mu = kMerge ? p.mean[0] : 0.f;
+    uint8_t* stg = gOut + ew * 4096;
+    const uint32_t stg_s = sOut + (uint32_t)ew * 4096u;
+    // raw scale inputs of this thread's block, loaded one tile ahead so their
+    // latency hides behind a whole tile of work
+    uint32_t nq = 0u;
+    float ns2 = 0.f;
+    auto fetch_scale = [&](int uu) {
+      if (!kMerge || uu >= units) return;
+      const int m = (uu / p.tiles_n) * 128 + row;
+      const int n = (uu % p.tiles_n) * 256 + 64 * bxi;
+      if (m < p.d && n < p.k) {
+        const int64_t b = (int64_t)m * kb + n / 64;
+        nq = p.absmax_q[b];
+        ns2 = p.scale2[b / kBlock2];
+      }
+    };
+    fetch_scale(blockIdx.x);
     int it = 0;
     for (int u = blockIdx.x; u < units; u += gridDim.x, ++it) {
       const int m0 = (u / p.tiles_n) * 128;
       const int n0 = (u % p.tiles_n) * 256;
       const int s = it & 1;
-      const int m = m0 + row;
-      // scales of the two 64-blocks this warp covers in its row: global loads
-      // issued before waiting for the tile so their latency overlaps the wait
-      float asc[2] = {0.f, 0.f};
-      if (kMerge && m < p.d) {
+      if (kMerge) {
+        // this lane's column of the table (only this lane reads it)
+        const float a = __fadd_rn(__fmul_rn(e4m3_to_f32((uint8_t)nq), ns2), mu);
 #pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          const int nb = n0 + 32 * c0 + 64 * j;
-          if (nb < p.k) asc[j] = block_scale(p.absmax_q, p.scale2, mu, (int64_t)m * kb + nb / 64);
+        for (int c = 0; c < 16; c += 2) {
+          const uint32_t pr = pack_bf16x2(__fmul_rn(s_lut[c], a), __fmul_rn(s_lut[c + 1], a));
+          s_wlut[kMerge ? ew : 0][c][lane] = bf16_bits_to_f32(pr & 0xFFFFu);
+          s_wlut[kMerge ? ew : 0][c + 1][lane] = bf16_bits_to_f32(pr >> 16);
         }
       }
+      fetch_scale(u + gridDim.x);
       bool ok = mbar_wait_bounded(smem_u32(&io_full[s]), (uint32_t)((it >> 1) & 1), abort_flag);
       ok = ok && mbar_wait_bounded(smem_u32(&acc_full[s]), (uint32_t)((it >> 1) & 1), abort_flag);
-      // every epilogue thread leaves together (the tile below uses named barriers)
-      if (named_bar_any(3, kEpiThreads, !ok)) break;
+      // the lanes leave together (the TMEM loads below are warp-collective)
+      if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
-      // the previous tile's store must have read its shared tile before this
-      // tile's results are written (merge: the one output tile; unmerge: the
-      // other input buffer, which the producer then refills)
-      if (it > 0) {
-        if (elected) {
-          bulk_wait_group_read0();
-          if (!kMerge) mbar_arrive(smem_u32(&io_empty[s ^ 1]));
-        }
-        named_bar_sync(2, kEpiThreads);
-      }
+      uint32_t vv[2][32];
       const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(s * 256);
+      tmem_ld_32x32b_x32(taddr + (uint32_t)(cA * 32), vv[0]);
+      tmem_ld_32x32b_x32(taddr + (uint32_t)((cA + 1) * 32), vv[1]);
+      // merge: the store that last read this warp's staging box is done
+      if (kMerge && it > 0 && lane == 0) bulk_wait_group_read0();
+      tmem_ld_wait();
+      // accumulator drained
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&acc_empty[s]));
       uint8_t* io = gIo + s * Cfg::kIo;
-      uint8_t* outt = kMerge ? gOut : io;
-      // two chunks per TMEM round trip: both loads are in flight before the wait
-#pragma unroll
-      for (int cp = 0; cp < 4; cp += 2) {
-        uint32_t vv[2][32];
-        tmem_ld_32x32b_x32(taddr + (uint32_t)((c0 + cp) * 32), vv[0]);
-        tmem_ld_32x32b_x32(taddr + (uint32_t)((c0 + cp + 1) * 32), vv[1]);
-        tmem_ld_wait();
+      // output rows of the box: merge -> staging (32 rows of 128 B); unmerge
+      // -> in place, rows quarter*32.. of the W box bxi
+      uint8_t* obox = kMerge ? stg : io + bxi * 16384 + quarter * 4096;
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
-        const int cc = cp + h;
-        const int c = c0 + cc;
         const uint32_t (&v)[32] = vv[h];
-        uint32_t w[16];                       // 32 bf16 inputs w' (merge) or W (unmerge)
+        float wf[32];                         // the 32 inputs w' (merge) or W (unmerge) as fp32
         if (kMerge) {
-          const uint4 cw = *reinterpret_cast<const uint4*>(io + sw128(row, c));
-          dequant32(cw, asc[cc >> 1], s_lut, w);
+          const uint4 cw = *reinterpret_cast<const uint4*>(io + sw128(row, cA + h));
+          const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const uint32_t lo = words[q] & 0x0F0F0F0Fu;          // byte j = code(8q + 2j)
+            const uint32_t hi = (words[q] >> 4) & 0x0F0F0F0Fu;   // byte j = code(8q + 2j + 1)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const uint32_t cl = __byte_perm(lo, 0u, 0x4440u + j);
+              const uint32_t ch = __byte_perm(hi, 0u, 0x4440u + j);
+              wf[8 * q + 2 * j] = s_wlut[kMerge ? ew : 0][cl][lane];
+              wf[8 * q + 2 * j + 1] = s_wlut[kMerge ? ew : 0][ch][lane];
+            }
+          }
         } else {
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            const uint4 x = *reinterpret_cast<const uint4*>(io + (c >> 1) * 16384 + sw128(row, (c & 1) * 4 + q));
-            w[4 * q + 0] = x.x; w[4 * q + 1] = x.y; w[4 * q + 2] = x.z; w[4 * q + 3] = x.w;
+            const uint4 x = *reinterpret_cast<const uint4*>(obox + sw128(lane, h * 4 + q));
+            const uint32_t xs[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              wf[8 * q + 2 * j] = bf16_bits_to_f32(xs[j] & 0xFFFFu);
+              wf[8 * q + 2 * j + 1] = bf16_bits_to_f32(xs[j] >> 16);
+            }
           }
         }
 #pragma unroll
@@ -277,32 +317,27 @@ __global__ void __launch_bounds__(kDeployThreads, 1)
           uint32_t r4[4];
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
-            const uint32_t wp = w[4 * q + j];
-            const float lo = __fmaf_rn(p.alpha, __uint_as_float(v[8 * q + 2 * j]), bf16_bits_to_f32(wp & 0xFFFFu));
-            const float hi = __fmaf_rn(p.alpha, __uint_as_float(v[8 * q + 2 * j + 1]), bf16_bits_to_f32(wp >> 16));
+            const float lo = __fmaf_rn(p.alpha, __uint_as_float(v[8 * q + 2 * j]), wf[8 * q + 2 * j]);
+            const float hi = __fmaf_rn(p.alpha, __uint_as_float(v[8 * q + 2 * j + 1]), wf[8 * q + 2 * j + 1]);
             r4[j] = pack_bf16x2(lo, hi);
           }
-          *reinterpret_cast<uint4*>(outt + (c >> 1) * 16384 + sw128(row, (c & 1) * 4 + q)) =
-              make_uint4(r4[0], r4[1], r4[2], r4[3]);
+          *reinterpret_cast<uint4*>(obox + sw128(lane, h * 4 + q)) = make_uint4(r4[0], r4[1], r4[2], r4[3]);
         }
       }
-      }
-      // accumulator drained
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&acc_empty[s]));
-      // all rows written: one thread stores the tile
+      // the box is written: lane 0 stores it
       fence_proxy_async_smem();
-      named_bar_sync(1, kEpiThreads);
-      if (elected) {
-        const uint32_t src = kMerge ? sOut : sIo + s * Cfg::kIo;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) tma_store_2d(&tmOut, src + i * 16384, n0 + 64 * i, m0);
+      __syncwarp();
+      if (lane == 0) {
+        const uint32_t src = kMerge ? stg_s : sIo + (uint32_t)(s * Cfg::kIo + bxi * 16384 + quarter * 4096);
+        tma_store_2d(&tmOut, src, n0 + 64 * bxi, m0 + quarter * 32);
         bulk_commit_group();
-        if (kMerge) mbar_arrive(smem_u32(&io_empty[s]));      // codes tile fully read
+        // input tile released: merge once the codes are read (they were, by
+        // the __syncwarp above); unmerge once the store has read it
+        if (!kMerge) bulk_wait_group_read0();
+        mbar_arrive(smem_u32(&io_empty[s]));
       }
     }
-    if (elected) bulk_wait_group0();
+    if (lane == 0) bulk_wait_group0();
   }
   tc_fence_before();
   __syncthreads();

@@ -95,6 +95,20 @@ HostTables build_tables() {
     if (inside > 1) t.enc_ok = false;      // the table form needs at most one per bin
     t.enc.base[j] = (uint8_t)base;
   }
+  // the fast encoder's coarser bins, rint(16 x) = j - 16, same construction
+  for (int j = 0; j < kFastBins; ++j) {
+    const double lo = ((double)j - 16.5) / 16.0;
+    const double hi = ((double)j - 15.5) / 16.0;
+    int base = 0, inside = 0;
+    for (int i = 0; i < 15; ++i) {
+      const double th = (double)t.thresholds[i];
+      if (th <= lo) ++base;
+      else if (th <= hi) ++inside;
+    }
+    if (inside > 1) t.enc_ok = false;
+    t.enc.fbase[j] = (uint32_t)base;
+    t.enc.fthr[j] = t.enc.thr[base];
+  }
   return t;
 }
 
@@ -263,7 +277,7 @@ int launch_deploy_t(const qlora_nf4_t* q, const uint16_t* W, const uint16_t* A, 
   CUtensorMap mA, mB, mIo, mOut;
   if (!make_map(&mA, Bp, r8, d, r8, 128)) return QLORA_ERR_CUDA;     // B rows, K-major
   if (!make_map(&mB, A, k, r, k, 64)) return QLORA_ERR_CUDA;         // A columns, MN-major
-  if (!make_map(&mOut, out, k, d, k, 128)) return QLORA_ERR_CUDA;
+  if (!make_map(&mOut, out, k, d, k, 32)) return QLORA_ERR_CUDA;      // per-warp 32 x 64 stores
   if (kMerge) {
     if (!make_map_u8(&mIo, q->codes, k / 2, d, k / 2, 128, 128)) return QLORA_ERR_CUDA;
   } else {
@@ -545,7 +559,7 @@ using namespace qlora;
 // name is only a stand-in for the device array; its device address comes from
 // cudaGetSymbolAddress, once per device.
 static constexpr size_t kNoallocScratchBytes =
-    (size_t)(QLORA_NOALLOC_MAX_WEIGHTS / 16) + (size_t)(QLORA_NOALLOC_MAX_WEIGHTS / 2048);
+    (size_t)(QLORA_NOALLOC_MAX_WEIGHTS / 16) + (size_t)(QLORA_NOALLOC_MAX_WEIGHTS / 2048) + 256;
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratchBytes];
 
 namespace {
@@ -604,7 +618,7 @@ size_t qlora_quantize_workspace_bytes(int64_t d, int64_t k) {
   if (d < 1 || k < 1) return 0;
   const int64_t n_b = d * k / kBlock;
   const int64_t n_g = cdiv(n_b, kBlock2);
-  return (size_t)(round_up(n_b * 4, 256) + round_up(n_g * 8, 256));
+  return (size_t)(round_up(n_b * 4, 256) + round_up(n_g * 8, 256) + 256);
 }
 
 int qlora_nf4_quantize(const float* W0, int64_t d, int64_t k, int block, qlora_nf4_t* out,
@@ -623,17 +637,17 @@ int qlora_nf4_quantize(const float* W0, int64_t d, int64_t k, int block, qlora_n
   Carver c{reinterpret_cast<uint8_t*>(ws)};
   float* absmax = (float*)c.take((size_t)(n_b * 4));
   double* gsum = (double*)c.take((size_t)(n_g * 8));
+  unsigned int* ticket = (unsigned int*)c.take(4);
   const auto& T = tables();
   const double bytes1 = (double)d * k * 4.5 + (double)n_b * 4;
+  if (cudaMemsetAsync(ticket, 0, sizeof(unsigned int), st) != cudaSuccess) return QLORA_ERR_CUDA;
   QLORA_TRY(launch("nf4_quantize_phase1", 0.0, bytes1, st, [&] {
     nf4_quantize_phase1<<<(unsigned)n_g, 256, 0, st>>>(W0, n_b, reinterpret_cast<uint32_t*>(out->codes),
-                                                       absmax, gsum, T.enc);
-  }));
-  QLORA_TRY(launch("nf4_quantize_mean", 0.0, (double)n_g * 8, st, [&] {
-    nf4_quantize_mean<<<1, 1024, 0, st>>>(gsum, n_g, n_b, out->mean);
+                                                       absmax, gsum, ticket, out->mean, T.enc);
   }));
   QLORA_TRY(launch("nf4_quantize_dq", 0.0, (double)n_b * 5 + n_g * 4, st, [&] {
-    nf4_quantize_dq<<<(unsigned)n_g, 256, 0, st>>>(absmax, n_b, out->mean, out->absmax_q, out->scale2);
+    nf4_quantize_dq<<<(unsigned)cdiv(n_g, kDqGroups), 256, 0, st>>>(absmax, n_g, n_b, out->mean,
+                                                                   out->absmax_q, out->scale2);
   }));
   return QLORA_OK;
 }

@@ -18,6 +18,7 @@ namespace qlora {
 constexpr int kBlock = 64;
 constexpr int kBlock2 = 256;
 constexpr int kEncBins = 129;     // rint(64 x) + 64, x in [-1, 1]
+constexpr int kFastBins = 33;     // rint(16 x) + 16, x in [-1, 1]
 
 // Encoder tables.  Bin j holds every x with rint(64 x) = j - 64, i.e. the
 // closed interval [(j - 64.5)/64, (j - 63.5)/64] (closed because a tie may
@@ -31,6 +32,11 @@ constexpr int kEncBins = 129;     // rint(64 x) + 64, x in [-1, 1]
 struct EncTable {
   uint8_t base[kEncBins + 3];
   float thr[16];
+  // The same construction on bins of width 1/16 (j = rint(16 x) + 16), which
+  // the gap between thresholds (> 1/16) still allows: 33 entries, so each
+  // table fits one word per shared-memory bank.
+  float fthr[kFastBins];
+  uint32_t fbase[kFastBins];
 };
 struct NF4Levels {
   float q[16];
@@ -59,23 +65,129 @@ __device__ __forceinline__ uint32_t enc_code(float x, const uint8_t* s_base, con
   return b + (x >= s_thr[b] ? 1u : 0u);
 }
 
+// The fast encoder reads {fthr[j], fbase[j]} of the coarse bins from two
+// 33-word shared arrays laid out back to back (fbase 33 words after fthr):
+// no two bins but the outermost pair share a bank, and both loads use one
+// address, bits(t) * 4 + K with t = x * 16 + 1.5 * 2^23 and
+// K = table - (0x4B400000 - 16) * 4 (mod 2^32).  It is used only where
+// |x| <= 1 is guaranteed, so the address needs no clamp.
+// Eight codes of one thread's weights, packed (element i in nibble i): all
+// quotients and addresses first, then the sixteen table loads, then the
+// assembly code = base + (x >= thr), each summed into its nibble.
+__device__ __forceinline__ uint32_t encode8_fast(const float (&w)[8], float m, uint32_t K) {
+  const float y = __frcp_rn(m);
+  float x[8];
+  uint32_t addr[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    x[i] = div_markstein(w[i], m, y);
+    addr[i] = (uint32_t)__float_as_int(__fmaf_rn(x[i], 16.0f, 12582912.0f)) * 4u + K;
+  }
+  float thr[8];
+  uint32_t base[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    asm("ld.shared.f32 %0, [%1];" : "=f"(thr[i]) : "r"(addr[i]));
+    asm("ld.shared.u32 %0, [%1+132];" : "=r"(base[i]) : "r"(addr[i]));
+  }
+  uint32_t packed = base[0];
+#pragma unroll
+  for (int i = 1; i < 8; ++i) packed += base[i] << (4 * i);
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    asm("{\n\t.reg .pred p;\n\tsetp.ge.f32 p, %1, %2;\n\t@p add.u32 %0, %0, %3;\n\t}"
+        : "+r"(packed) : "f"(x[i]), "f"(thr[i]), "r"(1u << (4 * i)));
+  return packed;
+}
+
+// Eight codes by the general route (any block absmax): IEEE division and the
+// clamped encoder; an all-zero (or NaN) block gives the zero level.
+__device__ __forceinline__ uint32_t encode8_general(const float (&w)[8], float m, const uint8_t* s_base,
+                                                    const float* s_thr) {
+  if (!(m > 0.f)) return 0x77777777u;
+  uint32_t packed = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) packed |= enc_code(__fdiv_rn(w[i], m), s_base, s_thr) << (4 * i);
+  return packed;
+}
+
+// max(a, |b|) that returns NaN if either operand is NaN.
+__device__ __forceinline__ float max_abs_nan(float a, float b) {
+  float r;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(fabsf(b)));
+  return r;
+}
+
+// ---------------------------------------------------------------------------
+// The mean of the block constants, formed by the last CTA of phase 1 (the one
+// that takes the final ticket, so every group sum is in memory): S is the
+// float64 pairwise tree over the n_g group sums padded with zeros to
+// P = max(2^ceil(log2 n_g), 1024) leaves (zero leaves and zero subtrees add
+// exactly nothing, so the padding does not change S).  Each warp takes
+// aligned chunks of 1024 leaves: lane l sums its 32 consecutive leaves as a
+// pairwise tree in registers and a shuffle tree joins the lanes; a
+// shared-memory tree then joins the P/1024 chunk sums.  mean = fp32(S / n_b).
+// ---------------------------------------------------------------------------
+constexpr int kMeanChunks = 1024;      // P / 1024 <= 1024 for n_g <= 2^20
+
+__device__ __noinline__ void pairwise_mean(const double* group_sum, int64_t n_g, int64_t n_b,
+                                           float* mean_out, double* s_v) {
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  int64_t P = 1024;
+  while (P < n_g) P <<= 1;
+  const int nch = (int)(P / 1024);
+  for (int c = warp; c < nch; c += (int)(blockDim.x >> 5)) {
+    const int64_t first = (int64_t)c * 1024 + lane * 32;
+    double a[32];
+#pragma unroll
+    for (int j = 0; j < 32; j += 2) {
+      const int64_t i = first + j;
+      if (i + 1 < n_g) {
+        const double2 t = __ldcg(reinterpret_cast<const double2*>(group_sum + i));
+        a[j] = t.x;
+        a[j + 1] = t.y;
+      } else {
+        a[j] = (i < n_g) ? __ldcg(group_sum + i) : 0.0;
+        a[j + 1] = 0.0;
+      }
+    }
+#pragma unroll
+    for (int st = 1; st < 32; st <<= 1)
+#pragma unroll
+      for (int j = 0; j < 32; j += 2 * st) a[j] = a[j] + a[j + st];
+    double sum = a[0];
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) sum = sum + __shfl_down_sync(0xffffffffu, sum, off);
+    if (lane == 0) s_v[c] = sum;
+  }
+  __syncthreads();
+  for (int st = 1; st < nch; st <<= 1) {
+    for (int j = 2 * st * tid; j < nch; j += 2 * st * (int)blockDim.x) s_v[j] = s_v[j] + s_v[j + st];
+    __syncthreads();
+  }
+  if (tid == 0) mean_out[0] = __double2float_rn(__ddiv_rn(s_v[0], (double)n_b));
+}
+
 // ---------------------------------------------------------------------------
 // Phase 1: one CTA per group of 256 blocks (16384 weights).  8 threads per
 // block, 8 consecutive weights per thread.  Writes packed codes, the fp32
 // block absmax (scratch) and the fp64 pairwise sum of the group's absmax.
+//
+// Fast path (every block of the warp has its absmax a in [2^-125, 2^125]):
+// x = w / a by Markstein's correction from y = RN(1/a) (all intermediates
+// normal in that range, and |x| <= 1 because |w| <= a), then encode8_fast.
+// Otherwise the warp takes the general route (needed for an all-zero,
+// subnormal or huge absmax, or a NaN, which the NaN-propagating maximum
+// exposes).  Both give RN(w / a) and the same code.  Only the last CTA
+// checks bounds.  The CTA that finishes last also forms the mean.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) nf4_quantize_phase1(
-    const float* __restrict__ W0, int64_t n_b, uint32_t* __restrict__ codes_u32,
-    float* __restrict__ absmax, double* __restrict__ group_sum, const __grid_constant__ EncTable tab) {
-  __shared__ uint8_t s_base[kEncBins + 3];
-  __shared__ float s_thr[16];
-  __shared__ float s_abs[kBlock2];
+template <bool kTail>
+__device__ __forceinline__ void quantize_group(const float* __restrict__ W0, int64_t n_b, int64_t g,
+                                               uint32_t* __restrict__ codes_u32, float* __restrict__ absmax,
+                                               float* s_abs, uint32_t K, const uint8_t* s_base,
+                                               const float* s_thr) {
   const int tid = threadIdx.x;
-  for (int i = tid; i < kEncBins + 3; i += blockDim.x) s_base[i] = tab.base[i];
-  if (tid < 16) s_thr[tid] = tab.thr[tid];
-  __syncthreads();
-
-  const int64_t g = blockIdx.x;
   const int sub = tid & 7;          // 8 threads per block
   const int lb0 = tid >> 3;         // 32 blocks per pass
 #pragma unroll 1
@@ -83,9 +195,8 @@ __global__ void __launch_bounds__(256) nf4_quantize_phase1(
     float4 v[4][2];
 #pragma unroll
     for (int p = 0; p < 4; ++p) {
-      const int lb = (half * 4 + p) * 32 + lb0;
-      const int64_t b = g * kBlock2 + lb;
-      if (b < n_b) {
+      const int64_t b = g * kBlock2 + (half * 4 + p) * 32 + lb0;
+      if (!kTail || b < n_b) {
         const float4* src = reinterpret_cast<const float4*>(W0 + b * kBlock + sub * 8);
         v[p][0] = __ldcs(src);
         v[p][1] = __ldcs(src + 1);
@@ -98,31 +209,51 @@ __global__ void __launch_bounds__(256) nf4_quantize_phase1(
     for (int p = 0; p < 4; ++p) {
       const int lb = (half * 4 + p) * 32 + lb0;
       const int64_t b = g * kBlock2 + lb;
-      float w[8] = {v[p][0].x, v[p][0].y, v[p][0].z, v[p][0].w,
-                    v[p][1].x, v[p][1].y, v[p][1].z, v[p][1].w};
-      float m = 0.f;
+      const float w[8] = {v[p][0].x, v[p][0].y, v[p][0].z, v[p][0].w,
+                          v[p][1].x, v[p][1].y, v[p][1].z, v[p][1].w};
+      float m = fabsf(w[0]);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(w[i]));
-      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
-      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
-      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
-      uint32_t packed = 0x77777777u;             // all-zero block: zero level (code 7)
-      if (m > 0.f) {
-        const float y = __frcp_rn(m);
-        packed = 0;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const float x = div_markstein(w[i], m, y);
-          packed |= enc_code(x, s_base, s_thr) << (4 * i);
-        }
-      }
-      if (b < n_b) {
+      for (int i = 1; i < 8; ++i) m = max_abs_nan(m, w[i]);
+      m = max_abs_nan(m, __shfl_xor_sync(0xffffffffu, m, 1));
+      m = max_abs_nan(m, __shfl_xor_sync(0xffffffffu, m, 2));
+      m = max_abs_nan(m, __shfl_xor_sync(0xffffffffu, m, 4));
+      const bool fast = m >= 0x1p-125f && m <= 0x1p125f;
+      // (the general route gives the same codes for blocks the fast one takes)
+      const uint32_t packed = __all_sync(0xffffffffu, fast) ? encode8_fast(w, m, K)
+                                                            : encode8_general(w, m, s_base, s_thr);
+      if (!kTail || b < n_b) {
         codes_u32[b * 8 + sub] = packed;
         if (sub == 0) absmax[b] = m;
       }
-      if (sub == 0) s_abs[lb] = (b < n_b) ? m : 0.f;
+      if (sub == 0) s_abs[lb] = (!kTail || b < n_b) ? m : 0.f;
     }
   }
+}
+
+__global__ void __launch_bounds__(256, 4) nf4_quantize_phase1(
+    const float* __restrict__ W0, int64_t n_b, uint32_t* __restrict__ codes_u32,
+    float* __restrict__ absmax, double* __restrict__ group_sum, unsigned int* __restrict__ ticket,
+    float* __restrict__ mean_out, const __grid_constant__ EncTable tab) {
+  __shared__ double s_v[kMeanChunks];
+  __shared__ bool s_last;
+  __shared__ uint32_t s_fast[2 * kFastBins];      // fthr (as bits), then fbase
+  __shared__ uint8_t s_base[kEncBins + 3];
+  __shared__ float s_thr[16];
+  __shared__ float s_abs[kBlock2];
+  const int tid = threadIdx.x;
+  if (tid < kFastBins) {
+    s_fast[tid] = __float_as_uint(tab.fthr[tid]);
+    s_fast[kFastBins + tid] = tab.fbase[tid];
+  }
+  if (tid < kEncBins + 3) s_base[tid] = tab.base[tid];
+  if (tid < 16) s_thr[tid] = tab.thr[tid];
+  __syncthreads();
+  const uint32_t K = smem_u32(s_fast) - (uint32_t)(0x4B400000 - 16) * 4u;
+  const int64_t g = blockIdx.x;
+  if ((g + 1) * kBlock2 <= n_b)
+    quantize_group<false>(W0, n_b, g, codes_u32, absmax, s_abs, K, s_base, s_thr);
+  else
+    quantize_group<true>(W0, n_b, g, codes_u32, absmax, s_abs, K, s_base, s_thr);
   __syncthreads();
   if (tid < 32) {
     // pairwise tree over the 256 constants: lane l sums leaves 8l..8l+7, then
@@ -133,78 +264,68 @@ __global__ void __launch_bounds__(256) nf4_quantize_phase1(
     double s = ((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]));
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) s = s + __shfl_down_sync(0xffffffffu, s, off);
-    if (tid == 0) group_sum[g] = s;
-  }
-}
-
-// ---------------------------------------------------------------------------
-// Phase 2: single CTA; pairwise tree over the group sums (padded with zeros
-// to a power of two), mean = fp32(S / n_b).
-// ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(1024) nf4_quantize_mean(const double* __restrict__ group_sum,
-                                                          int64_t n_g, int64_t n_b,
-                                                          float* __restrict__ mean_out) {
-  __shared__ double s_v[1024];
-  const int tid = threadIdx.x;
-  int64_t P = 1;
-  while (P < n_g) P <<= 1;
-  const int64_t C = (P > 1024) ? (P / 1024) : 1;     // leaves per thread (power of two)
-  double stack[24];
-  int level[24];
-  int sp = 0;
-  for (int64_t j = 0; j < C; ++j) {
-    const int64_t idx = (int64_t)tid * C + j;
-    double v = (idx < n_g) ? group_sum[idx] : 0.0;
-    int l = 0;
-    while (sp > 0 && level[sp - 1] == l) {
-      v = stack[sp - 1] + v;
-      --sp;
-      ++l;
+    if (tid == 0) {
+      group_sum[g] = s;
+      // publish the sum, then take a ticket: the CTA with the last ticket
+      // sees every group sum and forms the mean
+      __threadfence();
+      s_last = atomicAdd(ticket, 1u) == gridDim.x - 1;
     }
-    stack[sp] = v;
-    level[sp] = l;
-    ++sp;
   }
-  s_v[tid] = stack[0];
   __syncthreads();
-  for (int s = 1; s < 1024; s <<= 1) {
-    if ((tid % (2 * s)) == 0) s_v[tid] = s_v[tid] + s_v[tid + s];
-    __syncthreads();
+  if (s_last) {
+    __threadfence();
+    pairwise_mean(group_sum, (int64_t)gridDim.x, n_b, mean_out, s_v);
   }
-  if (tid == 0) mean_out[0] = __double2float_rn(__ddiv_rn(s_v[0], (double)n_b));
 }
 
 // ---------------------------------------------------------------------------
-// Phase 3: one CTA per group; second-level scale and E4M3 codes.
+// Phase 2: double quantisation, eight groups per CTA (thread t = block t of
+// each group):
+//   scale2_j   = fp32(max_b |fp32(a_b - mean)| / 448),
+//   absmax_q_b = E4M3_RN_satfinite(fp32(fp32(a_b - mean) / scale2_j)).
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) nf4_quantize_dq(const float* __restrict__ absmax,
+constexpr int kDqGroups = 8;
+
+__global__ void __launch_bounds__(256) nf4_quantize_dq(const float* __restrict__ absmax, int64_t n_g,
                                                        int64_t n_b, const float* __restrict__ mean,
                                                        uint8_t* __restrict__ absmax_q,
                                                        float* __restrict__ scale2) {
-  __shared__ float s_max[8];
-  const int64_t g = blockIdx.x;
+  __shared__ float s_max[kDqGroups][8];
   const int tid = threadIdx.x;
-  const int64_t b = g * kBlock2 + tid;
+  const int warp = tid >> 5, lane = tid & 31;
   const float mu = mean[0];
-  float cen = 0.f;
-  if (b < n_b) cen = __fsub_rn(absmax[b], mu);
-  float m = fabsf(cen);
+  const int64_t g0 = (int64_t)blockIdx.x * kDqGroups;
+  float cen[kDqGroups];
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-  if ((tid & 31) == 0) s_max[tid >> 5] = m;
+  for (int i = 0; i < kDqGroups; ++i) {
+    const int64_t b = (g0 + i) * kBlock2 + tid;
+    cen[i] = (b < n_b) ? __fsub_rn(absmax[b], mu) : 0.f;
+  }
+#pragma unroll
+  for (int i = 0; i < kDqGroups; ++i) {
+    float m = fabsf(cen[i]);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    if (lane == 0) s_max[i][warp] = m;
+  }
   __syncthreads();
-  float c1 = s_max[0];
 #pragma unroll
-  for (int i = 1; i < 8; ++i) c1 = fmaxf(c1, s_max[i]);
-  const float s1 = (c1 > 0.f) ? __fdiv_rn(c1, 448.0f) : 0.f;
-  if (tid == 0) scale2[g] = s1;
-  if (b < n_b) {
-    uint8_t code = 0;
-    if (s1 > 0.f) {
-      const float x = __fdiv_rn(cen, s1);
-      code = (uint8_t)__nv_cvt_float_to_fp8(x, __NV_SATFINITE, __NV_E4M3);
+  for (int i = 0; i < kDqGroups; ++i) {
+    const int64_t g = g0 + i;
+    if (g < n_g) {
+      float c1 = s_max[i][0];
+#pragma unroll
+      for (int w = 1; w < 8; ++w) c1 = fmaxf(c1, s_max[i][w]);
+      const float s1 = (c1 > 0.f) ? __fdiv_rn(c1, 448.0f) : 0.f;
+      if (tid == 0) scale2[g] = s1;
+      const int64_t b = g * kBlock2 + tid;
+      if (b < n_b) {
+        uint8_t code = 0;
+        if (s1 > 0.f) code = (uint8_t)__nv_cvt_float_to_fp8(__fdiv_rn(cen[i], s1), __NV_SATFINITE, __NV_E4M3);
+        absmax_q[b] = code;
+      }
     }
-    absmax_q[b] = code;
   }
 }
 

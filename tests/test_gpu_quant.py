@@ -121,6 +121,38 @@ def test_quantize_threshold_sweep():
     _check_full(W, qw, Wp)
 
 
+@pytest.mark.parametrize("a", [np.float32(1e-39), np.float32(2.0 ** -126), np.float32(2.0 ** -125),
+                               np.float32(2.0 ** 125), np.float32(2.0 ** 126), np.float32(3.0e38)],
+                         ids=["subnormal", "min_normal", "fast_lo", "fast_hi", "huge", "near_max"])
+def test_quantize_extreme_block_scales(a):
+    # blocks whose absmax sits at and beyond both ends of the normal range:
+    # quotients next to every threshold, plus one block of subnormal multiples
+    _, thr = q4.qlora_nf4_levels()
+    blocks = []
+    for t in thr:
+        xs = np.array(_near(np.float32(t), 3), np.float32)           # 7 values
+        blk = np.zeros(64, np.float32)
+        blk[:7] = (xs * a).astype(np.float32)
+        blk[7:14] = (-xs * a).astype(np.float32)
+        blk[14:20] = (a * (np.float32(0.3) / np.float32(7)
+                           * np.arange(1, 7, dtype=np.float32))).astype(np.float32)
+        blk[63] = a
+        blocks.append(blk)
+    tiny = (np.arange(64, dtype=np.float32) - np.float32(31)) * np.float32(2.0 ** -149)
+    blocks.append(tiny.astype(np.float32))
+    W = np.ascontiguousarray(np.stack(blocks).reshape(-1, 128))     # 16 blocks -> 8 x 128
+    qw = q4.qlora_nf4_quantize(f32_dev(W))
+    torch.cuda.synchronize()
+    assert q4.qlora_get_device_status() == 0
+    # storage only: the oracle's bf16 rounding covers the normal range, which
+    # the dequantised weights of these scales leave
+    ref = nf4.quantize(W)
+    assert np.array_equal(qw.codes.cpu().numpy(), ref["codes"])
+    assert np.array_equal(qw.absmax_q.cpu().numpy(), ref["absmax_q"])
+    assert np.array_equal(qw.scale2.cpu().numpy().view(np.uint32), ref["scale2"].view(np.uint32))
+    assert qw.mean.cpu().numpy().view(np.uint32)[0] == np.float32(ref["mean"]).view(np.uint32)
+
+
 def test_quantize_is_deterministic():
     lay = synthetic.make_layer(synthetic.config(2), with_acts=False)
     W = f32_dev(lay.W0)
