@@ -64,6 +64,62 @@ __device__ __forceinline__ uint32_t sw128(int row, int chunk) {
   return (uint32_t)(row * 128 + ((chunk ^ (row & 7)) << 4));
 }
 
+// Eight merged weights from one 32-bit word of codes (element 2j in the low
+// nibble of byte j) and their eight accumulator values, as one block of PTX:
+//   code -> this lane's level table column (lut + code * 128) -> w',
+//   W = bf16(fp32(w' + alpha * acc)), packed in pairs.
+__device__ __forceinline__ uint4 merge8(uint32_t codes, const uint32_t* acc, float alpha, uint32_t lut) {
+  uint4 o;
+  asm("{\n\t"
+      ".reg .b32 lo, hi, c<8>, a<8>;\n\t"
+      ".reg .f32 w<8>, v<8>;\n\t"
+      "and.b32 lo, %4, 0x0F0F0F0F;\n\t"
+      "shr.b32 hi, %4, 4;\n\t"
+      "and.b32 hi, hi, 0x0F0F0F0F;\n\t"
+      "prmt.b32 c0, lo, 0, 17472;\n\t"
+      "prmt.b32 c1, hi, 0, 17472;\n\t"
+      "prmt.b32 c2, lo, 0, 17473;\n\t"
+      "prmt.b32 c3, hi, 0, 17473;\n\t"
+      "prmt.b32 c4, lo, 0, 17474;\n\t"
+      "prmt.b32 c5, hi, 0, 17474;\n\t"
+      "prmt.b32 c6, lo, 0, 17475;\n\t"
+      "prmt.b32 c7, hi, 0, 17475;\n\t"
+      "mad.lo.u32 a0, c0, 128, %14;\n\t"
+      "mad.lo.u32 a1, c1, 128, %14;\n\t"
+      "mad.lo.u32 a2, c2, 128, %14;\n\t"
+      "mad.lo.u32 a3, c3, 128, %14;\n\t"
+      "mad.lo.u32 a4, c4, 128, %14;\n\t"
+      "mad.lo.u32 a5, c5, 128, %14;\n\t"
+      "mad.lo.u32 a6, c6, 128, %14;\n\t"
+      "mad.lo.u32 a7, c7, 128, %14;\n\t"
+      "ld.shared.f32 w0, [a0];\n\t"
+      "ld.shared.f32 w1, [a1];\n\t"
+      "ld.shared.f32 w2, [a2];\n\t"
+      "ld.shared.f32 w3, [a3];\n\t"
+      "ld.shared.f32 w4, [a4];\n\t"
+      "ld.shared.f32 w5, [a5];\n\t"
+      "ld.shared.f32 w6, [a6];\n\t"
+      "ld.shared.f32 w7, [a7];\n\t"
+      "fma.rn.f32 v0, %13, %5, w0;\n\t"
+      "fma.rn.f32 v1, %13, %6, w1;\n\t"
+      "fma.rn.f32 v2, %13, %7, w2;\n\t"
+      "fma.rn.f32 v3, %13, %8, w3;\n\t"
+      "fma.rn.f32 v4, %13, %9, w4;\n\t"
+      "fma.rn.f32 v5, %13, %10, w5;\n\t"
+      "fma.rn.f32 v6, %13, %11, w6;\n\t"
+      "fma.rn.f32 v7, %13, %12, w7;\n\t"
+      "cvt.rn.bf16x2.f32 %0, v1, v0;\n\t"
+      "cvt.rn.bf16x2.f32 %1, v3, v2;\n\t"
+      "cvt.rn.bf16x2.f32 %2, v5, v4;\n\t"
+      "cvt.rn.bf16x2.f32 %3, v7, v6;\n\t"
+      "}"
+      : "=r"(o.x), "=r"(o.y), "=r"(o.z), "=r"(o.w)
+      : "r"(codes), "f"(__uint_as_float(acc[0])), "f"(__uint_as_float(acc[1])), "f"(__uint_as_float(acc[2])),
+        "f"(__uint_as_float(acc[3])), "f"(__uint_as_float(acc[4])), "f"(__uint_as_float(acc[5])),
+        "f"(__uint_as_float(acc[6])), "f"(__uint_as_float(acc[7])), "f"(alpha), "r"(lut));
+  return o;
+}
+
 template <bool kMerge, int KS>
 __global__ void __launch_bounds__(kDeployThreads, 1)
     lora_deploy_kernel(const __grid_constant__ CUtensorMap tmOpA, const __grid_constant__ CUtensorMap tmOpB,
@@ -228,6 +284,7 @@ __global__ void __launch_bounds__(kDeployThreads, 1)
     const int row = quarter * 32 + lane;
     const int kb = p.k / kBlock;                  // blocks per row of W
     const float mu = kMerge ? p.mean[0] : 0.f;
+    const uint32_t lut_lane = smem_u32(&s_wlut[kMerge ? ew : 0][0][lane]);
     uint8_t* stg = gOut + ew * 4096;
     const uint32_t stg_s = sOut + (uint32_t)ew * 4096u;
     // raw scale inputs of this thread's block, loaded one tile ahead so their
@@ -266,40 +323,34 @@ __global__ void __launch_bounds__(kDeployThreads, 1)
       // the lanes leave together (the TMEM loads below are warp-collective)
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
-      uint32_t vv[2][32];
       const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(s * 256);
-      tmem_ld_32x32b_x32(taddr + (uint32_t)(cA * 32), vv[0]);
-      tmem_ld_32x32b_x32(taddr + (uint32_t)((cA + 1) * 32), vv[1]);
       // merge: the store that last read this warp's staging box is done
       if (kMerge && it > 0 && lane == 0) bulk_wait_group_read0();
-      tmem_ld_wait();
-      // accumulator drained
-      tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&acc_empty[s]));
       uint8_t* io = gIo + s * Cfg::kIo;
       // output rows of the box: merge -> staging (32 rows of 128 B); unmerge
       // -> in place, rows quarter*32.. of the W box bxi
       uint8_t* obox = kMerge ? stg : io + bxi * 16384 + quarter * 4096;
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
-        const uint32_t (&v)[32] = vv[h];
+        // one 32-column chunk per TMEM round trip keeps the register count low
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(taddr + (uint32_t)((cA + h) * 32), v);
+        tmem_ld_wait();
+        if (h == 1) {
+          // accumulator drained
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(smem_u32(&acc_empty[s]));
+        }
         float wf[32];                         // the 32 inputs w' (merge) or W (unmerge) as fp32
         if (kMerge) {
           const uint4 cw = *reinterpret_cast<const uint4*>(io + sw128(row, cA + h));
           const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const uint32_t lo = words[q] & 0x0F0F0F0Fu;          // byte j = code(8q + 2j)
-            const uint32_t hi = (words[q] >> 4) & 0x0F0F0F0Fu;   // byte j = code(8q + 2j + 1)
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const uint32_t cl = __byte_perm(lo, 0u, 0x4440u + j);
-              const uint32_t ch = __byte_perm(hi, 0u, 0x4440u + j);
-              wf[8 * q + 2 * j] = s_wlut[kMerge ? ew : 0][cl][lane];
-              wf[8 * q + 2 * j + 1] = s_wlut[kMerge ? ew : 0][ch][lane];
-            }
-          }
+          for (int q = 0; q < 4; ++q)
+            *reinterpret_cast<uint4*>(obox + sw128(lane, h * 4 + q)) = merge8(words[q], v + 8 * q, p.alpha, lut_lane);
+          continue;
         } else {
 #pragma unroll
           for (int q = 0; q < 4; ++q) {

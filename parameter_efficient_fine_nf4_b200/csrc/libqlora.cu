@@ -155,8 +155,14 @@ cudaError_t set_gemm_attrs() {
 
 template <bool kMerge, int KS>
 cudaError_t set_deploy_attrs() {
-  return cudaFuncSetAttribute(lora_deploy_kernel<kMerge, KS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              DeployCfg<kMerge, KS>::kSmemBytes);
+  const cudaError_t e = cudaFuncSetAttribute(lora_deploy_kernel<kMerge, KS>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             DeployCfg<kMerge, KS>::kSmemBytes);
+  if (e != cudaSuccess) return e;
+  // the kernel's register cap must leave room for its whole block
+  cudaFuncAttributes fa;
+  if (cudaFuncGetAttributes(&fa, lora_deploy_kernel<kMerge, KS>) != cudaSuccess) return cudaErrorInvalidValue;
+  return fa.maxThreadsPerBlock >= kDeployThreads ? cudaSuccess : cudaErrorLaunchOutOfResources;
 }
 
 int ensure_device() {
@@ -642,8 +648,8 @@ int qlora_nf4_quantize(const float* W0, int64_t d, int64_t k, int block, qlora_n
   const double bytes1 = (double)d * k * 4.5 + (double)n_b * 4;
   if (cudaMemsetAsync(ticket, 0, sizeof(unsigned int), st) != cudaSuccess) return QLORA_ERR_CUDA;
   QLORA_TRY(launch("nf4_quantize_phase1", 0.0, bytes1, st, [&] {
-    nf4_quantize_phase1<<<(unsigned)n_g, 256, 0, st>>>(W0, n_b, reinterpret_cast<uint32_t*>(out->codes),
-                                                       absmax, gsum, ticket, out->mean, T.enc);
+    nf4_quantize_phase1<<<(unsigned)std::min<int64_t>(n_g, 4 * (int64_t)current_sms()), 256, 0, st>>>(
+        W0, n_b, n_g, reinterpret_cast<uint32_t*>(out->codes), absmax, gsum, ticket, out->mean, T.enc);
   }));
   QLORA_TRY(launch("nf4_quantize_dq", 0.0, (double)n_b * 5 + n_g * 4, st, [&] {
     nf4_quantize_dq<<<(unsigned)cdiv(n_g, kDqGroups), 256, 0, st>>>(absmax, n_g, n_b, out->mean,

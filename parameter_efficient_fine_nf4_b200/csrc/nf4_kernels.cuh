@@ -71,38 +71,124 @@ __device__ __forceinline__ uint32_t enc_code(float x, const uint8_t* s_base, con
 // address, bits(t) * 4 + K with t = x * 16 + 1.5 * 2^23 and
 // K = table - (0x4B400000 - 16) * 4 (mod 2^32).  It is used only where
 // |x| <= 1 is guaranteed, so the address needs no clamp.
-// Eight codes of one thread's weights, packed (element i in nibble i): all
-// quotients and addresses first, then the sixteen table loads, then the
-// assembly code = base + (x >= thr), each summed into its nibble.
-__device__ __forceinline__ uint32_t encode8_fast(const float (&w)[8], float m, uint32_t K) {
-  const float y = __frcp_rn(m);
-  float x[8];
-  uint32_t addr[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    x[i] = div_markstein(w[i], m, y);
-    addr[i] = (uint32_t)__float_as_int(__fmaf_rn(x[i], 16.0f, 12582912.0f)) * 4u + K;
-  }
-  float thr[8];
-  uint32_t base[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    asm("ld.shared.f32 %0, [%1];" : "=f"(thr[i]) : "r"(addr[i]));
-    asm("ld.shared.u32 %0, [%1+132];" : "=r"(base[i]) : "r"(addr[i]));
-  }
-  uint32_t packed = base[0];
-#pragma unroll
-  for (int i = 1; i < 8; ++i) packed += base[i] << (4 * i);
-#pragma unroll
-  for (int i = 0; i < 8; ++i)
-    asm("{\n\t.reg .pred p;\n\tsetp.ge.f32 p, %1, %2;\n\t@p add.u32 %0, %0, %3;\n\t}"
-        : "+r"(packed) : "f"(x[i]), "f"(thr[i]), "r"(1u << (4 * i)));
+// Eight codes of one thread's weights, packed (element i in nibble i), as
+// one block of PTX so that nothing but the arithmetic below is emitted:
+//   x_i  = RN(w_i / m)   Markstein: q = w y, r = w - m q (exact), x = q + r y
+//   t_i  = x_i * 16 + 1.5 * 2^23        (rint(16 x_i) in the low bits)
+//   a_i  = bits(t_i) * 4 + K            (address of bin rint(16 x_i) + 16)
+//   code = fbase[a_i] + (x_i >= fthr[a_i]),  summed into nibble i (no carries)
+__device__ __forceinline__ uint32_t encode8_fast(const float* w, float m, float y, uint32_t K) {
+  uint32_t packed;
+  asm("{\n\t"
+      ".reg .f32 nm, q<8>, r<8>, x<8>, t<8>, th<8>;\n\t"
+      ".reg .b32 a<8>, b<8>;\n\t"
+      ".reg .pred p<8>;\n\t"
+      "neg.f32 nm, %9;\n\t"
+      "mul.rn.f32 q0, %1, %10;\n\t"
+      "fma.rn.f32 r0, nm, q0, %1;\n\t"
+      "fma.rn.f32 x0, r0, %10, q0;\n\t"
+      "fma.rn.f32 t0, x0, 0f41800000, 0f4B400000;\n\t"
+      "mov.b32 a0, t0;\n\t"
+      "mad.lo.u32 a0, a0, 4, %11;\n\t"
+      "mul.rn.f32 q1, %2, %10;\n\t"
+      "fma.rn.f32 r1, nm, q1, %2;\n\t"
+      "fma.rn.f32 x1, r1, %10, q1;\n\t"
+      "fma.rn.f32 t1, x1, 0f41800000, 0f4B400000;\n\t"
+      "mov.b32 a1, t1;\n\t"
+      "mad.lo.u32 a1, a1, 4, %11;\n\t"
+      "mul.rn.f32 q2, %3, %10;\n\t"
+      "fma.rn.f32 r2, nm, q2, %3;\n\t"
+      "fma.rn.f32 x2, r2, %10, q2;\n\t"
+      "fma.rn.f32 t2, x2, 0f41800000, 0f4B400000;\n\t"
+      "mov.b32 a2, t2;\n\t"
+      "mad.lo.u32 a2, a2, 4, %11;\n\t"
+      "mul.rn.f32 q3, %4, %10;\n\t"
+      "fma.rn.f32 r3, nm, q3, %4;\n\t"
+      "fma.rn.f32 x3, r3, %10, q3;\n\t"
+      "fma.rn.f32 t3, x3, 0f41800000, 0f4B400000;\n\t"
+      "mov.b32 a3, t3;\n\t"
+      "mad.lo.u32 a3, a3, 4, %11;\n\t"
+      "mul.rn.f32 q4, %5, %10;\n\t"
+      "fma.rn.f32 r4, nm, q4, %5;\n\t"
+      "fma.rn.f32 x4, r4, %10, q4;\n\t"
+      "fma.rn.f32 t4, x4, 0f41800000, 0f4B400000;\n\t"
+      "mov.b32 a4, t4;\n\t"
+      "mad.lo.u32 a4, a4, 4, %11;\n\t"
+      "mul.rn.f32 q5, %6, %10;\n\t"
+      "fma.rn.f32 r5, nm, q5, %6;\n\t"
+      "fma.rn.f32 x5, r5, %10, q5;\n\t"
+      "fma.rn.f32 t5, x5, 0f41800000, 0f4B400000;\n\t"
+      "mov.b32 a5, t5;\n\t"
+      "mad.lo.u32 a5, a5, 4, %11;\n\t"
+      "mul.rn.f32 q6, %7, %10;\n\t"
+      "fma.rn.f32 r6, nm, q6, %7;\n\t"
+      "fma.rn.f32 x6, r6, %10, q6;\n\t"
+      "fma.rn.f32 t6, x6, 0f41800000, 0f4B400000;\n\t"
+      "mov.b32 a6, t6;\n\t"
+      "mad.lo.u32 a6, a6, 4, %11;\n\t"
+      "mul.rn.f32 q7, %8, %10;\n\t"
+      "fma.rn.f32 r7, nm, q7, %8;\n\t"
+      "fma.rn.f32 x7, r7, %10, q7;\n\t"
+      "fma.rn.f32 t7, x7, 0f41800000, 0f4B400000;\n\t"
+      "mov.b32 a7, t7;\n\t"
+      "mad.lo.u32 a7, a7, 4, %11;\n\t"
+      "ld.shared.f32 th0, [a0];\n\t"
+      "ld.shared.u32 b0, [a0+132];\n\t"
+      "ld.shared.f32 th1, [a1];\n\t"
+      "ld.shared.u32 b1, [a1+132];\n\t"
+      "ld.shared.f32 th2, [a2];\n\t"
+      "ld.shared.u32 b2, [a2+132];\n\t"
+      "ld.shared.f32 th3, [a3];\n\t"
+      "ld.shared.u32 b3, [a3+132];\n\t"
+      "ld.shared.f32 th4, [a4];\n\t"
+      "ld.shared.u32 b4, [a4+132];\n\t"
+      "ld.shared.f32 th5, [a5];\n\t"
+      "ld.shared.u32 b5, [a5+132];\n\t"
+      "ld.shared.f32 th6, [a6];\n\t"
+      "ld.shared.u32 b6, [a6+132];\n\t"
+      "ld.shared.f32 th7, [a7];\n\t"
+      "ld.shared.u32 b7, [a7+132];\n\t"
+      "setp.ge.f32 p0, x0, th0;\n\t"
+      "setp.ge.f32 p1, x1, th1;\n\t"
+      "setp.ge.f32 p2, x2, th2;\n\t"
+      "setp.ge.f32 p3, x3, th3;\n\t"
+      "setp.ge.f32 p4, x4, th4;\n\t"
+      "setp.ge.f32 p5, x5, th5;\n\t"
+      "setp.ge.f32 p6, x6, th6;\n\t"
+      "setp.ge.f32 p7, x7, th7;\n\t"
+      "mov.u32 %0, b0;\n\t"
+      "shl.b32 b1, b1, 4;\n\t"
+      "add.u32 %0, %0, b1;\n\t"
+      "shl.b32 b2, b2, 8;\n\t"
+      "add.u32 %0, %0, b2;\n\t"
+      "shl.b32 b3, b3, 12;\n\t"
+      "add.u32 %0, %0, b3;\n\t"
+      "shl.b32 b4, b4, 16;\n\t"
+      "add.u32 %0, %0, b4;\n\t"
+      "shl.b32 b5, b5, 20;\n\t"
+      "add.u32 %0, %0, b5;\n\t"
+      "shl.b32 b6, b6, 24;\n\t"
+      "add.u32 %0, %0, b6;\n\t"
+      "shl.b32 b7, b7, 28;\n\t"
+      "add.u32 %0, %0, b7;\n\t"
+      "@p0 add.u32 %0, %0, 1;\n\t"
+      "@p1 add.u32 %0, %0, 16;\n\t"
+      "@p2 add.u32 %0, %0, 256;\n\t"
+      "@p3 add.u32 %0, %0, 4096;\n\t"
+      "@p4 add.u32 %0, %0, 65536;\n\t"
+      "@p5 add.u32 %0, %0, 1048576;\n\t"
+      "@p6 add.u32 %0, %0, 16777216;\n\t"
+      "@p7 add.u32 %0, %0, 268435456;\n\t"
+      "}"
+      : "=r"(packed)
+      : "f"(w[0]), "f"(w[1]), "f"(w[2]), "f"(w[3]), "f"(w[4]), "f"(w[5]), "f"(w[6]), "f"(w[7]),
+        "f"(m), "f"(y), "r"(K));
   return packed;
 }
 
 // Eight codes by the general route (any block absmax): IEEE division and the
 // clamped encoder; an all-zero (or NaN) block gives the zero level.
-__device__ __forceinline__ uint32_t encode8_general(const float (&w)[8], float m, const uint8_t* s_base,
+__device__ __forceinline__ uint32_t encode8_general(const float* w, float m, const uint8_t* s_base,
                                                     const float* s_thr) {
   if (!(m > 0.f)) return 0x77777777u;
   uint32_t packed = 0;
@@ -123,43 +209,51 @@ __device__ __forceinline__ float max_abs_nan(float a, float b) {
 // that takes the final ticket, so every group sum is in memory): S is the
 // float64 pairwise tree over the n_g group sums padded with zeros to
 // P = max(2^ceil(log2 n_g), 1024) leaves (zero leaves and zero subtrees add
-// exactly nothing, so the padding does not change S).  Each warp takes
-// aligned chunks of 1024 leaves: lane l sums its 32 consecutive leaves as a
-// pairwise tree in registers and a shuffle tree joins the lanes; a
-// shared-memory tree then joins the P/1024 chunk sums.  mean = fp32(S / n_b).
+// exactly nothing, so the padding does not change S).  mean = fp32(S / n_b).
 // ---------------------------------------------------------------------------
 constexpr int kMeanChunks = 1024;      // P / 1024 <= 1024 for n_g <= 2^20
 
-__device__ __noinline__ void pairwise_mean(const double* group_sum, int64_t n_g, int64_t n_b,
-                                           float* mean_out, double* s_v) {
+// Lane l of a warp: the pairwise tree over the 8 consecutive leaves
+// first + 8 l .. first + 8 l + 7 (zero beyond n), then the shuffle tree over
+// the lanes: lane 0 returns the tree over the 256 leaves from `first`.
+__device__ __forceinline__ double warp_tree256(const double* v, int64_t first, int64_t n, int lane) {
+  const int64_t i0 = first + 8 * lane;
+  double a[8];
+#pragma unroll
+  for (int j = 0; j < 8; j += 2) {
+    const int64_t i = i0 + j;
+    if (i + 1 < n) {
+      const double2 t = __ldcg(reinterpret_cast<const double2*>(v + i));
+      a[j] = t.x;
+      a[j + 1] = t.y;
+    } else {
+      a[j] = (i < n) ? __ldcg(v + i) : 0.0;
+      a[j + 1] = 0.0;
+    }
+  }
+  double s = ((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]));
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) s = s + __shfl_down_sync(0xffffffffu, s, off);
+  return s;
+}
+
+// Run by one whole CTA.  Each warp takes aligned chunks of 1024 leaves as
+// the tree of four 256-leaf subtrees; a shared-memory tree joins the P/1024
+// chunk sums in s_v.
+__device__ __forceinline__ void pairwise_mean(const double* group_sum, int64_t n_g, int64_t n_b,
+                                              float* mean_out, double* s_v) {
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
   int64_t P = 1024;
   while (P < n_g) P <<= 1;
   const int nch = (int)(P / 1024);
   for (int c = warp; c < nch; c += (int)(blockDim.x >> 5)) {
-    const int64_t first = (int64_t)c * 1024 + lane * 32;
-    double a[32];
-#pragma unroll
-    for (int j = 0; j < 32; j += 2) {
-      const int64_t i = first + j;
-      if (i + 1 < n_g) {
-        const double2 t = __ldcg(reinterpret_cast<const double2*>(group_sum + i));
-        a[j] = t.x;
-        a[j + 1] = t.y;
-      } else {
-        a[j] = (i < n_g) ? __ldcg(group_sum + i) : 0.0;
-        a[j + 1] = 0.0;
-      }
-    }
-#pragma unroll
-    for (int st = 1; st < 32; st <<= 1)
-#pragma unroll
-      for (int j = 0; j < 32; j += 2 * st) a[j] = a[j] + a[j + st];
-    double sum = a[0];
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) sum = sum + __shfl_down_sync(0xffffffffu, sum, off);
-    if (lane == 0) s_v[c] = sum;
+    const int64_t first = (int64_t)c * 1024;
+    const double s0 = warp_tree256(group_sum, first, n_g, lane);
+    const double s1 = warp_tree256(group_sum, first + 256, n_g, lane);
+    const double s2 = warp_tree256(group_sum, first + 512, n_g, lane);
+    const double s3 = warp_tree256(group_sum, first + 768, n_g, lane);
+    if (lane == 0) s_v[c] = (s0 + s1) + (s2 + s3);
   }
   __syncthreads();
   for (int st = 1; st < nch; st <<= 1) {
@@ -170,16 +264,17 @@ __device__ __noinline__ void pairwise_mean(const double* group_sum, int64_t n_g,
 }
 
 // ---------------------------------------------------------------------------
-// Phase 1: one CTA per group of 256 blocks (16384 weights).  8 threads per
-// block, 8 consecutive weights per thread.  Writes packed codes, the fp32
-// block absmax (scratch) and the fp64 pairwise sum of the group's absmax.
+// Phase 1: persistent CTAs, each taking groups of 256 blocks (16384 weights)
+// in turn.  8 threads per block, 8 consecutive weights per thread.  Writes
+// packed codes, the fp32 block absmax (scratch) and the fp64 pairwise sum of
+// each group's absmax.
 //
 // Fast path (every block of the warp has its absmax a in [2^-125, 2^125]):
 // x = w / a by Markstein's correction from y = RN(1/a) (all intermediates
 // normal in that range, and |x| <= 1 because |w| <= a), then encode8_fast.
 // Otherwise the warp takes the general route (needed for an all-zero,
 // subnormal or huge absmax, or a NaN, which the NaN-propagating maximum
-// exposes).  Both give RN(w / a) and the same code.  Only the last CTA
+// exposes).  Both give RN(w / a) and the same code.  Only the last group
 // checks bounds.  The CTA that finishes last also forms the mean.
 // ---------------------------------------------------------------------------
 template <bool kTail>
@@ -209,8 +304,7 @@ __device__ __forceinline__ void quantize_group(const float* __restrict__ W0, int
     for (int p = 0; p < 4; ++p) {
       const int lb = (half * 4 + p) * 32 + lb0;
       const int64_t b = g * kBlock2 + lb;
-      const float w[8] = {v[p][0].x, v[p][0].y, v[p][0].z, v[p][0].w,
-                          v[p][1].x, v[p][1].y, v[p][1].z, v[p][1].w};
+      const float* w = reinterpret_cast<const float*>(&v[p][0]);
       float m = fabsf(w[0]);
 #pragma unroll
       for (int i = 1; i < 8; ++i) m = max_abs_nan(m, w[i]);
@@ -219,7 +313,7 @@ __device__ __forceinline__ void quantize_group(const float* __restrict__ W0, int
       m = max_abs_nan(m, __shfl_xor_sync(0xffffffffu, m, 4));
       const bool fast = m >= 0x1p-125f && m <= 0x1p125f;
       // (the general route gives the same codes for blocks the fast one takes)
-      const uint32_t packed = __all_sync(0xffffffffu, fast) ? encode8_fast(w, m, K)
+      const uint32_t packed = __all_sync(0xffffffffu, fast) ? encode8_fast(w, m, __frcp_rn(m), K)
                                                             : encode8_general(w, m, s_base, s_thr);
       if (!kTail || b < n_b) {
         codes_u32[b * 8 + sub] = packed;
@@ -230,8 +324,8 @@ __device__ __forceinline__ void quantize_group(const float* __restrict__ W0, int
   }
 }
 
-__global__ void __launch_bounds__(256, 4) nf4_quantize_phase1(
-    const float* __restrict__ W0, int64_t n_b, uint32_t* __restrict__ codes_u32,
+__global__ void __launch_bounds__(256) nf4_quantize_phase1(
+    const float* __restrict__ W0, int64_t n_b, int64_t n_g, uint32_t* __restrict__ codes_u32,
     float* __restrict__ absmax, double* __restrict__ group_sum, unsigned int* __restrict__ ticket,
     float* __restrict__ mean_out, const __grid_constant__ EncTable tab) {
   __shared__ double s_v[kMeanChunks];
@@ -239,7 +333,7 @@ __global__ void __launch_bounds__(256, 4) nf4_quantize_phase1(
   __shared__ uint32_t s_fast[2 * kFastBins];      // fthr (as bits), then fbase
   __shared__ uint8_t s_base[kEncBins + 3];
   __shared__ float s_thr[16];
-  __shared__ float s_abs[kBlock2];
+  __shared__ float s_abs[2][kBlock2];             // block constants of two groups in turn
   const int tid = threadIdx.x;
   if (tid < kFastBins) {
     s_fast[tid] = __float_as_uint(tab.fthr[tid]);
@@ -249,33 +343,39 @@ __global__ void __launch_bounds__(256, 4) nf4_quantize_phase1(
   if (tid < 16) s_thr[tid] = tab.thr[tid];
   __syncthreads();
   const uint32_t K = smem_u32(s_fast) - (uint32_t)(0x4B400000 - 16) * 4u;
-  const int64_t g = blockIdx.x;
-  if ((g + 1) * kBlock2 <= n_b)
-    quantize_group<false>(W0, n_b, g, codes_u32, absmax, s_abs, K, s_base, s_thr);
-  else
-    quantize_group<true>(W0, n_b, g, codes_u32, absmax, s_abs, K, s_base, s_thr);
-  __syncthreads();
-  if (tid < 32) {
-    // pairwise tree over the 256 constants: lane l sums leaves 8l..8l+7, then
-    // the lanes are combined in halves (shfl_down by 1, 2, 4, 8, 16)
-    double a[8];
+  // persistent: this CTA takes groups blockIdx.x, blockIdx.x + gridDim.x, ...
+  int it = 0;
+  for (int64_t g = blockIdx.x; g < n_g; g += gridDim.x, ++it) {
+    float* sa = s_abs[it & 1];
+    if ((g + 1) * kBlock2 <= n_b)
+      quantize_group<false>(W0, n_b, g, codes_u32, absmax, sa, K, s_base, s_thr);
+    else
+      quantize_group<true>(W0, n_b, g, codes_u32, absmax, sa, K, s_base, s_thr);
+    // one barrier per group: warp 0 reads this group's constants while the
+    // other warps already fill the other half of s_abs with the next group
+    __syncthreads();
+    if (tid < 32) {
+      // pairwise tree over the 256 constants: lane l sums leaves 8l..8l+7,
+      // then the lanes are combined in halves (shfl_down by 1, 2, 4, 8, 16)
+      double a[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) a[i] = (double)s_abs[tid * 8 + i];
-    double s = ((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]));
+      for (int i = 0; i < 8; ++i) a[i] = (double)sa[tid * 8 + i];
+      double s = ((a[0] + a[1]) + (a[2] + a[3])) + ((a[4] + a[5]) + (a[6] + a[7]));
 #pragma unroll
-    for (int off = 1; off < 32; off <<= 1) s = s + __shfl_down_sync(0xffffffffu, s, off);
-    if (tid == 0) {
-      group_sum[g] = s;
-      // publish the sum, then take a ticket: the CTA with the last ticket
-      // sees every group sum and forms the mean
-      __threadfence();
-      s_last = atomicAdd(ticket, 1u) == gridDim.x - 1;
+      for (int off = 1; off < 32; off <<= 1) s = s + __shfl_down_sync(0xffffffffu, s, off);
+      if (tid == 0) group_sum[g] = s;
     }
+  }
+  // publish this CTA's sums, then take a ticket: the CTA with the last ticket
+  // sees every group sum and forms the mean
+  if (tid == 0) {
+    __threadfence();
+    s_last = atomicAdd(ticket, 1u) == gridDim.x - 1;
   }
   __syncthreads();
   if (s_last) {
     __threadfence();
-    pairwise_mean(group_sum, (int64_t)gridDim.x, n_b, mean_out, s_v);
+    pairwise_mean(group_sum, n_g, n_b, mean_out, s_v);
   }
 }
 
@@ -292,6 +392,7 @@ __global__ void __launch_bounds__(256) nf4_quantize_dq(const float* __restrict__
                                                        uint8_t* __restrict__ absmax_q,
                                                        float* __restrict__ scale2) {
   __shared__ float s_max[kDqGroups][8];
+  __shared__ float s_s1[kDqGroups], s_y1[kDqGroups];
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
   const float mu = mean[0];
@@ -310,21 +411,33 @@ __global__ void __launch_bounds__(256) nf4_quantize_dq(const float* __restrict__
     if (lane == 0) s_max[i][warp] = m;
   }
   __syncthreads();
+  if (tid < kDqGroups) {
+    // one thread per group: scale2 and, where it is a comfortably normal
+    // number, y = RN(1/scale2) for the quotients below
+    float c1 = s_max[tid][0];
+#pragma unroll
+    for (int w = 1; w < 8; ++w) c1 = fmaxf(c1, s_max[tid][w]);
+    const float s1 = (c1 > 0.f) ? __fdiv_rn(c1, 448.0f) : 0.f;
+    s_s1[tid] = s1;
+    s_y1[tid] = (s1 >= 0x1p-100f && s1 <= 0x1p100f) ? __frcp_rn(s1) : 0.f;
+    if (g0 + tid < n_g) scale2[g0 + tid] = s1;
+  }
+  __syncthreads();
 #pragma unroll
   for (int i = 0; i < kDqGroups; ++i) {
-    const int64_t g = g0 + i;
-    if (g < n_g) {
-      float c1 = s_max[i][0];
-#pragma unroll
-      for (int w = 1; w < 8; ++w) c1 = fmaxf(c1, s_max[i][w]);
-      const float s1 = (c1 > 0.f) ? __fdiv_rn(c1, 448.0f) : 0.f;
-      if (tid == 0) scale2[g] = s1;
-      const int64_t b = g * kBlock2 + tid;
-      if (b < n_b) {
-        uint8_t code = 0;
-        if (s1 > 0.f) code = (uint8_t)__nv_cvt_float_to_fp8(__fdiv_rn(cen[i], s1), __NV_SATFINITE, __NV_E4M3);
-        absmax_q[b] = code;
+    const int64_t b = (g0 + i) * kBlock2 + tid;
+    if (g0 + i < n_g && b < n_b) {
+      // x = RN(cen / scale2): Markstein's correction from y (|x| <= 448, and
+      // a quotient too small for the correction is below E4M3's smallest
+      // step, where both round to a zero of the same sign), else IEEE
+      // division
+      const float s1 = s_s1[i], y1 = s_y1[i];
+      uint8_t code = 0;
+      if (s1 > 0.f) {
+        const float x = (y1 != 0.f) ? div_markstein(cen[i], s1, y1) : __fdiv_rn(cen[i], s1);
+        code = (uint8_t)__nv_cvt_float_to_fp8(x, __NV_SATFINITE, __NV_E4M3);
       }
+      absmax_q[b] = code;
     }
   }
 }
@@ -465,7 +578,7 @@ __global__ void selftest_wait_kernel(unsigned long long limit_ns) {
   __syncthreads();
   if (threadIdx.x == 0) {
     const uint64_t start = globaltimer_ns();
-    while (!mbar_try_wait(smem_u32(&bar), 0)) {
+    while (!mbar_try_wait_suspend(smem_u32(&bar), 0, 100000u)) {
       if (globaltimer_ns() - start > limit_ns) {
         record_status(QLORA_ERR_TIMEOUT);
         break;

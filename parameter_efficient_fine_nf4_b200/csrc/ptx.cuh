@@ -66,24 +66,37 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Same test, but the thread may be suspended for up to `hint_ns` while the
+// phase is still incomplete (it resumes as soon as the phase completes), so
+// a waiting warp takes no issue slots from the warps doing work.
+__device__ __forceinline__ bool mbar_try_wait_suspend(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Wait for the phase with the given parity to complete.  Returns false (and
 // records a timeout) if it does not complete within the limit, or at once if
-// `abort_flag` is already set by another role of the same CTA.
+// `abort_flag` is already set by another role of the same CTA.  Each try may
+// suspend the thread for at most 0.1 ms, so the limit is checked often.
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
                                                   volatile int* abort_flag) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t start = globaltimer_ns();
   const uint64_t limit = g_wait_limit_ns;
-  uint32_t spins = 0;
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if (((++spins) & 63u) == 0u) {
-      if (abort_flag != nullptr && *abort_flag) return false;
-      if (globaltimer_ns() - start > limit) {
-        record_status(QLORA_ERR_TIMEOUT);
-        if (abort_flag != nullptr) *abort_flag = 1;
-        return false;
-      }
+    if (mbar_try_wait_suspend(bar, parity, 100000u)) return true;
+    if (abort_flag != nullptr && *abort_flag) return false;
+    if (globaltimer_ns() - start > limit) {
+      record_status(QLORA_ERR_TIMEOUT);
+      if (abort_flag != nullptr) *abort_flag = 1;
+      return false;
     }
   }
 }
