@@ -337,32 +337,65 @@ def run_ours(args):
     value = flops_rank * world / (ms / 1e3) / 1e12
     tokens_s = T * world / (ms / 1e3)
 
-    # ---- e2e through the public API with host buffers: per step, copy X and
-    # dY of every linear in from pinned memory, run the step, read dA and dB back
+    # ---- e2e through the public API with host buffers: every step copies X
+    # and dY of every linear in from pinned memory and reads dA and dB back.
+    # The copies run on a second stream into one of two device input sets, so
+    # the inputs of step i+1 (and of the second linear) arrive while step i
+    # computes, as a caller streaming micro-batches would run it.
     host_in = [(L["X"].cpu().pin_memory(), L["dY"].cpu().pin_memory()) for L in layers]
     host_out = [(torch.empty_like(L["dA"], device="cpu").pin_memory(),
                  torch.empty_like(L["dB"], device="cpu").pin_memory()) for L in layers]
     h2d = sum(x.numel() * x.element_size() + y.numel() * y.element_size() for x, y in host_in)
     d2h = sum(a.numel() * a.element_size() + b.numel() * b.element_size() for a, b in host_out)
-    e2e_ms = []
-    e2e_steps = max(3, min(args.steps, 5))
+    sets = [[(L["X"], L["dY"]) for L in layers],
+            [(torch.empty_like(L["X"]), torch.empty_like(L["dY"])) for L in layers]]
+    copy_stream = torch.cuda.Stream(device=dev)
+    ev_ready = [[torch.cuda.Event() for _ in layers] for _ in range(2)]
+    ev_free = [torch.cuda.Event() for _ in range(2)]
+
+    def run_layer(L, X, dY):
+        q4.qlora_nf4_quantize(L["W0"], out=L["qw"], ws=L["ws"])
+        q4.qlora_fwd(L["qw"], L["A"], L["B"], cfg.alpha, X, Y=L["Y"], U_save=L["U"], ws=L["ws"])
+        q4.qlora_bwd(L["qw"], L["A"], L["B"], cfg.alpha, X, L["U"], dY, dX=L["dX"],
+                     dA=L["dA"], dB=L["dB"], ws=L["ws"])
+        if world > 1:
+            dist.all_reduce(L["dA"])
+            dist.all_reduce(L["dB"])
+        q4.lora_merge(L["qw"], L["A"], L["B"], cfg.alpha, W_out=L["Wm"], ws=L["ws"])
+        q4.lora_unmerge(L["Wm"], L["A"], L["B"], cfg.alpha, W0_out=L["W0u"], ws=L["ws"])
+
+    def pipelined(n, start_ev):
+        copy_stream.wait_event(start_ev)
+        for i in range(n):
+            b = i % 2
+            with torch.cuda.stream(copy_stream):
+                if i >= 2:
+                    copy_stream.wait_event(ev_free[b])
+                for li, ((hx, hdy), (X, dY)) in enumerate(zip(host_in, sets[b])):
+                    X.copy_(hx, non_blocking=True)
+                    dY.copy_(hdy, non_blocking=True)
+                    ev_ready[b][li].record(copy_stream)
+            for li, L in enumerate(layers):
+                stream.wait_event(ev_ready[b][li])
+                run_layer(L, *sets[b][li])
+            ev_free[b].record(stream)
+            for L, (ha, hb) in zip(layers, host_out):
+                ha.copy_(L["dA"], non_blocking=True)
+                hb.copy_(L["dB"], non_blocking=True)
+
+    e2e_steps = max(3, min(args.steps, 8))
     barrier()
-    for i in range(e2e_steps + 1):
+    for timed in (False, True):
         flush.zero_()
         a = torch.cuda.Event(enable_timing=True)
-        b = torch.cuda.Event(enable_timing=True)
+        b_ev = torch.cuda.Event(enable_timing=True)
         a.record(stream)
-        for L, (hx, hdy) in zip(layers, host_in):
-            L["X"].copy_(hx, non_blocking=True)
-            L["dY"].copy_(hdy, non_blocking=True)
-        step()
-        for L, (ha, hb) in zip(layers, host_out):
-            ha.copy_(L["dA"], non_blocking=True)
-            hb.copy_(L["dB"], non_blocking=True)
-        b.record(stream)
-        b.synchronize()
-        if i > 0:
-            e2e_ms.append(a.elapsed_time(b))
+        pipelined(e2e_steps if timed else 2, a)
+        b_ev.record(stream)
+        b_ev.synchronize()
+        torch.cuda.synchronize(dev)
+        if timed:
+            e2e_ms = [a.elapsed_time(b_ev) / e2e_steps]
     barrier()
     te = torch.tensor([statistics.mean(e2e_ms)], device=dev, dtype=torch.float64)
     if world > 1:
@@ -442,7 +475,9 @@ def run_ours(args):
                          "peak_source": f"{peak_src} bf16_tflops_sustained",
                          "launches": g_launches, "ms_per_launch": g_ms / max(1, g_launches)},
             "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
-                    "d2h_bytes_per_step": d2h, "ms_per_step": float(te.item())},
+                    "d2h_bytes_per_step": d2h, "ms_per_step": float(te.item()), "steps": e2e_steps,
+                    "how": "public API, pinned host X/dY in and dA/dB out every step; copies on a "
+                           "second stream into two device input sets, overlapping compute"},
             "gpu_launches": launches // args.steps * args.steps,
             "gpu_launches_per_step": launches / args.steps,
             "clocks": clk,
@@ -460,6 +495,53 @@ def run_ours(args):
     return 0
 
 
+def run_deploy(args):
+    """The HBM-bound rows alone on the config's first linear: quantise, merge,
+    unmerge, doubleDequant (warm-up, then `steps` calls of each, CUDA-event
+    timing through the library profiler).  A diagnostic, not the bench line."""
+    import torch
+    import parameter_efficient_fine_nf4_b200 as q4
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    cfg, _ = workload(args.config)
+    lin = cfg.linears[0]
+    lay = synthetic.make_layer(cfg, 0, with_acts=False)
+    W0 = torch.from_numpy(lay.W0).to(dev)
+    A = torch.from_numpy(lay.A.view(np.int16)).view(torch.bfloat16).to(dev)
+    B = torch.from_numpy(lay.B.view(np.int16)).view(torch.bfloat16).to(dev)
+    qw = q4.NF4Weight(lin.d, lin.k, dev)
+    Wm = torch.empty(lin.d, lin.k, dtype=torch.bfloat16, device=dev)
+    W0u = torch.empty_like(Wm)
+    ws = q4.workspace(max(q4.qlora_quantize_workspace_bytes(lin.d, lin.k),
+                          q4.lora_merge_workspace_bytes(lin.d, lin.k, cfg.r)), dev)
+    ops = {"quantise": (lambda: q4.qlora_nf4_quantize(W0, out=qw, ws=ws), 4.5 + 1 / 64,
+                        ("nf4_quantize_phase1", "nf4_quantize_dq")),
+           "merge": (lambda: q4.lora_merge(qw, A, B, cfg.alpha, W_out=Wm, ws=ws), 2.5 + 1 / 64,
+                     ("lora_merge",)),
+           "unmerge": (lambda: q4.lora_unmerge(Wm, A, B, cfg.alpha, W0_out=W0u, ws=ws), 4.0,
+                       ("lora_unmerge",)),
+           "dequantise": (lambda: q4.qlora_nf4_dequantize(qw, W_out=W0u), 2.5 + 1 / 64,
+                          ("nf4_dequantize",))}
+    peaks, src = read_peaks()
+    hbm = float(peaks.get("hbm_gbs"))
+    out = {"mode": "deploy-only", "config": {"workload": f"{lin.name}: d={lin.d}, k={lin.k}, r={cfg.r}"},
+           "peak_gbs": hbm, "peak_source": f"{src} hbm_gbs"}
+    for name, (fn, bpw, kernels) in ops.items():
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize(dev)
+        q4.qlora_profile_begin()
+        for _ in range(args.steps):
+            fn()
+        st = q4.qlora_profile_end()
+        ms = sum(x["total_ms"] for x in st if x["name"] in kernels) / args.steps
+        gbs = lin.d * lin.k * bpw / 1e9 / (ms / 1e3)
+        out[name] = {"us_per_call": 1e3 * ms, "gbs": gbs, "frac": gbs / hbm, "bytes_per_weight": bpw}
+    assert q4.qlora_get_device_status() == 0
+    print(json.dumps(out), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -468,11 +550,15 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", type=int, default=4)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--deploy-only", action="store_true",
+                    help="time only quantise, merge, unmerge and doubleDequant of the first linear")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
     if args.impl == "reference":
         return run_reference(args)
+    if args.deploy_only:
+        return run_deploy(args)
     return run_ours(args)
 
 
