@@ -280,21 +280,37 @@ def run_ours(args):
                      q4.qlora_bwd_workspace_bytes(lin.d, lin.k, cfg.r, T),
                      q4.lora_merge_workspace_bytes(lin.d, lin.k, cfg.r))
         L["ws"] = q4.workspace(nbytes, dev)
+        if args.base == "bf16":
+            L["Wb"] = L["W0"].to(torch.bfloat16)
         layers.append(L)
     flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    def step():
-        for L in layers:
+    plain = args.base == "bf16"
+
+    def run_layer(L, X, dY):
+        """One pass of the path over one linear: QLoRA (quantise, forward,
+        backward, merge, unmerge) or, with --base bf16, plain LoRA (forward,
+        backward on the bf16 base)."""
+        if plain:
+            q4.lora_fwd(L["Wb"], L["A"], L["B"], cfg.alpha, X, Y=L["Y"], U_save=L["U"], ws=L["ws"])
+            q4.lora_bwd(L["Wb"], L["A"], L["B"], cfg.alpha, X, L["U"], dY, dX=L["dX"],
+                        dA=L["dA"], dB=L["dB"], ws=L["ws"])
+        else:
             q4.qlora_nf4_quantize(L["W0"], out=L["qw"], ws=L["ws"])
-            q4.qlora_fwd(L["qw"], L["A"], L["B"], cfg.alpha, L["X"], Y=L["Y"], U_save=L["U"], ws=L["ws"])
-            q4.qlora_bwd(L["qw"], L["A"], L["B"], cfg.alpha, L["X"], L["U"], L["dY"], dX=L["dX"],
+            q4.qlora_fwd(L["qw"], L["A"], L["B"], cfg.alpha, X, Y=L["Y"], U_save=L["U"], ws=L["ws"])
+            q4.qlora_bwd(L["qw"], L["A"], L["B"], cfg.alpha, X, L["U"], dY, dX=L["dX"],
                          dA=L["dA"], dB=L["dB"], ws=L["ws"])
-            if world > 1:
-                dist.all_reduce(L["dA"])
-                dist.all_reduce(L["dB"])
+        if world > 1:
+            dist.all_reduce(L["dA"])
+            dist.all_reduce(L["dB"])
+        if not plain:
             q4.lora_merge(L["qw"], L["A"], L["B"], cfg.alpha, W_out=L["Wm"], ws=L["ws"])
             q4.lora_unmerge(L["Wm"], L["A"], L["B"], cfg.alpha, W0_out=L["W0u"], ws=L["ws"])
+
+    def step():
+        for L in layers:
+            run_layer(L, L["X"], L["dY"])
 
     def barrier():
         if world > 1:
@@ -353,17 +369,6 @@ def run_ours(args):
     ev_ready = [[torch.cuda.Event() for _ in layers] for _ in range(2)]
     ev_free = [torch.cuda.Event() for _ in range(2)]
 
-    def run_layer(L, X, dY):
-        q4.qlora_nf4_quantize(L["W0"], out=L["qw"], ws=L["ws"])
-        q4.qlora_fwd(L["qw"], L["A"], L["B"], cfg.alpha, X, Y=L["Y"], U_save=L["U"], ws=L["ws"])
-        q4.qlora_bwd(L["qw"], L["A"], L["B"], cfg.alpha, X, L["U"], dY, dX=L["dX"],
-                     dA=L["dA"], dB=L["dB"], ws=L["ws"])
-        if world > 1:
-            dist.all_reduce(L["dA"])
-            dist.all_reduce(L["dB"])
-        q4.lora_merge(L["qw"], L["A"], L["B"], cfg.alpha, W_out=L["Wm"], ws=L["ws"])
-        q4.lora_unmerge(L["Wm"], L["A"], L["B"], cfg.alpha, W0_out=L["W0u"], ws=L["ws"])
-
     def pipelined(n, start_ev):
         copy_stream.wait_event(start_ev)
         for i in range(n):
@@ -415,7 +420,7 @@ def run_ours(args):
         return sum(x["total_ms"] for x in st if x["name"] in names) / calls
 
     alone = {}
-    for name, fn in (("quantise", lambda L: q4.qlora_nf4_quantize(L["W0"], out=L["qw"], ws=L["ws"])),
+    for name, fn in () if plain else (("quantise", lambda L: q4.qlora_nf4_quantize(L["W0"], out=L["qw"], ws=L["ws"])),
                      ("merge", lambda L: q4.lora_merge(L["qw"], L["A"], L["B"], cfg.alpha, W_out=L["Wm"],
                                                        ws=L["ws"])),
                      ("unmerge", lambda L: q4.lora_unmerge(L["Wm"], L["A"], L["B"], cfg.alpha,
@@ -432,11 +437,16 @@ def run_ours(args):
         alone[name] = per_call_ms(st_alone, kernels[name], 5)
     assert q4.qlora_get_device_status() == 0
 
+    fb_names = ("nf4_dequantize", "gemm_lora_down", "gemm_fwd_main", "pad_cols_bf16", "scale_f32_to_bf16_hilo",
+                "gemm_lora_g", "gemm_lora_dB", "splitk_reduce_f32", "gemm_lora_dA", "gemm_bwd_dx")
+    fb_ms = sum(x["total_ms"] for x in stats if x["name"] in fb_names) / args.steps
+    fwd_bwd_value = flops_rank * world / (fb_ms / 1e3) / 1e12 if fb_ms > 0 else None
+
     # ---- roofline of the dominant kernel (the tcgen05 GEMM: forward main and dX)
     peaks, peak_src = read_peaks()
     hbm = float(peaks.get("hbm_gbs"))
     hbm_rows = {}
-    for name in bpw:
+    for name in () if plain else bpw:
         calls = args.steps * (2 if name == "dequantise" else 1)
         ms_step = per_call_ms(stats, kernels[name], calls)
         gb = weights * bpw[name] / 1e9
@@ -464,11 +474,16 @@ def run_ours(args):
             "data": "synthetic (seeded W0/A/B from the config recipe, X and dY ~ N(0,1) drawn on device)",
             "config": {"workload": workload_name(cfg, T), "tokens_per_gpu": T,
                        "global_tokens": T * world, "r": cfg.r, "alpha": cfg.alpha,
-                       "step": "per linear: nf4_quantize, qlora_fwd, qlora_bwd, lora_merge, lora_unmerge"
+                       "step": ("per linear: lora_fwd, lora_bwd on the bf16 base (plain LoRA)" if plain else
+                                "per linear: nf4_quantize, qlora_fwd, qlora_bwd, lora_merge, lora_unmerge")
                                + (" + all-reduce(dA, dB)" if world > 1 else ""),
+                       "base": "bf16" if plain else "nf4",
                        "l2": "inputs larger than L2; L2 flushed (256 MB write) between timed steps",
                        "parallelism": f"dp{world}"},
             "tokens_per_s": tokens_s,
+            "fwd_bwd_only": {"value": fwd_bwd_value, "unit": "TFLOP/s",
+                             "note": "same flops over the forward and backward kernels of the step alone "
+                                     "(quantise, merge and unmerge launches left out)"},
             "roofline": {"kernel": "gemm_tc_kernel<256> (fwd main + dX)", "bound": "tensor",
                          "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                          "frac": achieved / peak if peak else None, "traffic": traffic,
@@ -550,6 +565,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", type=int, default=4)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--base", choices=["nf4", "bf16"], default="nf4",
+                    help="nf4: the QLoRA path (default); bf16: plain LoRA on the bf16 base")
     ap.add_argument("--deploy-only", action="store_true",
                     help="time only quantise, merge, unmerge and doubleDequant of the first linear")
     args = ap.parse_args()

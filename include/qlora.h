@@ -204,6 +204,29 @@ QLORA_API int qlora_bwd(const qlora_nf4_t* q, const uint16_t* A, const uint16_t*
               uint16_t* dX, float* dA, float* dB, void* workspace, size_t workspace_bytes,
               qlora_stream_t stream);
 
+/* ------------------------------------------- plain LoRA on a bf16 base */
+
+/*
+ * The same layer on an unquantised bf16 base W ([P2] "The LoRA hypothesis":
+ * h = W0 x + (alpha/r) B A x with W0 frozen; [P2] "QLoRA: shrink the frozen
+ * part too": QLoRA buys its memory saving with a dequantisation of the base
+ * in every step, which LoRA on a 16-bit base does not pay).  Same arguments,
+ * results and errors as qlora_fwd / qlora_bwd with W in place of W' and its
+ * shape passed as d, k.  W: bf16 d x k, device, 16-byte aligned, k % 8 == 0
+ * (rows 16-byte aligned for TMA), caller-owned and only read.  The workspace
+ * holds no copy of the weight, so it is smaller than the QLoRA one.
+ */
+QLORA_API size_t lora_fwd_workspace_bytes(int64_t d, int64_t k, int r, int64_t T);
+QLORA_API int lora_fwd(const uint16_t* W, int64_t d, int64_t k, const uint16_t* A, const uint16_t* B, int r,
+             float alpha, const uint16_t* X, int64_t T, uint16_t* Y, float* U_save, void* workspace,
+             size_t workspace_bytes, qlora_stream_t stream);
+
+QLORA_API size_t lora_bwd_workspace_bytes(int64_t d, int64_t k, int r, int64_t T);
+QLORA_API int lora_bwd(const uint16_t* W, int64_t d, int64_t k, const uint16_t* A, const uint16_t* B, int r,
+             float alpha, const uint16_t* X, const float* U_saved, const uint16_t* dY, int64_t T,
+             uint16_t* dX, float* dA, float* dB, void* workspace, size_t workspace_bytes,
+             qlora_stream_t stream);
+
 /* ---------------------------------------------------------------- deploy */
 
 QLORA_API size_t lora_merge_workspace_bytes(int64_t d, int64_t k, int r);

@@ -65,6 +65,11 @@ _SIGNATURES = {
     "qlora_bwd_workspace_bytes": (_SIZE, [_I64, _I64, _INT, _I64]),
     "qlora_bwd": (_INT, [_NF4P, _VP, _VP, _INT, _F, _VP, _VP, _VP, _I64, _VP, _VP, _VP, _VP,
                          _SIZE, _VP]),
+    "lora_fwd_workspace_bytes": (_SIZE, [_I64, _I64, _INT, _I64]),
+    "lora_fwd": (_INT, [_VP, _I64, _I64, _VP, _VP, _INT, _F, _VP, _I64, _VP, _VP, _VP, _SIZE, _VP]),
+    "lora_bwd_workspace_bytes": (_SIZE, [_I64, _I64, _INT, _I64]),
+    "lora_bwd": (_INT, [_VP, _I64, _I64, _VP, _VP, _INT, _F, _VP, _VP, _VP, _I64, _VP, _VP, _VP, _VP,
+                        _SIZE, _VP]),
     "lora_merge_workspace_bytes": (_SIZE, [_I64, _I64, _INT]),
     "lora_merge": (_INT, [_NF4P, _VP, _VP, _INT, _F, _VP, _VP, _SIZE, _VP]),
     "lora_unmerge": (_INT, [_VP, _VP, _VP, _INT, _F, _I64, _I64, _VP, _VP, _SIZE, _VP]),
@@ -272,6 +277,66 @@ def qlora_bwd(q: NF4Weight, A: torch.Tensor, B: torch.Tensor, alpha: float, X: t
                          _ptr(U_saved), _ptr(dY), T, _ptr(dX), _ptr(dA), _ptr(dB), _ptr(ws),
                          ws.numel(), _stream(stream))
     _check(st, "qlora_bwd")
+    return dX, dA, dB
+
+
+def lora_fwd_workspace_bytes(d: int, k: int, r: int, T: int) -> int:
+    return lib().lora_fwd_workspace_bytes(d, k, r, T)
+
+
+def lora_bwd_workspace_bytes(d: int, k: int, r: int, T: int) -> int:
+    return lib().lora_bwd_workspace_bytes(d, k, r, T)
+
+
+def lora_fwd(W: torch.Tensor, A: torch.Tensor, B: torch.Tensor, alpha: float, X: torch.Tensor,
+             Y: Optional[torch.Tensor] = None, U_save: Optional[torch.Tensor] = None,
+             ws: Optional[torch.Tensor] = None, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Plain LoRA forward on a bf16 base W (d x k); see lora_fwd in qlora.h."""
+    d, k = W.shape
+    r = A.shape[0]
+    T = X.shape[0]
+    _need(W, torch.bfloat16, (d, k), "W")
+    _need(A, torch.bfloat16, (r, k), "A")
+    _need(B, torch.bfloat16, (d, r), "B")
+    _need(X, torch.bfloat16, (T, k), "X")
+    dev = X.device
+    Y = torch.empty(T, d, dtype=torch.bfloat16, device=dev) if Y is None else Y
+    U_save = torch.empty(T, r, dtype=torch.float32, device=dev) if U_save is None else U_save
+    _need(Y, torch.bfloat16, (T, d), "Y")
+    _need(U_save, torch.float32, (T, r), "U_save")
+    ws = workspace(lora_fwd_workspace_bytes(d, k, r, T), dev) if ws is None else ws
+    st = lib().lora_fwd(_ptr(W), d, k, _ptr(A), _ptr(B), r, float(alpha), _ptr(X), T, _ptr(Y),
+                        _ptr(U_save), _ptr(ws), ws.numel(), _stream(stream))
+    _check(st, "lora_fwd")
+    return Y, U_save
+
+
+def lora_bwd(W: torch.Tensor, A: torch.Tensor, B: torch.Tensor, alpha: float, X: torch.Tensor,
+             U_saved: torch.Tensor, dY: torch.Tensor, dX: Optional[torch.Tensor] = None,
+             dA: Optional[torch.Tensor] = None, dB: Optional[torch.Tensor] = None,
+             ws: Optional[torch.Tensor] = None, stream=None):
+    """Plain LoRA backward on a bf16 base W (d x k); see lora_bwd in qlora.h."""
+    d, k = W.shape
+    r = A.shape[0]
+    T = X.shape[0]
+    _need(W, torch.bfloat16, (d, k), "W")
+    _need(A, torch.bfloat16, (r, k), "A")
+    _need(B, torch.bfloat16, (d, r), "B")
+    _need(X, torch.bfloat16, (T, k), "X")
+    _need(U_saved, torch.float32, (T, r), "U_saved")
+    _need(dY, torch.bfloat16, (T, d), "dY")
+    dev = X.device
+    dX = torch.empty(T, k, dtype=torch.bfloat16, device=dev) if dX is None else dX
+    dA = torch.empty(r, k, dtype=torch.float32, device=dev) if dA is None else dA
+    dB = torch.empty(d, r, dtype=torch.float32, device=dev) if dB is None else dB
+    _need(dX, torch.bfloat16, (T, k), "dX")
+    _need(dA, torch.float32, (r, k), "dA")
+    _need(dB, torch.float32, (d, r), "dB")
+    ws = workspace(lora_bwd_workspace_bytes(d, k, r, T), dev) if ws is None else ws
+    st = lib().lora_bwd(_ptr(W), d, k, _ptr(A), _ptr(B), r, float(alpha), _ptr(X), _ptr(U_saved),
+                        _ptr(dY), T, _ptr(dX), _ptr(dA), _ptr(dB), _ptr(ws), ws.numel(),
+                        _stream(stream))
+    _check(st, "lora_bwd")
     return dX, dA, dB
 
 

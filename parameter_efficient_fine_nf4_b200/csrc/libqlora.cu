@@ -461,11 +461,13 @@ const uint16_t* padded_B(const uint16_t* B, int64_t d, int r, int r8, uint16_t* 
 struct FwdWs {
   uint16_t* Wdq; uint16_t* sU; uint16_t* Bp; size_t bytes;
 };
-FwdWs carve_fwd(void* ws, int64_t d, int64_t k, int r, int64_t T) {
+// `dequant`: room for the bf16 W' that the QLoRA entry points dequantise into
+// (the plain-LoRA entry points read the caller's bf16 W instead).
+FwdWs carve_fwd(void* ws, int64_t d, int64_t k, int r, int64_t T, bool dequant = true) {
   Carver c{reinterpret_cast<uint8_t*>(ws)};
   const int64_t r8 = round_up(r, 8);
   FwdWs w;
-  w.Wdq = (uint16_t*)c.take((size_t)(d * k * 2));
+  w.Wdq = (uint16_t*)c.take((size_t)(dequant ? d * k * 2 : 0));
   w.sU = (uint16_t*)c.take((size_t)(std::max<int64_t>(T, 1) * r8 * 2));
   w.Bp = (uint16_t*)c.take((size_t)(d * r8 * 2));
   w.bytes = c.off;
@@ -494,14 +496,14 @@ struct BwdWs {
 // 2*rp columns (rp = r rounded up to 32); with rp <= 128 one GEMM with N = 2*rp
 // multiplies both and the epilogue adds the paired columns, otherwise the two
 // halves run as two GEMMs whose partial outputs are summed.
-BwdWs carve_bwd(void* ws, int64_t d, int64_t k, int r, int64_t T) {
+BwdWs carve_bwd(void* ws, int64_t d, int64_t k, int r, int64_t T, bool dequant = true) {
   Carver c{reinterpret_cast<uint8_t*>(ws)};
   const int64_t r8 = round_up(r, 8);
   const int64_t Tm = std::max<int64_t>(T, 1);
   BwdWs w;
   w.rp = (int)round_up(r, 32);
   w.halves = w.rp > 128 ? 2 : 1;
-  w.Wdq = (uint16_t*)c.take((size_t)(d * k * 2));
+  w.Wdq = (uint16_t*)c.take((size_t)(dequant ? d * k * 2 : 0));
   w.Us2 = (uint16_t*)c.take((size_t)(Tm * 2 * w.rp * 2));
   w.Gs2 = (uint16_t*)c.take((size_t)(Tm * 2 * w.rp * 2));
   w.Bp = (uint16_t*)c.take((size_t)(d * r8 * 2));
@@ -555,6 +557,108 @@ int adapter_grad_gemm(const char* name, const uint16_t* big, int64_t M, int64_t 
   return QLORA_OK;
 }
 
+// Forward on a bf16 d x k weight W (W' of the QLoRA path, or the caller's W).
+int fwd_core(const uint16_t* W, int64_t d, int64_t k, const uint16_t* A, const uint16_t* B, int r,
+             float alpha, const uint16_t* X, int64_t T, uint16_t* Y, float* U_save, const FwdWs& w,
+             cudaStream_t st) {
+  const float s = alpha / (float)r;
+  const int r8 = (int)round_up(r, 8);
+  int pst = QLORA_OK;
+  const uint16_t* Bp = padded_B(B, d, r, r8, w.Bp, st, &pst);
+  QLORA_TRY(pst);
+
+  // U = X A^T (fp32 to U_save), sU = bf16(s U) (operand of the extension)
+  {
+    GemmPlan g;
+    g.M = (int)T; g.N = r; g.K0 = (int)k; g.bn = bn_for_rank(r);
+    g.a0 = kmajor(X, k, T, k);
+    g.b0 = kmajor(A, k, r, k);
+    GemmArgs a = blank_args();
+    a.epi = EPI_F32; a.out = U_save; a.ldo = r; a.alpha = 1.0f; a.n_store = r;
+    a.out2 = w.sU; a.ldo2 = r8; a.alpha2 = s; a.n_store2 = r8;
+    QLORA_TRY(launch_gemm("gemm_lora_down", g, a, st));
+  }
+  // Y = [X | sU] [W | B]^T
+  {
+    GemmPlan g;
+    g.M = (int)T; g.N = (int)d; g.K0 = (int)k; g.K1 = r; g.bn = 256;
+    g.a0 = kmajor(X, k, T, k);
+    g.b0 = kmajor(W, k, d, k);
+    g.a1 = kmajor(w.sU, r8, T, r8);
+    g.b1 = kmajor(Bp, r8, d, r8);
+    GemmArgs a = blank_args();
+    a.epi = EPI_BF16; a.out = Y; a.ldo = d; a.n_store = (int)d;
+    QLORA_TRY(launch_gemm("gemm_fwd_main", g, a, st));
+  }
+  return QLORA_OK;
+}
+
+// Backward on a bf16 d x k weight W (W' of the QLoRA path, or the caller's W).
+int bwd_core(const uint16_t* W, int64_t d, int64_t k, const uint16_t* A, const uint16_t* B, int r,
+             float alpha, const uint16_t* X, const float* U_saved, const uint16_t* dY, int64_t T,
+             uint16_t* dX, float* dA, float* dB, const BwdWs& w, cudaStream_t st) {
+  const float s = alpha / (float)r;
+  const int r8 = (int)round_up(r, 8);
+  const int bnr = bn_for_rank(r);
+
+  int pst = QLORA_OK;
+  const uint16_t* Bp = padded_B(B, d, r, r8, w.Bp, st, &pst);
+  QLORA_TRY(pst);
+  const int rp = w.rp;
+  // Us2 = hi/lo of bf16(s U)
+  QLORA_TRY(launch("scale_f32_to_bf16_hilo", 0.0, (double)T * r * 8, st, [&] {
+    scale_f32_to_bf16_hilo<<<grid_for(T * rp, 256), 256, 0, st>>>(U_saved, T, r, s, w.Us2, rp);
+  }));
+  // G = dY B  ->  Gs2 = hi/lo of bf16(s G)
+  {
+    GemmPlan g;
+    g.M = (int)T; g.N = r; g.K0 = (int)d; g.bn = bnr;
+    g.a0 = kmajor(dY, d, T, d);
+    g.b0 = mnmajor(Bp, r8, d, r8);
+    GemmArgs a = blank_args();
+    a.epi = EPI_F32; a.out = nullptr; a.n_store = 0;
+    a.out2 = w.Gs2; a.ldo2 = 2 * rp; a.alpha2 = s; a.n_store2 = rp; a.lo_offset = rp;
+    QLORA_TRY(launch_gemm("gemm_lora_g", g, a, st));
+  }
+  // dB = dY^T (s U)   (M = d, N = r, K = T)
+  QLORA_TRY(adapter_grad_gemm("gemm_lora_dB", dY, d, T, w.Us2, r, rp, w.halves, w.splitsB,
+                              false, dB, w.partB, st));
+  // dA^T = X^T (s G)  (M = k, N = r, K = T), stored transposed into dA (r x k)
+  QLORA_TRY(adapter_grad_gemm("gemm_lora_dA", X, k, T, w.Gs2, r, rp, w.halves, w.splitsA,
+                              true, dA, w.partA, st));
+  // dX = [dY | sG] [W ; A]   (M = T, N = k, K = d + r)
+  {
+    GemmPlan g;
+    g.M = (int)T; g.N = (int)k; g.K0 = (int)d; g.K1 = r; g.bn = 256;
+    g.a0 = kmajor(dY, d, T, d);
+    g.b0 = mnmajor(W, k, d, k);
+    g.a1 = kmajor(w.Gs2, r, T, 2 * rp);          // hi part of s G
+    g.b1 = mnmajor(A, k, r, k);
+    GemmArgs a = blank_args();
+    a.epi = EPI_BF16; a.out = dX; a.ldo = k; a.n_store = (int)k;
+    QLORA_TRY(launch_gemm("gemm_bwd_dx", g, a, st));
+  }
+  return QLORA_OK;
+}
+
+// Shared argument checks of the two backward entry points (T > 0).
+int check_bwd_args(const uint16_t* A, const uint16_t* X, const float* U_saved, const uint16_t* dY,
+                   uint16_t* dX, float* dA, float* dB, void* ws, int64_t d, int64_t T) {
+  if (!X || !U_saved || !dY || !dX || !ws) return QLORA_ERR_INVALID_ARG;
+  if (!aligned16(A) || !aligned16(X) || !aligned16(dY) || !aligned16(dX) || !aligned16(dA) ||
+      !aligned16(dB) || !aligned16(U_saved) || !aligned16(ws))
+    return QLORA_ERR_MISALIGNED;
+  if (T > ((int64_t)1 << 31)) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (d % 8 != 0) return QLORA_ERR_UNSUPPORTED_SHAPE;   // dY rows must be 16-byte aligned for TMA
+  return QLORA_OK;
+}
+
+int zero_adapter_grads(float* dA, float* dB, int64_t d, int64_t k, int r, cudaStream_t st) {
+  QLORA_TRY(ensure_device());
+  if (cudaMemsetAsync(dA, 0, (size_t)r * k * 4, st) != cudaSuccess) return QLORA_ERR_CUDA;
+  if (cudaMemsetAsync(dB, 0, (size_t)d * r * 4, st) != cudaSuccess) return QLORA_ERR_CUDA;
+  return QLORA_OK;
+}
 }  // namespace
 }  // namespace qlora
 
@@ -680,6 +784,7 @@ size_t qlora_fwd_workspace_bytes(int64_t d, int64_t k, int r, int64_t T) {
   return carve_fwd(nullptr, d, k, r, T).bytes;
 }
 
+
 int qlora_fwd(const qlora_nf4_t* q, const uint16_t* A, const uint16_t* B, int r, float alpha,
               const uint16_t* X, int64_t T, uint16_t* Y, float* U_save, void* ws, size_t ws_bytes,
               qlora_stream_t stream) {
@@ -696,44 +801,38 @@ int qlora_fwd(const qlora_nf4_t* q, const uint16_t* A, const uint16_t* B, int r,
   if (ws_bytes < w.bytes) return QLORA_ERR_WORKSPACE_TOO_SMALL;
   QLORA_TRY(ensure_device());
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const float s = alpha / (float)r;
-  const int r8 = (int)round_up(r, 8);
-
   QLORA_TRY(dequantize_into(q, w.Wdq, st));
-  int pst = QLORA_OK;
-  const uint16_t* Bp = padded_B(B, d, r, r8, w.Bp, st, &pst);
-  QLORA_TRY(pst);
+  return fwd_core(w.Wdq, d, k, A, B, r, alpha, X, T, Y, U_save, w, st);
+}
 
-  // U = X A^T (fp32 to U_save), sU = bf16(s U) (operand of the extension)
-  {
-    GemmPlan g;
-    g.M = (int)T; g.N = r; g.K0 = (int)k; g.bn = bn_for_rank(r);
-    g.a0 = kmajor(X, k, T, k);
-    g.b0 = kmajor(A, k, r, k);
-    GemmArgs a = blank_args();
-    a.epi = EPI_F32; a.out = U_save; a.ldo = r; a.alpha = 1.0f; a.n_store = r;
-    a.out2 = w.sU; a.ldo2 = r8; a.alpha2 = s; a.n_store2 = r8;
-    QLORA_TRY(launch_gemm("gemm_lora_down", g, a, st));
-  }
-  // Y = [X | sU] [W' | B]^T
-  {
-    GemmPlan g;
-    g.M = (int)T; g.N = (int)d; g.K0 = (int)k; g.K1 = r; g.bn = 256;
-    g.a0 = kmajor(X, k, T, k);
-    g.b0 = kmajor(w.Wdq, k, d, k);
-    g.a1 = kmajor(w.sU, r8, T, r8);
-    g.b1 = kmajor(Bp, r8, d, r8);
-    GemmArgs a = blank_args();
-    a.epi = EPI_BF16; a.out = Y; a.ldo = d; a.n_store = (int)d;
-    QLORA_TRY(launch_gemm("gemm_fwd_main", g, a, st));
-  }
-  return QLORA_OK;
+size_t lora_fwd_workspace_bytes(int64_t d, int64_t k, int r, int64_t T) {
+  if (d < 1 || k < 1 || r < 1 || T < 0) return 0;
+  return carve_fwd(nullptr, d, k, r, T, false).bytes;
+}
+
+int lora_fwd(const uint16_t* W, int64_t d, int64_t k, const uint16_t* A, const uint16_t* B, int r,
+             float alpha, const uint16_t* X, int64_t T, uint16_t* Y, float* U_save, void* ws,
+             size_t ws_bytes, qlora_stream_t stream) {
+  QLORA_TRY(check_rank(r, alpha));
+  if (d < 1 || k < 1 || T < 0) return QLORA_ERR_INVALID_ARG;
+  if (T == 0) return QLORA_OK;
+  if (!W || !A || !B || !X || !Y || !U_save || !ws) return QLORA_ERR_INVALID_ARG;
+  if (k % 8 != 0 || d > ((int64_t)1 << 31) || k > ((int64_t)1 << 31) || T > ((int64_t)1 << 31))
+    return QLORA_ERR_UNSUPPORTED_SHAPE;
+  if (!aligned16(W) || !aligned16(A) || !aligned16(X) || !aligned16(Y) || !aligned16(U_save) ||
+      !aligned16(ws))
+    return QLORA_ERR_MISALIGNED;
+  FwdWs w = carve_fwd(ws, d, k, r, T, false);
+  if (ws_bytes < w.bytes) return QLORA_ERR_WORKSPACE_TOO_SMALL;
+  QLORA_TRY(ensure_device());
+  return fwd_core(W, d, k, A, B, r, alpha, X, T, Y, U_save, w, reinterpret_cast<cudaStream_t>(stream));
 }
 
 size_t qlora_bwd_workspace_bytes(int64_t d, int64_t k, int r, int64_t T) {
   if (d < 1 || k < 1 || r < 1 || T < 0) return 0;
   return carve_bwd(nullptr, d, k, r, T).bytes;
 }
+
 
 int qlora_bwd(const qlora_nf4_t* q, const uint16_t* A, const uint16_t* B, int r, float alpha,
               const uint16_t* X, const float* U_saved, const uint16_t* dY, int64_t T, uint16_t* dX,
@@ -744,64 +843,35 @@ int qlora_bwd(const qlora_nf4_t* q, const uint16_t* A, const uint16_t* B, int r,
   if (!A || !B || !dA || !dB) return QLORA_ERR_INVALID_ARG;
   const int64_t d = q->d, k = q->k;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (T == 0) {
-    QLORA_TRY(ensure_device());
-    if (cudaMemsetAsync(dA, 0, (size_t)r * k * 4, st) != cudaSuccess) return QLORA_ERR_CUDA;
-    if (cudaMemsetAsync(dB, 0, (size_t)d * r * 4, st) != cudaSuccess) return QLORA_ERR_CUDA;
-    return QLORA_OK;
-  }
-  if (!X || !U_saved || !dY || !dX || !ws) return QLORA_ERR_INVALID_ARG;
-  if (!aligned16(A) || !aligned16(X) || !aligned16(dY) || !aligned16(dX) || !aligned16(dA) ||
-      !aligned16(dB) || !aligned16(U_saved) || !aligned16(ws))
-    return QLORA_ERR_MISALIGNED;
-  if (T > ((int64_t)1 << 31)) return QLORA_ERR_UNSUPPORTED_SHAPE;
-  if (d % 8 != 0) return QLORA_ERR_UNSUPPORTED_SHAPE;   // dY rows must be 16-byte aligned for TMA
+  if (T == 0) return zero_adapter_grads(dA, dB, d, k, r, st);
+  QLORA_TRY(check_bwd_args(A, X, U_saved, dY, dX, dA, dB, ws, d, T));
   BwdWs w = carve_bwd(ws, d, k, r, T);
   if (ws_bytes < w.bytes) return QLORA_ERR_WORKSPACE_TOO_SMALL;
   QLORA_TRY(ensure_device());
-  const float s = alpha / (float)r;
-  const int r8 = (int)round_up(r, 8);
-  const int bnr = bn_for_rank(r);
-
   QLORA_TRY(dequantize_into(q, w.Wdq, st));
-  int pst = QLORA_OK;
-  const uint16_t* Bp = padded_B(B, d, r, r8, w.Bp, st, &pst);
-  QLORA_TRY(pst);
-  const int rp = w.rp;
-  // Us2 = hi/lo of bf16(s U)
-  QLORA_TRY(launch("scale_f32_to_bf16_hilo", 0.0, (double)T * r * 8, st, [&] {
-    scale_f32_to_bf16_hilo<<<grid_for(T * rp, 256), 256, 0, st>>>(U_saved, T, r, s, w.Us2, rp);
-  }));
-  // G = dY B  ->  Gs2 = hi/lo of bf16(s G)
-  {
-    GemmPlan g;
-    g.M = (int)T; g.N = r; g.K0 = (int)d; g.bn = bnr;
-    g.a0 = kmajor(dY, d, T, d);
-    g.b0 = mnmajor(Bp, r8, d, r8);
-    GemmArgs a = blank_args();
-    a.epi = EPI_F32; a.out = nullptr; a.n_store = 0;
-    a.out2 = w.Gs2; a.ldo2 = 2 * rp; a.alpha2 = s; a.n_store2 = rp; a.lo_offset = rp;
-    QLORA_TRY(launch_gemm("gemm_lora_g", g, a, st));
-  }
-  // dB = dY^T (s U)   (M = d, N = r, K = T)
-  QLORA_TRY(adapter_grad_gemm("gemm_lora_dB", dY, d, T, w.Us2, r, rp, w.halves, w.splitsB,
-                              false, dB, w.partB, st));
-  // dA^T = X^T (s G)  (M = k, N = r, K = T), stored transposed into dA (r x k)
-  QLORA_TRY(adapter_grad_gemm("gemm_lora_dA", X, k, T, w.Gs2, r, rp, w.halves, w.splitsA,
-                              true, dA, w.partA, st));
-  // dX = [dY | sG] [W' ; A]   (M = T, N = k, K = d + r)
-  {
-    GemmPlan g;
-    g.M = (int)T; g.N = (int)k; g.K0 = (int)d; g.K1 = r; g.bn = 256;
-    g.a0 = kmajor(dY, d, T, d);
-    g.b0 = mnmajor(w.Wdq, k, d, k);
-    g.a1 = kmajor(w.Gs2, r, T, 2 * rp);          // hi part of s G
-    g.b1 = mnmajor(A, k, r, k);
-    GemmArgs a = blank_args();
-    a.epi = EPI_BF16; a.out = dX; a.ldo = k; a.n_store = (int)k;
-    QLORA_TRY(launch_gemm("gemm_bwd_dx", g, a, st));
-  }
-  return QLORA_OK;
+  return bwd_core(w.Wdq, d, k, A, B, r, alpha, X, U_saved, dY, T, dX, dA, dB, w, st);
+}
+
+size_t lora_bwd_workspace_bytes(int64_t d, int64_t k, int r, int64_t T) {
+  if (d < 1 || k < 1 || r < 1 || T < 0) return 0;
+  return carve_bwd(nullptr, d, k, r, T, false).bytes;
+}
+
+int lora_bwd(const uint16_t* W, int64_t d, int64_t k, const uint16_t* A, const uint16_t* B, int r,
+             float alpha, const uint16_t* X, const float* U_saved, const uint16_t* dY, int64_t T,
+             uint16_t* dX, float* dA, float* dB, void* ws, size_t ws_bytes, qlora_stream_t stream) {
+  QLORA_TRY(check_rank(r, alpha));
+  if (d < 1 || k < 1 || T < 0) return QLORA_ERR_INVALID_ARG;
+  if (!W || !A || !B || !dA || !dB) return QLORA_ERR_INVALID_ARG;
+  if (k % 8 != 0 || d > ((int64_t)1 << 31) || k > ((int64_t)1 << 31)) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (T == 0) return zero_adapter_grads(dA, dB, d, k, r, st);
+  if (!aligned16(W)) return QLORA_ERR_MISALIGNED;
+  QLORA_TRY(check_bwd_args(A, X, U_saved, dY, dX, dA, dB, ws, d, T));
+  BwdWs w = carve_bwd(ws, d, k, r, T, false);
+  if (ws_bytes < w.bytes) return QLORA_ERR_WORKSPACE_TOO_SMALL;
+  QLORA_TRY(ensure_device());
+  return bwd_core(W, d, k, A, B, r, alpha, X, U_saved, dY, T, dX, dA, dB, w, st);
 }
 
 size_t lora_merge_workspace_bytes(int64_t d, int64_t k, int r) {

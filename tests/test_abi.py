@@ -70,6 +70,11 @@ def test_workspace_queries(lib):
     assert q4.qlora_bwd_workspace_bytes(22016, 8192, 64, 16384) >= 22016 * 8192 * 2
     assert q4.lora_merge_workspace_bytes(256, 256, 8) >= 256 * 8 * 2
     assert q4.qlora_fwd_workspace_bytes(0, 256, 8, 16) == 0
+    # the plain-LoRA workspace holds no copy of the weight
+    for fn_q, fn_p in ((q4.qlora_fwd_workspace_bytes, q4.lora_fwd_workspace_bytes),
+                       (q4.qlora_bwd_workspace_bytes, q4.lora_bwd_workspace_bytes)):
+        assert fn_q(22016, 8192, 64, 16384) - fn_p(22016, 8192, 64, 16384) == 22016 * 8192 * 2
+    assert q4.lora_fwd_workspace_bytes(4096, 4096, 8, 0) > 0
 
 
 def test_argument_validation_without_device(lib):
@@ -89,3 +94,12 @@ def test_argument_validation_without_device(lib):
     nf_bad = q4._NF4(16, 16, 16, 16, 256, 256, 32, 256)           # block != 64
     assert L.qlora_nf4_dequantize(ctypes.byref(nf_bad), 16, None) == 2
     assert q4.strerror(6) == "device wait timed out"
+    # plain LoRA: k % 8, alignment, rank and workspace are checked on the host
+    assert L.lora_fwd(16, 256, 100, 16, 16, 8, 16.0, 16, 16, 16, 16, 16, 1 << 20, None) == 2      # k % 8
+    assert L.lora_fwd(17, 256, 256, 16, 16, 8, 16.0, 16, 16, 16, 16, 16, 1 << 20, None) == 3      # W
+    assert L.lora_fwd(16, 256, 256, 16, 16, 0, 16.0, 16, 16, 16, 16, 16, 1 << 20, None) == 2      # r = 0
+    assert L.lora_fwd(16, 256, 256, 16, 16, 8, 16.0, 16, 16, 16, 16, 16, 64, None) == 4           # workspace
+    assert L.lora_bwd(16, 130, 256, 16, 16, 8, 16.0, 16, 16, 16, 16, 16, 16, 16, 16, 1 << 20,
+                      None) == 2                                                                  # d % 8
+    assert L.lora_bwd(None, 256, 256, 16, 16, 8, 16.0, 16, 16, 16, 16, 16, 16, 16, 16, 1 << 20,
+                      None) == 1                                                                  # null W
