@@ -17,4 +17,4 @@ function whose numbers the pages do not fix is the absolute value of the NF4
 levels (the outermost quantile probability is not printed): its structure is
 pinned, its digits are "parity unpinned" beyond that structure.
 """
-from . import nf4, lora  # noqa: F401
+from . import nf4, lora, adam  # noqa: F401
