@@ -512,8 +512,9 @@ def run_ours(args):
 
 def run_deploy(args):
     """The HBM-bound rows alone on the config's first linear: quantise, merge,
-    unmerge, doubleDequant (warm-up, then `steps` calls of each, CUDA-event
-    timing through the library profiler).  A diagnostic, not the bench line."""
+    unmerge, doubleDequant and the Adam step on its A and B (warm-up, then
+    `steps` calls of each, CUDA-event timing through the library profiler).
+    A diagnostic, not the bench line."""
     import torch
     import parameter_efficient_fine_nf4_b200 as q4
     dev = torch.device("cuda", 0)
@@ -537,6 +538,19 @@ def run_deploy(args):
                        ("lora_unmerge",)),
            "dequantise": (lambda: q4.qlora_nf4_dequantize(qw, W_out=W0u), 2.5 + 1 / 64,
                           ("nf4_dequantize",))}
+    # the optimiser step on the adapter factors (A and B together, one call each)
+    opt = []
+    for shape in ((cfg.r, lin.k), (lin.d, cfg.r)):
+        master = torch.randn(shape, device=dev) * 0.02
+        opt.append((master, master.to(torch.bfloat16), torch.zeros_like(master), torch.zeros_like(master),
+                    torch.randn(shape, device=dev) * 1e-3))
+    n_opt = sum(o[0].numel() for o in opt)
+
+    def adam_both():
+        for master, w16, m, v, g in opt:
+            q4.lora_adam_step(master, w16, m, v, g, step=1, lr=2e-4)
+
+    ops["adam"] = (adam_both, 30.0 * n_opt / (lin.d * lin.k), ("lora_adam_step",))
     peaks, src = read_peaks()
     hbm = float(peaks.get("hbm_gbs"))
     out = {"mode": "deploy-only", "config": {"workload": f"{lin.name}: d={lin.d}, k={lin.k}, r={cfg.r}"},
@@ -568,7 +582,8 @@ def main():
     ap.add_argument("--base", choices=["nf4", "bf16"], default="nf4",
                     help="nf4: the QLoRA path (default); bf16: plain LoRA on the bf16 base")
     ap.add_argument("--deploy-only", action="store_true",
-                    help="time only quantise, merge, unmerge and doubleDequant of the first linear")
+                    help="time only quantise, merge, unmerge, doubleDequant and the Adam step "
+                         "of the first linear")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)

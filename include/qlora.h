@@ -227,6 +227,28 @@ QLORA_API int lora_bwd(const uint16_t* W, int64_t d, int64_t k, const uint16_t* 
              uint16_t* dX, float* dA, float* dB, void* workspace, size_t workspace_bytes,
              qlora_stream_t stream);
 
+/* ------------------------------------------------- optimiser (next row) */
+
+/*
+ * One Adam step on a trainable fp32 tensor, e.g. A (n = r*k) or B (n = d*r)
+ * with their gradients dA, dB ([P1] "The update LoRA is allowed to learn":
+ * only A and B carry optimiser state; [P2] "Why full fine-tuning costs so
+ * much": a 16-bit forward copy, an fp32 master copy and fp32 moments m, v per
+ * parameter).  The pages print no update rule; this is bias-corrected Adam
+ * (Kingma and Ba 2015) with decoupled weight decay (Loshchilov and Hutter
+ * 2019), computed in fp32:
+ *   m = beta1 m + (1 - beta1) g;   v = beta2 v + (1 - beta2) g^2;
+ *   master -= lr (m / (1 - beta1^step) / (sqrt(v / (1 - beta2^step)) + eps)
+ *                 + weight_decay master);
+ *   weight_bf16 = bf16_RN(master)   (the copy the forward and backward read).
+ * All five arrays are device, n elements, 16-byte aligned and updated in
+ * place (grad is only read).  step counts from 1; lr, eps, weight_decay >= 0;
+ * 0 <= beta1, beta2 < 1.  Returns QLORA_ERR_INVALID_ARG otherwise.
+ */
+QLORA_API int lora_adam_step(float* master, uint16_t* weight_bf16, float* m, float* v, const float* grad,
+                             int64_t n, int64_t step, float lr, float beta1, float beta2, float eps,
+                             float weight_decay, qlora_stream_t stream);
+
 /* ---------------------------------------------------------------- deploy */
 
 QLORA_API size_t lora_merge_workspace_bytes(int64_t d, int64_t k, int r);

@@ -70,6 +70,7 @@ _SIGNATURES = {
     "lora_bwd_workspace_bytes": (_SIZE, [_I64, _I64, _INT, _I64]),
     "lora_bwd": (_INT, [_VP, _I64, _I64, _VP, _VP, _INT, _F, _VP, _VP, _VP, _I64, _VP, _VP, _VP, _VP,
                         _SIZE, _VP]),
+    "lora_adam_step": (_INT, [_VP, _VP, _VP, _VP, _VP, _I64, _I64, _F, _F, _F, _F, _F, _VP]),
     "lora_merge_workspace_bytes": (_SIZE, [_I64, _I64, _INT]),
     "lora_merge": (_INT, [_NF4P, _VP, _VP, _INT, _F, _VP, _VP, _SIZE, _VP]),
     "lora_unmerge": (_INT, [_VP, _VP, _VP, _INT, _F, _I64, _I64, _VP, _VP, _SIZE, _VP]),
@@ -338,6 +339,20 @@ def lora_bwd(W: torch.Tensor, A: torch.Tensor, B: torch.Tensor, alpha: float, X:
                         _stream(stream))
     _check(st, "lora_bwd")
     return dX, dA, dB
+
+
+def lora_adam_step(master: torch.Tensor, weight_bf16: torch.Tensor, m: torch.Tensor, v: torch.Tensor,
+                   grad: torch.Tensor, step: int, lr: float, beta1: float = 0.9, beta2: float = 0.999,
+                   eps: float = 1e-8, weight_decay: float = 0.0, stream=None) -> None:
+    """One Adam step in place on (master, m, v) and the bf16 copy; see qlora.h."""
+    n = master.numel()
+    _need(master, torch.float32, tuple(master.shape), "master")
+    for t, dt, name in ((weight_bf16, torch.bfloat16, "weight_bf16"), (m, torch.float32, "m"),
+                        (v, torch.float32, "v"), (grad, torch.float32, "grad")):
+        _need(t, dt, tuple(master.shape), name)
+    _check(lib().lora_adam_step(_ptr(master), _ptr(weight_bf16), _ptr(m), _ptr(v), _ptr(grad), n, int(step),
+                                float(lr), float(beta1), float(beta2), float(eps), float(weight_decay),
+                                _stream(stream)), "lora_adam_step")
 
 
 def lora_merge(q: NF4Weight, A: torch.Tensor, B: torch.Tensor, alpha: float,

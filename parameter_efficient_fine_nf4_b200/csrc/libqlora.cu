@@ -16,6 +16,7 @@
 #include <cuda_runtime.h>
 
 #include "../../include/qlora.h"
+#include "adam_kernels.cuh"
 #include "deploy_kernels.cuh"
 #include "gemm_tc.cuh"
 #include "nf4_kernels.cuh"
@@ -915,6 +916,30 @@ int lora_merge(const qlora_nf4_t* q, const uint16_t* A, const uint16_t* B, int r
   QLORA_TRY(check_rank(r, alpha));
   return merge_common(q, nullptr, A, B, r, alpha, q->d, q->k, W_out, ws, ws_bytes,
                       reinterpret_cast<cudaStream_t>(stream), true);
+}
+
+int lora_adam_step(float* master, uint16_t* weight_bf16, float* m, float* v, const float* grad, int64_t n,
+                   int64_t step, float lr, float beta1, float beta2, float eps, float weight_decay,
+                   qlora_stream_t stream) {
+  if (!master || !weight_bf16 || !m || !v || !grad || n < 0 || step < 1) return QLORA_ERR_INVALID_ARG;
+  if (!(lr >= 0.f) || !(beta1 >= 0.f && beta1 < 1.f) || !(beta2 >= 0.f && beta2 < 1.f) || !(eps >= 0.f) ||
+      !(weight_decay >= 0.f))
+    return QLORA_ERR_INVALID_ARG;
+  if (!aligned16(master) || !aligned16(weight_bf16) || !aligned16(m) || !aligned16(v) || !aligned16(grad))
+    return QLORA_ERR_MISALIGNED;
+  if (n == 0) return QLORA_OK;
+  QLORA_TRY(ensure_device());
+  AdamArgs a;
+  a.lr = lr; a.beta1 = beta1; a.beta2 = beta2;
+  a.omb1 = (float)(1.0 - (double)beta1);
+  a.omb2 = (float)(1.0 - (double)beta2);
+  a.c1 = (float)(1.0 / (1.0 - std::pow((double)beta1, (double)step)));
+  a.c2 = (float)(1.0 / (1.0 - std::pow((double)beta2, (double)step)));
+  a.eps = eps; a.wd = weight_decay;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  return launch("lora_adam_step", 0.0, 30.0 * (double)n, st, [&] {
+    adam_step_kernel<<<grid_for(cdiv(n, 4), 256), 256, 0, st>>>(master, weight_bf16, m, v, grad, n, a);
+  });
 }
 
 int lora_unmerge(const uint16_t* W, const uint16_t* A, const uint16_t* B, int r, float alpha,
