@@ -8,7 +8,7 @@ equation with doubleDequant(c1 FP32, c2 k-bit, W NF4)), [P2] section
 "QLoRA: shrink the frozen part too", and [P1] "What to choose and why"
 (NF4, block size 64, double-quant block size 256).
 
-Readings taken where the pages are silent (each also listed in the design doc):
+Readings taken where the pages are silent:
   R1  outermost quantile probability p_max = 1 - (1/2)(1/(2*16) + 1/(2*15)).
   R2  blocks are consecutive runs of 64 elements of row-major W0.
   R3  an all-zero block encodes every element as the zero level.
