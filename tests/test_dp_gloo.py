@@ -58,3 +58,55 @@ def test_two_rank_token_sharding_sums_to_full_batch(tmp_path):
     mp.start_processes(_worker, args=(2, _free_port(), out), nprocs=2, join=True,
                        start_method="spawn")
     assert open(out).read() == "ok"
+
+
+def _adam_worker(rank, world, port, out_path):
+    """Two data-parallel ranks take three optimiser steps: per step each rank forms
+    the adapter gradients of its token shard, the ranks sum them (the one
+    exchange), and each applies the same Adam step to its own replica of A
+    and B.  The replicas stay identical and equal a single process that sees
+    the whole batch."""
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        from oracle import adam
+        lay = synthetic.custom_layer(seed=77, d=96, k=64, r=4, T=64, alpha=8.0)
+        X = nf4.bf16_to_f64(lay.X)
+        dY = nf4.bf16_to_f64(lay.dY)
+        Wp = np.zeros((lay.d, lay.k))
+        shard = np.array_split(np.arange(lay.T), world)[rank]
+        mine = {"A": nf4.bf16_to_f64(lay.A), "B": nf4.bf16_to_f64(lay.B)}
+        ref = {n: v.copy() for n, v in mine.items()}
+        st_m = {n: (np.zeros_like(v), np.zeros_like(v)) for n, v in mine.items()}
+        ref_m = {n: (np.zeros_like(v), np.zeros_like(v)) for n, v in ref.items()}
+        for t in range(1, 4):
+            g = lora.grad_adapters(X[shard], mine["A"], mine["B"], lay.s, dY[shard])
+            grads = {"A": torch.from_numpy(g["dA"].copy()), "B": torch.from_numpy(g["dB"].copy())}
+            for n in ("A", "B"):
+                dist.all_reduce(grads[n])
+                out = adam.adam_step(mine[n], *st_m[n], grads[n].numpy(), t=t, lr=1e-3)
+                mine[n], st_m[n] = out["theta"], (out["m"], out["v"])
+            gf = lora.grad_adapters(X, ref["A"], ref["B"], lay.s, dY)
+            for n, gn in (("A", gf["dA"]), ("B", gf["dB"])):
+                out = adam.adam_step(ref[n], *ref_m[n], gn, t=t, lr=1e-3)
+                ref[n], ref_m[n] = out["theta"], (out["m"], out["v"])
+        # replicas agree across ranks bit for bit, and match the whole-batch run
+        both = {n: [torch.zeros(v.shape, dtype=torch.float64) for _ in range(world)] for n, v in mine.items()}
+        for n in mine:
+            dist.all_gather(both[n], torch.from_numpy(mine[n].copy()))
+        if rank == 0:
+            same = all(torch.equal(both[n][0], both[n][1]) for n in mine)
+            close = all(np.allclose(mine[n], ref[n], rtol=1e-10, atol=1e-12) for n in mine)
+            with open(out_path, "w") as f:
+                f.write("ok" if same and close else f"same={same} close={close}")
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_rank_adam_keeps_replicas_identical(tmp_path):
+    out = str(tmp_path / "adam.txt")
+    mp.start_processes(_adam_worker, args=(2, _free_port(), out), nprocs=2, join=True,
+                       start_method="spawn")
+    assert open(out).read() == "ok"
