@@ -11,6 +11,8 @@ Equations followed:
     Y = X doubleDequant(c1, c2, W) + X L1 L2 (row-vector form, so L1 = A^T,
     L2 = B^T with the alpha/r scale s folded in); the activation gradient is
     also formed through the bf16-dequantised W.
+  * [P5] "LoRA vs QLoRA: Parameter-Efficient Fine-Tuning Explained", run
+    configuration: LoRA dropout (reading in the dropout section below).
   * [P1] deploy paragraph and [P2] "The LoRA hypothesis": W = W0 + (alpha/r) B A;
     switching tasks subtracts B A.  [P2] "What actually goes wrong": merge into
     the 16-bit base, keep the adapter separate (so the merged output is bf16
@@ -59,6 +61,39 @@ def grad_adapters(X: np.ndarray, A: np.ndarray, B: np.ndarray, s: float, dY: np.
         U = X @ A.T
     G = dY @ B
     return {"dA": s * (G.T @ X), "dB": s * (dY.T @ U)}
+
+
+# ---------------------------------------------------------------------------
+# LoRA dropout on the adapter input.  [P5] "LoRA vs QLoRA: Parameter-Efficient
+# Fine-Tuning Explained", run configuration list: a LoRA dropout of 0.05-0.1
+# is used for regularisation.  The pages give no formula; reading taken: the
+# adapter path sees X dropped out element-wise with inverted scaling,
+# D(X) = X * keep / (1 - p), keep a 0/1 mask drawn with probability 1 - p of a
+# one, while the frozen path sees X itself.  The mask is an input here.
+# ---------------------------------------------------------------------------
+def dropout_input(X: np.ndarray, keep: np.ndarray, p: float) -> np.ndarray:
+    """D(X) = X * keep / (1 - p)."""
+    if not 0.0 <= p < 1.0:
+        raise ValueError("dropout probability must be in [0, 1)")
+    return X * keep / (1.0 - p)
+
+
+def forward_dropout(X: np.ndarray, Wp: np.ndarray, A: np.ndarray, B: np.ndarray, s: float,
+                    keep: np.ndarray, p: float) -> Dict[str, np.ndarray]:
+    """U = D(X) A^T;  Y = X W'^T + s U B^T."""
+    U = dropout_input(X, keep, p) @ A.T
+    return {"U": U, "Y": X @ Wp.T + s * (U @ B.T)}
+
+
+def backward_dropout(X: np.ndarray, Wp: np.ndarray, A: np.ndarray, B: np.ndarray, s: float,
+                     dY: np.ndarray, keep: np.ndarray, p: float) -> Dict[str, np.ndarray]:
+    """Gradients of <dY, Y> for forward_dropout:
+    G = dY B;  dX = dY W' + D(s G A)  (the adapter term passes back through the
+    same mask and scale);  dA = s G^T D(X);  dB = s dY^T (D(X) A^T)."""
+    G = dY @ B
+    Xd = dropout_input(X, keep, p)
+    return {"G": G, "dX": dY @ Wp + dropout_input(s * (G @ A), keep, p),
+            "dA": s * (G.T @ Xd), "dB": s * (dY.T @ (Xd @ A.T))}
 
 
 def merge(Wp: np.ndarray, A: np.ndarray, B: np.ndarray, s: float) -> np.ndarray:

@@ -5,6 +5,7 @@ import json
 import os
 
 import numpy as np
+import pytest
 
 from oracle import lora, nf4
 import synthetic
@@ -124,3 +125,72 @@ def test_flop_formula():
     T, d, k, r = 16384, 22016, 8192, 64
     assert lora.algorithmic_flops(T, d, k, r) == 4 * T * d * k + 6 * T * r * (d + k)
     assert round(lora.algorithmic_flops(T, d, k, r) / 1e8) == 120098   # 1.20098e13
+
+
+# ---------------------------------------------------------------------------
+# LoRA dropout (mask passed in): pins by special case, linearity and a
+# directional derivative
+# ---------------------------------------------------------------------------
+def _small(seed=3, T=24, d=20, k=16, r=4):
+    rng = np.random.default_rng(seed)
+    X = rng.standard_normal((T, k))
+    Wp = rng.standard_normal((d, k)) * 0.1
+    A = rng.standard_normal((r, k)) * 0.3
+    B = rng.standard_normal((d, r)) * 0.2
+    dY = rng.standard_normal((T, d))
+    keep = (rng.random((T, k)) < 0.5).astype(np.float64)
+    return X, Wp, A, B, dY, keep
+
+
+def test_dropout_zero_is_plain_lora():
+    X, Wp, A, B, dY, _ = _small()
+    ones = np.ones_like(X)
+    f0, f1 = lora.forward(X, Wp, A, B, 0.5), lora.forward_dropout(X, Wp, A, B, 0.5, ones, 0.0)
+    np.testing.assert_array_equal(f0["Y"], f1["Y"])
+    b0, b1 = lora.backward(X, Wp, A, B, 0.5, dY), lora.backward_dropout(X, Wp, A, B, 0.5, dY, ones, 0.0)
+    for key in ("dX", "dA", "dB"):
+        np.testing.assert_allclose(b0[key], b1[key], rtol=1e-14, atol=1e-14)
+
+
+def test_complementary_masks_add_up_to_twice_the_undropped_adapter():
+    # p = 1/2: D_M(X) + D_{1-M}(X) = 2 X, and everything adapter-side is linear in D(X)
+    X, Wp, A, B, dY, keep = _small()
+    s = 0.75
+    a = lora.forward_dropout(X, Wp, A, B, s, keep, 0.5)
+    b = lora.forward_dropout(X, Wp, A, B, s, 1.0 - keep, 0.5)
+    base = X @ Wp.T
+    full = lora.forward(X, Wp, A, B, s)
+    np.testing.assert_allclose((a["Y"] - base) + (b["Y"] - base), 2 * (full["Y"] - base), rtol=1e-12, atol=1e-12)
+    ga = lora.backward_dropout(X, Wp, A, B, s, dY, keep, 0.5)
+    gb = lora.backward_dropout(X, Wp, A, B, s, dY, 1.0 - keep, 0.5)
+    gf = lora.backward(X, Wp, A, B, s, dY)
+    for key in ("dA", "dB"):
+        np.testing.assert_allclose(ga[key] + gb[key], 2 * gf[key], rtol=1e-12, atol=1e-12)
+    base_dx = dY @ Wp
+    np.testing.assert_allclose((ga["dX"] - base_dx) + (gb["dX"] - base_dx), 2 * (gf["dX"] - base_dx),
+                               rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("wrt", ["X", "A", "B"])
+def test_dropout_gradients_match_directional_derivatives(wrt):
+    # L = <dY, Y> is linear in X and bilinear in (A, B): the central difference is exact
+    # up to rounding for any step, so every mask and scale has to be in the right place
+    X, Wp, A, B, dY, keep = _small(seed=9)
+    s, p = 0.6, 0.1
+    args = {"X": X, "A": A, "B": B}
+    E = np.random.default_rng(1).standard_normal(args[wrt].shape)
+
+    def loss(v):
+        a = dict(args, **{wrt: v})
+        return np.sum(dY * lora.forward_dropout(a["X"], Wp, a["A"], a["B"], s, keep, p)["Y"])
+
+    h = 1e-3
+    num = (loss(args[wrt] + h * E) - loss(args[wrt] - h * E)) / (2 * h)
+    g = lora.backward_dropout(X, Wp, A, B, s, dY, keep, p)["d" + wrt]
+    assert abs(num - np.sum(g * E)) <= 1e-8 * (1 + abs(num))
+
+
+def test_dropout_rejects_p_one():
+    X, Wp, A, B, dY, keep = _small()
+    with pytest.raises(ValueError):
+        lora.forward_dropout(X, Wp, A, B, 1.0, keep, 1.0)
