@@ -103,3 +103,11 @@ def test_argument_validation_without_device(lib):
                       None) == 2                                                                  # d % 8
     assert L.lora_bwd(None, 256, 256, 16, 16, 8, 16.0, 16, 16, 16, 16, 16, 16, 16, 16, 1 << 20,
                       None) == 1                                                                  # null W
+    # Adam: step, betas, lr and alignment are checked on the host; n = 0 is a no-op
+    assert L.lora_adam_step(16, 16, 16, 16, 16, 8, 0, 1e-3, 0.9, 0.999, 1e-8, 0.0, None) == 1     # step 0
+    assert L.lora_adam_step(16, 16, 16, 16, 16, 8, 1, 1e-3, 1.0, 0.999, 1e-8, 0.0, None) == 1     # beta1 = 1
+    assert L.lora_adam_step(16, 16, 16, 16, 16, 8, 1, -1.0, 0.9, 0.999, 1e-8, 0.0, None) == 1     # lr < 0
+    assert L.lora_adam_step(16, 16, 16, 16, 16, 8, 1, float("nan"), 0.9, 0.999, 1e-8, 0.0, None) == 1
+    assert L.lora_adam_step(16, 20, 16, 16, 16, 8, 1, 1e-3, 0.9, 0.999, 1e-8, 0.0, None) == 3     # bf16 copy
+    assert L.lora_adam_step(None, 16, 16, 16, 16, 8, 1, 1e-3, 0.9, 0.999, 1e-8, 0.0, None) == 1   # null
+    assert L.lora_adam_step(16, 16, 16, 16, 16, 0, 1, 1e-3, 0.9, 0.999, 1e-8, 0.0, None) == 0     # n = 0
