@@ -13,6 +13,8 @@ Equations followed:
     also formed through the bf16-dequantised W.
   * [P5] "LoRA vs QLoRA: Parameter-Efficient Fine-Tuning Explained", run
     configuration: LoRA dropout (reading in the dropout section below).
+  * [P2] "The LoRA hypothesis" and [P1] "What to choose and why": many
+    unmerged adapters over one base (reading in the multi-adapter section).
   * [P1] deploy paragraph and [P2] "The LoRA hypothesis": W = W0 + (alpha/r) B A;
     switching tasks subtracts B A.  [P2] "What actually goes wrong": merge into
     the 16-bit base, keep the adapter separate (so the merged output is bf16
@@ -94,6 +96,46 @@ def backward_dropout(X: np.ndarray, Wp: np.ndarray, A: np.ndarray, B: np.ndarray
     Xd = dropout_input(X, keep, p)
     return {"G": G, "dX": dY @ Wp + dropout_input(s * (G @ A), keep, p),
             "dA": s * (G.T @ Xd), "dB": s * (dY.T @ (Xd @ A.T))}
+
+
+# ---------------------------------------------------------------------------
+# Several unmerged adapters over one frozen base in one batch.  [P2] "The LoRA
+# hypothesis": serving many tasks keeps the adapters unmerged, one frozen base
+# in memory with a stack of small adapters chosen per request; [P1] "What to
+# choose and why": one deployed base, a small B A per task.  Reading taken:
+# token t uses adapter idx[t] of a stack (A_i r x k, B_i d x r, scale s_i),
+# the frozen path is shared.
+# ---------------------------------------------------------------------------
+def forward_multi(X: np.ndarray, Wp: np.ndarray, As: np.ndarray, Bs: np.ndarray, ss: np.ndarray,
+                  idx: np.ndarray) -> Dict[str, np.ndarray]:
+    """Y[t] = X[t] W'^T + s_i (X[t] A_i^T) B_i^T with i = idx[t]; U[t] = X[t] A_i^T.
+    As: n x r x k, Bs: n x d x r, ss: n scales, idx: T adapter indices."""
+    T = X.shape[0]
+    U = np.zeros((T, As.shape[1]))
+    Y = X @ Wp.T
+    for t in range(T):
+        i = int(idx[t])
+        U[t] = As[i] @ X[t]
+        Y[t] = Y[t] + ss[i] * (Bs[i] @ U[t])
+    return {"U": U, "Y": Y}
+
+
+def backward_multi(X: np.ndarray, Wp: np.ndarray, As: np.ndarray, Bs: np.ndarray, ss: np.ndarray,
+                   idx: np.ndarray, dY: np.ndarray) -> Dict[str, np.ndarray]:
+    """Gradients of <dY, Y> for forward_multi, token by token:
+    G[t] = dY[t] B_i;  dX[t] = dY[t] W' + s_i G[t] A_i;
+    dA_i = s_i sum over tokens of adapter i of G[t]^T X[t];
+    dB_i = s_i sum over those tokens of dY[t]^T (X[t] A_i^T)."""
+    dX = dY @ Wp
+    dAs = np.zeros_like(As, dtype=np.float64)
+    dBs = np.zeros_like(Bs, dtype=np.float64)
+    for t in range(X.shape[0]):
+        i = int(idx[t])
+        G = dY[t] @ Bs[i]
+        dX[t] = dX[t] + ss[i] * (G @ As[i])
+        dAs[i] += ss[i] * np.outer(G, X[t])
+        dBs[i] += ss[i] * np.outer(dY[t], As[i] @ X[t])
+    return {"dX": dX, "dA": dAs, "dB": dBs}
 
 
 def merge(Wp: np.ndarray, A: np.ndarray, B: np.ndarray, s: float) -> np.ndarray:

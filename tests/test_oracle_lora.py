@@ -194,3 +194,73 @@ def test_dropout_rejects_p_one():
     X, Wp, A, B, dY, keep = _small()
     with pytest.raises(ValueError):
         lora.forward_dropout(X, Wp, A, B, 1.0, keep, 1.0)
+
+
+# ---------------------------------------------------------------------------
+# Several unmerged adapters in one batch: pins by reduction to the single-
+# adapter routines (pinned above), permutation and directional derivatives
+# ---------------------------------------------------------------------------
+def _multi(seed=4, T=30, d=18, k=12, r=3, n=3):
+    rng = np.random.default_rng(seed)
+    X = rng.standard_normal((T, k))
+    Wp = rng.standard_normal((d, k)) * 0.1
+    As = rng.standard_normal((n, r, k)) * 0.3
+    Bs = rng.standard_normal((n, d, r)) * 0.2
+    ss = np.array([0.5, 2.0, 1.25])[:n]
+    idx = rng.integers(0, n, T)
+    dY = rng.standard_normal((T, d))
+    return X, Wp, As, Bs, ss, idx, dY
+
+
+def test_multi_with_one_adapter_is_plain_lora():
+    X, Wp, As, Bs, ss, _, dY = _multi()
+    idx = np.zeros(X.shape[0], int)
+    f = lora.forward_multi(X, Wp, As, Bs, ss, idx)
+    f1 = lora.forward(X, Wp, As[0], Bs[0], ss[0])
+    np.testing.assert_allclose(f["Y"], f1["Y"], rtol=1e-13, atol=1e-13)
+    b = lora.backward_multi(X, Wp, As, Bs, ss, idx, dY)
+    b1 = lora.backward(X, Wp, As[0], Bs[0], ss[0], dY)
+    for key in ("dX", "dA", "dB"):
+        got = b[key] if key == "dX" else b[key][0]
+        np.testing.assert_allclose(got, b1[key], rtol=1e-12, atol=1e-12)
+    assert np.all(b["dA"][1:] == 0) and np.all(b["dB"][1:] == 0)
+
+
+def test_multi_equals_separate_runs_per_adapter():
+    X, Wp, As, Bs, ss, idx, dY = _multi()
+    f = lora.forward_multi(X, Wp, As, Bs, ss, idx)
+    b = lora.backward_multi(X, Wp, As, Bs, ss, idx, dY)
+    for i in range(As.shape[0]):
+        rows = np.nonzero(idx == i)[0]
+        fi = lora.forward(X[rows], Wp, As[i], Bs[i], ss[i])
+        np.testing.assert_allclose(f["Y"][rows], fi["Y"], rtol=1e-12, atol=1e-12)
+        gi = lora.backward(X[rows], Wp, As[i], Bs[i], ss[i], dY[rows])
+        np.testing.assert_allclose(b["dX"][rows], gi["dX"], rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(b["dA"][i], gi["dA"], rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(b["dB"][i], gi["dB"], rtol=1e-12, atol=1e-12)
+
+
+def test_multi_is_invariant_to_token_order():
+    X, Wp, As, Bs, ss, idx, dY = _multi(seed=8)
+    perm = np.random.default_rng(2).permutation(X.shape[0])
+    a = lora.backward_multi(X, Wp, As, Bs, ss, idx, dY)
+    b = lora.backward_multi(X[perm], Wp, As, Bs, ss, idx[perm], dY[perm])
+    np.testing.assert_allclose(a["dX"][perm], b["dX"], rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(a["dA"], b["dA"], rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(a["dB"], b["dB"], rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("wrt", ["X", "As", "Bs"])
+def test_multi_gradients_match_directional_derivatives(wrt):
+    X, Wp, As, Bs, ss, idx, dY = _multi(seed=12)
+    args = {"X": X, "As": As, "Bs": Bs}
+    E = np.random.default_rng(5).standard_normal(args[wrt].shape)
+
+    def loss(v):
+        a = dict(args, **{wrt: v})
+        return np.sum(dY * lora.forward_multi(a["X"], Wp, a["As"], a["Bs"], ss, idx)["Y"])
+
+    h = 1e-3
+    num = (loss(args[wrt] + h * E) - loss(args[wrt] - h * E)) / (2 * h)
+    g = lora.backward_multi(X, Wp, As, Bs, ss, idx, dY)[{"X": "dX", "As": "dA", "Bs": "dB"}[wrt]]
+    assert abs(num - np.sum(g * E)) <= 1e-8 * (1 + abs(num))
