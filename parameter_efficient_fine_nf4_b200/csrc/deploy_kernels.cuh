@@ -14,8 +14,9 @@
 //     accumulators;
 //   * warps 2-9 combine accumulator and input row by row; each warp writes
 //     its 32 x 128 part of the bf16 result into swizzled shared boxes of its
-//     own (in place over W for unmerge) and stores them with TMA itself, so
-//     the eight warps never wait for one another.
+//     own (in place over W for unmerge) and stores them with TMA itself
+//     (lines marked evict-first in L2), so the warps never wait for one
+//     another.
 // Rows or columns beyond d or k are zero-filled by the loads and clipped by
 // the stores, so no element masks are needed.
 #pragma once
@@ -57,6 +58,24 @@ struct DeployCfg {
 constexpr int kEpiWarps = 16;
 constexpr int kEpiThreads = kEpiWarps * 32;
 constexpr int kDeployThreads = 64 + kEpiThreads;
+
+// L2 policy marking lines for early eviction: the output is written once and
+// not read again here, so it should not displace other lines.
+__device__ __forceinline__ uint64_t l2_policy_evict_first() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
+// 2-D tiled TMA store from this CTA's shared memory with an L2 cache policy.
+__device__ __forceinline__ void tma_store_2d_hint(const CUtensorMap* map, uint32_t src, int32_t x, int32_t y,
+                                                  uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.global.shared::cta.bulk_group.L2::cache_hint [%0, {%2, %3}], [%1], %4;" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(src), "r"(x), "r"(y), "l"(pol)
+      : "memory");
+}
 
 // Byte offset of 16-byte chunk `chunk` (0..7) of row `row` in a 128-byte-row,
 // 128B-swizzled tile.
@@ -286,6 +305,7 @@ __global__ void __launch_bounds__(kDeployThreads, 1)
     const float mu = kMerge ? p.mean[0] : 0.f;
     const uint32_t lut_lane = smem_u32(&s_wlut[kMerge ? ew : 0][0][lane]);
     uint8_t* stg = gOut + ew * 4096;
+    const uint64_t out_policy = l2_policy_evict_first();
     const uint32_t stg_s = sOut + (uint32_t)ew * 4096u;
     // raw scale inputs of this thread's block, loaded one tile ahead so their
     // latency hides behind a whole tile of work
@@ -380,7 +400,7 @@ __global__ void __launch_bounds__(kDeployThreads, 1)
       __syncwarp();
       if (lane == 0) {
         const uint32_t src = kMerge ? stg_s : sIo + (uint32_t)(s * Cfg::kIo + bxi * 16384 + quarter * 4096);
-        tma_store_2d(&tmOut, src, n0 + 64 * bxi, m0 + quarter * 32);
+        tma_store_2d_hint(&tmOut, src, n0 + 64 * bxi, m0 + quarter * 32, out_policy);
         bulk_commit_group();
         // input tile released: merge once the codes are read (they were, by
         // the __syncwarp above); unmerge once the store has read it
