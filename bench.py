@@ -43,6 +43,23 @@ def algorithmic_flops(T, d, k, r):
     return 4 * T * d * k + 6 * T * r * (d + k)
 
 
+def nf4_bytes(d, k):
+    """Stored bytes of one NF4 weight: codes, E4M3 constants, group scales, mean."""
+    n_b = d * k // 64
+    return d * k // 2 + n_b + 4 * ((n_b + 255) // 256) + 4
+
+
+def algorithmic_bytes(T, d, k, r):
+    """Least HBM traffic of one forward plus one backward call: the NF4 weight
+    is read by each; A and B are read by each; the forward reads X and writes
+    Y and U (fp32); the backward reads X, U and dY and writes dX, dA and dB
+    (fp32)."""
+    weights = 2 * nf4_bytes(d, k)
+    adapters = 2 * 2 * (r * k + d * r) + 4 * (r * k + d * r)
+    acts = (2 * T * k + 2 * T * d + 4 * T * r) + (2 * T * k + 4 * T * r + 2 * T * d + 2 * T * k)
+    return weights + adapters + acts
+
+
 def workload(config_index: int):
     cfg = synthetic.config(config_index)
     T = cfg.tokens[0]
@@ -210,11 +227,12 @@ def run_reference(args):
 
 
 # --------------------------------------------------------------------------- GPU arm
-# The files the roofline kernel (gemm_tc_kernel) is built from: its header,
+# The files the roofline kernel (gemm_nf4_kernel) is built from: its header,
 # the headers that one includes, the C ABI header, and the host file that sets
 # its launch parameters.  Its recorded DRAM traffic stays valid while these
 # are unchanged (other kernels of the library live in other headers).
-GEMM_SOURCES = ("parameter_efficient_fine_nf4_b200/csrc/gemm_tc.cuh",
+GEMM_SOURCES = ("parameter_efficient_fine_nf4_b200/csrc/nf4_gemm.cuh",
+                "parameter_efficient_fine_nf4_b200/csrc/gemm_tc.cuh",
                 "parameter_efficient_fine_nf4_b200/csrc/ptx.cuh",
                 "parameter_efficient_fine_nf4_b200/csrc/nf4_kernels.cuh",
                 "parameter_efficient_fine_nf4_b200/csrc/libqlora.cu",
@@ -242,6 +260,148 @@ def read_traffic(kernel: str):
         return t.get("kernels", {}).get(kernel)
     except Exception:
         return None
+
+
+FWD_BWD_KERNELS = ("gemm_lora_down", "gemm_fwd_main", "gemm_nf4_fwd", "gemm_nf4_small_fwd", "pad_cols_bf16",
+                   "scale_f32_to_bf16_hilo", "gemm_lora_g", "gemm_lora_dB", "splitk_reduce_f32", "gemm_lora_dA",
+                   "gemm_bwd_dx", "gemm_nf4_dx", "gemm_nf4_small_dx", "memset")
+
+
+def measure_write_ceiling(torch, dev, stream, nbytes=512 << 20, reps=5):
+    """A plain fill of a buffer larger than L2 (a torch kernel): the rate at
+    which this GPU writes HBM, the ceiling of write-dominated kernels."""
+    buf = torch.empty(nbytes // 4, dtype=torch.float32, device=dev)
+    buf.fill_(1.0)
+    torch.cuda.synchronize(dev)
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(reps):
+        buf.fill_(0.5)
+    b.record(stream)
+    b.synchronize()
+    ms = a.elapsed_time(b) / reps
+    del buf
+    return {"gbs": nbytes / 1e9 / (ms / 1e3), "how": f"torch fill_ of {nbytes >> 20} MiB, {reps} calls"}
+
+
+def make_device_layers(torch, q4, cfg, T, dev, rank=0):
+    """Device tensors of every linear of `cfg` with T tokens: the frozen W0 drawn
+    from the config's distribution (quantised once here), A and B from the
+    seeded host recipe, X and dY ~ N(0, 1) drawn on the device."""
+    out = []
+
+    def bf16_host(bits):
+        return torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(dev)
+
+    for li, lin in enumerate(cfg.linears):
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(synthetic.seed_for(cfg.index, "W0", li))
+        W0 = torch.randn(lin.d, lin.k, generator=gen, device=dev, dtype=torch.float32) * cfg.sigma_w
+        A = bf16_host(synthetic.normal_bf16(synthetic.seed_for(cfg.index, "A", li), (cfg.r, lin.k), cfg.sigma_a))
+        B = bf16_host(synthetic.normal_bf16(synthetic.seed_for(cfg.index, "B", li), (lin.d, cfg.r), cfg.sigma_b))
+        gen.manual_seed(synthetic.seed_for(cfg.index, "X", li) + 1000 * rank)
+        X = torch.randn(T, lin.k, generator=gen, device=dev, dtype=torch.float32).to(torch.bfloat16)
+        dY = torch.randn(T, lin.d, generator=gen, device=dev, dtype=torch.float32).to(torch.bfloat16)
+        qw = q4.qlora_nf4_quantize(W0)
+        del W0
+        nbytes = max(q4.qlora_fwd_workspace_bytes(lin.d, lin.k, cfg.r, T),
+                     q4.qlora_bwd_workspace_bytes(lin.d, lin.k, cfg.r, T),
+                     q4.lora_merge_workspace_bytes(lin.d, lin.k, cfg.r))
+        out.append({"lin": lin, "qw": qw, "A": A, "B": B, "X": X, "dY": dY,
+                    "Y": torch.empty(T, lin.d, dtype=torch.bfloat16, device=dev),
+                    "U": torch.empty(T, cfg.r, dtype=torch.float32, device=dev),
+                    "dX": torch.empty(T, lin.k, dtype=torch.bfloat16, device=dev),
+                    "dA": torch.empty(cfg.r, lin.k, dtype=torch.float32, device=dev),
+                    "dB": torch.empty(lin.d, cfg.r, dtype=torch.float32, device=dev),
+                    "ws": q4.workspace(nbytes, dev)})
+    return out
+
+
+def config_block(torch, q4, dev, stream, flush, peaks, write_ceiling, steps=10, warmup=3):
+    """fwd+bwd of every linear of configs 1, 2, 3 and 5 (T = 4096 and T = 16),
+    timed like the headline (CUDA events per step on the launch stream, L2
+    flushed between steps outside the events), plus merge and unmerge of
+    config 3 alone.  Returns the per-config entries of the JSON line."""
+    hbm = float(peaks.get("hbm_gbs"))
+    burst = float(peaks.get("bf16_tflops"))
+    sustained = float(peaks.get("bf16_tflops_sustained", burst))
+    out = {}
+    cases = [(1, 16), (2, 4096), (3, 8192), (5, 4096), (5, 16)]
+    for ci, T in cases:
+        cfg = synthetic.config(ci)
+        layers = make_device_layers(torch, q4, cfg, T, dev)
+
+        def step():
+            for L in layers:
+                q4.qlora_fwd(L["qw"], L["A"], L["B"], cfg.alpha, L["X"], Y=L["Y"], U_save=L["U"], ws=L["ws"])
+                q4.qlora_bwd(L["qw"], L["A"], L["B"], cfg.alpha, L["X"], L["U"], L["dY"], dX=L["dX"],
+                             dA=L["dA"], dB=L["dB"], ws=L["ws"])
+
+        for _ in range(warmup):
+            step()
+        torch.cuda.synchronize(dev)
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        n0 = q4.qlora_launch_count()
+        for i in range(steps):
+            flush.zero_()
+            evs[i][0].record(stream)
+            step()
+            evs[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+        launches = (q4.qlora_launch_count() - n0) / steps
+        assert q4.qlora_get_device_status() == 0
+        ms = statistics.median(a.elapsed_time(b) for a, b in evs)
+        flops = sum(algorithmic_flops(T, L["lin"].d, L["lin"].k, cfg.r) for L in layers)
+        nbytes = sum(algorithmic_bytes(T, L["lin"].d, L["lin"].k, cfg.r) for L in layers)
+        key = f"config{ci}_T{T}"
+        e = {"linears": [f"{L['lin'].name} {L['lin'].k}->{L['lin'].d}" for L in layers], "r": cfg.r,
+             "tokens": T, "ms_fwd_bwd": ms, "us_fwd_bwd": 1e3 * ms, "tflops": flops / (ms / 1e3) / 1e12,
+             "frac_of_dense_burst": flops / (ms / 1e3) / 1e12 / burst,
+             "frac_of_sustained": flops / (ms / 1e3) / 1e12 / sustained,
+             "tokens_per_s": T / (ms / 1e3), "launches_per_step": launches,
+             "algorithmic_bytes": nbytes, "gbs": nbytes / 1e9 / (ms / 1e3),
+             "frac_of_hbm": nbytes / 1e9 / (ms / 1e3) / hbm}
+        e["bound"] = "hbm" if T <= 64 else "tensor"
+        # per-kernel device time of one more step (library profiler: events on
+        # the launch stream around every launch)
+        flush.zero_()
+        torch.cuda.synchronize(dev)
+        q4.qlora_profile_begin()
+        step()
+        st = q4.qlora_profile_end()
+        e["kernels_us"] = {x["name"]: round(1e3 * x["total_ms"], 2) for x in st}
+        out[key] = e
+        if cfg.merge:
+            L = layers[0]
+            lin = L["lin"]
+            Wm = torch.empty(lin.d, lin.k, dtype=torch.bfloat16, device=dev)
+            W0u = torch.empty_like(Wm)
+            for name, fn, bpw, kern in (
+                    ("merge", lambda: q4.lora_merge(L["qw"], L["A"], L["B"], cfg.alpha, W_out=Wm, ws=L["ws"]),
+                     2.5 + 1 / 64, "lora_merge"),
+                    ("unmerge", lambda: q4.lora_unmerge(Wm, L["A"], L["B"], cfg.alpha, W0_out=W0u, ws=L["ws"]),
+                     4.0, "lora_unmerge")):
+                for _ in range(warmup):
+                    fn()
+                torch.cuda.synchronize(dev)
+                times = []
+                for _ in range(steps):
+                    flush.zero_()
+                    q4.qlora_profile_begin()
+                    fn()
+                    st = q4.qlora_profile_end()
+                    times.append(sum(x["total_ms"] for x in st if x["name"] == kern))
+                ms1 = statistics.median(times)
+                gbs = lin.d * lin.k * bpw / 1e9 / (ms1 / 1e3)
+                m = {"us": 1e3 * ms1, "gbs": gbs, "frac_of_hbm": gbs / hbm, "bytes_per_weight": bpw}
+                if name == "merge" and write_ceiling:
+                    m["frac_of_write_ceiling"] = gbs / write_ceiling["gbs"]
+                out[f"config{ci}_{name}"] = m
+            del Wm, W0u
+        del layers
+        torch.cuda.empty_cache()
+    return out
 
 
 def run_ours(args):
@@ -447,29 +607,41 @@ def run_ours(args):
         alone[name] = per_call_ms(st_alone, kernels[name], 5)
     assert q4.qlora_get_device_status() == 0
 
-    fb_names = ("nf4_dequantize", "gemm_lora_down", "gemm_fwd_main", "pad_cols_bf16", "scale_f32_to_bf16_hilo",
-                "gemm_lora_g", "gemm_lora_dB", "splitk_reduce_f32", "gemm_lora_dA", "gemm_bwd_dx")
+    fb_names = FWD_BWD_KERNELS
     fb_ms = sum(x["total_ms"] for x in stats if x["name"] in fb_names) / args.steps
     fwd_bwd_value = flops_rank * world / (fb_ms / 1e3) / 1e12 if fb_ms > 0 else None
 
-    # ---- roofline of the dominant kernel (the tcgen05 GEMM: forward main and dX)
+    # ---- roofline of the dominant kernel (the tcgen05 base GEMM: forward and dX)
     peaks, peak_src = read_peaks()
     hbm = float(peaks.get("hbm_gbs"))
+    write_ceiling = None if plain else measure_write_ceiling(torch, dev, stream)
     hbm_rows = {}
     for name in () if plain else bpw:
-        calls = args.steps * (2 if name == "dequantise" else 1)
-        ms_step = per_call_ms(stats, kernels[name], calls)
         gb = weights * bpw[name] / 1e9
-        hbm_rows[name] = {"bytes_per_weight": round(bpw[name], 4),
-                          "in_step_gbs": gb / (ms_step / 1e3), "in_step_frac": gb / (ms_step / 1e3) / hbm,
-                          "alone_gbs": gb / (alone[name] / 1e3), "alone_frac": gb / (alone[name] / 1e3) / hbm}
-    gemm = [s for s in stats if s["name"] in ("gemm_fwd_main", "gemm_bwd_dx")]
+        row = {"bytes_per_weight": round(bpw[name], 4),
+               "alone_gbs": gb / (alone[name] / 1e3), "alone_frac": gb / (alone[name] / 1e3) / hbm}
+        if name in ("merge", "dequantise") and write_ceiling:
+            # 2 of the 2.5 bytes per weight are writes: also against a plain fill
+            row["alone_frac_of_write_ceiling"] = row["alone_gbs"] / write_ceiling["gbs"]
+        ms_step = per_call_ms(stats, kernels[name], args.steps)
+        if ms_step > 0:
+            row["in_step_gbs"] = gb / (ms_step / 1e3)
+            row["in_step_frac"] = gb / (ms_step / 1e3) / hbm
+        else:
+            row["in_step"] = "not part of the step (the GEMMs dequantise internally)"
+        hbm_rows[name] = row
+    gemm_names = ("gemm_fwd_main", "gemm_bwd_dx") if plain else ("gemm_nf4_fwd", "gemm_nf4_dx")
+    gemm = [s for s in stats if s["name"] in gemm_names]
     g_ms = sum(s["total_ms"] for s in gemm)
     g_launches = sum(s["launches"] for s in gemm)
     g_flops = sum(s["flops"] for s in gemm)
     achieved = g_flops / (g_ms / 1e3) / 1e12 if g_ms > 0 else 0.0
     peak = float(peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops")))
-    traffic = read_traffic("gemm_tc_kernel")
+    peak_burst = float(peaks.get("bf16_tflops"))
+    traffic = read_traffic("gemm_tc_kernel" if plain else "gemm_nf4_kernel")
+    per_config = None
+    if rank == 0 and world == 1 and not args.no_configs and not plain:
+        per_config = config_block(torch, q4, dev, stream, flush, peaks, write_ceiling)
     rows = {s["name"]: {"launches": s["launches"], "ms_per_step": s["total_ms"] / args.steps,
                         "share": s["total_ms"] / max(1e-9, sum(x["total_ms"] for x in stats))}
             for s in stats}
@@ -494,10 +666,15 @@ def run_ours(args):
             "fwd_bwd_only": {"value": fwd_bwd_value, "unit": "TFLOP/s",
                              "note": "same flops over the forward and backward kernels of the step alone "
                                      "(quantise, merge and unmerge launches left out)"},
-            "roofline": {"kernel": "gemm_tc_kernel<256> (fwd main + dX)", "bound": "tensor",
+            "roofline": {"kernel": ("gemm_tc_kernel<256> (fwd main + dX on the bf16 base)" if plain else
+                                    "gemm_nf4_kernel (fwd + dX, NF4 dequantised inside the GEMM)"),
+                         "bound": "tensor",
                          "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                          "frac": achieved / peak if peak else None, "traffic": traffic,
-                         "peak_source": f"{peak_src} bf16_tflops_sustained",
+                         "peak_source": f"{peak_src} bf16_tflops_sustained (kernel timed inside a long, "
+                                        "power-capped step)",
+                         "frac_of_dense_burst": achieved / peak_burst if peak_burst else None,
+                         "dense_burst_peak": peak_burst,
                          "launches": g_launches, "ms_per_launch": g_ms / max(1, g_launches)},
             "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": float(te.item()), "steps": e2e_steps,
@@ -508,9 +685,12 @@ def run_ours(args):
             "clocks": clk,
             "rows": rows,
             "hbm_rows": {"peak_gbs": hbm, "peak_source": f"{peak_src} hbm_gbs",
+                         "write_ceiling": write_ceiling,
                          "note": "in the step (clocks held down by the power-capped GEMMs) and alone "
                                  "(5 calls back to back after the timed region)", **hbm_rows},
         }
+        if per_config is not None:
+            line["configs"] = per_config
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(cfg)
         print(json.dumps(line), flush=True)
@@ -589,6 +769,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", type=int, default=4)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the per-config block (configs 1, 2, 3, 5) of the JSON line")
     ap.add_argument("--base", choices=["nf4", "bf16"], default="nf4",
                     help="nf4: the QLoRA path (default); bf16: plain LoRA on the bf16 base")
     ap.add_argument("--deploy-only", action="store_true",

@@ -154,8 +154,10 @@ QLORA_API int qlora_nf4_dequantize(const qlora_nf4_t* q, uint16_t* W_out, qlora_
  * QLORA_ERR_EXCEEDS_STATIC_SCRATCH before anything is launched.
  *
  * The first call on a device looks up the array's device address (with that
- * device current) and caches it; make that first call before any stream
- * capture begins.  All calls share the one array, which keeps the contents
+ * device current) and caches it with the id of the current CUDA context; make
+ * that first call before any stream capture begins.  After a device reset the
+ * next call runs in a new context and looks the address up again (the array's
+ * contents start over then).  All calls share the one array, which keeps the contents
  * of the last call; every byte a call reads from it is first written by the
  * same call, so nothing needs clearing.  Calls that overlap on the GPU (on
  * different streams, or from different threads) race on the array and must
@@ -203,6 +205,34 @@ QLORA_API int qlora_bwd(const qlora_nf4_t* q, const uint16_t* A, const uint16_t*
               const uint16_t* X, const float* U_saved, const uint16_t* dY, int64_t T,
               uint16_t* dX, float* dA, float* dB, void* workspace, size_t workspace_bytes,
               qlora_stream_t stream);
+
+/* ------------------------------------------------ LoRA dropout (next row) */
+
+/*
+ * The layer with LoRA dropout on the adapter input ([P5] "LoRA vs QLoRA:
+ * Parameter-Efficient Fine-Tuning Explained", run configuration: a LoRA
+ * dropout of 0.05-0.1).  The pages give no formula; this library applies
+ * inverted dropout to the input of the adapter path only:
+ *   D(X) = X * keep / (1 - p),   U = D(X) A^T,   Y = X W'^T + s U B^T
+ * and the matching gradients
+ *   G = dY B,  dX = dY W' + D(s G A),  dA = s G^T D(X),  dB = s dY^T U.
+ * keep: device, bit-packed T x k mask drawn by the caller (bit j % 8 of byte
+ * (t*k + j) / 8 is 1 where element (t, j) is kept), 16-byte aligned; the
+ * forward and the backward of one step must get the same mask.  0 <= p < 1;
+ * p == 0 ignores `keep` and is exactly qlora_fwd / qlora_bwd.  U_save holds
+ * the dropped-out U for the backward.  Otherwise the arguments, results and
+ * errors are those of qlora_fwd / qlora_bwd; the workspaces also hold the
+ * masked input (T x k bf16).
+ */
+QLORA_API size_t qlora_fwd_dropout_workspace_bytes(int64_t d, int64_t k, int r, int64_t T);
+QLORA_API int qlora_fwd_dropout(const qlora_nf4_t* q, const uint16_t* A, const uint16_t* B, int r, float alpha,
+                                const uint16_t* X, const uint8_t* keep, float p, int64_t T, uint16_t* Y,
+                                float* U_save, void* workspace, size_t workspace_bytes, qlora_stream_t stream);
+QLORA_API size_t qlora_bwd_dropout_workspace_bytes(int64_t d, int64_t k, int r, int64_t T);
+QLORA_API int qlora_bwd_dropout(const qlora_nf4_t* q, const uint16_t* A, const uint16_t* B, int r, float alpha,
+                                const uint16_t* X, const uint8_t* keep, float p, const float* U_saved,
+                                const uint16_t* dY, int64_t T, uint16_t* dX, float* dA, float* dB,
+                                void* workspace, size_t workspace_bytes, qlora_stream_t stream);
 
 /* ------------------------------------------- plain LoRA on a bf16 base */
 

@@ -147,20 +147,29 @@ def e4m3_value(codes: np.ndarray) -> np.ndarray:
 # --------------------------------------------------------------------------
 # bf16 rounding (own definition: 8 significant bits, ties to even)
 # --------------------------------------------------------------------------
+BF16_MIN_NORMAL = 2.0 ** -126
+BF16_SUBNORMAL_STEP = 2.0 ** -133     # 7 fraction bits below the smallest normal
+BF16_MAX = (2.0 - 2.0 ** -7) * 2.0 ** 127
+
+
 def to_bf16_bits(x: np.ndarray) -> np.ndarray:
     """Round float64 values to bf16 (nearest, ties to even); return uint16 bits.
 
     A bf16 number has an 8-bit significand and float32's exponent range.  With
-    x = m * 2^e, 0.5 <= |m| < 1, the rounded value is rint(m * 256) / 256 * 2^e
-    (numpy's rint rounds half to even).  Values here are normal numbers far
-    from the exponent limits; that is asserted.
+    x = m * 2^e, 0.5 <= |m| < 1, a normal result is rint(m * 256) / 256 * 2^e
+    (numpy's rint rounds half to even).  Below the smallest normal 2^-126 the
+    representable values are the multiples of 2^-133 (exponent field 0, seven
+    fraction bits), so the result is rint(x / 2^-133) * 2^-133; a value that
+    rounds up to 2^-126 is the smallest normal.  Results beyond the largest
+    finite bf16 are outside this oracle (asserted).
     """
     x = np.asarray(x, dtype=np.float64)
     m, e = np.frexp(x)
     r = np.ldexp(np.rint(m * 256.0), e - 8)
-    nz = r != 0
-    assert np.all(np.abs(r[nz]) > 2.0 ** -126) and np.all(np.abs(r) < 3.0e38)
-    f = r.astype(np.float32)                      # exact: 8 significant bits
+    sub = np.abs(x) < BF16_MIN_NORMAL
+    r = np.where(sub, np.rint(x / BF16_SUBNORMAL_STEP) * BF16_SUBNORMAL_STEP, r)
+    assert np.all(np.abs(r) <= BF16_MAX)
+    f = r.astype(np.float32)                      # exact: at most 8 significant bits
     bits = (f.view(np.uint32) >> 16).astype(np.uint16)
     # zero keeps the sign of the input
     bits = np.where(r == 0, np.where(np.signbit(x), 0x8000, 0).astype(np.uint16), bits)

@@ -65,6 +65,11 @@ _SIGNATURES = {
     "qlora_bwd_workspace_bytes": (_SIZE, [_I64, _I64, _INT, _I64]),
     "qlora_bwd": (_INT, [_NF4P, _VP, _VP, _INT, _F, _VP, _VP, _VP, _I64, _VP, _VP, _VP, _VP,
                          _SIZE, _VP]),
+    "qlora_fwd_dropout_workspace_bytes": (_SIZE, [_I64, _I64, _INT, _I64]),
+    "qlora_fwd_dropout": (_INT, [_NF4P, _VP, _VP, _INT, _F, _VP, _VP, _F, _I64, _VP, _VP, _VP, _SIZE, _VP]),
+    "qlora_bwd_dropout_workspace_bytes": (_SIZE, [_I64, _I64, _INT, _I64]),
+    "qlora_bwd_dropout": (_INT, [_NF4P, _VP, _VP, _INT, _F, _VP, _VP, _F, _VP, _VP, _I64, _VP, _VP, _VP, _VP,
+                                 _SIZE, _VP]),
     "lora_fwd_workspace_bytes": (_SIZE, [_I64, _I64, _INT, _I64]),
     "lora_fwd": (_INT, [_VP, _I64, _I64, _VP, _VP, _INT, _F, _VP, _I64, _VP, _VP, _VP, _SIZE, _VP]),
     "lora_bwd_workspace_bytes": (_SIZE, [_I64, _I64, _INT, _I64]),
@@ -278,6 +283,72 @@ def qlora_bwd(q: NF4Weight, A: torch.Tensor, B: torch.Tensor, alpha: float, X: t
                          _ptr(U_saved), _ptr(dY), T, _ptr(dX), _ptr(dA), _ptr(dB), _ptr(ws),
                          ws.numel(), _stream(stream))
     _check(st, "qlora_bwd")
+    return dX, dA, dB
+
+
+def qlora_fwd_dropout_workspace_bytes(d: int, k: int, r: int, T: int) -> int:
+    return lib().qlora_fwd_dropout_workspace_bytes(d, k, r, T)
+
+
+def qlora_bwd_dropout_workspace_bytes(d: int, k: int, r: int, T: int) -> int:
+    return lib().qlora_bwd_dropout_workspace_bytes(d, k, r, T)
+
+
+def _need_keep(keep: Optional[torch.Tensor], T: int, k: int, p: float):
+    if p == 0.0 and keep is None:
+        return None
+    _need(keep, torch.uint8, (T * k // 8,), "keep")
+    return _ptr(keep)
+
+
+def qlora_fwd_dropout(q: NF4Weight, A: torch.Tensor, B: torch.Tensor, alpha: float, X: torch.Tensor,
+                      keep: Optional[torch.Tensor], p: float, Y: Optional[torch.Tensor] = None,
+                      U_save: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None,
+                      stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Forward with LoRA dropout on the adapter input (keep: bit-packed T*k/8 bytes)."""
+    r = A.shape[0]
+    T = X.shape[0]
+    _need(A, torch.bfloat16, (r, q.k), "A")
+    _need(B, torch.bfloat16, (q.d, r), "B")
+    _need(X, torch.bfloat16, (T, q.k), "X")
+    kp = _need_keep(keep, T, q.k, p)
+    dev = X.device
+    Y = torch.empty(T, q.d, dtype=torch.bfloat16, device=dev) if Y is None else Y
+    U_save = torch.empty(T, r, dtype=torch.float32, device=dev) if U_save is None else U_save
+    _need(Y, torch.bfloat16, (T, q.d), "Y")
+    _need(U_save, torch.float32, (T, r), "U_save")
+    ws = workspace(qlora_fwd_dropout_workspace_bytes(q.d, q.k, r, T), dev) if ws is None else ws
+    st = lib().qlora_fwd_dropout(ctypes.byref(q.cstruct), _ptr(A), _ptr(B), r, float(alpha), _ptr(X), kp,
+                                 float(p), T, _ptr(Y), _ptr(U_save), _ptr(ws), ws.numel(), _stream(stream))
+    _check(st, "qlora_fwd_dropout")
+    return Y, U_save
+
+
+def qlora_bwd_dropout(q: NF4Weight, A: torch.Tensor, B: torch.Tensor, alpha: float, X: torch.Tensor,
+                      keep: Optional[torch.Tensor], p: float, U_saved: torch.Tensor, dY: torch.Tensor,
+                      dX: Optional[torch.Tensor] = None, dA: Optional[torch.Tensor] = None,
+                      dB: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None, stream=None):
+    """Backward of qlora_fwd_dropout with the same keep mask."""
+    r = A.shape[0]
+    T = X.shape[0]
+    _need(A, torch.bfloat16, (r, q.k), "A")
+    _need(B, torch.bfloat16, (q.d, r), "B")
+    _need(X, torch.bfloat16, (T, q.k), "X")
+    _need(U_saved, torch.float32, (T, r), "U_saved")
+    _need(dY, torch.bfloat16, (T, q.d), "dY")
+    kp = _need_keep(keep, T, q.k, p)
+    dev = X.device
+    dX = torch.empty(T, q.k, dtype=torch.bfloat16, device=dev) if dX is None else dX
+    dA = torch.empty(r, q.k, dtype=torch.float32, device=dev) if dA is None else dA
+    dB = torch.empty(q.d, r, dtype=torch.float32, device=dev) if dB is None else dB
+    _need(dX, torch.bfloat16, (T, q.k), "dX")
+    _need(dA, torch.float32, (r, q.k), "dA")
+    _need(dB, torch.float32, (q.d, r), "dB")
+    ws = workspace(qlora_bwd_dropout_workspace_bytes(q.d, q.k, r, T), dev) if ws is None else ws
+    st = lib().qlora_bwd_dropout(ctypes.byref(q.cstruct), _ptr(A), _ptr(B), r, float(alpha), _ptr(X), kp,
+                                 float(p), _ptr(U_saved), _ptr(dY), T, _ptr(dX), _ptr(dA), _ptr(dB), _ptr(ws),
+                                 ws.numel(), _stream(stream))
+    _check(st, "qlora_bwd_dropout")
     return dX, dA, dB
 
 

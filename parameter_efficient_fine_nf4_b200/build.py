@@ -17,7 +17,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libqlora.so")
 SOURCES = ["libqlora.cu"]
-HEADERS = ["ptx.cuh", "nf4_kernels.cuh", "gemm_tc.cuh", "deploy_kernels.cuh", "adam_kernels.cuh"]
+HEADERS = ["ptx.cuh", "nf4_kernels.cuh", "gemm_tc.cuh", "nf4_gemm.cuh", "deploy_kernels.cuh", "adam_kernels.cuh"]
 
 NVCC_FLAGS = [
     "-O3", "-std=c++17",

@@ -12,11 +12,12 @@
 //     128-byte-swizzled form, double-buffered;
 //   * warp 1 computes (B A) for the tile with tcgen05 into one of two TMEM
 //     accumulators;
-//   * warps 2-9 combine accumulator and input row by row; each warp writes
-//     its 32 x 128 part of the bf16 result into swizzled shared boxes of its
-//     own (in place over W for unmerge) and stores them with TMA itself
-//     (lines marked evict-first in L2), so the warps never wait for one
-//     another.
+//   * sixteen epilogue warps (2-17, four per TMEM lane quarter) each combine
+//     accumulator and input for one 32-row x 64-column box of the tile (one
+//     quantisation block wide), write the bf16 result into a swizzled 4 KB
+//     shared box of their own (in place over W for unmerge) and store it with
+//     TMA themselves (lines marked evict-first in L2), so the warps never
+//     wait for one another.
 // Rows or columns beyond d or k are zero-filled by the loads and clipped by
 // the stores, so no element masks are needed.
 #pragma once

@@ -30,7 +30,8 @@ enum EpiKind : int {
   EPI_F32 = 1,       // out fp32 [M][ldo] = alpha*acc ; out2 bf16 = alpha2*acc
   EPI_F32_T = 2,     // out fp32 [N][ldo] = alpha*acc (transposed store)
   EPI_MERGE = 3,     // out bf16 = bf16(alpha*acc + dequant(codes))
-  EPI_UNMERGE = 4    // out bf16 = bf16(alpha*acc + w_in)
+  EPI_UNMERGE = 4,   // out bf16 = bf16(alpha*acc + w_in)
+  EPI_DROPOUT = 5    // out bf16 = bf16(out + keep * alpha*acc), in place (the masked rank-r term of dX)
 };
 
 struct GemmArgs {
@@ -58,6 +59,8 @@ struct GemmArgs {
   const float* mean;
   const uint16_t* w_in;
   int64_t ldw;
+  const uint8_t* keep;        // EPI_DROPOUT: bit (m * ldk + n) of this array keeps element (m, n)
+  int64_t ldk;
   float levels[16];
 };
 
@@ -170,6 +173,17 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& p, uint32_t (&v)[
         r4[j] = pack_bf16x2(lo, hi);
       }
       o4[i] = make_uint4(r4[0], r4[1], r4[2], r4[3]);
+    }
+  } else if (p.epi == EPI_DROPOUT) {
+    // 32 keep bits of row m, columns n..n+31 (n is a multiple of 32 and ldk of
+    // 32, so the word is aligned); bit i keeps column n + i
+    uint16_t* out = reinterpret_cast<uint16_t*>(p.out) + (int64_t)m * p.ldo + n;
+    const uint32_t bits = *reinterpret_cast<const uint32_t*>(p.keep + ((int64_t)m * p.ldk + n) / 8);
+    for (int i = 0; i < 32 && n + i < p.n_store; ++i) {
+      const float base = bf16_bits_to_f32(out[i]);
+      const float add = ((bits >> i) & 1u) ? __fmul_rn(p.alpha, __uint_as_float(v[i])) : 0.f;
+      const __nv_bfloat16 h = __float2bfloat16_rn(__fadd_rn(base, add));
+      out[i] = *reinterpret_cast<const uint16_t*>(&h);
     }
   } else if (p.epi == EPI_UNMERGE) {
     const uint4* w4 = reinterpret_cast<const uint4*>(p.w_in + (int64_t)m * p.ldw + n);

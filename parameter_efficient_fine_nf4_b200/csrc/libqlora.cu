@@ -19,6 +19,7 @@
 #include "adam_kernels.cuh"
 #include "deploy_kernels.cuh"
 #include "gemm_tc.cuh"
+#include "nf4_gemm.cuh"
 #include "nf4_kernels.cuh"
 #include "ptx.cuh"
 
@@ -138,7 +139,38 @@ EncodeTiledFn encode_fn() {
 
 std::mutex g_init_mu;
 bool g_dev_ready[kMaxDevices] = {false};
+unsigned long long g_dev_ctx[kMaxDevices] = {0};
 int g_dev_sms[kMaxDevices] = {0};
+
+// Unique id of the calling thread's current CUDA context, 0 if there is none
+// yet.  Ids are never reused within a process, so a device reset (which
+// destroys the context; the next runtime call creates a new one) changes it.
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+unsigned long long current_ctx_id() {
+  static const CtxGetCurrentFn get_cur = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return (CtxGetCurrentFn) nullptr;
+    return reinterpret_cast<CtxGetCurrentFn>(p);
+  }();
+  static const CtxGetIdFn get_id = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return (CtxGetIdFn) nullptr;
+    return reinterpret_cast<CtxGetIdFn>(p);
+  }();
+  if (get_cur == nullptr || get_id == nullptr) return 0;
+  CUcontext c = nullptr;
+  if (get_cur(&c) != CUDA_SUCCESS || c == nullptr) return 0;
+  unsigned long long id = 0;
+  if (get_id(c, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
 
 // SM count of the current device (persistent grids are sized to it).
 int current_sms() {
@@ -152,6 +184,41 @@ template <int BN>
 cudaError_t set_gemm_attrs() {
   return cudaFuncSetAttribute(gemm_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               GemmCfg<BN>::kSmemBytes);
+}
+
+template <bool kDx>
+cudaError_t set_nf4_gemm_attrs() {
+  const cudaError_t e = cudaFuncSetAttribute(gemm_nf4_kernel<kDx>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             kNf4SmemBytes);
+  if (e != cudaSuccess) return e;
+  cudaFuncAttributes fa;
+  if (cudaFuncGetAttributes(&fa, gemm_nf4_kernel<kDx>) != cudaSuccess) return cudaErrorInvalidValue;
+  return fa.maxThreadsPerBlock >= kNf4Threads ? cudaSuccess : cudaErrorLaunchOutOfResources;
+}
+
+template <int kSrc, int kOut, int TN>
+cudaError_t set_small_attrs_one() {
+  const cudaError_t e = cudaFuncSetAttribute(gemm_nf4_small_kernel<kSrc, kOut, TN>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, SmallCfg<TN>::kSmem);
+  if (e != cudaSuccess) return e;
+  cudaFuncAttributes fa;
+  if (cudaFuncGetAttributes(&fa, gemm_nf4_small_kernel<kSrc, kOut, TN>) != cudaSuccess)
+    return cudaErrorInvalidValue;
+  return fa.maxThreadsPerBlock >= kSmThreads ? cudaSuccess : cudaErrorLaunchOutOfResources;
+}
+template <int kSrc, int kOut>
+cudaError_t set_small_attrs_tn() {
+  cudaError_t e = set_small_attrs_one<kSrc, kOut, 16>();
+  if (e == cudaSuccess) e = set_small_attrs_one<kSrc, kOut, 32>();
+  if (e == cudaSuccess) e = set_small_attrs_one<kSrc, kOut, 64>();
+  return e;
+}
+cudaError_t set_small_attrs() {
+  cudaError_t e = set_small_attrs_tn<SRC_NF4_ROWS, OUT_BF16>();
+  if (e == cudaSuccess) e = set_small_attrs_tn<SRC_NF4_COLS, OUT_BF16>();
+  if (e == cudaSuccess) e = set_small_attrs_tn<SRC_TMA_K, OUT_U>();
+  if (e == cudaSuccess) e = set_small_attrs_tn<SRC_TMA_MN, OUT_HILO>();
+  return e;
 }
 
 template <bool kMerge, int KS>
@@ -171,7 +238,11 @@ int ensure_device() {
   if (cudaGetDevice(&dev) != cudaSuccess) return QLORA_ERR_NO_DEVICE;
   if (dev < 0 || dev >= kMaxDevices) return QLORA_ERR_NO_DEVICE;
   std::lock_guard<std::mutex> lk(g_init_mu);
-  if (g_dev_ready[dev]) return QLORA_OK;
+  // the kernel attributes below belong to the context: set them again when
+  // the context has changed (after a device reset)
+  const unsigned long long ctx = current_ctx_id();
+  if (g_dev_ready[dev] && ctx != 0 && ctx == g_dev_ctx[dev]) return QLORA_OK;
+  g_dev_ready[dev] = false;
   int major = 0, minor = 0;
   cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
   cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
@@ -182,8 +253,10 @@ int ensure_device() {
   if (set_gemm_attrs<64>() != cudaSuccess || set_gemm_attrs<128>() != cudaSuccess ||
       set_gemm_attrs<256>() != cudaSuccess || set_deploy_attrs<true, 1>() != cudaSuccess ||
       set_deploy_attrs<true, 2>() != cudaSuccess || set_deploy_attrs<false, 1>() != cudaSuccess ||
-      set_deploy_attrs<false, 2>() != cudaSuccess)
+      set_deploy_attrs<false, 2>() != cudaSuccess || set_nf4_gemm_attrs<false>() != cudaSuccess ||
+      set_nf4_gemm_attrs<true>() != cudaSuccess || set_small_attrs() != cudaSuccess)
     return QLORA_ERR_CUDA;
+  g_dev_ctx[dev] = current_ctx_id();
   g_dev_ready[dev] = true;
   return QLORA_OK;
 }
@@ -240,6 +313,12 @@ int launch(const char* name, double flops, double bytes, cudaStream_t stream, F&
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline int64_t round_up(int64_t a, int64_t b) { return (a + b - 1) / b * b; }
 inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+// fp32 product rounded once (the double product of two floats is exact)
+inline float mul_rn_f32(float a, float b) { return (float)((double)a * (double)b); }
+inline int64_t nf4_storage_bytes(int64_t d, int64_t k) {
+  const int64_t n_b = d * k / 64;
+  return d * k / 2 + n_b + 4 * ((n_b + 255) / 256) + 4;
+}
 inline int grid_for(int64_t n, int threads) {
   int64_t g = cdiv(n, threads);
   const int64_t cap = (int64_t)kSMs * 16;
@@ -264,15 +343,15 @@ bool make_map(CUtensorMap* map, const void* base, int64_t inner, int64_t outer, 
 }
 
 // uint8 2-D tensor map (for the NF4 codes): `inner` bytes per row, `outer`
-// rows, `ld` bytes between rows, 128-byte swizzle.
+// rows, `ld` bytes between rows; 128-byte swizzle unless given.
 bool make_map_u8(CUtensorMap* map, const void* base, int64_t inner, int64_t outer, int64_t ld,
-                 int box_inner, int box_outer) {
+                 int box_inner, int box_outer, CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B) {
   cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)outer};
   cuuint64_t strides[1] = {(cuuint64_t)ld};
   cuuint32_t box[2] = {(cuuint32_t)box_inner, (cuuint32_t)box_outer};
   cuuint32_t estr[2] = {1u, 1u};
   CUresult r = encode_fn()(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides,
-                           box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                           box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -459,18 +538,56 @@ const uint16_t* padded_B(const uint16_t* B, int64_t d, int r, int r8, uint16_t* 
   return ws;
 }
 
-struct FwdWs {
-  uint16_t* Wdq; uint16_t* sU; uint16_t* Bp; size_t bytes;
+// Few-token plan of gemm_nf4_small_kernel: tokens padded to TN, 128-row
+// tiles of the Mw output features, the main depth split so that about three
+// CTAs per SM are busy while every split keeps at least four K-steps.
+constexpr int64_t kSmallT = 64;
+struct SmallPlan {
+  int tn = 16, tiles_m = 1, splits = 1, sps = 1;
 };
-// `dequant`: room for the bf16 W' that the QLoRA entry points dequantise into
-// (the plain-LoRA entry points read the caller's bf16 W instead).
-FwdWs carve_fwd(void* ws, int64_t d, int64_t k, int r, int64_t T, bool dequant = true) {
+SmallPlan small_plan(int64_t Mw, int64_t K0, int64_t T) {
+  SmallPlan sp;
+  sp.tn = T <= 16 ? 16 : (T <= 32 ? 32 : 64);
+  sp.tiles_m = (int)cdiv(Mw, 128);
+  const int steps0 = (int)cdiv(K0, 64);
+  const int want = (int)cdiv(3 * kSMs, sp.tiles_m);
+  const int splits = std::max(1, std::min(want, steps0 / 4));
+  sp.sps = (int)cdiv(steps0, splits);
+  sp.splits = (int)cdiv(steps0, sp.sps);
+  return sp;
+}
+
+// Forward workspace: bf16 s*U (the rank-r operand of the extension), B
+// padded to r8 columns, and for T <= 64 the split partials of the few-token
+// kernels (U and Y) with their completion tickets in one array.  No copy of
+// the weight: the QLoRA path dequantises inside the GEMM and plain LoRA reads
+// the caller's W.
+struct FwdWs {
+  uint16_t* sU; uint16_t* Bp;
+  float* part_u; float* part_y; unsigned int* tickets; int n_tickets; int tickets_y_off;
+  uint16_t* Xm;            // LoRA dropout: the masked adapter input
+  size_t bytes;
+};
+FwdWs carve_fwd(void* ws, int64_t d, int64_t k, int r, int64_t T, bool dropout = false) {
   Carver c{reinterpret_cast<uint8_t*>(ws)};
   const int64_t r8 = round_up(r, 8);
   FwdWs w;
-  w.Wdq = (uint16_t*)c.take((size_t)(dequant ? d * k * 2 : 0));
   w.sU = (uint16_t*)c.take((size_t)(std::max<int64_t>(T, 1) * r8 * 2));
   w.Bp = (uint16_t*)c.take((size_t)(d * r8 * 2));
+  w.part_u = w.part_y = nullptr;
+  w.tickets = nullptr;
+  w.n_tickets = w.tickets_y_off = 0;
+  if (T >= 1 && T <= kSmallT) {
+    // U runs over r8 accumulator rows so that the padding columns of sU are
+    // written (as zeros)
+    const SmallPlan su = small_plan(r8, k, T), sy = small_plan(d, k, T);
+    w.part_u = (float*)c.take((size_t)(su.splits > 1 ? (int64_t)su.splits * T * r8 * 4 : 0));
+    w.part_y = (float*)c.take((size_t)(sy.splits > 1 ? (int64_t)sy.splits * T * d * 4 : 0));
+    w.tickets_y_off = su.tiles_m;
+    w.n_tickets = su.tiles_m + sy.tiles_m;
+    w.tickets = (unsigned int*)c.take((size_t)w.n_tickets * 4);
+  }
+  w.Xm = dropout ? (uint16_t*)c.take((size_t)(std::max<int64_t>(T, 1) * k * 2)) : nullptr;
   w.bytes = c.off;
   return w;
 }
@@ -489,7 +606,9 @@ int eff_splits(int64_t K, int splits) {
 }
 
 struct BwdWs {
-  uint16_t* Wdq; uint16_t* Us2; uint16_t* Gs2; uint16_t* Bp; float* partA; float* partB;
+  uint16_t* Us2; uint16_t* Gs2; uint16_t* Bp; float* partA; float* partB;
+  float* part_g; float* part_x; unsigned int* tickets; int n_tickets; int tickets_x_off;
+  uint16_t* Xm;            // LoRA dropout: the masked adapter input
   int rp, halves, splitsA, splitsB; size_t bytes;
 };
 // Backward workspace.  U and G enter the T-reductions (dB, dA) as two bf16
@@ -497,14 +616,13 @@ struct BwdWs {
 // 2*rp columns (rp = r rounded up to 32); with rp <= 128 one GEMM with N = 2*rp
 // multiplies both and the epilogue adds the paired columns, otherwise the two
 // halves run as two GEMMs whose partial outputs are summed.
-BwdWs carve_bwd(void* ws, int64_t d, int64_t k, int r, int64_t T, bool dequant = true) {
+BwdWs carve_bwd(void* ws, int64_t d, int64_t k, int r, int64_t T, bool dropout = false) {
   Carver c{reinterpret_cast<uint8_t*>(ws)};
   const int64_t r8 = round_up(r, 8);
   const int64_t Tm = std::max<int64_t>(T, 1);
   BwdWs w;
   w.rp = (int)round_up(r, 32);
   w.halves = w.rp > 128 ? 2 : 1;
-  w.Wdq = (uint16_t*)c.take((size_t)(dequant ? d * k * 2 : 0));
   w.Us2 = (uint16_t*)c.take((size_t)(Tm * 2 * w.rp * 2));
   w.Gs2 = (uint16_t*)c.take((size_t)(Tm * 2 * w.rp * 2));
   w.Bp = (uint16_t*)c.take((size_t)(d * r8 * 2));
@@ -513,6 +631,20 @@ BwdWs carve_bwd(void* ws, int64_t d, int64_t k, int r, int64_t T, bool dequant =
   const int64_t pa = (int64_t)w.splitsA * w.halves, pb = (int64_t)w.splitsB * w.halves;
   w.partA = (float*)c.take((size_t)(pa > 1 ? pa * r * k * 4 : 0));
   w.partB = (float*)c.take((size_t)(pb > 1 ? pb * d * r * 4 : 0));
+  w.part_g = w.part_x = nullptr;
+  w.tickets = nullptr;
+  w.n_tickets = w.tickets_x_off = 0;
+  if (T >= 1 && T <= kSmallT) {
+    // G runs over rp accumulator rows so that the padding columns of both
+    // halves of sG are written (as zeros)
+    const SmallPlan sg = small_plan(w.rp, d, T), sx = small_plan(k, d, T);
+    w.part_g = (float*)c.take((size_t)(sg.splits > 1 ? (int64_t)sg.splits * T * w.rp * 4 : 0));
+    w.part_x = (float*)c.take((size_t)(sx.splits > 1 ? (int64_t)sx.splits * T * k * 4 : 0));
+    w.tickets_x_off = sg.tiles_m;
+    w.n_tickets = sg.tiles_m + sx.tiles_m;
+    w.tickets = (unsigned int*)c.take((size_t)w.n_tickets * 4);
+  }
+  w.Xm = dropout ? (uint16_t*)c.take((size_t)(Tm * k * 2)) : nullptr;
   w.bytes = c.off;
   return w;
 }
@@ -522,7 +654,7 @@ BwdWs carve_bwd(void* ws, int64_t d, int64_t k, int r, int64_t T, bool dequant =
 // T x 2rp hi/lo operand.  Deterministic: partials are reduced in fixed order.
 int adapter_grad_gemm(const char* name, const uint16_t* big, int64_t M, int64_t T, const uint16_t* hilo,
                       int r, int rp, int halves, int splits, bool transposed, float* out,
-                      float* part, cudaStream_t st) {
+                      float* part, cudaStream_t st, float alpha = 1.0f) {
   const int nparts = splits * halves;
   const int64_t plane = M * r;
   for (int h = 0; h < halves; ++h) {
@@ -531,7 +663,7 @@ int adapter_grad_gemm(const char* name, const uint16_t* big, int64_t M, int64_t 
     g.a0 = mnmajor(big, M, T, M);
     GemmArgs a = blank_args();
     a.epi = transposed ? EPI_F32_T : EPI_F32;
-    a.alpha = 1.0f;
+    a.alpha = alpha;
     a.n_store = r;
     a.ldo = transposed ? M : r;
     if (halves == 1) {
@@ -558,28 +690,235 @@ int adapter_grad_gemm(const char* name, const uint16_t* big, int64_t M, int64_t 
   return QLORA_OK;
 }
 
-// Forward on a bf16 d x k weight W (W' of the QLoRA path, or the caller's W).
-int fwd_core(const uint16_t* W, int64_t d, int64_t k, const uint16_t* A, const uint16_t* B, int r,
+// Base GEMM on the NF4 weight with the rank-r extension (gemm_nf4_kernel):
+//   forward (dx = false): out = Y (T x d)  = [X | sU][W' | B]^T,  a1 = sU (T x r8, ld r8), b1 = B (d x r8)
+//   dX      (dx = true):  out = dX (T x k) = [dY | sG][W' ; A],    a1 = sG (T x r, ld a1_ld), b1 = A (r x k)
+int launch_nf4_gemm(bool dx, const qlora_nf4_t* q, const uint16_t* act, int64_t T, const uint16_t* a1,
+                    int64_t a1_inner, int64_t a1_ld, const uint16_t* b1, int r, int r8, uint16_t* out,
+                    cudaStream_t st) {
+  const int64_t d = q->d, k = q->k;
+  Nf4GemmArgs a;
+  memset(&a, 0, sizeof(a));
+  a.M = (int)T;
+  a.N = (int)(dx ? k : d);
+  a.K0 = (int)(dx ? d : k);
+  a.K1 = r;
+  a.tiles_m = (int)cdiv(T, 256);
+  a.tiles_n = (int)cdiv(a.N, 256);
+  a.group_m = 8;
+  a.absmax_q = q->absmax_q;
+  a.scale2 = q->scale2;
+  a.mean = q->mean;
+  a.kb = k / kBlock;
+  a.wd = (int)d;
+  a.wk = (int)k;
+  memcpy(a.levels, tables().levels, sizeof(a.levels));
+  CUtensorMap mA0, mC, mA1, mB1, mO;
+  if (!make_map(&mA0, act, a.K0, T, a.K0, 128)) return QLORA_ERR_CUDA;
+  if (dx) {
+    if (!make_map_u8(&mC, q->codes, k / 2, d, k / 2, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
+  } else {
+    if (!make_map_u8(&mC, q->codes, k / 2, d, k / 2, 32, 256, CU_TENSOR_MAP_SWIZZLE_32B)) return QLORA_ERR_CUDA;
+  }
+  if (r == 0) {
+    mA1 = mA0;
+    mB1 = mA0;
+  } else {
+    if (!make_map(&mA1, a1, a1_inner, T, a1_ld, 128)) return QLORA_ERR_CUDA;
+    if (dx) {
+      if (!make_map(&mB1, b1, k, r, k, 64)) return QLORA_ERR_CUDA;        // A columns, MN-major
+    } else {
+      if (!make_map(&mB1, b1, r8, d, r8, 256)) return QLORA_ERR_CUDA;     // B rows, K-major
+    }
+  }
+  mO = mA0;
+  a.out = out;
+  a.ldo = a.N;
+  a.tma_store = 0;
+  if (aligned16(out) && (a.N % 8) == 0) {
+    if (!make_map(&mO, out, a.N, T, a.N, 32)) return QLORA_ERR_CUDA;
+    a.tma_store = 1;
+  }
+  const int64_t units = (int64_t)a.tiles_m * a.tiles_n;
+  const dim3 grid((unsigned)std::min<int64_t>(units, current_sms()));
+  const double flops = 2.0 * (double)T * a.N * ((double)a.K0 + r);
+  const char* name = dx ? "gemm_nf4_dx" : "gemm_nf4_fwd";
+  return launch(name, flops, 0.0, st, [&] {
+    if (dx)
+      gemm_nf4_kernel<true><<<grid, kNf4Threads, kNf4SmemBytes, st>>>(mA0, mC, mA1, mB1, mO, a);
+    else
+      gemm_nf4_kernel<false><<<grid, kNf4Threads, kNf4SmemBytes, st>>>(mA0, mC, mA1, mB1, mO, a);
+  });
+}
+
+// One few-token GEMM (gemm_nf4_small_kernel): out^T (Mw x T) = Wside * act^T
+// over K0 (+ the rank-r extension for the NF4 products), depth split over
+// CTAs, partials summed in split order by the last CTA of each row tile.
+struct SmallJob {
+  int src = SRC_NF4_ROWS, out = OUT_BF16;
+  const char* name = "";
+  const qlora_nf4_t* q = nullptr;                         // NF4 sources
+  const void* w = nullptr;                                // bf16 sources: the tensor tiles are cut from
+  int64_t w_inner = 0, w_outer = 0, w_ld = 0;
+  const uint16_t* act = nullptr;                          // T x K0 activations (row stride K0)
+  int64_t K0 = 0, Mw = 0;
+  int r = 0, r8 = 0;                                      // extension (NF4 sources)
+  const uint16_t* a1 = nullptr;
+  int64_t a1_inner = 0, a1_ld = 0;
+  const uint16_t* w1 = nullptr;
+  float* f32_out = nullptr;
+  int ldf = 0, nf = 0;
+  uint16_t* b16_out = nullptr;
+  int ldb = 0, nb = 0, lo_off = 0;
+  float scale = 1.0f, f32_scale = 1.0f;
+  float* part = nullptr;
+  unsigned int* tickets = nullptr;
+};
+
+template <int kSrc, int kOut>
+void small_dispatch(int tn, dim3 grid, cudaStream_t st, const CUtensorMap& a, const CUtensorMap& w,
+                    const CUtensorMap& w1, const CUtensorMap& a1, const Nf4SmallArgs& p) {
+  switch (tn) {
+    case 16:
+      gemm_nf4_small_kernel<kSrc, kOut, 16><<<grid, kSmThreads, SmallCfg<16>::kSmem, st>>>(a, w, w1, a1, p);
+      break;
+    case 32:
+      gemm_nf4_small_kernel<kSrc, kOut, 32><<<grid, kSmThreads, SmallCfg<32>::kSmem, st>>>(a, w, w1, a1, p);
+      break;
+    default:
+      gemm_nf4_small_kernel<kSrc, kOut, 64><<<grid, kSmThreads, SmallCfg<64>::kSmem, st>>>(a, w, w1, a1, p);
+      break;
+  }
+}
+
+int launch_small(const SmallJob& j, int64_t T, cudaStream_t st) {
+  const SmallPlan sp = small_plan(j.Mw, j.K0, T);
+  Nf4SmallArgs a;
+  memset(&a, 0, sizeof(a));
+  a.T = (int)T;
+  a.Mw = (int)j.Mw;
+  a.K0 = (int)j.K0;
+  a.K1 = j.r;
+  a.tiles_m = sp.tiles_m;
+  a.splits = sp.splits;
+  a.steps_per_split = sp.sps;
+  a.part = j.part;
+  a.tickets = j.tickets;
+  a.f32_out = j.f32_out;
+  a.ldf = j.ldf;
+  a.nf = j.nf;
+  a.b16_out = j.b16_out;
+  a.ldb = j.ldb;
+  a.nb = j.nb;
+  a.lo_off = j.lo_off;
+  a.scale = j.scale;
+  a.f32_scale = j.f32_scale;
+  memcpy(a.levels, tables().levels, sizeof(a.levels));
+  CUtensorMap mAct, mW, mW1, mAct1;
+  if (!make_map(&mAct, j.act, j.K0, T, j.K0, sp.tn)) return QLORA_ERR_CUDA;
+  double bytes = 0.0;
+  if (j.src == SRC_NF4_ROWS || j.src == SRC_NF4_COLS) {
+    const int64_t d = j.q->d, k = j.q->k;
+    a.absmax_q = j.q->absmax_q;
+    a.scale2 = j.q->scale2;
+    a.mean = j.q->mean;
+    a.kb = k / kBlock;
+    a.wd = (int)d;
+    a.wk = (int)k;
+    bytes = (double)nf4_storage_bytes(d, k);
+    if (j.src == SRC_NF4_COLS) {
+      if (!make_map_u8(&mW, j.q->codes, k / 2, d, k / 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_64B)) return QLORA_ERR_CUDA;
+    } else {
+      if (!make_map_u8(&mW, j.q->codes, k / 2, d, k / 2, 32, 128, CU_TENSOR_MAP_SWIZZLE_32B)) return QLORA_ERR_CUDA;
+    }
+    if (j.r == 0) {
+      mW1 = mW;
+      mAct1 = mAct;
+    } else {
+      if (j.src == SRC_NF4_COLS) {
+        if (!make_map(&mW1, j.w1, k, j.r, k, 64)) return QLORA_ERR_CUDA;          // A columns, MN-major
+      } else {
+        if (!make_map(&mW1, j.w1, j.r8, d, j.r8, 128)) return QLORA_ERR_CUDA;     // B rows, K-major
+      }
+      if (!make_map(&mAct1, j.a1, j.a1_inner, T, j.a1_ld, sp.tn)) return QLORA_ERR_CUDA;
+    }
+  } else {
+    const int box_outer = j.src == SRC_TMA_MN ? 64 : 128;
+    if (!make_map(&mW, j.w, j.w_inner, j.w_outer, j.w_ld, box_outer)) return QLORA_ERR_CUDA;
+    mW1 = mW;
+    mAct1 = mAct;
+  }
+  const dim3 grid((unsigned)(sp.tiles_m * sp.splits));
+  const double flops = 2.0 * (double)T * j.Mw * ((double)j.K0 + j.r);
+  return launch(j.name, flops, bytes, st, [&] {
+    switch (j.src) {
+      case SRC_NF4_ROWS: small_dispatch<SRC_NF4_ROWS, OUT_BF16>(sp.tn, grid, st, mAct, mW, mW1, mAct1, a); break;
+      case SRC_NF4_COLS: small_dispatch<SRC_NF4_COLS, OUT_BF16>(sp.tn, grid, st, mAct, mW, mW1, mAct1, a); break;
+      case SRC_TMA_K: small_dispatch<SRC_TMA_K, OUT_U>(sp.tn, grid, st, mAct, mW, mW1, mAct1, a); break;
+      default: small_dispatch<SRC_TMA_MN, OUT_HILO>(sp.tn, grid, st, mAct, mW, mW1, mAct1, a); break;
+    }
+  });
+}
+
+int zero_tickets(unsigned int* t, int n, cudaStream_t st) {
+  return launch("memset", 0.0, 0.0, st, [&] { cudaMemsetAsync(t, 0, (size_t)n * sizeof(unsigned int), st); });
+}
+
+// Forward on a bf16 d x k weight W (plain LoRA: the caller's W) or, when `q`
+// is given, on the NF4 weight dequantised inside the GEMM (W unused).
+// With LoRA dropout (`keep` given, rate p): the adapter path reads the masked
+// input X * keep (in the workspace) and U is scaled by c = 1 / (1 - p), so
+// U = D(X) A^T with D(X) = X * keep / (1 - p); the frozen path reads X.
+int fwd_core(const qlora_nf4_t* q, const uint16_t* W, int64_t d, int64_t k, const uint16_t* A, const uint16_t* B, int r,
              float alpha, const uint16_t* X, int64_t T, uint16_t* Y, float* U_save, const FwdWs& w,
-             cudaStream_t st) {
+             cudaStream_t st, const uint8_t* keep = nullptr, float c = 1.0f) {
   const float s = alpha / (float)r;
+  const uint16_t* Xa = X;
+  if (keep) {
+    QLORA_TRY(launch("apply_keep_bf16", 0.0, (double)T * k * 4.125, st, [&] {
+      apply_keep_bf16<<<grid_for(T * k / 8, 256), 256, 0, st>>>(reinterpret_cast<const uint4*>(X), keep, T * k / 8,
+                                                                reinterpret_cast<uint4*>(w.Xm));
+    }));
+    Xa = w.Xm;
+  }
+  const float su = keep ? mul_rn_f32(s, c) : s;
   const int r8 = (int)round_up(r, 8);
   int pst = QLORA_OK;
   const uint16_t* Bp = padded_B(B, d, r, r8, w.Bp, st, &pst);
   QLORA_TRY(pst);
 
+  if (T <= kSmallT) QLORA_TRY(zero_tickets(w.tickets, w.n_tickets, st));
   // U = X A^T (fp32 to U_save), sU = bf16(s U) (operand of the extension)
-  {
+  if (T <= kSmallT) {
+    SmallJob j;
+    j.src = SRC_TMA_K; j.out = OUT_U; j.name = "gemm_lora_down_small";
+    j.w = A; j.w_inner = k; j.w_outer = r; j.w_ld = k;
+    j.act = Xa; j.K0 = k; j.Mw = r8;
+    j.f32_out = U_save; j.ldf = r; j.nf = r; j.f32_scale = c;
+    j.b16_out = w.sU; j.ldb = r8; j.nb = r8; j.scale = su;
+    j.part = w.part_u; j.tickets = w.tickets;
+    QLORA_TRY(launch_small(j, T, st));
+  } else {
     GemmPlan g;
     g.M = (int)T; g.N = r; g.K0 = (int)k; g.bn = bn_for_rank(r);
-    g.a0 = kmajor(X, k, T, k);
+    g.a0 = kmajor(Xa, k, T, k);
     g.b0 = kmajor(A, k, r, k);
     GemmArgs a = blank_args();
-    a.epi = EPI_F32; a.out = U_save; a.ldo = r; a.alpha = 1.0f; a.n_store = r;
-    a.out2 = w.sU; a.ldo2 = r8; a.alpha2 = s; a.n_store2 = r8;
+    a.epi = EPI_F32; a.out = U_save; a.ldo = r; a.alpha = c; a.n_store = r;
+    a.out2 = w.sU; a.ldo2 = r8; a.alpha2 = su; a.n_store2 = r8;
     QLORA_TRY(launch_gemm("gemm_lora_down", g, a, st));
   }
   // Y = [X | sU] [W | B]^T
+  if (q && T <= kSmallT) {
+    SmallJob j;
+    j.src = SRC_NF4_ROWS; j.out = OUT_BF16; j.name = "gemm_nf4_small_fwd";
+    j.q = q; j.act = X; j.K0 = k; j.Mw = d;
+    j.r = r; j.r8 = r8; j.a1 = w.sU; j.a1_inner = r8; j.a1_ld = r8; j.w1 = Bp;
+    j.b16_out = Y; j.ldb = (int)d; j.nb = (int)d;
+    j.part = w.part_y; j.tickets = w.tickets + w.tickets_y_off;
+    return launch_small(j, T, st);
+  }
+  if (q) return launch_nf4_gemm(false, q, X, T, w.sU, r8, r8, Bp, r, r8, Y, st);
   {
     GemmPlan g;
     g.M = (int)T; g.N = (int)d; g.K0 = (int)k; g.K1 = r; g.bn = 256;
@@ -594,11 +933,30 @@ int fwd_core(const uint16_t* W, int64_t d, int64_t k, const uint16_t* A, const u
   return QLORA_OK;
 }
 
-// Backward on a bf16 d x k weight W (W' of the QLoRA path, or the caller's W).
-int bwd_core(const uint16_t* W, int64_t d, int64_t k, const uint16_t* A, const uint16_t* B, int r,
+// Backward on a bf16 d x k weight W (plain LoRA) or, when `q` is given, on
+// the NF4 weight dequantised inside the dX GEMM (W unused).
+int bwd_dx_base(const qlora_nf4_t* q, const uint16_t* W, int64_t d, int64_t k, const uint16_t* A, int r, int r8,
+                int rp, const uint16_t* dY, int64_t T, uint16_t* dX, const BwdWs& w, cudaStream_t st,
+                bool with_rank);
+
+// With LoRA dropout (`keep` given, c = 1 / (1 - p)), the gradients of the
+// forward above: dA = c s G^T (X * keep), dB as without dropout (U_saved is
+// the dropped-out U), and the adapter term of dX passes back through the same
+// mask, dX = dY W' + keep * (c s G A), added onto the base product by a
+// second rank-r GEMM because the mask is elementwise.
+int bwd_core(const qlora_nf4_t* q, const uint16_t* W, int64_t d, int64_t k, const uint16_t* A, const uint16_t* B, int r,
              float alpha, const uint16_t* X, const float* U_saved, const uint16_t* dY, int64_t T,
-             uint16_t* dX, float* dA, float* dB, const BwdWs& w, cudaStream_t st) {
+             uint16_t* dX, float* dA, float* dB, const BwdWs& w, cudaStream_t st,
+             const uint8_t* keep = nullptr, float c = 1.0f) {
   const float s = alpha / (float)r;
+  const uint16_t* Xa = X;
+  if (keep) {
+    QLORA_TRY(launch("apply_keep_bf16", 0.0, (double)T * k * 4.125, st, [&] {
+      apply_keep_bf16<<<grid_for(T * k / 8, 256), 256, 0, st>>>(reinterpret_cast<const uint4*>(X), keep, T * k / 8,
+                                                                reinterpret_cast<uint4*>(w.Xm));
+    }));
+    Xa = w.Xm;
+  }
   const int r8 = (int)round_up(r, 8);
   const int bnr = bn_for_rank(r);
 
@@ -606,12 +964,21 @@ int bwd_core(const uint16_t* W, int64_t d, int64_t k, const uint16_t* A, const u
   const uint16_t* Bp = padded_B(B, d, r, r8, w.Bp, st, &pst);
   QLORA_TRY(pst);
   const int rp = w.rp;
+  if (T <= kSmallT) QLORA_TRY(zero_tickets(w.tickets, w.n_tickets, st));
   // Us2 = hi/lo of bf16(s U)
   QLORA_TRY(launch("scale_f32_to_bf16_hilo", 0.0, (double)T * r * 8, st, [&] {
     scale_f32_to_bf16_hilo<<<grid_for(T * rp, 256), 256, 0, st>>>(U_saved, T, r, s, w.Us2, rp);
   }));
   // G = dY B  ->  Gs2 = hi/lo of bf16(s G)
-  {
+  if (T <= kSmallT) {
+    SmallJob j;
+    j.src = SRC_TMA_MN; j.out = OUT_HILO; j.name = "gemm_lora_g_small";
+    j.w = Bp; j.w_inner = r8; j.w_outer = d; j.w_ld = r8;
+    j.act = dY; j.K0 = d; j.Mw = rp;
+    j.b16_out = w.Gs2; j.ldb = 2 * rp; j.nb = rp; j.lo_off = rp; j.scale = s;
+    j.part = w.part_g; j.tickets = w.tickets;
+    QLORA_TRY(launch_small(j, T, st));
+  } else {
     GemmPlan g;
     g.M = (int)T; g.N = r; g.K0 = (int)d; g.bn = bnr;
     g.a0 = kmajor(dY, d, T, d);
@@ -625,12 +992,43 @@ int bwd_core(const uint16_t* W, int64_t d, int64_t k, const uint16_t* A, const u
   QLORA_TRY(adapter_grad_gemm("gemm_lora_dB", dY, d, T, w.Us2, r, rp, w.halves, w.splitsB,
                               false, dB, w.partB, st));
   // dA^T = X^T (s G)  (M = k, N = r, K = T), stored transposed into dA (r x k)
-  QLORA_TRY(adapter_grad_gemm("gemm_lora_dA", X, k, T, w.Gs2, r, rp, w.halves, w.splitsA,
-                              true, dA, w.partA, st));
+  QLORA_TRY(adapter_grad_gemm("gemm_lora_dA", Xa, k, T, w.Gs2, r, rp, w.halves, w.splitsA,
+                              true, dA, w.partA, st, c));
+  if (keep) {
+    // dX = dY W' first (no rank-r extension), then += keep * c (s G) A
+    QLORA_TRY(bwd_dx_base(q, W, d, k, A, r, r8, rp, dY, T, dX, w, st, false));
+    GemmPlan g;
+    g.M = (int)T; g.N = (int)k; g.K0 = r; g.bn = 256;
+    g.a0 = kmajor(w.Gs2, r, T, 2 * rp);          // hi part of s G
+    g.b0 = mnmajor(A, k, r, k);
+    GemmArgs a = blank_args();
+    a.epi = EPI_DROPOUT; a.out = dX; a.ldo = k; a.n_store = (int)k; a.alpha = c;
+    a.keep = keep; a.ldk = k;
+    return launch_gemm("gemm_dropout_dx", g, a, st);
+  }
+  return bwd_dx_base(q, W, d, k, A, r, r8, rp, dY, T, dX, w, st, true);
+}
+
+// dX = dY W' (+ (s G) A when `with_rank` is set): the base GEMM of the
+// backward, on the NF4 weight or on a bf16 W.
+int bwd_dx_base(const qlora_nf4_t* q, const uint16_t* W, int64_t d, int64_t k, const uint16_t* A, int r, int r8,
+                int rp, const uint16_t* dY, int64_t T, uint16_t* dX, const BwdWs& w, cudaStream_t st,
+                bool with_rank) {
+  const int re = with_rank ? r : 0;
   // dX = [dY | sG] [W ; A]   (M = T, N = k, K = d + r)
+  if (q && T <= kSmallT) {
+    SmallJob j;
+    j.src = SRC_NF4_COLS; j.out = OUT_BF16; j.name = "gemm_nf4_small_dx";
+    j.q = q; j.act = dY; j.K0 = d; j.Mw = k;
+    j.r = re; j.r8 = r8; j.a1 = w.Gs2; j.a1_inner = r; j.a1_ld = 2 * rp; j.w1 = A;
+    j.b16_out = dX; j.ldb = (int)k; j.nb = (int)k;
+    j.part = w.part_x; j.tickets = w.tickets + w.tickets_x_off;
+    return launch_small(j, T, st);
+  }
+  if (q) return launch_nf4_gemm(true, q, dY, T, w.Gs2, r, 2 * rp, A, re, r8, dX, st);
   {
     GemmPlan g;
-    g.M = (int)T; g.N = (int)k; g.K0 = (int)d; g.K1 = r; g.bn = 256;
+    g.M = (int)T; g.N = (int)k; g.K0 = (int)d; g.K1 = re; g.bn = 256;
     g.a0 = kmajor(dY, d, T, d);
     g.b0 = mnmajor(W, k, d, k);
     g.a1 = kmajor(w.Gs2, r, T, 2 * rp);          // hi part of s G
@@ -676,17 +1074,23 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratch
 namespace {
 std::mutex g_noalloc_mu;
 void* g_noalloc_ptr[64] = {nullptr};
+unsigned long long g_noalloc_ctx[64] = {0};
 
-// Device address of g_noalloc_scratch on the current device (looked up on the
-// first call per device, with that device current, then cached).
+// Device address of g_noalloc_scratch on the current device: looked up on the
+// first call per device (with that device current) and cached together with
+// the id of the context it belongs to; a call in another context (after a
+// device reset) looks it up again instead of using a stale address.
 int noalloc_scratch(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return QLORA_ERR_NO_DEVICE;
+  const unsigned long long ctx = current_ctx_id();
+  if (ctx == 0) return QLORA_ERR_NO_DEVICE;
   std::lock_guard<std::mutex> lk(g_noalloc_mu);
-  if (g_noalloc_ptr[dev] == nullptr) {
+  if (g_noalloc_ptr[dev] == nullptr || g_noalloc_ctx[dev] != ctx) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return QLORA_ERR_CUDA;
     g_noalloc_ptr[dev] = p;
+    g_noalloc_ctx[dev] = ctx;
   }
   *out = g_noalloc_ptr[dev];
   return QLORA_OK;
@@ -802,13 +1206,12 @@ int qlora_fwd(const qlora_nf4_t* q, const uint16_t* A, const uint16_t* B, int r,
   if (ws_bytes < w.bytes) return QLORA_ERR_WORKSPACE_TOO_SMALL;
   QLORA_TRY(ensure_device());
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  QLORA_TRY(dequantize_into(q, w.Wdq, st));
-  return fwd_core(w.Wdq, d, k, A, B, r, alpha, X, T, Y, U_save, w, st);
+  return fwd_core(q, nullptr, d, k, A, B, r, alpha, X, T, Y, U_save, w, st);
 }
 
 size_t lora_fwd_workspace_bytes(int64_t d, int64_t k, int r, int64_t T) {
   if (d < 1 || k < 1 || r < 1 || T < 0) return 0;
-  return carve_fwd(nullptr, d, k, r, T, false).bytes;
+  return carve_fwd(nullptr, d, k, r, T).bytes;
 }
 
 int lora_fwd(const uint16_t* W, int64_t d, int64_t k, const uint16_t* A, const uint16_t* B, int r,
@@ -823,10 +1226,10 @@ int lora_fwd(const uint16_t* W, int64_t d, int64_t k, const uint16_t* A, const u
   if (!aligned16(W) || !aligned16(A) || !aligned16(X) || !aligned16(Y) || !aligned16(U_save) ||
       !aligned16(ws))
     return QLORA_ERR_MISALIGNED;
-  FwdWs w = carve_fwd(ws, d, k, r, T, false);
+  FwdWs w = carve_fwd(ws, d, k, r, T);
   if (ws_bytes < w.bytes) return QLORA_ERR_WORKSPACE_TOO_SMALL;
   QLORA_TRY(ensure_device());
-  return fwd_core(W, d, k, A, B, r, alpha, X, T, Y, U_save, w, reinterpret_cast<cudaStream_t>(stream));
+  return fwd_core(nullptr, W, d, k, A, B, r, alpha, X, T, Y, U_save, w, reinterpret_cast<cudaStream_t>(stream));
 }
 
 size_t qlora_bwd_workspace_bytes(int64_t d, int64_t k, int r, int64_t T) {
@@ -849,13 +1252,73 @@ int qlora_bwd(const qlora_nf4_t* q, const uint16_t* A, const uint16_t* B, int r,
   BwdWs w = carve_bwd(ws, d, k, r, T);
   if (ws_bytes < w.bytes) return QLORA_ERR_WORKSPACE_TOO_SMALL;
   QLORA_TRY(ensure_device());
-  QLORA_TRY(dequantize_into(q, w.Wdq, st));
-  return bwd_core(w.Wdq, d, k, A, B, r, alpha, X, U_saved, dY, T, dX, dA, dB, w, st);
+  return bwd_core(q, nullptr, d, k, A, B, r, alpha, X, U_saved, dY, T, dX, dA, dB, w, st);
+}
+
+static int check_dropout(const uint8_t* keep, float p) {
+  if (!(p >= 0.0f && p < 1.0f)) return QLORA_ERR_INVALID_ARG;
+  if (p > 0.0f && !keep) return QLORA_ERR_INVALID_ARG;
+  if (p > 0.0f && !aligned16(keep)) return QLORA_ERR_MISALIGNED;
+  return QLORA_OK;
+}
+
+// c = fp32(1 / (1 - p)), the inverted-dropout scale of the kept elements
+static float dropout_scale(float p) { return (float)(1.0 / (1.0 - (double)p)); }
+
+size_t qlora_fwd_dropout_workspace_bytes(int64_t d, int64_t k, int r, int64_t T) {
+  if (d < 1 || k < 1 || r < 1 || T < 0) return 0;
+  return carve_fwd(nullptr, d, k, r, T, true).bytes;
+}
+
+int qlora_fwd_dropout(const qlora_nf4_t* q, const uint16_t* A, const uint16_t* B, int r, float alpha,
+                      const uint16_t* X, const uint8_t* keep, float p, int64_t T, uint16_t* Y, float* U_save,
+                      void* ws, size_t ws_bytes, qlora_stream_t stream) {
+  QLORA_TRY(check_dropout(keep, p));
+  if (p == 0.0f) return qlora_fwd(q, A, B, r, alpha, X, T, Y, U_save, ws, ws_bytes, stream);
+  QLORA_TRY(check_nf4(q));
+  QLORA_TRY(check_rank(r, alpha));
+  if (T < 0) return QLORA_ERR_INVALID_ARG;
+  if (T == 0) return QLORA_OK;
+  if (!A || !B || !X || !Y || !U_save || !ws) return QLORA_ERR_INVALID_ARG;
+  if (!aligned16(A) || !aligned16(X) || !aligned16(Y) || !aligned16(U_save) || !aligned16(ws))
+    return QLORA_ERR_MISALIGNED;
+  const int64_t d = q->d, k = q->k;
+  if (T > ((int64_t)1 << 31)) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  FwdWs w = carve_fwd(ws, d, k, r, T, true);
+  if (ws_bytes < w.bytes) return QLORA_ERR_WORKSPACE_TOO_SMALL;
+  QLORA_TRY(ensure_device());
+  return fwd_core(q, nullptr, d, k, A, B, r, alpha, X, T, Y, U_save, w, reinterpret_cast<cudaStream_t>(stream),
+                  keep, dropout_scale(p));
+}
+
+size_t qlora_bwd_dropout_workspace_bytes(int64_t d, int64_t k, int r, int64_t T) {
+  if (d < 1 || k < 1 || r < 1 || T < 0) return 0;
+  return carve_bwd(nullptr, d, k, r, T, true).bytes;
+}
+
+int qlora_bwd_dropout(const qlora_nf4_t* q, const uint16_t* A, const uint16_t* B, int r, float alpha,
+                      const uint16_t* X, const uint8_t* keep, float p, const float* U_saved, const uint16_t* dY,
+                      int64_t T, uint16_t* dX, float* dA, float* dB, void* ws, size_t ws_bytes,
+                      qlora_stream_t stream) {
+  QLORA_TRY(check_dropout(keep, p));
+  if (p == 0.0f) return qlora_bwd(q, A, B, r, alpha, X, U_saved, dY, T, dX, dA, dB, ws, ws_bytes, stream);
+  QLORA_TRY(check_nf4(q));
+  QLORA_TRY(check_rank(r, alpha));
+  if (T < 0) return QLORA_ERR_INVALID_ARG;
+  if (!A || !B || !dA || !dB) return QLORA_ERR_INVALID_ARG;
+  const int64_t d = q->d, k = q->k;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (T == 0) return zero_adapter_grads(dA, dB, d, k, r, st);
+  QLORA_TRY(check_bwd_args(A, X, U_saved, dY, dX, dA, dB, ws, d, T));
+  BwdWs w = carve_bwd(ws, d, k, r, T, true);
+  if (ws_bytes < w.bytes) return QLORA_ERR_WORKSPACE_TOO_SMALL;
+  QLORA_TRY(ensure_device());
+  return bwd_core(q, nullptr, d, k, A, B, r, alpha, X, U_saved, dY, T, dX, dA, dB, w, st, keep, dropout_scale(p));
 }
 
 size_t lora_bwd_workspace_bytes(int64_t d, int64_t k, int r, int64_t T) {
   if (d < 1 || k < 1 || r < 1 || T < 0) return 0;
-  return carve_bwd(nullptr, d, k, r, T, false).bytes;
+  return carve_bwd(nullptr, d, k, r, T).bytes;
 }
 
 int lora_bwd(const uint16_t* W, int64_t d, int64_t k, const uint16_t* A, const uint16_t* B, int r,
@@ -869,10 +1332,10 @@ int lora_bwd(const uint16_t* W, int64_t d, int64_t k, const uint16_t* A, const u
   if (T == 0) return zero_adapter_grads(dA, dB, d, k, r, st);
   if (!aligned16(W)) return QLORA_ERR_MISALIGNED;
   QLORA_TRY(check_bwd_args(A, X, U_saved, dY, dX, dA, dB, ws, d, T));
-  BwdWs w = carve_bwd(ws, d, k, r, T, false);
+  BwdWs w = carve_bwd(ws, d, k, r, T);
   if (ws_bytes < w.bytes) return QLORA_ERR_WORKSPACE_TOO_SMALL;
   QLORA_TRY(ensure_device());
-  return bwd_core(W, d, k, A, B, r, alpha, X, U_saved, dY, T, dX, dA, dB, w, st);
+  return bwd_core(nullptr, W, d, k, A, B, r, alpha, X, U_saved, dY, T, dX, dA, dB, w, st);
 }
 
 size_t lora_merge_workspace_bytes(int64_t d, int64_t k, int r) {

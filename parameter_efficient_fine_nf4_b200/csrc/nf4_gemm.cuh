@@ -1,0 +1,977 @@
+// Tensor-core GEMMs whose weight operand is dequantised from NF4 inside the
+// kernel ([P1] "What QLoRA freezes, and in how many bits": W is stored as NF4
+// with double-quantised block constants and is dequantised to BF16 for the
+// multiply, in the forward pass and again for the activation gradient).
+//
+//   forward  Y  = [X | sU] [W' | B]^T      (M = T, N = d, K = k (+ r))
+//   backward dX = [dY | sG] [W' ; A]       (M = T, N = k, K = d (+ r))
+//
+// W' never exists in global memory.  Dequantising warps read the packed codes
+// of one K-step (staged in shared memory by TMA, read back with 128-bit
+// loads), form per 64-weight block the 16 products bf16(level[i] * a') once,
+// select each weight's value from them with byte permutes on registers, and
+// write the bf16 tile in exactly the 128B-swizzled layout a TMA load of W'
+// would have produced (K-major rows for the forward, MN-major for dX).  So the
+// MMA sees the same operand bytes as on a dequantised weight and the result
+// is bit-identical to the plain-LoRA GEMM on W'.
+//
+// Tiles: one CTA per SM, each work unit is 256 rows of M (two 128-row MMA
+// tiles, two TMEM accumulators) by 256 columns of N, so one dequantised
+// weight tile feeds 256 x 256 x 64 of MMA work per K-step: the decode costs
+// 16 weights per MMA cycle-equivalent instead of 32.
+//
+// Warps: 0 TMA (activations, codes, rank-r operands), 1 TMEM + MMA issue,
+// 2-5 epilogue, 6-13 dequantisation (thread i owns weight-tile row i).
+#pragma once
+#include "gemm_tc.cuh"
+#include "nf4_kernels.cuh"
+#include "ptx.cuh"
+
+namespace qlora {
+
+// ------------------------------------------------------------------ decode
+// Per-block tables: entry i = bf16(level[i] * a') split into its low bytes
+// (lo[j] holds entries 4j..4j+3) and high bytes (hi[j]).
+struct Nf4Lut {
+  uint32_t lo[4], hi[4];
+};
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+
+__device__ __forceinline__ Nf4Lut nf4_block_lut(float a, const float (&lv)[16]) {
+  uint32_t P[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    // one fp32 product per level, one round-to-nearest-even to bf16
+    const float e0 = __fmul_rn(lv[2 * j], a);
+    const float e1 = __fmul_rn(lv[2 * j + 1], a);
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(P[j]) : "f"(e1), "f"(e0));
+  }
+  Nf4Lut t;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    t.lo[j] = prmt(P[2 * j], P[2 * j + 1], 0x6420u);
+    t.hi[j] = prmt(P[2 * j], P[2 * j + 1], 0x7531u);
+  }
+  return t;
+}
+
+// Eight codes (nibble e of w = element e) -> eight bf16 values, packed in
+// pairs (element 2i in the low half of word i).  The low three bits of each
+// code pick a byte from entries 0-7 and from entries 8-15 (one permute each
+// for the low and the high bytes); the code's top bit then selects between
+// the two; a last permute interleaves low and high bytes.
+__device__ __forceinline__ uint4 nf4_decode8(uint32_t w, const Nf4Lut& t) {
+  uint4 o;
+  asm("{\n\t"
+      ".reg .b32 m, mh, x, s, sh, a0, a1, b0, b1, la, ha, lb, hb;\n\t"
+      "and.b32 m, %4, 0x77777777;\n\t"
+      "shr.u32 mh, m, 16;\n\t"
+      "shr.u32 x, %4, 1;\n\t"
+      "lop3.b32 s, x, 0x44444444, 0x32103210, 0xEA;\n\t"   // (x & 0x4..) | 0x3210..
+      "shr.u32 sh, s, 16;\n\t"
+      "prmt.b32 a0, %5, %6, m;\n\t"
+      "prmt.b32 a1, %7, %8, m;\n\t"
+      "prmt.b32 la, a0, a1, s;\n\t"
+      "prmt.b32 b0, %9, %10, m;\n\t"
+      "prmt.b32 b1, %11, %12, m;\n\t"
+      "prmt.b32 ha, b0, b1, s;\n\t"
+      "prmt.b32 %0, la, ha, 0x5140;\n\t"
+      "prmt.b32 %1, la, ha, 0x7362;\n\t"
+      "prmt.b32 a0, %5, %6, mh;\n\t"
+      "prmt.b32 a1, %7, %8, mh;\n\t"
+      "prmt.b32 lb, a0, a1, sh;\n\t"
+      "prmt.b32 b0, %9, %10, mh;\n\t"
+      "prmt.b32 b1, %11, %12, mh;\n\t"
+      "prmt.b32 hb, b0, b1, sh;\n\t"
+      "prmt.b32 %2, lb, hb, 0x5140;\n\t"
+      "prmt.b32 %3, lb, hb, 0x7362;\n\t"
+      "}"
+      : "=r"(o.x), "=r"(o.y), "=r"(o.z), "=r"(o.w)
+      : "r"(w), "r"(t.lo[0]), "r"(t.lo[1]), "r"(t.lo[2]), "r"(t.lo[3]), "r"(t.hi[0]), "r"(t.hi[1]),
+        "r"(t.hi[2]), "r"(t.hi[3]));
+  return o;
+}
+
+// A whole 64-weight block: 32 code bytes as two 16-byte words -> eight
+// 16-byte chunks of bf16 (chunk j = elements 8j .. 8j+7).
+__device__ __forceinline__ void nf4_decode_block(uint4 c0, uint4 c1, float a, const float (&lv)[16],
+                                                 uint4 (&o)[8]) {
+  const Nf4Lut t = nf4_block_lut(a, lv);
+  o[0] = nf4_decode8(c0.x, t);
+  o[1] = nf4_decode8(c0.y, t);
+  o[2] = nf4_decode8(c0.z, t);
+  o[3] = nf4_decode8(c0.w, t);
+  o[4] = nf4_decode8(c1.x, t);
+  o[5] = nf4_decode8(c1.y, t);
+  o[6] = nf4_decode8(c1.z, t);
+  o[7] = nf4_decode8(c1.w, t);
+}
+
+// Raw inputs of one block's scale a' = fp32(fp32(E4M3(q) * scale2) + mean),
+// loaded ahead of use.  `ok` = 0 for blocks outside W (their scale is 0, so
+// their decoded weights are zeros).
+struct ScaleIn {
+  uint32_t q;
+  float s2;
+  uint32_t ok;
+};
+__device__ __forceinline__ ScaleIn load_scale_in(const uint8_t* absmax_q, const float* scale2, int64_t b,
+                                                 bool ok) {
+  ScaleIn r;
+  r.q = 0u;
+  r.s2 = 0.f;
+  r.ok = ok ? 1u : 0u;
+  if (ok) {
+    r.q = __ldg(absmax_q + b);
+    r.s2 = __ldg(scale2 + (b >> 8));
+  }
+  return r;
+}
+__device__ __forceinline__ float scale_of(const ScaleIn& s, float mu) {
+  return s.ok ? __fadd_rn(__fmul_rn(e4m3_to_f32((uint8_t)s.q), s.s2), mu) : 0.f;
+}
+
+// ------------------------------------------------------------------ kernel
+struct Nf4GemmArgs {
+  int M, N, K0, K1;           // M tokens, N output columns, K0 main depth, K1 = r
+  int tiles_m, tiles_n;       // tiles_m counts 256-row units
+  int group_m;                // raster: units walk group_m tile rows per column
+  int tma_store;              // bf16 output through shared staging + TMA stores
+  uint16_t* out;              // direct-store fallback (rows not 16-byte aligned)
+  int64_t ldo;
+  const uint8_t* absmax_q;
+  const float* scale2;
+  const float* mean;
+  int64_t kb;                 // quantisation blocks per row of W (k / 64)
+  int wd, wk;                 // W is wd x wk
+  float levels[16];
+};
+
+constexpr int kNf4DqWarps = 8;
+constexpr int kNf4Threads = (6 + kNf4DqWarps) * 32;     // 448
+constexpr int kNf4SA = 3;          // activation stages: two 128 x 64 bf16 tiles (32 KB)
+constexpr int kNf4SB = 2;          // weight stages: 256 x 64 bf16 (32 KB), dequantised or (rank-r) TMA
+constexpr int kNf4SC = 4;          // code stages: 8 KB
+constexpr int kNf4ABytes = 32768;
+constexpr int kNf4BBytes = 32768;
+constexpr int kNf4CBytes = 8192;
+constexpr int kNf4StgBoxes = 2;                         // epilogue staging: 4 KB boxes per warp
+constexpr int kNf4Stage = 4 * kNf4StgBoxes * 4096;
+constexpr int kNf4SmemBytes =
+    kNf4SA * kNf4ABytes + kNf4SB * kNf4BBytes + kNf4SC * kNf4CBytes + kNf4Stage + 1024 /*align*/ + 512 /*bars*/;
+
+struct Nf4Unit {
+  int m0, n0;
+};
+__device__ __forceinline__ Nf4Unit nf4_unit(const Nf4GemmArgs& p, int u) {
+  const int per_group = p.group_m * p.tiles_n;
+  const int gidx = u / per_group;
+  const int first_m = gidx * p.group_m;
+  const int gsize = min(p.group_m, p.tiles_m - first_m);
+  const int in_group = u - gidx * per_group;
+  Nf4Unit r;
+  r.m0 = (first_m + in_group % gsize) * 256;
+  r.n0 = (in_group / gsize) * 256;
+  return r;
+}
+
+// Waits for a phase with a short limit, used only to let copies already in
+// flight land before an aborting CTA exits.
+__device__ __forceinline__ void mbar_wait_drain(uint32_t bar, uint32_t parity) {
+  const uint64_t start = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - start > 10000000ull) return;
+  }
+}
+
+// kDx = false: forward (W' rows are N, K-major tiles); true: dX (W' rows are
+// K, MN-major tiles).
+template <bool kDx>
+__global__ void __launch_bounds__(kNf4Threads, 1)
+    gemm_nf4_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmC,
+                    const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
+                    const __grid_constant__ CUtensorMap tmOut, const __grid_constant__ Nf4GemmArgs p) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  const uint32_t pad = (1024u - (raw_addr & 1023u)) & 1023u;
+  uint8_t* smem = smem_raw + pad;
+  const uint32_t sbase = raw_addr + pad;
+  const uint32_t sA = sbase;
+  const uint32_t sB = sA + kNf4SA * kNf4ABytes;
+  const uint32_t sC = sB + kNf4SB * kNf4BBytes;
+  const uint32_t sStg = sC + kNf4SC * kNf4CBytes;
+  uint8_t* stg_ptr = smem + (sStg - sbase);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (sStg - sbase) + kNf4Stage);
+  uint64_t* a_full = bars;
+  uint64_t* a_empty = a_full + kNf4SA;
+  uint64_t* b_full = a_empty + kNf4SA;
+  uint64_t* b_empty = b_full + kNf4SB;
+  uint64_t* c_full = b_empty + kNf4SB;
+  uint64_t* c_empty = c_full + kNf4SC;
+  uint64_t* acc_full = c_empty + kNf4SC;
+  uint64_t* acc_empty = acc_full + 1;
+  uint64_t* drain_bar = acc_empty + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_bar + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int units = p.tiles_m * p.tiles_n;
+  const int steps0 = (p.K0 + 63) / 64;
+  const int steps1 = (p.K1 + 63) / 64;
+  const int steps = steps0 + steps1;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kNf4SA; ++i) {
+      mbar_init(smem_u32(&a_full[i]), 1);
+      mbar_init(smem_u32(&a_empty[i]), 1);
+    }
+    for (int i = 0; i < kNf4SB; ++i) {
+      mbar_init(smem_u32(&b_full[i]), kNf4DqWarps);
+      mbar_init(smem_u32(&b_empty[i]), 1);
+    }
+    for (int i = 0; i < kNf4SC; ++i) {
+      mbar_init(smem_u32(&c_full[i]), 1);
+      mbar_init(smem_u32(&c_empty[i]), kNf4DqWarps);
+    }
+    mbar_init(smem_u32(acc_full), 1);
+    mbar_init(smem_u32(acc_empty), 4);
+    mbar_init(smem_u32(drain_bar), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA0);
+    tma_prefetch_desc(&tmC);
+    if (steps1 > 0) {
+      tma_prefetch_desc(&tmA1);
+      tma_prefetch_desc(&tmB1);
+    }
+    if (p.tma_store) tma_prefetch_desc(&tmOut);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int a_iss[kNf4SA], c_iss[kNf4SC];
+      int b_last[kNf4SB];              // ring use index of this warp's last weight-tile load per stage
+      for (int i = 0; i < kNf4SA; ++i) a_iss[i] = 0;
+      for (int i = 0; i < kNf4SC; ++i) c_iss[i] = 0;
+      for (int i = 0; i < kNf4SB; ++i) b_last[i] = -1;
+      int g = 0, gc = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+        const Nf4Unit c = nf4_unit(p, u);
+        const bool has2 = c.m0 + 128 < p.M;
+        for (int step = 0; step < steps; ++step, ++g) {
+          const int sa = g % kNf4SA;
+          if (!mbar_wait_bounded(smem_u32(&a_empty[sa]), (uint32_t)(((g / kNf4SA) & 1) ^ 1), abort_flag)) {
+            ok = false;
+            break;
+          }
+          const bool ext = step >= steps0;
+          const int e = step - steps0;
+          const uint32_t fa = smem_u32(&a_full[sa]);
+          mbar_arrive_expect_tx(fa, has2 ? 2u * 16384u : 16384u);
+          const CUtensorMap* ma = ext ? &tmA1 : &tmA0;
+          const int x = ext ? e * 64 : step * 64;
+          tma_load_2d(sA + sa * kNf4ABytes, ma, fa, x, c.m0);
+          if (has2) tma_load_2d(sA + sa * kNf4ABytes + 16384, ma, fa, x, c.m0 + 128);
+          a_iss[sa] += 1;
+          if (!ext) {
+            const int sc = gc % kNf4SC;
+            if (!mbar_wait_bounded(smem_u32(&c_empty[sc]), (uint32_t)(((gc / kNf4SC) & 1) ^ 1), abort_flag)) {
+              ok = false;
+              break;
+            }
+            const uint32_t fc = smem_u32(&c_full[sc]);
+            mbar_arrive_expect_tx(fc, (uint32_t)kNf4CBytes);
+            if (kDx)
+              tma_load_2d(sC + sc * kNf4CBytes, &tmC, fc, c.n0 / 2, step * 64);
+            else
+              tma_load_2d(sC + sc * kNf4CBytes, &tmC, fc, step * 32, c.n0);
+            c_iss[sc] += 1;
+            ++gc;
+          } else {
+            // rank-r weight operand: B rows (forward) or A columns (dX) by TMA
+            const int sb = g % kNf4SB;
+            if (!mbar_wait_bounded(smem_u32(&b_empty[sb]), (uint32_t)(((g / kNf4SB) & 1) ^ 1), abort_flag)) {
+              ok = false;
+              break;
+            }
+            const uint32_t fb = smem_u32(&b_full[sb]);
+            mbar_arrive_expect_tx(fb, (uint32_t)kNf4BBytes);
+            mbar_arrive_count(fb, kNf4DqWarps - 1);
+            if (kDx) {
+#pragma unroll
+              for (int i = 0; i < 4; ++i)
+                tma_load_2d(sB + sb * kNf4BBytes + i * 8192, &tmB1, fb, c.n0 + 64 * i, e * 64);
+            } else {
+              tma_load_2d(sB + sb * kNf4BBytes, &tmB1, fb, e * 64, c.n0);
+            }
+            b_last[sb] = g / kNf4SB;
+          }
+        }
+      }
+      if (*abort_flag) {
+        // let copies already in flight land before the CTA exits
+        for (int i = 0; i < kNf4SA; ++i)
+          if (a_iss[i] > 0) mbar_wait_drain(smem_u32(&a_full[i]), (uint32_t)((a_iss[i] - 1) & 1));
+        for (int i = 0; i < kNf4SC; ++i)
+          if (c_iss[i] > 0) mbar_wait_drain(smem_u32(&c_full[i]), (uint32_t)((c_iss[i] - 1) & 1));
+        for (int i = 0; i < kNf4SB; ++i)
+          if (b_last[i] >= 0) mbar_wait_drain(smem_u32(&b_full[i]), (uint32_t)(b_last[i] & 1));
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint64_t adesc = smem_desc_sw128(sA, 16, 1024);
+      const uint64_t bdesc = kDx ? smem_desc_sw128(sB, 8192, 1024) : smem_desc_sw128(sB, 16, 1024);
+      const uint32_t bstep = kDx ? 128u : 2u;
+      const uint32_t idesc = idesc_bf16_f32(128, 256, 0, kDx ? 1 : 0);
+      bool ok = true;
+      int issued_any = 0;
+      int g = 0, it = 0;
+      for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++it) {
+        const Nf4Unit c = nf4_unit(p, u);
+        const bool has2 = c.m0 + 128 < p.M;
+        if (!mbar_wait_bounded(smem_u32(acc_empty), (uint32_t)((it & 1) ^ 1), abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        for (int step = 0; step < steps; ++step, ++g) {
+          const int sa = g % kNf4SA;
+          const int sb = g % kNf4SB;
+          if (!mbar_wait_bounded(smem_u32(&a_full[sa]), (uint32_t)((g / kNf4SA) & 1), abort_flag) ||
+              !mbar_wait_bounded(smem_u32(&b_full[sb]), (uint32_t)((g / kNf4SB) & 1), abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const bool ext = step >= steps0;
+          const int nsub = ext ? min(4, (p.K1 - (step - steps0) * 64 + 15) / 16) : 4;
+          const uint64_t a0 = adesc + (uint64_t)((sa * kNf4ABytes) >> 4);
+          const uint64_t b0 = bdesc + (uint64_t)((sb * kNf4BBytes) >> 4);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            if (j < nsub) {
+              const uint32_t acc = (step == 0 && j == 0) ? 0u : 1u;
+              umma_bf16(tmem_base, a0 + (uint64_t)(2 * j), b0 + (uint64_t)(j * bstep), idesc, acc);
+              if (has2)
+                umma_bf16(tmem_base + 256u, a0 + (uint64_t)(1024 + 2 * j), b0 + (uint64_t)(j * bstep), idesc,
+                          acc);
+            }
+          }
+          issued_any = 1;
+          umma_commit(smem_u32(&a_empty[sa]));
+          umma_commit(smem_u32(&b_empty[sb]));
+        }
+        if (ok) umma_commit(smem_u32(acc_full));
+      }
+      if (!ok && issued_any) {
+        umma_commit(smem_u32(drain_bar));
+        mbar_wait_bounded(smem_u32(drain_bar), 0, nullptr);
+      }
+    }
+  } else if (warp < 6) {
+    // ------------------------------------------------------------ epilogue
+    const int quarter = warp & 3;
+    uint8_t* stg = stg_ptr + (warp - 2) * (kNf4StgBoxes * 4096);
+    const uint32_t stg_s = sStg + (uint32_t)((warp - 2) * (kNf4StgBoxes * 4096));
+    int it = 0, nbox = 0;
+    for (int u = blockIdx.x; u < units; u += gridDim.x, ++it) {
+      const Nf4Unit c = nf4_unit(p, u);
+      const bool has2 = c.m0 + 128 < p.M;
+      const bool ok = mbar_wait_bounded(smem_u32(acc_full), (uint32_t)(it & 1), abort_flag);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      for (int t = 0; t < (has2 ? 2 : 1); ++t) {
+        const int mrow0 = c.m0 + t * 128 + quarter * 32;
+        const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(t * 256);
+        if (p.tma_store) {
+#pragma unroll 1
+          for (int b = 0; b < 4; ++b, ++nbox) {
+            uint32_t v0[32], v1[32];
+            tmem_ld_32x32b_x32(taddr + (uint32_t)(b * 64), v0);
+            tmem_ld_32x32b_x32(taddr + (uint32_t)(b * 64 + 32), v1);
+            tmem_ld_wait();
+            if (nbox >= kNf4StgBoxes) {
+              // the store that used this buffer has read it
+              if (lane == 0) {
+                if (kNf4StgBoxes == 2)
+                  bulk_wait_group_read1();
+                else
+                  bulk_wait_group_read0();
+              }
+              __syncwarp();
+            }
+            const int slot = nbox % kNf4StgBoxes;
+            uint8_t* box = stg + slot * 4096;
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              const uint32_t(&v)[32] = q < 4 ? v0 : v1;
+              const int o = (q & 3) * 8;
+              uint4 w;
+              w.x = pack_bf16x2(__uint_as_float(v[o + 0]), __uint_as_float(v[o + 1]));
+              w.y = pack_bf16x2(__uint_as_float(v[o + 2]), __uint_as_float(v[o + 3]));
+              w.z = pack_bf16x2(__uint_as_float(v[o + 4]), __uint_as_float(v[o + 5]));
+              w.w = pack_bf16x2(__uint_as_float(v[o + 6]), __uint_as_float(v[o + 7]));
+              *reinterpret_cast<uint4*>(box + lane * 128 + ((q ^ (lane & 7)) << 4)) = w;
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&tmOut, stg_s + (uint32_t)(slot * 4096), c.n0 + 64 * b, mrow0);
+              bulk_commit_group();
+            }
+          }
+        } else {
+          const int m = mrow0 + lane;
+#pragma unroll 1
+          for (int ch = 0; ch < 8; ++ch) {
+            uint32_t v[32];
+            tmem_ld_32x32b_x32(taddr + (uint32_t)(ch * 32), v);
+            tmem_ld_wait();
+            const int n = c.n0 + ch * 32;
+            if (m < p.M) {
+              uint16_t* o = p.out + (int64_t)m * p.ldo + n;
+              for (int i = 0; i < 32 && n + i < p.N; ++i) {
+                const __nv_bfloat16 h = __float2bfloat16_rn(__uint_as_float(v[i]));
+                o[i] = *reinterpret_cast<const uint16_t*>(&h);
+              }
+            }
+          }
+        }
+      }
+      // the accumulators may be overwritten once all four warps are done
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(acc_empty));
+    }
+    if (p.tma_store && lane == 0) bulk_wait_group0();
+  } else {
+    // ------------------------------------------------------------ dequantisation
+    // Thread i of these warps owns one 64-weight block of each K-step's
+    // weight tile.  Forward: tile row i (W' row n0 + i, block column = the
+    // K-step).  dX: K-row kk = i % 64 (W' row 64 * step + kk) and MN chunk
+    // c = i / 64 (W' block column n0 / 64 + c).
+    const int i = threadIdx.x - 192;
+    const int kk = i & 63, cc = i >> 6;
+    const float mu = __ldg(p.mean);
+    int g = 0, gc = 0;
+    for (int u = blockIdx.x; u < units; u += gridDim.x) {
+      const Nf4Unit c = nf4_unit(p, u);
+      // block index b(step) = b0 + step * bstride; validity per step
+      int64_t b0, bstride;
+      bool col_ok;
+      if (kDx) {
+        const int64_t col = (int64_t)(c.n0 >> 6) + cc;
+        col_ok = col < p.kb;
+        b0 = (int64_t)kk * p.kb + col;
+        bstride = 64 * p.kb;
+      } else {
+        col_ok = c.n0 + i < p.wd;
+        b0 = (int64_t)(c.n0 + i) * p.kb;
+        bstride = 1;
+      }
+      auto fetch = [&](int s) -> ScaleIn {
+        const bool ok = col_ok && s < steps0 && (!kDx || s * 64 + kk < p.wd);
+        return load_scale_in(p.absmax_q, p.scale2, b0 + (int64_t)s * bstride, ok);
+      };
+      ScaleIn s_cur = fetch(0), s_n1 = fetch(1), s_n2 = fetch(2);
+      bool live = true;
+      for (int step = 0; step < steps0; ++step, ++g, ++gc) {
+        const int sc = gc % kNf4SC;
+        bool ok = mbar_wait_bounded(smem_u32(&c_full[sc]), (uint32_t)((gc / kNf4SC) & 1), abort_flag);
+        if (!__all_sync(0xffffffffu, ok)) {
+          live = false;
+          break;
+        }
+        uint4 c0, c1;
+        const uint32_t cs = sC + sc * kNf4CBytes;
+        if (kDx) {
+          // 128-byte rows (K-rows), 128B swizzle: 16-byte chunk j at (j ^ (row & 7))
+          const uint32_t row = cs + kk * 128;
+          const int sw = kk & 7;
+          c0 = ld_shared_v4(row + (((2 * cc) ^ sw) << 4));
+          c1 = ld_shared_v4(row + (((2 * cc + 1) ^ sw) << 4));
+        } else {
+          // 32-byte rows, 32B swizzle: chunk j at (j ^ ((row >> 2) & 1))
+          const uint32_t row = cs + i * 32;
+          const int sw = (i >> 2) & 1;
+          c0 = ld_shared_v4(row + ((0 ^ sw) << 4));
+          c1 = ld_shared_v4(row + ((1 ^ sw) << 4));
+        }
+        const float a = scale_of(s_cur, mu);
+        s_cur = s_n1;
+        s_n1 = s_n2;
+        s_n2 = fetch(step + 3);
+        uint4 o[8];
+        nf4_decode_block(c0, c1, a, p.levels, o);
+        // the codes are consumed (the decode read them): release the stage
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&c_empty[sc]));
+        const int sb = g % kNf4SB;
+        ok = mbar_wait_bounded(smem_u32(&b_empty[sb]), (uint32_t)(((g / kNf4SB) & 1) ^ 1), abort_flag);
+        if (!__all_sync(0xffffffffu, ok)) {
+          live = false;
+          break;
+        }
+        uint32_t dst;
+        int sw;
+        if (kDx) {
+          dst = sB + sb * kNf4BBytes + cc * 8192 + kk * 128;
+          sw = kk & 7;
+        } else {
+          dst = sB + sb * kNf4BBytes + i * 128;
+          sw = i & 7;
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) st_shared_v4(dst + ((j ^ sw) << 4), o[j]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&b_full[sb]));
+      }
+      if (!live) break;
+      g += steps1;     // the rank-r weight tiles arrive by TMA
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) tmem_dealloc(tmem_base, 512);
+}
+
+// ===========================================================================
+// Few tokens (T <= 64): the products with the operands swapped, so that the
+// weight side is the 128-row MMA operand and the tokens are the (16, 32 or
+// 64 wide) N side:
+//   forward   Y^T  = [W' | B ] [X | sU]^T      (M = d,  K = k (+ r))
+//   dX        dX^T = [W'^T | A^T] [dY | sG]^T  (M = k,  K = d (+ r))
+//   U         U^T  = A X^T                     (M = r,  K = k)
+//   G         G^T  = B^T dY^T                  (M = r,  K = d)
+// With few tokens the layer is bound by the weight stream (0.52 bytes per NF4
+// weight), so the depth is split across CTAs to put every SM to work; each CTA
+// writes fp32 partials and the last CTA of a row tile (a completion ticket)
+// sums them in split order, so results are deterministic.
+// Warps: 0 TMA, 1 TMEM + MMA, 2-5 dequantisation (NF4 sources), then all four
+// run the epilogue.
+// ===========================================================================
+enum SmallSrc : int {
+  SRC_NF4_ROWS = 0,   // W' rows (forward), K-major tiles dequantised in the kernel
+  SRC_NF4_COLS = 1,   // W' columns (dX), MN-major tiles dequantised in the kernel
+  SRC_TMA_K = 2,      // a bf16 matrix whose rows are M (A for U), K-major tiles by TMA
+  SRC_TMA_MN = 3      // a bf16 matrix whose rows are K (B for G), MN-major tiles by TMA
+};
+enum SmallOut : int {
+  OUT_BF16 = 0,       // b16[t][m] = bf16(v)                         (Y, dX)
+  OUT_U = 1,          // f32[t][m] = v, b16[t][m] = bf16(scale v)    (U and s U)
+  OUT_HILO = 2        // b16[t][m] = hi, b16[t][lo_off + m] = lo of scale v   (s G)
+};
+
+struct Nf4SmallArgs {
+  int T;                      // tokens (MMA N side, at most TN)
+  int Mw;                     // output features (rows of the accumulator)
+  int K0, K1;                 // main depth and r (rank-r extension of the NF4 products)
+  int tiles_m, splits, steps_per_split;
+  float* part;                // fp32 partials [splits][T][Mw] when splits > 1
+  unsigned int* tickets;      // one counter per row tile, zero at launch
+  float* f32_out;             // OUT_U
+  int ldf, nf;
+  uint16_t* b16_out;
+  int ldb, nb;                // row stride and columns written
+  int lo_off;                 // OUT_HILO
+  float scale;                // OUT_U / OUT_HILO: bf16 output = bf16(scale v)
+  float f32_scale;            // OUT_U: fp32 output = f32_scale v
+  const uint8_t* absmax_q;
+  const float* scale2;
+  const float* mean;
+  int64_t kb;
+  int wd, wk;
+  float levels[16];
+};
+
+constexpr int kSmDqWarps = 4;
+constexpr int kSmThreads = (2 + kSmDqWarps) * 32;       // 192
+
+template <int TN>
+struct SmallCfg {
+  static constexpr int SA = 3;                 // weight tiles, 128 x 64 bf16
+  static constexpr int SC = 4;                 // codes, 4 KB
+  static constexpr int SB = 4;                 // activation tiles, TN x 64 bf16
+  static constexpr int kABytes = 16384;
+  static constexpr int kCBytes = 4096;
+  static constexpr int kBBytes = TN * 128;
+  static constexpr int kSmem = SA * kABytes + SC * kCBytes + SB * kBBytes + 1024 + 256;
+  static constexpr int kTmemCols = TN < 32 ? 32 : TN;
+};
+
+template <int kOut>
+__device__ __forceinline__ void small_emit(const Nf4SmallArgs& p, int m, int t, float v) {
+  if (kOut == OUT_BF16) {
+    if (m < p.nb) {
+      const __nv_bfloat16 h = __float2bfloat16_rn(v);
+      p.b16_out[(int64_t)t * p.ldb + m] = *reinterpret_cast<const uint16_t*>(&h);
+    }
+  } else {
+    if (kOut == OUT_U && m < p.nf) p.f32_out[(int64_t)t * p.ldf + m] = __fmul_rn(p.f32_scale, v);
+    if (m < p.nb) {
+      const float x = __fmul_rn(p.scale, v);
+      const __nv_bfloat16 h = __float2bfloat16_rn(x);
+      p.b16_out[(int64_t)t * p.ldb + m] = *reinterpret_cast<const uint16_t*>(&h);
+      if (kOut == OUT_HILO) {
+        const __nv_bfloat16 l = __float2bfloat16_rn(__fsub_rn(x, __bfloat162float(h)));
+        p.b16_out[(int64_t)t * p.ldb + p.lo_off + m] = *reinterpret_cast<const uint16_t*>(&l);
+      }
+    }
+  }
+}
+
+template <int kSrc, int kOut, int TN>
+__global__ void __launch_bounds__(kSmThreads, 1)
+    gemm_nf4_small_kernel(const __grid_constant__ CUtensorMap tmAct, const __grid_constant__ CUtensorMap tmW,
+                          const __grid_constant__ CUtensorMap tmW1, const __grid_constant__ CUtensorMap tmAct1,
+                          const __grid_constant__ Nf4SmallArgs p) {
+  using Cfg = SmallCfg<TN>;
+  constexpr bool kNf4 = kSrc == SRC_NF4_ROWS || kSrc == SRC_NF4_COLS;
+  constexpr bool kMnA = kSrc == SRC_NF4_COLS || kSrc == SRC_TMA_MN;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  const uint32_t pad = (1024u - (raw_addr & 1023u)) & 1023u;
+  uint8_t* smem = smem_raw + pad;
+  const uint32_t sA = raw_addr + pad;                       // weight tiles
+  const uint32_t sB = sA + Cfg::SA * Cfg::kABytes;          // activation tiles
+  const uint32_t sC = sB + Cfg::SB * Cfg::kBBytes;          // codes
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Cfg::SA * Cfg::kABytes + Cfg::SB * Cfg::kBBytes +
+                                               Cfg::SC * Cfg::kCBytes);
+  uint64_t* a_full = bars;
+  uint64_t* a_empty = a_full + Cfg::SA;
+  uint64_t* b_full = a_empty + Cfg::SA;
+  uint64_t* b_empty = b_full + Cfg::SB;
+  uint64_t* c_full = b_empty + Cfg::SB;
+  uint64_t* c_empty = c_full + Cfg::SC;
+  uint64_t* acc_full = c_empty + Cfg::SC;
+  uint64_t* drain_bar = acc_full + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_bar + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* last_flag = const_cast<int*>(abort_flag) + 1;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int tile = blockIdx.x / p.splits;
+  const int split = blockIdx.x - tile * p.splits;
+  const int m0 = tile * 128;
+  const int steps0 = (p.K0 + 63) / 64;
+  const int s_begin = split * p.steps_per_split;
+  const int nmain = max(0, min(steps0, s_begin + p.steps_per_split) - s_begin);
+  const int steps1 = (kNf4 && split == 0) ? (p.K1 + 63) / 64 : 0;
+  const int steps = nmain + steps1;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < Cfg::SA; ++i) {
+      mbar_init(smem_u32(&a_full[i]), kSmDqWarps);
+      mbar_init(smem_u32(&a_empty[i]), 1);
+    }
+    for (int i = 0; i < Cfg::SB; ++i) {
+      mbar_init(smem_u32(&b_full[i]), 1);
+      mbar_init(smem_u32(&b_empty[i]), 1);
+    }
+    for (int i = 0; i < Cfg::SC; ++i) {
+      mbar_init(smem_u32(&c_full[i]), 1);
+      mbar_init(smem_u32(&c_empty[i]), kSmDqWarps);
+    }
+    mbar_init(smem_u32(acc_full), 1);
+    mbar_init(smem_u32(drain_bar), 1);
+    *abort_flag = 0;
+    *last_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), Cfg::kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmAct);
+    tma_prefetch_desc(&tmW);
+    if (steps1 > 0) {
+      tma_prefetch_desc(&tmW1);
+      tma_prefetch_desc(&tmAct1);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int b_iss[Cfg::SB], c_iss[Cfg::SC];
+      int a_last[Cfg::SA];
+      for (int i = 0; i < Cfg::SB; ++i) b_iss[i] = 0;
+      for (int i = 0; i < Cfg::SC; ++i) c_iss[i] = 0;
+      for (int i = 0; i < Cfg::SA; ++i) a_last[i] = -1;
+      for (int step = 0; step < steps; ++step) {
+        const bool main = step < nmain;
+        const int ks = s_begin + step;
+        const int e = step - nmain;
+        const int sb = step % Cfg::SB;
+        if (!mbar_wait_bounded(smem_u32(&b_empty[sb]), (uint32_t)(((step / Cfg::SB) & 1) ^ 1), abort_flag)) break;
+        const uint32_t fb = smem_u32(&b_full[sb]);
+        mbar_arrive_expect_tx(fb, (uint32_t)Cfg::kBBytes);
+        if (main)
+          tma_load_2d(sB + sb * Cfg::kBBytes, &tmAct, fb, ks * 64, 0);
+        else
+          tma_load_2d(sB + sb * Cfg::kBBytes, &tmAct1, fb, e * 64, 0);
+        b_iss[sb] += 1;
+        if (main && kNf4) {
+          const int sc = step % Cfg::SC;
+          if (!mbar_wait_bounded(smem_u32(&c_empty[sc]), (uint32_t)(((step / Cfg::SC) & 1) ^ 1), abort_flag))
+            break;
+          const uint32_t fc = smem_u32(&c_full[sc]);
+          mbar_arrive_expect_tx(fc, (uint32_t)Cfg::kCBytes);
+          if (kSrc == SRC_NF4_COLS)
+            tma_load_2d(sC + sc * Cfg::kCBytes, &tmW, fc, m0 / 2, ks * 64);
+          else
+            tma_load_2d(sC + sc * Cfg::kCBytes, &tmW, fc, ks * 32, m0);
+          c_iss[sc] += 1;
+        } else {
+          // a bf16 weight-side tile by TMA: the main operand of U / G, or the
+          // rank-r operand (B rows / A columns) of the NF4 products
+          const int sa = step % Cfg::SA;
+          if (!mbar_wait_bounded(smem_u32(&a_empty[sa]), (uint32_t)(((step / Cfg::SA) & 1) ^ 1), abort_flag))
+            break;
+          const uint32_t fa = smem_u32(&a_full[sa]);
+          mbar_arrive_expect_tx(fa, (uint32_t)Cfg::kABytes);
+          mbar_arrive_count(fa, kSmDqWarps - 1);
+          const CUtensorMap* mw = main ? &tmW : &tmW1;
+          const int kx = main ? ks * 64 : e * 64;
+          if (kMnA) {
+            tma_load_2d(sA + sa * Cfg::kABytes, mw, fa, m0, kx);
+            tma_load_2d(sA + sa * Cfg::kABytes + 8192, mw, fa, m0 + 64, kx);
+          } else {
+            tma_load_2d(sA + sa * Cfg::kABytes, mw, fa, kx, m0);
+          }
+          a_last[sa] = step / Cfg::SA;
+        }
+      }
+      if (*abort_flag) {
+        for (int i = 0; i < Cfg::SB; ++i)
+          if (b_iss[i] > 0) mbar_wait_drain(smem_u32(&b_full[i]), (uint32_t)((b_iss[i] - 1) & 1));
+        for (int i = 0; i < Cfg::SC; ++i)
+          if (c_iss[i] > 0) mbar_wait_drain(smem_u32(&c_full[i]), (uint32_t)((c_iss[i] - 1) & 1));
+        for (int i = 0; i < Cfg::SA; ++i)
+          if (a_last[i] >= 0) mbar_wait_drain(smem_u32(&a_full[i]), (uint32_t)(a_last[i] & 1));
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint64_t adesc = kMnA ? smem_desc_sw128(sA, 8192, 1024) : smem_desc_sw128(sA, 16, 1024);
+      const uint32_t astep = kMnA ? 128u : 2u;
+      const uint64_t bdesc = smem_desc_sw128(sB, 16, 1024);
+      const uint32_t idesc = idesc_bf16_f32(128, TN, kMnA ? 1 : 0, 0);
+      bool ok = true;
+      int issued_any = 0;
+      for (int step = 0; step < steps; ++step) {
+        const int sa = step % Cfg::SA;
+        const int sb = step % Cfg::SB;
+        if (!mbar_wait_bounded(smem_u32(&a_full[sa]), (uint32_t)((step / Cfg::SA) & 1), abort_flag) ||
+            !mbar_wait_bounded(smem_u32(&b_full[sb]), (uint32_t)((step / Cfg::SB) & 1), abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const bool ext = step >= nmain;
+        const int nsub = ext ? min(4, (p.K1 - (step - nmain) * 64 + 15) / 16) : 4;
+        const uint64_t a0 = adesc + (uint64_t)((sa * Cfg::kABytes) >> 4);
+        const uint64_t b0 = bdesc + (uint64_t)((sb * Cfg::kBBytes) >> 4);
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if (j < nsub)
+            umma_bf16(tmem_base, a0 + (uint64_t)(j * astep), b0 + (uint64_t)(2 * j), idesc,
+                      (step == 0 && j == 0) ? 0u : 1u);
+        issued_any = 1;
+        umma_commit(smem_u32(&a_empty[sa]));
+        umma_commit(smem_u32(&b_empty[sb]));
+      }
+      if (ok) {
+        umma_commit(smem_u32(acc_full));
+      } else if (issued_any) {
+        umma_commit(smem_u32(drain_bar));
+        mbar_wait_bounded(smem_u32(drain_bar), 0, nullptr);
+      }
+    }
+  } else {
+    bool live = true;
+    if (kNf4) {
+      // -------------------------------------------------------- dequantisation
+      // Thread i owns one block per K-step.  Rows: tile row i (W' row m0 + i,
+      // block column = the K-step).  Columns: K-row kk = i % 64 (W' row
+      // 64 * ks + kk) and MN chunk cc = i / 64 (W' block column m0 / 64 + cc).
+      const int i = threadIdx.x - 64;
+      const int kk = i & 63, cc = i >> 6;
+      const float mu = __ldg(p.mean);
+      int64_t b0, bstride;
+      bool col_ok;
+      if (kSrc == SRC_NF4_COLS) {
+        const int64_t col = (int64_t)(m0 >> 6) + cc;
+        col_ok = col < p.kb;
+        b0 = (int64_t)kk * p.kb + col;
+        bstride = 64 * p.kb;
+      } else {
+        col_ok = m0 + i < p.wd;
+        b0 = (int64_t)(m0 + i) * p.kb;
+        bstride = 1;
+      }
+      auto fetch = [&](int step) -> ScaleIn {
+        const int ks = s_begin + step;
+        const bool ok = col_ok && step < nmain && (kSrc != SRC_NF4_COLS || ks * 64 + kk < p.wd);
+        return load_scale_in(p.absmax_q, p.scale2, b0 + (int64_t)ks * bstride, ok);
+      };
+      ScaleIn s_cur = fetch(0), s_n1 = fetch(1), s_n2 = fetch(2);
+      for (int step = 0; step < nmain; ++step) {
+        const int sc = step % Cfg::SC;
+        bool ok = mbar_wait_bounded(smem_u32(&c_full[sc]), (uint32_t)((step / Cfg::SC) & 1), abort_flag);
+        if (!__all_sync(0xffffffffu, ok)) {
+          live = false;
+          break;
+        }
+        uint4 c0, c1;
+        const uint32_t cs = sC + sc * Cfg::kCBytes;
+        if (kSrc == SRC_NF4_COLS) {
+          // 64-byte rows, 64B swizzle: chunk j at (j ^ ((row >> 1) & 3))
+          const uint32_t row = cs + kk * 64;
+          const int sw = (kk >> 1) & 3;
+          c0 = ld_shared_v4(row + (((2 * cc) ^ sw) << 4));
+          c1 = ld_shared_v4(row + (((2 * cc + 1) ^ sw) << 4));
+        } else {
+          const uint32_t row = cs + i * 32;
+          const int sw = (i >> 2) & 1;
+          c0 = ld_shared_v4(row + ((0 ^ sw) << 4));
+          c1 = ld_shared_v4(row + ((1 ^ sw) << 4));
+        }
+        const float a = scale_of(s_cur, mu);
+        s_cur = s_n1;
+        s_n1 = s_n2;
+        s_n2 = fetch(step + 3);
+        uint4 o[8];
+        nf4_decode_block(c0, c1, a, p.levels, o);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&c_empty[sc]));
+        const int sa = step % Cfg::SA;
+        ok = mbar_wait_bounded(smem_u32(&a_empty[sa]), (uint32_t)(((step / Cfg::SA) & 1) ^ 1), abort_flag);
+        if (!__all_sync(0xffffffffu, ok)) {
+          live = false;
+          break;
+        }
+        uint32_t dst;
+        int sw;
+        if (kSrc == SRC_NF4_COLS) {
+          dst = sA + sa * Cfg::kABytes + cc * 8192 + kk * 128;
+          sw = kk & 7;
+        } else {
+          dst = sA + sa * Cfg::kABytes + i * 128;
+          sw = i & 7;
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) st_shared_v4(dst + ((j ^ sw) << 4), o[j]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&a_full[sa]));
+      }
+    }
+    // ---------------------------------------------------------- epilogue
+    // lane quarter of this warp: accumulator rows m0 + 32 q .. + 31
+    const int quarter = warp & 3;
+    const int m = m0 + quarter * 32 + lane;
+    bool ok = live && mbar_wait_bounded(smem_u32(acc_full), 0u, abort_flag);
+    ok = __all_sync(0xffffffffu, ok);
+    if (ok) {
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16);
+#pragma unroll 1
+      for (int t0 = 0; t0 < TN; t0 += 16) {
+        uint32_t v[16];
+        tmem_ld_32x32b_x16(taddr + (uint32_t)t0, v);
+        tmem_ld_wait();
+        if (m < p.Mw) {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int t = t0 + j;
+            if (t < p.T) {
+              if (p.splits == 1)
+                small_emit<kOut>(p, m, t, __uint_as_float(v[j]));
+              else
+                p.part[((int64_t)split * p.T + t) * p.Mw + m] = __uint_as_float(v[j]);
+            }
+          }
+        }
+      }
+    }
+    if (p.splits > 1) {
+      // completion ticket: the last CTA of this row tile sums the partials
+      __threadfence();
+      named_bar_sync(1, kSmDqWarps * 32);
+      if (threadIdx.x == 64) {
+        const unsigned int prev = atomicAdd(p.tickets + tile, 1u);
+        *last_flag = (prev == (unsigned int)(p.splits - 1)) ? 1 : 0;
+      }
+      named_bar_sync(1, kSmDqWarps * 32);
+      if (*last_flag && ok) {
+        __threadfence();
+        if (m < p.Mw) {
+          const int64_t zs = (int64_t)p.T * p.Mw;
+          for (int t0 = 0; t0 < p.T; t0 += 16) {
+            // 16 tokens at a time; two splits' loads in flight per round,
+            // added in split order
+            const float* src = p.part + (int64_t)t0 * p.Mw + m;
+            const int nt = min(16, p.T - t0);
+            float acc[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) acc[j] = j < nt ? __ldcg(src + (int64_t)j * p.Mw) : 0.f;
+            int z = 1;
+            for (; z + 1 < p.splits; z += 2) {
+              float v0[16], v1[16];
+#pragma unroll
+              for (int j = 0; j < 16; ++j) {
+                v0[j] = j < nt ? __ldcg(src + z * zs + (int64_t)j * p.Mw) : 0.f;
+                v1[j] = j < nt ? __ldcg(src + (z + 1) * zs + (int64_t)j * p.Mw) : 0.f;
+              }
+#pragma unroll
+              for (int j = 0; j < 16; ++j) acc[j] = __fadd_rn(__fadd_rn(acc[j], v0[j]), v1[j]);
+            }
+            if (z < p.splits) {
+#pragma unroll
+              for (int j = 0; j < 16; ++j)
+                acc[j] = __fadd_rn(acc[j], j < nt ? __ldcg(src + z * zs + (int64_t)j * p.Mw) : 0.f);
+            }
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+              if (j < nt) small_emit<kOut>(p, m, t0 + j, acc[j]);
+          }
+        }
+        if (threadIdx.x == 64) p.tickets[tile] = 0u;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) tmem_dealloc(tmem_base, Cfg::kTmemCols);
+}
+
+}  // namespace qlora

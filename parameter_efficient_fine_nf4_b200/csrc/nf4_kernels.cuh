@@ -568,6 +568,24 @@ __global__ void splitk_reduce_f32(const float* __restrict__ part, int splits, in
   }
 }
 
+// LoRA dropout on the adapter input: Xm = X with every element whose keep bit
+// is 0 set to +0 (bf16 bit patterns; the kept elements are copied exactly).
+// Unit = 8 consecutive elements: one 16-byte load of X, one byte of the
+// bit-packed mask (bit i keeps element 8u + i), one 16-byte store.
+__global__ void apply_keep_bf16(const uint4* __restrict__ X, const uint8_t* __restrict__ keep, int64_t n_units,
+                                uint4* __restrict__ Xm) {
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t u = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; u < n_units; u += stride) {
+    const uint4 x = __ldcs(X + u);
+    const uint32_t b = keep[u];
+    const uint32_t m0 = ((b & 1u) ? 0x0000FFFFu : 0u) | ((b & 2u) ? 0xFFFF0000u : 0u);
+    const uint32_t m1 = ((b & 4u) ? 0x0000FFFFu : 0u) | ((b & 8u) ? 0xFFFF0000u : 0u);
+    const uint32_t m2 = ((b & 16u) ? 0x0000FFFFu : 0u) | ((b & 32u) ? 0xFFFF0000u : 0u);
+    const uint32_t m3 = ((b & 64u) ? 0x0000FFFFu : 0u) | ((b & 128u) ? 0xFFFF0000u : 0u);
+    Xm[u] = make_uint4(x.x & m0, x.y & m1, x.z & m2, x.w & m3);
+  }
+}
+
 // Bounded-wait self test: waits on a barrier that nothing completes.
 __global__ void selftest_wait_kernel(unsigned long long limit_ns) {
   __shared__ __align__(8) uint64_t bar;

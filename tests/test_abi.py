@@ -66,14 +66,17 @@ def test_library_levels_equal_oracle_bit_for_bit(lib):
 
 def test_workspace_queries(lib):
     assert q4.qlora_quantize_workspace_bytes(256, 256) >= (256 * 256 // 64) * 4
-    assert q4.qlora_fwd_workspace_bytes(22016, 8192, 64, 16384) >= 22016 * 8192 * 2
-    assert q4.qlora_bwd_workspace_bytes(22016, 8192, 64, 16384) >= 22016 * 8192 * 2
     assert q4.lora_merge_workspace_bytes(256, 256, 8) >= 256 * 8 * 2
     assert q4.qlora_fwd_workspace_bytes(0, 256, 8, 16) == 0
-    # the plain-LoRA workspace holds no copy of the weight
+    # the weight is dequantised inside the GEMM: neither workspace holds a
+    # 16-bit copy of it (sU / hi-lo pairs, padded B and split-K partials only)
+    # and the QLoRA workspaces equal the plain-LoRA ones
+    d, k, r, T = 22016, 8192, 64, 16384
     for fn_q, fn_p in ((q4.qlora_fwd_workspace_bytes, q4.lora_fwd_workspace_bytes),
                        (q4.qlora_bwd_workspace_bytes, q4.lora_bwd_workspace_bytes)):
-        assert fn_q(22016, 8192, 64, 16384) - fn_p(22016, 8192, 64, 16384) == 22016 * 8192 * 2
+        assert fn_q(d, k, r, T) == fn_p(d, k, r, T)
+        assert fn_q(d, k, r, T) < d * k * 2 // 4
+    assert q4.qlora_fwd_workspace_bytes(d, k, r, T) >= T * r * 2
     assert q4.lora_fwd_workspace_bytes(4096, 4096, 8, 0) > 0
 
 
@@ -103,6 +106,20 @@ def test_argument_validation_without_device(lib):
                       None) == 2                                                                  # d % 8
     assert L.lora_bwd(None, 256, 256, 16, 16, 8, 16.0, 16, 16, 16, 16, 16, 16, 16, 16, 1 << 20,
                       None) == 1                                                                  # null W
+    # LoRA dropout: the rate and the mask are checked on the host first
+    nf = q4._NF4(16, 16, 16, 16, 256, 256, 64, 256)
+    for p in (1.0, 1.5, -0.1, float("nan")):
+        assert L.qlora_fwd_dropout(ctypes.byref(nf), 16, 16, 8, 16.0, 16, 16, p, 16, 16, 16, 16,
+                                   1 << 20, None) == 1
+    assert L.qlora_fwd_dropout(ctypes.byref(nf), 16, 16, 8, 16.0, 16, None, 0.1, 16, 16, 16, 16,
+                               1 << 20, None) == 1                                             # no mask
+    assert L.qlora_fwd_dropout(ctypes.byref(nf), 16, 16, 8, 16.0, 16, 17, 0.1, 16, 16, 16, 16,
+                               1 << 20, None) == 3                                             # misaligned mask
+    assert L.qlora_bwd_dropout(ctypes.byref(nf), 16, 16, 8, 16.0, 16, None, 0.1, 16, 16, 16, 16, 16, 16,
+                               16, 1 << 20, None) == 1
+    assert L.qlora_fwd_dropout(ctypes.byref(nf), 16, 16, 8, 16.0, 16, 16, 0.1, 16, 16, 16, 16,
+                               64, None) == 4                                                  # workspace
+    assert q4.qlora_fwd_dropout_workspace_bytes(256, 256, 8, 16) > q4.qlora_fwd_workspace_bytes(256, 256, 8, 16)
     # Adam: step, betas, lr and alignment are checked on the host; n = 0 is a no-op
     assert L.lora_adam_step(16, 16, 16, 16, 16, 8, 0, 1e-3, 0.9, 0.999, 1e-8, 0.0, None) == 1     # step 0
     assert L.lora_adam_step(16, 16, 16, 16, 16, 8, 1, 1e-3, 1.0, 0.999, 1e-8, 0.0, None) == 1     # beta1 = 1

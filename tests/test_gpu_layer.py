@@ -84,6 +84,31 @@ def test_config1_b_zero_init():
     rows_within(bf16_host_f64(c.Y), X @ Wp.T, what="Y base")
 
 
+@pytest.mark.parametrize("T", [16, 300])
+def test_b_zero_adds_exactly_nothing(T):
+    # [P1] "The update LoRA is allowed to learn": with B = 0 the adapted layer
+    # is the base layer.  On the GPU the rank-r term then adds +0 to every
+    # fp32 accumulator, so Y and dX are bit-identical whatever A holds (A = 0
+    # as well), and dA is exactly zero.
+    cfg = synthetic.config(1)
+    lay = synthetic.make_layer(cfg, T=T, zero_b=True)
+    qw = q4.qlora_nf4_quantize(f32_dev(lay.W0))
+    A, B, X, dY = bf16_dev(lay.A), bf16_dev(lay.B), bf16_dev(lay.X), bf16_dev(lay.dY)
+    A0 = torch.zeros_like(A)
+    Y, U = q4.qlora_fwd(qw, A, B, cfg.alpha, X)
+    dX, dA, dB = q4.qlora_bwd(qw, A, B, cfg.alpha, X, U, dY)
+    Y0, U0 = q4.qlora_fwd(qw, A0, B, cfg.alpha, X)
+    dX0, dA0, dB0 = q4.qlora_bwd(qw, A0, B, cfg.alpha, X, U0, dY)
+    torch.cuda.synchronize()
+    assert torch.equal(Y, Y0) and torch.equal(dX, dX0)
+    assert torch.count_nonzero(dA).item() == 0 and torch.count_nonzero(dA0).item() == 0
+    assert torch.count_nonzero(U0).item() == 0 and torch.count_nonzero(dB0).item() == 0
+    # and the base product alone is what the oracle gives
+    Wp = oracle_Wp(lay.W0)
+    rows_within(bf16_host_f64(Y), nf4.bf16_to_f64(lay.X) @ Wp.T, what="Y base")
+    rows_within(bf16_host_f64(dX), nf4.bf16_to_f64(lay.dY) @ Wp, what="dX base")
+
+
 @pytest.mark.parametrize("d,k,r,T", [
     (320, 192, 5, 200),      # ragged M and N tiles, r not a multiple of 8
     (64, 64, 1, 1),          # one token, rank 1
@@ -235,3 +260,40 @@ def test_merged_layer_matches_unmerged_forward():
     Y_merged = (c.X.float() @ W.float().T)
     torch.cuda.synchronize()
     rows_within(Y_merged.double().cpu().numpy(), bf16_host_f64(c.Y).astype(np.float64), what="merged")
+
+
+def test_merge_unmerge_full_size_sampled_rows():
+    # the merge the benchmark times: 22016 x 8192, r = 64.  The oracle's own
+    # storage for the sampled rows (constants and mean from every block,
+    # codes of the sampled rows), merged in float64; the GPU unmerge is fed
+    # the oracle's merged rows at those positions.
+    cfg = synthetic.config(4)
+    lay = synthetic.make_layer(cfg, 0, with_acts=False)
+    d, k, r, s = lay.d, lay.k, lay.r, cfg.s
+    qw = q4.qlora_nf4_quantize(f32_dev(lay.W0))
+    A, B = bf16_dev(lay.A), bf16_dev(lay.B)
+    W = q4.lora_merge(qw, A, B, cfg.alpha)
+    torch.cuda.synchronize()
+    assert q4.qlora_get_device_status() == 0
+    rows = synthetic.sample_rows(4040, d, 48)
+    kb = k // 64
+    blocks = (rows[:, None] * kb + np.arange(kb)[None, :]).ravel()
+    a = nf4.block_absmax(lay.W0)
+    mu = nf4.block_mean(a)
+    c2, s1 = nf4.double_quant(a, mu)
+    packed = np.zeros(d * k // 2, np.uint8)
+    packed.reshape(-1, 32)[blocks] = nf4.pack_codes(
+        nf4.encode_blocks(lay.W0.reshape(-1, 64)[blocks], a[blocks]).ravel()).reshape(-1, 32)
+    Wp_rows = nf4.bf16_to_f64(nf4.dequantize_blocks(packed, c2, s1, mu, blocks)).reshape(rows.size, k)
+    Af = nf4.bf16_to_f64(lay.A)
+    Bf = nf4.bf16_to_f64(lay.B)[rows]
+    ref = lora.merge(Wp_rows, Af, Bf, s)
+    extra = r * 2.0 ** -22 * s * (np.abs(Bf) @ np.abs(Af)) + 2.0 ** -23 * np.abs(Wp_rows)
+    within_one_bf16_ulp(bf16_host_bits(W)[rows], ref, "merge 22016x8192", abs_extra=extra)
+    W_in = W.clone()
+    W_in[torch.from_numpy(rows).cuda()] = bf16_dev(ref)
+    W0pp = q4.lora_unmerge(W_in, A, B, cfg.alpha)
+    torch.cuda.synchronize()
+    ref_back = lora.unmerge(nf4.bf16_to_f64(ref), Af, Bf, s)
+    within_one_bf16_ulp(bf16_host_bits(W0pp)[rows], ref_back, "unmerge 22016x8192", abs_extra=extra)
+    assert q4.qlora_get_device_status() == 0

@@ -142,15 +142,17 @@ def test_quantize_extreme_block_scales(a):
     blocks.append(tiny.astype(np.float32))
     W = np.ascontiguousarray(np.stack(blocks).reshape(-1, 128))     # 16 blocks -> 8 x 128
     qw = q4.qlora_nf4_quantize(f32_dev(W))
+    Wp = q4.qlora_nf4_dequantize(qw)
     torch.cuda.synchronize()
     assert q4.qlora_get_device_status() == 0
-    # storage only: the oracle's bf16 rounding covers the normal range, which
-    # the dequantised weights of these scales leave
     ref = nf4.quantize(W)
     assert np.array_equal(qw.codes.cpu().numpy(), ref["codes"])
     assert np.array_equal(qw.absmax_q.cpu().numpy(), ref["absmax_q"])
     assert np.array_equal(qw.scale2.cpu().numpy().view(np.uint32), ref["scale2"].view(np.uint32))
     assert qw.mean.cpu().numpy().view(np.uint32)[0] == np.float32(ref["mean"]).view(np.uint32)
+    # the dequantised weights too, subnormal results included (the oracle
+    # rounds to bf16 over the whole finite range)
+    assert np.array_equal(bf16_host_bits(Wp), nf4.dequantize(ref))
 
 
 def test_quantize_is_deterministic():

@@ -175,6 +175,27 @@ def test_bf16_rounding_matches_torch():
     assert np.array_equal(ours, ref)
 
 
+def test_bf16_rounding_subnormal_range():
+    # below 2^-126 the bf16 grid is the multiples of 2^-133; every fp32
+    # subnormal pattern class (random bits, exact ties between grid points,
+    # values rounding up into the normal range) against torch's conversion
+    torch = pytest.importorskip("torch")
+    rng = np.random.Generator(np.random.Philox(key=12))
+    rand = rng.integers(1, 0x00800000, 50000).astype(np.uint32)
+    ties = (rng.integers(0, 0x80, 2000).astype(np.uint32) << 16) | 0x8000
+    edge = np.array([0x007F8000, 0x007FFFFF, 0x00008000, 0x00018000, 0x00000001], np.uint32)
+    bits = np.concatenate([rand, ties, edge])
+    x = np.concatenate([bits, bits | 0x80000000]).view(np.float32)
+    ours = nf4.to_bf16_bits(x.astype(np.float64))
+    ref = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(ours, ref)
+    # closed forms: half the smallest step rounds to (signed) zero, 1.5 steps to 2
+    step = 2.0 ** -133
+    assert nf4.to_bf16_bits(np.array([0.5 * step, -0.5 * step, 1.5 * step])).tolist() == [0x0000, 0x8000, 0x0002]
+    # just below the smallest normal rounds up to it (exponent field 1)
+    assert nf4.to_bf16_bits(np.array([2.0 ** -126 - 0.25 * step])).tolist() == [0x0080]
+
+
 # ---------------------------------------------------------------------- mean
 def test_pairwise_sum_exact_on_integers_and_close_to_fsum():
     v = np.arange(1, 1001, dtype=np.float64)
