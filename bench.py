@@ -363,6 +363,35 @@ def config_block(torch, q4, dev, stream, flush, peaks, write_ceiling, steps=10, 
              "algorithmic_bytes": nbytes, "gbs": nbytes / 1e9 / (ms / 1e3),
              "frac_of_hbm": nbytes / 1e9 / (ms / 1e3) / hbm}
         e["bound"] = "hbm" if T <= 64 else "tensor"
+        if T <= 64:
+            # a decode-like step is launch-bound on the host: replay it as one
+            # CUDA graph (the library's launches are stream-ordered and
+            # capturable; tensor maps are baked into the kernel parameters)
+            g = torch.cuda.CUDAGraph()
+            side = torch.cuda.Stream(device=dev)
+            side.wait_stream(stream)
+            with torch.cuda.stream(side):
+                step()
+            stream.wait_stream(side)
+            torch.cuda.synchronize(dev)
+            with torch.cuda.graph(g):
+                step()
+            for _ in range(warmup):
+                g.replay()
+            torch.cuda.synchronize(dev)
+            gev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+            for i in range(steps):
+                flush.zero_()
+                gev[i][0].record(stream)
+                g.replay()
+                gev[i][1].record(stream)
+            torch.cuda.synchronize(dev)
+            assert q4.qlora_get_device_status() == 0
+            gms = statistics.median(a.elapsed_time(b) for a, b in gev)
+            e["graph"] = {"us_fwd_bwd": 1e3 * gms, "tflops": flops / (gms / 1e3) / 1e12,
+                          "gbs": nbytes / 1e9 / (gms / 1e3), "frac_of_hbm": nbytes / 1e9 / (gms / 1e3) / hbm,
+                          "how": "the fwd+bwd step of every linear captured once as a CUDA graph, replayed"}
+            del g
         # per-kernel device time of one more step (library profiler: events on
         # the launch stream around every launch)
         flush.zero_()

@@ -234,6 +234,36 @@ QLORA_API int qlora_bwd_dropout(const qlora_nf4_t* q, const uint16_t* A, const u
                                 const uint16_t* dY, int64_t T, uint16_t* dX, float* dA, float* dB,
                                 void* workspace, size_t workspace_bytes, qlora_stream_t stream);
 
+/* ------------------------------------- several unmerged adapters (next row) */
+
+/*
+ * One frozen base with a stack of unmerged adapters, each token using its own
+ * ([P2] "The LoRA hypothesis": serving many tasks keeps the adapters unmerged,
+ * one base in memory and a few-MB adapter chosen per request; [P1] "What to
+ * choose and why": one deployed base, a small B A per task).  The pages give
+ * no batching rule; here token t uses adapter idx[t] of the stack:
+ *   U[t] = X[t] A_i^T,   Y[t] = X[t] W'^T + s_i U[t] B_i^T,   i = idx[t], s_i = alphas[i] / r
+ * and the backward gives dX and, per adapter, dA_i = s_i sum_{t: idx[t]=i} G[t]^T X[t],
+ * dB_i = s_i sum_{t: idx[t]=i} dY[t]^T U[t] with G[t] = dY[t] B_i (an adapter
+ * no token uses gets dA_i = dB_i = 0 exactly).
+ * As: device, n x r x k bf16 (adapter i's A at As + i r k); Bs: device,
+ * n x d x r bf16; alphas: HOST array of n floats (> 0); idx: device int32[T]
+ * (a token whose index is outside [0, n) gets no adapter term and a zero U
+ * row); U_save: T x r fp32, the token's own U.  dAs (n x r x k) and dBs
+ * (n x d x r) are fp32 and overwritten.  1 <= n <= 64 and n r <= 256.  With
+ * n = 1 and every idx 0 the results are bit-identical to qlora_fwd /
+ * qlora_bwd.  Other arguments and errors as for qlora_fwd / qlora_bwd.
+ */
+QLORA_API size_t qlora_fwd_multi_workspace_bytes(int64_t d, int64_t k, int n, int r, int64_t T);
+QLORA_API int qlora_fwd_multi(const qlora_nf4_t* q, int n, const uint16_t* As, const uint16_t* Bs, int r,
+                              const float* alphas, const int32_t* idx, const uint16_t* X, int64_t T, uint16_t* Y,
+                              float* U_save, void* workspace, size_t workspace_bytes, qlora_stream_t stream);
+QLORA_API size_t qlora_bwd_multi_workspace_bytes(int64_t d, int64_t k, int n, int r, int64_t T);
+QLORA_API int qlora_bwd_multi(const qlora_nf4_t* q, int n, const uint16_t* As, const uint16_t* Bs, int r,
+                              const float* alphas, const int32_t* idx, const uint16_t* X, const float* U_saved,
+                              const uint16_t* dY, int64_t T, uint16_t* dX, float* dAs, float* dBs,
+                              void* workspace, size_t workspace_bytes, qlora_stream_t stream);
+
 /* ------------------------------------------- plain LoRA on a bf16 base */
 
 /*

@@ -70,6 +70,11 @@ _SIGNATURES = {
     "qlora_bwd_dropout_workspace_bytes": (_SIZE, [_I64, _I64, _INT, _I64]),
     "qlora_bwd_dropout": (_INT, [_NF4P, _VP, _VP, _INT, _F, _VP, _VP, _F, _VP, _VP, _I64, _VP, _VP, _VP, _VP,
                                  _SIZE, _VP]),
+    "qlora_fwd_multi_workspace_bytes": (_SIZE, [_I64, _I64, _INT, _INT, _I64]),
+    "qlora_fwd_multi": (_INT, [_NF4P, _INT, _VP, _VP, _INT, _VP, _VP, _VP, _I64, _VP, _VP, _VP, _SIZE, _VP]),
+    "qlora_bwd_multi_workspace_bytes": (_SIZE, [_I64, _I64, _INT, _INT, _I64]),
+    "qlora_bwd_multi": (_INT, [_NF4P, _INT, _VP, _VP, _INT, _VP, _VP, _VP, _VP, _VP, _I64, _VP, _VP, _VP, _VP,
+                               _SIZE, _VP]),
     "lora_fwd_workspace_bytes": (_SIZE, [_I64, _I64, _INT, _I64]),
     "lora_fwd": (_INT, [_VP, _I64, _I64, _VP, _VP, _INT, _F, _VP, _I64, _VP, _VP, _VP, _SIZE, _VP]),
     "lora_bwd_workspace_bytes": (_SIZE, [_I64, _I64, _INT, _I64]),
@@ -350,6 +355,68 @@ def qlora_bwd_dropout(q: NF4Weight, A: torch.Tensor, B: torch.Tensor, alpha: flo
                                  ws.numel(), _stream(stream))
     _check(st, "qlora_bwd_dropout")
     return dX, dA, dB
+
+
+def _host_alphas(alphas):
+    arr = (ctypes.c_float * len(alphas))(*[float(a) for a in alphas])
+    return arr
+
+
+def qlora_fwd_multi(q: NF4Weight, As: torch.Tensor, Bs: torch.Tensor, alphas, idx: torch.Tensor,
+                    X: torch.Tensor, Y: Optional[torch.Tensor] = None, U_save: Optional[torch.Tensor] = None,
+                    ws: Optional[torch.Tensor] = None, stream=None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """Forward with a stack of n adapters (As n x r x k, Bs n x d x r), token t
+    using adapter idx[t] (int32, device) with scale alphas[idx[t]] / r."""
+    n, r = As.shape[0], As.shape[1]
+    T = X.shape[0]
+    _need(As, torch.bfloat16, (n, r, q.k), "As")
+    _need(Bs, torch.bfloat16, (n, q.d, r), "Bs")
+    _need(idx, torch.int32, (T,), "idx")
+    _need(X, torch.bfloat16, (T, q.k), "X")
+    if len(alphas) != n:
+        raise ValueError("one alpha per adapter")
+    dev = X.device
+    Y = torch.empty(T, q.d, dtype=torch.bfloat16, device=dev) if Y is None else Y
+    U_save = torch.empty(T, r, dtype=torch.float32, device=dev) if U_save is None else U_save
+    _need(Y, torch.bfloat16, (T, q.d), "Y")
+    _need(U_save, torch.float32, (T, r), "U_save")
+    ws = workspace(lib().qlora_fwd_multi_workspace_bytes(q.d, q.k, n, r, T), dev) if ws is None else ws
+    al = _host_alphas(alphas)
+    st = lib().qlora_fwd_multi(ctypes.byref(q.cstruct), n, _ptr(As), _ptr(Bs), r, ctypes.addressof(al), _ptr(idx),
+                               _ptr(X), T, _ptr(Y), _ptr(U_save), _ptr(ws), ws.numel(), _stream(stream))
+    _check(st, "qlora_fwd_multi")
+    return Y, U_save
+
+
+def qlora_bwd_multi(q: NF4Weight, As: torch.Tensor, Bs: torch.Tensor, alphas, idx: torch.Tensor,
+                    X: torch.Tensor, U_saved: torch.Tensor, dY: torch.Tensor, dX: Optional[torch.Tensor] = None,
+                    dAs: Optional[torch.Tensor] = None, dBs: Optional[torch.Tensor] = None,
+                    ws: Optional[torch.Tensor] = None, stream=None):
+    """Backward of qlora_fwd_multi: dX and per-adapter dAs (n x r x k), dBs (n x d x r)."""
+    n, r = As.shape[0], As.shape[1]
+    T = X.shape[0]
+    _need(As, torch.bfloat16, (n, r, q.k), "As")
+    _need(Bs, torch.bfloat16, (n, q.d, r), "Bs")
+    _need(idx, torch.int32, (T,), "idx")
+    _need(X, torch.bfloat16, (T, q.k), "X")
+    _need(U_saved, torch.float32, (T, r), "U_saved")
+    _need(dY, torch.bfloat16, (T, q.d), "dY")
+    if len(alphas) != n:
+        raise ValueError("one alpha per adapter")
+    dev = X.device
+    dX = torch.empty(T, q.k, dtype=torch.bfloat16, device=dev) if dX is None else dX
+    dAs = torch.empty(n, r, q.k, dtype=torch.float32, device=dev) if dAs is None else dAs
+    dBs = torch.empty(n, q.d, r, dtype=torch.float32, device=dev) if dBs is None else dBs
+    _need(dX, torch.bfloat16, (T, q.k), "dX")
+    _need(dAs, torch.float32, (n, r, q.k), "dAs")
+    _need(dBs, torch.float32, (n, q.d, r), "dBs")
+    ws = workspace(lib().qlora_bwd_multi_workspace_bytes(q.d, q.k, n, r, T), dev) if ws is None else ws
+    al = _host_alphas(alphas)
+    st = lib().qlora_bwd_multi(ctypes.byref(q.cstruct), n, _ptr(As), _ptr(Bs), r, ctypes.addressof(al), _ptr(idx),
+                               _ptr(X), _ptr(U_saved), _ptr(dY), T, _ptr(dX), _ptr(dAs), _ptr(dBs), _ptr(ws),
+                               ws.numel(), _stream(stream))
+    _check(st, "qlora_bwd_multi")
+    return dX, dAs, dBs
 
 
 def lora_fwd_workspace_bytes(d: int, k: int, r: int, T: int) -> int:

@@ -218,6 +218,7 @@ cudaError_t set_small_attrs() {
   if (e == cudaSuccess) e = set_small_attrs_tn<SRC_NF4_COLS, OUT_BF16>();
   if (e == cudaSuccess) e = set_small_attrs_tn<SRC_TMA_K, OUT_U>();
   if (e == cudaSuccess) e = set_small_attrs_tn<SRC_TMA_MN, OUT_HILO>();
+  if (e == cudaSuccess) e = set_small_attrs_tn<SRC_TMA_MN, OUT_U>();
   return e;
 }
 
@@ -355,6 +356,27 @@ bool make_map_u8(CUtensorMap* map, const void* base, int64_t inner, int64_t oute
                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
+
+// fp32 2-D tensor map without swizzle: `inner` contiguous elements per row,
+// `outer` rows, `ld` elements between rows (a multiple of 4), box
+// box_inner x box_outer (box_inner * 4 a multiple of 16 bytes).
+bool make_map_f32(CUtensorMap* map, const void* base, int64_t inner, int64_t outer, int64_t ld, int box_inner,
+                  int box_outer) {
+  cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)outer};
+  cuuint64_t strides[1] = {(cuuint64_t)(ld * 4)};
+  cuuint32_t box[2] = {(cuuint32_t)box_inner, (cuuint32_t)box_outer};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = encode_fn()(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(base), dims, strides, box,
+                           estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// Layouts of the per-call block scales (nf4_block_scales): the forward reads
+// them transposed (block column s: rows n contiguous, row stride round4(d)),
+// dX row-major (row n: block columns contiguous, row stride round4(k / 64)).
+inline int64_t scales_ld_fwd(int64_t d) { return (d + 3) / 4 * 4; }
+inline int64_t scales_ld_dx(int64_t k) { return (k / 64 + 3) / 4 * 4; }
 
 // Merge / unmerge through the bulk-copy deploy kernel (r <= 128).
 template <bool kMerge, int KS>
@@ -540,7 +562,9 @@ const uint16_t* padded_B(const uint16_t* B, int64_t d, int r, int r8, uint16_t* 
 
 // Few-token plan of gemm_nf4_small_kernel: tokens padded to TN, 128-row
 // tiles of the Mw output features, the main depth split so that about three
-// CTAs per SM are busy while every split keeps at least four K-steps.
+// CTAs per SM are busy, while every split keeps at least eight K-steps and a
+// row tile has at most kSmMaxSplits splits (the last CTA's reduction keeps
+// all of them in flight).
 constexpr int64_t kSmallT = 64;
 struct SmallPlan {
   int tn = 16, tiles_m = 1, splits = 1, sps = 1;
@@ -551,7 +575,7 @@ SmallPlan small_plan(int64_t Mw, int64_t K0, int64_t T) {
   sp.tiles_m = (int)cdiv(Mw, 128);
   const int steps0 = (int)cdiv(K0, 64);
   const int want = (int)cdiv(3 * kSMs, sp.tiles_m);
-  const int splits = std::max(1, std::min(want, steps0 / 4));
+  const int splits = std::max(1, std::min(std::min(want, steps0 / 8), kSmMaxSplits));
   sp.sps = (int)cdiv(steps0, splits);
   sp.splits = (int)cdiv(steps0, sp.sps);
   return sp;
@@ -566,9 +590,12 @@ struct FwdWs {
   uint16_t* sU; uint16_t* Bp;
   float* part_u; float* part_y; unsigned int* tickets; int n_tickets; int tickets_y_off;
   uint16_t* Xm;            // LoRA dropout: the masked adapter input
+  uint16_t* Bcat; float* Uall;   // several adapters: B_0..B_{n-1} side by side, U of every adapter
+  float* scales;           // fp32 block scales of the NF4 weight (forward layout)
   size_t bytes;
 };
-FwdWs carve_fwd(void* ws, int64_t d, int64_t k, int r, int64_t T, bool dropout = false) {
+// `r` is the rank seen by the GEMMs (n r for a stack of n adapters of rank r).
+FwdWs carve_fwd(void* ws, int64_t d, int64_t k, int r, int64_t T, bool dropout = false, bool multi = false) {
   Carver c{reinterpret_cast<uint8_t*>(ws)};
   const int64_t r8 = round_up(r, 8);
   FwdWs w;
@@ -588,6 +615,9 @@ FwdWs carve_fwd(void* ws, int64_t d, int64_t k, int r, int64_t T, bool dropout =
     w.tickets = (unsigned int*)c.take((size_t)w.n_tickets * 4);
   }
   w.Xm = dropout ? (uint16_t*)c.take((size_t)(std::max<int64_t>(T, 1) * k * 2)) : nullptr;
+  w.Bcat = multi ? (uint16_t*)c.take((size_t)(d * r * 2)) : nullptr;
+  w.Uall = multi ? (float*)c.take((size_t)(std::max<int64_t>(T, 1) * r * 4)) : nullptr;
+  w.scales = (float*)c.take((size_t)(k / 64 * scales_ld_fwd(d) * 4));
   w.bytes = c.off;
   return w;
 }
@@ -609,6 +639,8 @@ struct BwdWs {
   uint16_t* Us2; uint16_t* Gs2; uint16_t* Bp; float* partA; float* partB;
   float* part_g; float* part_x; unsigned int* tickets; int n_tickets; int tickets_x_off;
   uint16_t* Xm;            // LoRA dropout: the masked adapter input
+  uint16_t* Bcat; float* Gall; float* dBcat;   // several adapters
+  float* scales;           // fp32 block scales of the NF4 weight (dX layout)
   int rp, halves, splitsA, splitsB; size_t bytes;
 };
 // Backward workspace.  U and G enter the T-reductions (dB, dA) as two bf16
@@ -616,7 +648,7 @@ struct BwdWs {
 // 2*rp columns (rp = r rounded up to 32); with rp <= 128 one GEMM with N = 2*rp
 // multiplies both and the epilogue adds the paired columns, otherwise the two
 // halves run as two GEMMs whose partial outputs are summed.
-BwdWs carve_bwd(void* ws, int64_t d, int64_t k, int r, int64_t T, bool dropout = false) {
+BwdWs carve_bwd(void* ws, int64_t d, int64_t k, int r, int64_t T, bool dropout = false, bool multi = false) {
   Carver c{reinterpret_cast<uint8_t*>(ws)};
   const int64_t r8 = round_up(r, 8);
   const int64_t Tm = std::max<int64_t>(T, 1);
@@ -645,6 +677,10 @@ BwdWs carve_bwd(void* ws, int64_t d, int64_t k, int r, int64_t T, bool dropout =
     w.tickets = (unsigned int*)c.take((size_t)w.n_tickets * 4);
   }
   w.Xm = dropout ? (uint16_t*)c.take((size_t)(Tm * k * 2)) : nullptr;
+  w.Bcat = multi ? (uint16_t*)c.take((size_t)(d * r * 2)) : nullptr;
+  w.Gall = multi ? (float*)c.take((size_t)(Tm * r * 4)) : nullptr;
+  w.dBcat = multi ? (float*)c.take((size_t)(d * r * 4)) : nullptr;
+  w.scales = (float*)c.take((size_t)(d * scales_ld_dx(k) * 4));
   w.bytes = c.off;
   return w;
 }
@@ -693,9 +729,9 @@ int adapter_grad_gemm(const char* name, const uint16_t* big, int64_t M, int64_t 
 // Base GEMM on the NF4 weight with the rank-r extension (gemm_nf4_kernel):
 //   forward (dx = false): out = Y (T x d)  = [X | sU][W' | B]^T,  a1 = sU (T x r8, ld r8), b1 = B (d x r8)
 //   dX      (dx = true):  out = dX (T x k) = [dY | sG][W' ; A],    a1 = sG (T x r, ld a1_ld), b1 = A (r x k)
-int launch_nf4_gemm(bool dx, const qlora_nf4_t* q, const uint16_t* act, int64_t T, const uint16_t* a1,
-                    int64_t a1_inner, int64_t a1_ld, const uint16_t* b1, int r, int r8, uint16_t* out,
-                    cudaStream_t st) {
+int launch_nf4_gemm(bool dx, const qlora_nf4_t* q, const float* scales, const uint16_t* act, int64_t T,
+                    const uint16_t* a1, int64_t a1_inner, int64_t a1_ld, const uint16_t* b1, int r, int r8,
+                    uint16_t* out, cudaStream_t st) {
   const int64_t d = q->d, k = q->k;
   Nf4GemmArgs a;
   memset(&a, 0, sizeof(a));
@@ -706,14 +742,13 @@ int launch_nf4_gemm(bool dx, const qlora_nf4_t* q, const uint16_t* act, int64_t 
   a.tiles_m = (int)cdiv(T, 256);
   a.tiles_n = (int)cdiv(a.N, 256);
   a.group_m = 8;
-  a.absmax_q = q->absmax_q;
-  a.scale2 = q->scale2;
-  a.mean = q->mean;
-  a.kb = k / kBlock;
-  a.wd = (int)d;
-  a.wk = (int)k;
   memcpy(a.levels, tables().levels, sizeof(a.levels));
-  CUtensorMap mA0, mC, mA1, mB1, mO;
+  CUtensorMap mA0, mC, mS, mA1, mB1, mO;
+  if (dx) {
+    if (!make_map_f32(&mS, scales, k / 64, d, scales_ld_dx(k), 4, 64)) return QLORA_ERR_CUDA;
+  } else {
+    if (!make_map_f32(&mS, scales, d, k / 64, scales_ld_fwd(d), 256, 1)) return QLORA_ERR_CUDA;
+  }
   if (!make_map(&mA0, act, a.K0, T, a.K0, 128)) return QLORA_ERR_CUDA;
   if (dx) {
     if (!make_map_u8(&mC, q->codes, k / 2, d, k / 2, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
@@ -745,9 +780,9 @@ int launch_nf4_gemm(bool dx, const qlora_nf4_t* q, const uint16_t* act, int64_t 
   const char* name = dx ? "gemm_nf4_dx" : "gemm_nf4_fwd";
   return launch(name, flops, 0.0, st, [&] {
     if (dx)
-      gemm_nf4_kernel<true><<<grid, kNf4Threads, kNf4SmemBytes, st>>>(mA0, mC, mA1, mB1, mO, a);
+      gemm_nf4_kernel<true><<<grid, kNf4Threads, kNf4SmemBytes, st>>>(mA0, mC, mS, mA1, mB1, mO, a);
     else
-      gemm_nf4_kernel<false><<<grid, kNf4Threads, kNf4SmemBytes, st>>>(mA0, mC, mA1, mB1, mO, a);
+      gemm_nf4_kernel<false><<<grid, kNf4Threads, kNf4SmemBytes, st>>>(mA0, mC, mS, mA1, mB1, mO, a);
   });
 }
 
@@ -758,6 +793,7 @@ struct SmallJob {
   int src = SRC_NF4_ROWS, out = OUT_BF16;
   const char* name = "";
   const qlora_nf4_t* q = nullptr;                         // NF4 sources
+  const float* scales = nullptr;                          // their block scales (nf4_block_scales)
   const void* w = nullptr;                                // bf16 sources: the tensor tiles are cut from
   int64_t w_inner = 0, w_outer = 0, w_ld = 0;
   const uint16_t* act = nullptr;                          // T x K0 activations (row stride K0)
@@ -777,16 +813,16 @@ struct SmallJob {
 
 template <int kSrc, int kOut>
 void small_dispatch(int tn, dim3 grid, cudaStream_t st, const CUtensorMap& a, const CUtensorMap& w,
-                    const CUtensorMap& w1, const CUtensorMap& a1, const Nf4SmallArgs& p) {
+                    const CUtensorMap& sc, const CUtensorMap& w1, const CUtensorMap& a1, const Nf4SmallArgs& p) {
   switch (tn) {
     case 16:
-      gemm_nf4_small_kernel<kSrc, kOut, 16><<<grid, kSmThreads, SmallCfg<16>::kSmem, st>>>(a, w, w1, a1, p);
+      gemm_nf4_small_kernel<kSrc, kOut, 16><<<grid, kSmThreads, SmallCfg<16>::kSmem, st>>>(a, w, sc, w1, a1, p);
       break;
     case 32:
-      gemm_nf4_small_kernel<kSrc, kOut, 32><<<grid, kSmThreads, SmallCfg<32>::kSmem, st>>>(a, w, w1, a1, p);
+      gemm_nf4_small_kernel<kSrc, kOut, 32><<<grid, kSmThreads, SmallCfg<32>::kSmem, st>>>(a, w, sc, w1, a1, p);
       break;
     default:
-      gemm_nf4_small_kernel<kSrc, kOut, 64><<<grid, kSmThreads, SmallCfg<64>::kSmem, st>>>(a, w, w1, a1, p);
+      gemm_nf4_small_kernel<kSrc, kOut, 64><<<grid, kSmThreads, SmallCfg<64>::kSmem, st>>>(a, w, sc, w1, a1, p);
       break;
   }
 }
@@ -814,22 +850,19 @@ int launch_small(const SmallJob& j, int64_t T, cudaStream_t st) {
   a.scale = j.scale;
   a.f32_scale = j.f32_scale;
   memcpy(a.levels, tables().levels, sizeof(a.levels));
-  CUtensorMap mAct, mW, mW1, mAct1;
+  CUtensorMap mAct, mW, mS, mW1, mAct1;
   if (!make_map(&mAct, j.act, j.K0, T, j.K0, sp.tn)) return QLORA_ERR_CUDA;
+  mS = mAct;
   double bytes = 0.0;
   if (j.src == SRC_NF4_ROWS || j.src == SRC_NF4_COLS) {
     const int64_t d = j.q->d, k = j.q->k;
-    a.absmax_q = j.q->absmax_q;
-    a.scale2 = j.q->scale2;
-    a.mean = j.q->mean;
-    a.kb = k / kBlock;
-    a.wd = (int)d;
-    a.wk = (int)k;
     bytes = (double)nf4_storage_bytes(d, k);
     if (j.src == SRC_NF4_COLS) {
       if (!make_map_u8(&mW, j.q->codes, k / 2, d, k / 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_64B)) return QLORA_ERR_CUDA;
+      if (!make_map_f32(&mS, j.scales, k / 64, d, scales_ld_dx(k), 4, 64)) return QLORA_ERR_CUDA;
     } else {
       if (!make_map_u8(&mW, j.q->codes, k / 2, d, k / 2, 32, 128, CU_TENSOR_MAP_SWIZZLE_32B)) return QLORA_ERR_CUDA;
+      if (!make_map_f32(&mS, j.scales, d, k / 64, scales_ld_fwd(d), 128, 1)) return QLORA_ERR_CUDA;
     }
     if (j.r == 0) {
       mW1 = mW;
@@ -852,10 +885,15 @@ int launch_small(const SmallJob& j, int64_t T, cudaStream_t st) {
   const double flops = 2.0 * (double)T * j.Mw * ((double)j.K0 + j.r);
   return launch(j.name, flops, bytes, st, [&] {
     switch (j.src) {
-      case SRC_NF4_ROWS: small_dispatch<SRC_NF4_ROWS, OUT_BF16>(sp.tn, grid, st, mAct, mW, mW1, mAct1, a); break;
-      case SRC_NF4_COLS: small_dispatch<SRC_NF4_COLS, OUT_BF16>(sp.tn, grid, st, mAct, mW, mW1, mAct1, a); break;
-      case SRC_TMA_K: small_dispatch<SRC_TMA_K, OUT_U>(sp.tn, grid, st, mAct, mW, mW1, mAct1, a); break;
-      default: small_dispatch<SRC_TMA_MN, OUT_HILO>(sp.tn, grid, st, mAct, mW, mW1, mAct1, a); break;
+      case SRC_NF4_ROWS: small_dispatch<SRC_NF4_ROWS, OUT_BF16>(sp.tn, grid, st, mAct, mW, mS, mW1, mAct1, a); break;
+      case SRC_NF4_COLS: small_dispatch<SRC_NF4_COLS, OUT_BF16>(sp.tn, grid, st, mAct, mW, mS, mW1, mAct1, a); break;
+      case SRC_TMA_K: small_dispatch<SRC_TMA_K, OUT_U>(sp.tn, grid, st, mAct, mW, mS, mW1, mAct1, a); break;
+      default:
+        if (j.out == OUT_U)
+          small_dispatch<SRC_TMA_MN, OUT_U>(sp.tn, grid, st, mAct, mW, mS, mW1, mAct1, a);
+        else
+          small_dispatch<SRC_TMA_MN, OUT_HILO>(sp.tn, grid, st, mAct, mW, mS, mW1, mAct1, a);
+        break;
     }
   });
 }
@@ -864,14 +902,37 @@ int zero_tickets(unsigned int* t, int n, cudaStream_t st) {
   return launch("memset", 0.0, 0.0, st, [&] { cudaMemsetAsync(t, 0, (size_t)n * sizeof(unsigned int), st); });
 }
 
+// a' of every block of q into `out`, transposed (forward) or row-major (dX),
+// and zero `tickets` (n words) on the way.
+int block_scales(const qlora_nf4_t* q, bool transposed, float* out, unsigned int* tickets, int n,
+                 cudaStream_t st) {
+  const int64_t d = q->d, kb = q->k / 64;
+  const int64_t ld = transposed ? scales_ld_fwd(d) : scales_ld_dx(q->k);
+  const dim3 grid((unsigned)cdiv(kb, 32), (unsigned)cdiv(d, 32));
+  return launch("nf4_block_scales", 0.0, (double)d * kb * 5, st, [&] {
+    nf4_block_scales<<<grid, 256, 0, st>>>(q->absmax_q, q->scale2, q->mean, d, kb, transposed ? 1 : 0, ld, out,
+                                          tickets, tickets ? n : 0);
+  });
+}
+
 // Forward on a bf16 d x k weight W (plain LoRA: the caller's W) or, when `q`
 // is given, on the NF4 weight dequantised inside the GEMM (W unused).
+// A stack of n unmerged adapters of rank ra chosen per token (idx[t]); the
+// GEMMs then see rank n ra with A = [A_0; ...; A_{n-1}] and B = [B_0 | ... ],
+// and every rank-r operand is scattered into the token's block.
+struct MultiAdapter {
+  int n, ra;
+  const int32_t* idx;
+  AdapterScales sc;
+};
+
 // With LoRA dropout (`keep` given, rate p): the adapter path reads the masked
 // input X * keep (in the workspace) and U is scaled by c = 1 / (1 - p), so
 // U = D(X) A^T with D(X) = X * keep / (1 - p); the frozen path reads X.
 int fwd_core(const qlora_nf4_t* q, const uint16_t* W, int64_t d, int64_t k, const uint16_t* A, const uint16_t* B, int r,
              float alpha, const uint16_t* X, int64_t T, uint16_t* Y, float* U_save, const FwdWs& w,
-             cudaStream_t st, const uint8_t* keep = nullptr, float c = 1.0f) {
+             cudaStream_t st, const uint8_t* keep = nullptr, float c = 1.0f,
+             const MultiAdapter* ma = nullptr) {
   const float s = alpha / (float)r;
   const uint16_t* Xa = X;
   if (keep) {
@@ -887,15 +948,20 @@ int fwd_core(const qlora_nf4_t* q, const uint16_t* W, int64_t d, int64_t k, cons
   const uint16_t* Bp = padded_B(B, d, r, r8, w.Bp, st, &pst);
   QLORA_TRY(pst);
 
-  if (T <= kSmallT) QLORA_TRY(zero_tickets(w.tickets, w.n_tickets, st));
+  if (q) {
+    // block scales for the dequantising GEMM (and the few-token tickets)
+    QLORA_TRY(block_scales(q, true, w.scales, T <= kSmallT ? w.tickets : nullptr, w.n_tickets, st));
+  } else if (T <= kSmallT) {
+    QLORA_TRY(zero_tickets(w.tickets, w.n_tickets, st));
+  }
   // U = X A^T (fp32 to U_save), sU = bf16(s U) (operand of the extension)
   if (T <= kSmallT) {
     SmallJob j;
     j.src = SRC_TMA_K; j.out = OUT_U; j.name = "gemm_lora_down_small";
     j.w = A; j.w_inner = k; j.w_outer = r; j.w_ld = k;
     j.act = Xa; j.K0 = k; j.Mw = r8;
-    j.f32_out = U_save; j.ldf = r; j.nf = r; j.f32_scale = c;
-    j.b16_out = w.sU; j.ldb = r8; j.nb = r8; j.scale = su;
+    j.f32_out = ma ? w.Uall : U_save; j.ldf = r; j.nf = r; j.f32_scale = c;
+    j.b16_out = w.sU; j.ldb = r8; j.nb = ma ? 0 : r8; j.scale = su;
     j.part = w.part_u; j.tickets = w.tickets;
     QLORA_TRY(launch_small(j, T, st));
   } else {
@@ -904,21 +970,28 @@ int fwd_core(const qlora_nf4_t* q, const uint16_t* W, int64_t d, int64_t k, cons
     g.a0 = kmajor(Xa, k, T, k);
     g.b0 = kmajor(A, k, r, k);
     GemmArgs a = blank_args();
-    a.epi = EPI_F32; a.out = U_save; a.ldo = r; a.alpha = c; a.n_store = r;
-    a.out2 = w.sU; a.ldo2 = r8; a.alpha2 = su; a.n_store2 = r8;
+    a.epi = EPI_F32; a.out = ma ? w.Uall : U_save; a.ldo = r; a.alpha = c; a.n_store = r;
+    if (!ma) { a.out2 = w.sU; a.ldo2 = r8; a.alpha2 = su; a.n_store2 = r8; }
     QLORA_TRY(launch_gemm("gemm_lora_down", g, a, st));
+  }
+  if (ma) {
+    // each token's own U and its scaled block of sU
+    QLORA_TRY(launch("scatter_adapter_u", 0.0, 0.0, st, [&] {
+      scatter_adapter_u<<<grid_for(T * r8, 256), 256, 0, st>>>(w.Uall, ma->idx, T, ma->ra, ma->n, r8, ma->sc,
+                                                               U_save, w.sU);
+    }));
   }
   // Y = [X | sU] [W | B]^T
   if (q && T <= kSmallT) {
     SmallJob j;
     j.src = SRC_NF4_ROWS; j.out = OUT_BF16; j.name = "gemm_nf4_small_fwd";
-    j.q = q; j.act = X; j.K0 = k; j.Mw = d;
+    j.q = q; j.scales = w.scales; j.act = X; j.K0 = k; j.Mw = d;
     j.r = r; j.r8 = r8; j.a1 = w.sU; j.a1_inner = r8; j.a1_ld = r8; j.w1 = Bp;
     j.b16_out = Y; j.ldb = (int)d; j.nb = (int)d;
     j.part = w.part_y; j.tickets = w.tickets + w.tickets_y_off;
     return launch_small(j, T, st);
   }
-  if (q) return launch_nf4_gemm(false, q, X, T, w.sU, r8, r8, Bp, r, r8, Y, st);
+  if (q) return launch_nf4_gemm(false, q, w.scales, X, T, w.sU, r8, r8, Bp, r, r8, Y, st);
   {
     GemmPlan g;
     g.M = (int)T; g.N = (int)d; g.K0 = (int)k; g.K1 = r; g.bn = 256;
@@ -947,7 +1020,7 @@ int bwd_dx_base(const qlora_nf4_t* q, const uint16_t* W, int64_t d, int64_t k, c
 int bwd_core(const qlora_nf4_t* q, const uint16_t* W, int64_t d, int64_t k, const uint16_t* A, const uint16_t* B, int r,
              float alpha, const uint16_t* X, const float* U_saved, const uint16_t* dY, int64_t T,
              uint16_t* dX, float* dA, float* dB, const BwdWs& w, cudaStream_t st,
-             const uint8_t* keep = nullptr, float c = 1.0f) {
+             const uint8_t* keep = nullptr, float c = 1.0f, const MultiAdapter* ma = nullptr) {
   const float s = alpha / (float)r;
   const uint16_t* Xa = X;
   if (keep) {
@@ -964,11 +1037,22 @@ int bwd_core(const qlora_nf4_t* q, const uint16_t* W, int64_t d, int64_t k, cons
   const uint16_t* Bp = padded_B(B, d, r, r8, w.Bp, st, &pst);
   QLORA_TRY(pst);
   const int rp = w.rp;
-  if (T <= kSmallT) QLORA_TRY(zero_tickets(w.tickets, w.n_tickets, st));
+  if (q) {
+    QLORA_TRY(block_scales(q, false, w.scales, T <= kSmallT ? w.tickets : nullptr, w.n_tickets, st));
+  } else if (T <= kSmallT) {
+    QLORA_TRY(zero_tickets(w.tickets, w.n_tickets, st));
+  }
   // Us2 = hi/lo of bf16(s U)
-  QLORA_TRY(launch("scale_f32_to_bf16_hilo", 0.0, (double)T * r * 8, st, [&] {
-    scale_f32_to_bf16_hilo<<<grid_for(T * rp, 256), 256, 0, st>>>(U_saved, T, r, s, w.Us2, rp);
-  }));
+  if (ma) {
+    QLORA_TRY(launch("scatter_adapter_hilo", 0.0, 0.0, st, [&] {
+      scatter_adapter_hilo<<<grid_for(T * rp, 256), 256, 0, st>>>(U_saved, 1, ma->idx, T, ma->ra, ma->n, rp,
+                                                                  ma->sc, w.Us2);
+    }));
+  } else {
+    QLORA_TRY(launch("scale_f32_to_bf16_hilo", 0.0, (double)T * r * 8, st, [&] {
+      scale_f32_to_bf16_hilo<<<grid_for(T * rp, 256), 256, 0, st>>>(U_saved, T, r, s, w.Us2, rp);
+    }));
+  }
   // G = dY B  ->  Gs2 = hi/lo of bf16(s G)
   if (T <= kSmallT) {
     SmallJob j;
@@ -976,6 +1060,11 @@ int bwd_core(const qlora_nf4_t* q, const uint16_t* W, int64_t d, int64_t k, cons
     j.w = Bp; j.w_inner = r8; j.w_outer = d; j.w_ld = r8;
     j.act = dY; j.K0 = d; j.Mw = rp;
     j.b16_out = w.Gs2; j.ldb = 2 * rp; j.nb = rp; j.lo_off = rp; j.scale = s;
+    if (ma) {
+      // every adapter's G in fp32, scattered below
+      j.out = OUT_U; j.name = "gemm_lora_g_small";
+      j.f32_out = w.Gall; j.ldf = r; j.nf = r; j.nb = 0; j.lo_off = 0;
+    }
     j.part = w.part_g; j.tickets = w.tickets;
     QLORA_TRY(launch_small(j, T, st));
   } else {
@@ -984,13 +1073,29 @@ int bwd_core(const qlora_nf4_t* q, const uint16_t* W, int64_t d, int64_t k, cons
     g.a0 = kmajor(dY, d, T, d);
     g.b0 = mnmajor(Bp, r8, d, r8);
     GemmArgs a = blank_args();
-    a.epi = EPI_F32; a.out = nullptr; a.n_store = 0;
-    a.out2 = w.Gs2; a.ldo2 = 2 * rp; a.alpha2 = s; a.n_store2 = rp; a.lo_offset = rp;
+    if (ma) {
+      a.epi = EPI_F32; a.out = w.Gall; a.ldo = r; a.n_store = r; a.alpha = 1.0f;
+    } else {
+      a.epi = EPI_F32; a.out = nullptr; a.n_store = 0;
+      a.out2 = w.Gs2; a.ldo2 = 2 * rp; a.alpha2 = s; a.n_store2 = rp; a.lo_offset = rp;
+    }
     QLORA_TRY(launch_gemm("gemm_lora_g", g, a, st));
   }
-  // dB = dY^T (s U)   (M = d, N = r, K = T)
+  if (ma) {
+    QLORA_TRY(launch("scatter_adapter_hilo", 0.0, 0.0, st, [&] {
+      scatter_adapter_hilo<<<grid_for(T * rp, 256), 256, 0, st>>>(w.Gall, 0, ma->idx, T, ma->ra, ma->n, rp,
+                                                                  ma->sc, w.Gs2);
+    }));
+  }
+  // dB = dY^T (s U)   (M = d, N = r, K = T); several adapters: every
+  // adapter's dB side by side, then split into the stack
   QLORA_TRY(adapter_grad_gemm("gemm_lora_dB", dY, d, T, w.Us2, r, rp, w.halves, w.splitsB,
-                              false, dB, w.partB, st));
+                              false, ma ? w.dBcat : dB, w.partB, st));
+  if (ma) {
+    QLORA_TRY(launch("uncat_adapters_db", 0.0, 0.0, st, [&] {
+      uncat_adapters_db<<<grid_for(d * r, 256), 256, 0, st>>>(w.dBcat, d, ma->ra, ma->n, dB);
+    }));
+  }
   // dA^T = X^T (s G)  (M = k, N = r, K = T), stored transposed into dA (r x k)
   QLORA_TRY(adapter_grad_gemm("gemm_lora_dA", Xa, k, T, w.Gs2, r, rp, w.halves, w.splitsA,
                               true, dA, w.partA, st, c));
@@ -1019,13 +1124,13 @@ int bwd_dx_base(const qlora_nf4_t* q, const uint16_t* W, int64_t d, int64_t k, c
   if (q && T <= kSmallT) {
     SmallJob j;
     j.src = SRC_NF4_COLS; j.out = OUT_BF16; j.name = "gemm_nf4_small_dx";
-    j.q = q; j.act = dY; j.K0 = d; j.Mw = k;
+    j.q = q; j.scales = w.scales; j.act = dY; j.K0 = d; j.Mw = k;
     j.r = re; j.r8 = r8; j.a1 = w.Gs2; j.a1_inner = r; j.a1_ld = 2 * rp; j.w1 = A;
     j.b16_out = dX; j.ldb = (int)k; j.nb = (int)k;
     j.part = w.part_x; j.tickets = w.tickets + w.tickets_x_off;
     return launch_small(j, T, st);
   }
-  if (q) return launch_nf4_gemm(true, q, dY, T, w.Gs2, r, 2 * rp, A, re, r8, dX, st);
+  if (q) return launch_nf4_gemm(true, q, w.scales, dY, T, w.Gs2, r, 2 * rp, A, re, r8, dX, st);
   {
     GemmPlan g;
     g.M = (int)T; g.N = (int)k; g.K0 = (int)d; g.K1 = re; g.bn = 256;
@@ -1253,6 +1358,82 @@ int qlora_bwd(const qlora_nf4_t* q, const uint16_t* A, const uint16_t* B, int r,
   if (ws_bytes < w.bytes) return QLORA_ERR_WORKSPACE_TOO_SMALL;
   QLORA_TRY(ensure_device());
   return bwd_core(q, nullptr, d, k, A, B, r, alpha, X, U_saved, dY, T, dX, dA, dB, w, st);
+}
+
+// Several adapters: host-side checks and the stack descriptor.
+static int make_multi(int n, int r, const float* alphas, const int32_t* idx, MultiAdapter* ma) {
+  if (n < 1 || n > kMaxAdapters || !alphas || !idx) return QLORA_ERR_INVALID_ARG;
+  if (r < 1 || (int64_t)n * r > 256) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  ma->n = n;
+  ma->ra = r;
+  ma->idx = idx;
+  memset(&ma->sc, 0, sizeof(ma->sc));
+  for (int i = 0; i < n; ++i) {
+    if (!(alphas[i] > 0.0f) || !std::isfinite(alphas[i])) return QLORA_ERR_INVALID_ARG;
+    ma->sc.s[i] = alphas[i] / (float)r;
+  }
+  return QLORA_OK;
+}
+
+size_t qlora_fwd_multi_workspace_bytes(int64_t d, int64_t k, int n, int r, int64_t T) {
+  if (d < 1 || k < 1 || n < 1 || r < 1 || T < 0) return 0;
+  return carve_fwd(nullptr, d, k, n * r, T, false, true).bytes;
+}
+
+int qlora_fwd_multi(const qlora_nf4_t* q, int n, const uint16_t* As, const uint16_t* Bs, int r,
+                    const float* alphas, const int32_t* idx, const uint16_t* X, int64_t T, uint16_t* Y,
+                    float* U_save, void* ws, size_t ws_bytes, qlora_stream_t stream) {
+  QLORA_TRY(check_nf4(q));
+  MultiAdapter ma;
+  QLORA_TRY(make_multi(n, r, alphas, idx, &ma));
+  if (T < 0) return QLORA_ERR_INVALID_ARG;
+  if (T == 0) return QLORA_OK;
+  if (!As || !Bs || !X || !Y || !U_save || !ws) return QLORA_ERR_INVALID_ARG;
+  if (!aligned16(As) || !aligned16(X) || !aligned16(Y) || !aligned16(U_save) || !aligned16(ws) ||
+      (reinterpret_cast<uintptr_t>(idx) & 3u) != 0)
+    return QLORA_ERR_MISALIGNED;
+  const int64_t d = q->d, k = q->k;
+  if (T > ((int64_t)1 << 31)) return QLORA_ERR_UNSUPPORTED_SHAPE;
+  const int R = n * r;
+  FwdWs w = carve_fwd(ws, d, k, R, T, false, true);
+  if (ws_bytes < w.bytes) return QLORA_ERR_WORKSPACE_TOO_SMALL;
+  QLORA_TRY(ensure_device());
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  QLORA_TRY(launch("cat_adapters_b", 0.0, 0.0, st, [&] {
+    cat_adapters_b<<<grid_for(d * R, 256), 256, 0, st>>>(Bs, d, r, n, w.Bcat);
+  }));
+  // alpha only sets s = alpha / R, which the stack path does not use
+  return fwd_core(q, nullptr, d, k, As, w.Bcat, R, (float)R, X, T, Y, U_save, w, st, nullptr, 1.0f, &ma);
+}
+
+size_t qlora_bwd_multi_workspace_bytes(int64_t d, int64_t k, int n, int r, int64_t T) {
+  if (d < 1 || k < 1 || n < 1 || r < 1 || T < 0) return 0;
+  return carve_bwd(nullptr, d, k, n * r, T, false, true).bytes;
+}
+
+int qlora_bwd_multi(const qlora_nf4_t* q, int n, const uint16_t* As, const uint16_t* Bs, int r,
+                    const float* alphas, const int32_t* idx, const uint16_t* X, const float* U_saved,
+                    const uint16_t* dY, int64_t T, uint16_t* dX, float* dAs, float* dBs, void* ws,
+                    size_t ws_bytes, qlora_stream_t stream) {
+  QLORA_TRY(check_nf4(q));
+  MultiAdapter ma;
+  QLORA_TRY(make_multi(n, r, alphas, idx, &ma));
+  if (T < 0) return QLORA_ERR_INVALID_ARG;
+  if (!As || !Bs || !dAs || !dBs) return QLORA_ERR_INVALID_ARG;
+  const int64_t d = q->d, k = q->k;
+  const int R = n * r;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (T == 0) return zero_adapter_grads(dAs, dBs, d, k, R, st);
+  QLORA_TRY(check_bwd_args(As, X, U_saved, dY, dX, dAs, dBs, ws, d, T));
+  if ((reinterpret_cast<uintptr_t>(idx) & 3u) != 0) return QLORA_ERR_MISALIGNED;
+  BwdWs w = carve_bwd(ws, d, k, R, T, false, true);
+  if (ws_bytes < w.bytes) return QLORA_ERR_WORKSPACE_TOO_SMALL;
+  QLORA_TRY(ensure_device());
+  QLORA_TRY(launch("cat_adapters_b", 0.0, 0.0, st, [&] {
+    cat_adapters_b<<<grid_for(d * R, 256), 256, 0, st>>>(Bs, d, r, n, w.Bcat);
+  }));
+  return bwd_core(q, nullptr, d, k, As, w.Bcat, R, (float)R, X, U_saved, dY, T, dX, dAs, dBs, w, st, nullptr,
+                  1.0f, &ma);
 }
 
 static int check_dropout(const uint8_t* keep, float p) {

@@ -7,8 +7,10 @@
 //   backward dX = [dY | sG] [W' ; A]       (M = T, N = k, K = d (+ r))
 //
 // W' never exists in global memory.  Dequantising warps read the packed codes
-// of one K-step (staged in shared memory by TMA, read back with 128-bit
-// loads), form per 64-weight block the 16 products bf16(level[i] * a') once,
+// of one K-step and the fp32 block scales a' of its blocks (both staged in
+// shared memory by TMA, the codes read back with 128-bit loads; the scales are
+// formed once per call by nf4_block_scales in a TMA-friendly layout), form per
+// 64-weight block the 16 products bf16(level[i] * a') once,
 // select each weight's value from them with byte permutes on registers, and
 // write the bf16 tile in exactly the 128B-swizzled layout a TMA load of W'
 // would have produced (K-major rows for the forward, MN-major for dX).  So the
@@ -112,30 +114,6 @@ __device__ __forceinline__ void nf4_decode_block(uint4 c0, uint4 c1, float a, co
   o[7] = nf4_decode8(c1.w, t);
 }
 
-// Raw inputs of one block's scale a' = fp32(fp32(E4M3(q) * scale2) + mean),
-// loaded ahead of use.  `ok` = 0 for blocks outside W (their scale is 0, so
-// their decoded weights are zeros).
-struct ScaleIn {
-  uint32_t q;
-  float s2;
-  uint32_t ok;
-};
-__device__ __forceinline__ ScaleIn load_scale_in(const uint8_t* absmax_q, const float* scale2, int64_t b,
-                                                 bool ok) {
-  ScaleIn r;
-  r.q = 0u;
-  r.s2 = 0.f;
-  r.ok = ok ? 1u : 0u;
-  if (ok) {
-    r.q = __ldg(absmax_q + b);
-    r.s2 = __ldg(scale2 + (b >> 8));
-  }
-  return r;
-}
-__device__ __forceinline__ float scale_of(const ScaleIn& s, float mu) {
-  return s.ok ? __fadd_rn(__fmul_rn(e4m3_to_f32((uint8_t)s.q), s.s2), mu) : 0.f;
-}
-
 // ------------------------------------------------------------------ kernel
 struct Nf4GemmArgs {
   int M, N, K0, K1;           // M tokens, N output columns, K0 main depth, K1 = r
@@ -144,11 +122,6 @@ struct Nf4GemmArgs {
   int tma_store;              // bf16 output through shared staging + TMA stores
   uint16_t* out;              // direct-store fallback (rows not 16-byte aligned)
   int64_t ldo;
-  const uint8_t* absmax_q;
-  const float* scale2;
-  const float* mean;
-  int64_t kb;                 // quantisation blocks per row of W (k / 64)
-  int wd, wk;                 // W is wd x wk
   float levels[16];
 };
 
@@ -156,10 +129,11 @@ constexpr int kNf4DqWarps = 8;
 constexpr int kNf4Threads = (6 + kNf4DqWarps) * 32;     // 448
 constexpr int kNf4SA = 3;          // activation stages: two 128 x 64 bf16 tiles (32 KB)
 constexpr int kNf4SB = 2;          // weight stages: 256 x 64 bf16 (32 KB), dequantised or (rank-r) TMA
-constexpr int kNf4SC = 4;          // code stages: 8 KB
+constexpr int kNf4SC = 3;          // code stages: 8 KB of codes + 1 KB of block scales
 constexpr int kNf4ABytes = 32768;
 constexpr int kNf4BBytes = 32768;
-constexpr int kNf4CBytes = 8192;
+constexpr int kNf4CodeBytes = 8192;
+constexpr int kNf4CBytes = kNf4CodeBytes + 1024;
 constexpr int kNf4StgBoxes = 2;                         // epilogue staging: 4 KB boxes per warp
 constexpr int kNf4Stage = 4 * kNf4StgBoxes * 4096;
 constexpr int kNf4SmemBytes =
@@ -194,8 +168,9 @@ __device__ __forceinline__ void mbar_wait_drain(uint32_t bar, uint32_t parity) {
 template <bool kDx>
 __global__ void __launch_bounds__(kNf4Threads, 1)
     gemm_nf4_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmC,
-                    const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
-                    const __grid_constant__ CUtensorMap tmOut, const __grid_constant__ Nf4GemmArgs p) {
+                    const __grid_constant__ CUtensorMap tmS, const __grid_constant__ CUtensorMap tmA1,
+                    const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmOut,
+                    const __grid_constant__ Nf4GemmArgs p) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   const uint32_t pad = (1024u - (raw_addr & 1023u)) & 1023u;
@@ -252,6 +227,7 @@ __global__ void __launch_bounds__(kNf4Threads, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmA0);
     tma_prefetch_desc(&tmC);
+    tma_prefetch_desc(&tmS);
     if (steps1 > 0) {
       tma_prefetch_desc(&tmA1);
       tma_prefetch_desc(&tmB1);
@@ -298,11 +274,16 @@ __global__ void __launch_bounds__(kNf4Threads, 1)
               break;
             }
             const uint32_t fc = smem_u32(&c_full[sc]);
-            mbar_arrive_expect_tx(fc, (uint32_t)kNf4CBytes);
-            if (kDx)
+            mbar_arrive_expect_tx(fc, (uint32_t)(kNf4CodeBytes + 1024));
+            if (kDx) {
               tma_load_2d(sC + sc * kNf4CBytes, &tmC, fc, c.n0 / 2, step * 64);
-            else
+              // scales of the tile's 64 K-rows x 4 block columns
+              tma_load_2d(sC + sc * kNf4CBytes + kNf4CodeBytes, &tmS, fc, c.n0 / 64, step * 64);
+            } else {
               tma_load_2d(sC + sc * kNf4CBytes, &tmC, fc, step * 32, c.n0);
+              // scales of the tile's 256 rows at block column `step`
+              tma_load_2d(sC + sc * kNf4CBytes + kNf4CodeBytes, &tmS, fc, c.n0, step);
+            }
             c_iss[sc] += 1;
             ++gc;
           } else {
@@ -472,28 +453,8 @@ __global__ void __launch_bounds__(kNf4Threads, 1)
     // c = i / 64 (W' block column n0 / 64 + c).
     const int i = threadIdx.x - 192;
     const int kk = i & 63, cc = i >> 6;
-    const float mu = __ldg(p.mean);
     int g = 0, gc = 0;
     for (int u = blockIdx.x; u < units; u += gridDim.x) {
-      const Nf4Unit c = nf4_unit(p, u);
-      // block index b(step) = b0 + step * bstride; validity per step
-      int64_t b0, bstride;
-      bool col_ok;
-      if (kDx) {
-        const int64_t col = (int64_t)(c.n0 >> 6) + cc;
-        col_ok = col < p.kb;
-        b0 = (int64_t)kk * p.kb + col;
-        bstride = 64 * p.kb;
-      } else {
-        col_ok = c.n0 + i < p.wd;
-        b0 = (int64_t)(c.n0 + i) * p.kb;
-        bstride = 1;
-      }
-      auto fetch = [&](int s) -> ScaleIn {
-        const bool ok = col_ok && s < steps0 && (!kDx || s * 64 + kk < p.wd);
-        return load_scale_in(p.absmax_q, p.scale2, b0 + (int64_t)s * bstride, ok);
-      };
-      ScaleIn s_cur = fetch(0), s_n1 = fetch(1), s_n2 = fetch(2);
       bool live = true;
       for (int step = 0; step < steps0; ++step, ++g, ++gc) {
         const int sc = gc % kNf4SC;
@@ -504,26 +465,26 @@ __global__ void __launch_bounds__(kNf4Threads, 1)
         }
         uint4 c0, c1;
         const uint32_t cs = sC + sc * kNf4CBytes;
+        const float* scl = reinterpret_cast<const float*>(smem + (cs - sbase) + kNf4CodeBytes);
+        float a;
         if (kDx) {
           // 128-byte rows (K-rows), 128B swizzle: 16-byte chunk j at (j ^ (row & 7))
           const uint32_t row = cs + kk * 128;
           const int sw = kk & 7;
           c0 = ld_shared_v4(row + (((2 * cc) ^ sw) << 4));
           c1 = ld_shared_v4(row + (((2 * cc + 1) ^ sw) << 4));
+          a = scl[kk * 4 + cc];
         } else {
           // 32-byte rows, 32B swizzle: chunk j at (j ^ ((row >> 2) & 1))
           const uint32_t row = cs + i * 32;
           const int sw = (i >> 2) & 1;
           c0 = ld_shared_v4(row + ((0 ^ sw) << 4));
           c1 = ld_shared_v4(row + ((1 ^ sw) << 4));
+          a = scl[i];
         }
-        const float a = scale_of(s_cur, mu);
-        s_cur = s_n1;
-        s_n1 = s_n2;
-        s_n2 = fetch(step + 3);
         uint4 o[8];
         nf4_decode_block(c0, c1, a, p.levels, o);
-        // the codes are consumed (the decode read them): release the stage
+        // the codes and scales are consumed (the decode read them): release the stage
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&c_empty[sc]));
         const int sb = g % kNf4SB;
@@ -597,24 +558,21 @@ struct Nf4SmallArgs {
   int lo_off;                 // OUT_HILO
   float scale;                // OUT_U / OUT_HILO: bf16 output = bf16(scale v)
   float f32_scale;            // OUT_U: fp32 output = f32_scale v
-  const uint8_t* absmax_q;
-  const float* scale2;
-  const float* mean;
-  int64_t kb;
-  int wd, wk;
   float levels[16];
 };
 
 constexpr int kSmDqWarps = 4;
 constexpr int kSmThreads = (2 + kSmDqWarps) * 32;       // 192
+constexpr int kSmMaxSplits = 16;                         // depth splits per row tile (host plan caps it)
 
 template <int TN>
 struct SmallCfg {
   static constexpr int SA = 3;                 // weight tiles, 128 x 64 bf16
-  static constexpr int SC = 4;                 // codes, 4 KB
+  static constexpr int SC = 3;                 // codes (4 KB) + block scales (up to 1 KB)
   static constexpr int SB = 4;                 // activation tiles, TN x 64 bf16
   static constexpr int kABytes = 16384;
-  static constexpr int kCBytes = 4096;
+  static constexpr int kCodeBytes = 4096;
+  static constexpr int kCBytes = kCodeBytes + 1024;
   static constexpr int kBBytes = TN * 128;
   static constexpr int kSmem = SA * kABytes + SC * kCBytes + SB * kBBytes + 1024 + 256;
   static constexpr int kTmemCols = TN < 32 ? 32 : TN;
@@ -644,8 +602,8 @@ __device__ __forceinline__ void small_emit(const Nf4SmallArgs& p, int m, int t, 
 template <int kSrc, int kOut, int TN>
 __global__ void __launch_bounds__(kSmThreads, 1)
     gemm_nf4_small_kernel(const __grid_constant__ CUtensorMap tmAct, const __grid_constant__ CUtensorMap tmW,
-                          const __grid_constant__ CUtensorMap tmW1, const __grid_constant__ CUtensorMap tmAct1,
-                          const __grid_constant__ Nf4SmallArgs p) {
+                          const __grid_constant__ CUtensorMap tmS, const __grid_constant__ CUtensorMap tmW1,
+                          const __grid_constant__ CUtensorMap tmAct1, const __grid_constant__ Nf4SmallArgs p) {
   using Cfg = SmallCfg<TN>;
   constexpr bool kNf4 = kSrc == SRC_NF4_ROWS || kSrc == SRC_NF4_COLS;
   constexpr bool kMnA = kSrc == SRC_NF4_COLS || kSrc == SRC_TMA_MN;
@@ -707,6 +665,7 @@ __global__ void __launch_bounds__(kSmThreads, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmAct);
     tma_prefetch_desc(&tmW);
+    if (kNf4) tma_prefetch_desc(&tmS);
     if (steps1 > 0) {
       tma_prefetch_desc(&tmW1);
       tma_prefetch_desc(&tmAct1);
@@ -743,11 +702,18 @@ __global__ void __launch_bounds__(kSmThreads, 1)
           if (!mbar_wait_bounded(smem_u32(&c_empty[sc]), (uint32_t)(((step / Cfg::SC) & 1) ^ 1), abort_flag))
             break;
           const uint32_t fc = smem_u32(&c_full[sc]);
-          mbar_arrive_expect_tx(fc, (uint32_t)Cfg::kCBytes);
-          if (kSrc == SRC_NF4_COLS)
+          if (kSrc == SRC_NF4_COLS) {
+            mbar_arrive_expect_tx(fc, (uint32_t)(Cfg::kCodeBytes + 1024));
             tma_load_2d(sC + sc * Cfg::kCBytes, &tmW, fc, m0 / 2, ks * 64);
-          else
+            // scales of 64 K-rows x 4 block columns from a 16-byte aligned
+            // column (the tile's two columns sit at (m0 / 64) % 4)
+            tma_load_2d(sC + sc * Cfg::kCBytes + Cfg::kCodeBytes, &tmS, fc, (m0 >> 6) & ~3, ks * 64);
+          } else {
+            mbar_arrive_expect_tx(fc, (uint32_t)(Cfg::kCodeBytes + 512));
             tma_load_2d(sC + sc * Cfg::kCBytes, &tmW, fc, ks * 32, m0);
+            // scales of the tile's 128 rows at block column ks
+            tma_load_2d(sC + sc * Cfg::kCBytes + Cfg::kCodeBytes, &tmS, fc, m0, ks);
+          }
           c_iss[sc] += 1;
         } else {
           // a bf16 weight-side tile by TMA: the main operand of U / G, or the
@@ -825,25 +791,6 @@ __global__ void __launch_bounds__(kSmThreads, 1)
       // 64 * ks + kk) and MN chunk cc = i / 64 (W' block column m0 / 64 + cc).
       const int i = threadIdx.x - 64;
       const int kk = i & 63, cc = i >> 6;
-      const float mu = __ldg(p.mean);
-      int64_t b0, bstride;
-      bool col_ok;
-      if (kSrc == SRC_NF4_COLS) {
-        const int64_t col = (int64_t)(m0 >> 6) + cc;
-        col_ok = col < p.kb;
-        b0 = (int64_t)kk * p.kb + col;
-        bstride = 64 * p.kb;
-      } else {
-        col_ok = m0 + i < p.wd;
-        b0 = (int64_t)(m0 + i) * p.kb;
-        bstride = 1;
-      }
-      auto fetch = [&](int step) -> ScaleIn {
-        const int ks = s_begin + step;
-        const bool ok = col_ok && step < nmain && (kSrc != SRC_NF4_COLS || ks * 64 + kk < p.wd);
-        return load_scale_in(p.absmax_q, p.scale2, b0 + (int64_t)ks * bstride, ok);
-      };
-      ScaleIn s_cur = fetch(0), s_n1 = fetch(1), s_n2 = fetch(2);
       for (int step = 0; step < nmain; ++step) {
         const int sc = step % Cfg::SC;
         bool ok = mbar_wait_bounded(smem_u32(&c_full[sc]), (uint32_t)((step / Cfg::SC) & 1), abort_flag);
@@ -853,22 +800,23 @@ __global__ void __launch_bounds__(kSmThreads, 1)
         }
         uint4 c0, c1;
         const uint32_t cs = sC + sc * Cfg::kCBytes;
+        const float* scl =
+            reinterpret_cast<const float*>(smem + (cs - sA) + Cfg::kCodeBytes);
+        float a;
         if (kSrc == SRC_NF4_COLS) {
           // 64-byte rows, 64B swizzle: chunk j at (j ^ ((row >> 1) & 3))
           const uint32_t row = cs + kk * 64;
           const int sw = (kk >> 1) & 3;
           c0 = ld_shared_v4(row + (((2 * cc) ^ sw) << 4));
           c1 = ld_shared_v4(row + (((2 * cc + 1) ^ sw) << 4));
+          a = scl[kk * 4 + ((m0 >> 6) & 3) + cc];
         } else {
           const uint32_t row = cs + i * 32;
           const int sw = (i >> 2) & 1;
           c0 = ld_shared_v4(row + ((0 ^ sw) << 4));
           c1 = ld_shared_v4(row + ((1 ^ sw) << 4));
+          a = scl[i];
         }
-        const float a = scale_of(s_cur, mu);
-        s_cur = s_n1;
-        s_n1 = s_n2;
-        s_n2 = fetch(step + 3);
         uint4 o[8];
         nf4_decode_block(c0, c1, a, p.levels, o);
         __syncwarp();
@@ -935,34 +883,26 @@ __global__ void __launch_bounds__(kSmThreads, 1)
       if (*last_flag && ok) {
         __threadfence();
         if (m < p.Mw) {
+          // four tokens at a time with every split's partial in flight
+          // (at most kSmMaxSplits), then summed in split order
           const int64_t zs = (int64_t)p.T * p.Mw;
-          for (int t0 = 0; t0 < p.T; t0 += 16) {
-            // 16 tokens at a time; two splits' loads in flight per round,
-            // added in split order
+          for (int t0 = 0; t0 < p.T; t0 += 4) {
+            const int nt = min(4, p.T - t0);
             const float* src = p.part + (int64_t)t0 * p.Mw + m;
-            const int nt = min(16, p.T - t0);
-            float acc[16];
+            float v[kSmMaxSplits][4];
 #pragma unroll
-            for (int j = 0; j < 16; ++j) acc[j] = j < nt ? __ldcg(src + (int64_t)j * p.Mw) : 0.f;
-            int z = 1;
-            for (; z + 1 < p.splits; z += 2) {
-              float v0[16], v1[16];
+            for (int z = 0; z < kSmMaxSplits; ++z)
 #pragma unroll
-              for (int j = 0; j < 16; ++j) {
-                v0[j] = j < nt ? __ldcg(src + z * zs + (int64_t)j * p.Mw) : 0.f;
-                v1[j] = j < nt ? __ldcg(src + (z + 1) * zs + (int64_t)j * p.Mw) : 0.f;
-              }
+              for (int j = 0; j < 4; ++j)
+                v[z][j] = (z < p.splits && j < nt) ? __ldcg(src + z * zs + (int64_t)j * p.Mw) : 0.f;
 #pragma unroll
-              for (int j = 0; j < 16; ++j) acc[j] = __fadd_rn(__fadd_rn(acc[j], v0[j]), v1[j]);
+            for (int j = 0; j < 4; ++j) {
+              float acc = v[0][j];
+#pragma unroll
+              for (int z = 1; z < kSmMaxSplits; ++z)
+                if (z < p.splits) acc = __fadd_rn(acc, v[z][j]);
+              if (j < nt) small_emit<kOut>(p, m, t0 + j, acc);
             }
-            if (z < p.splits) {
-#pragma unroll
-              for (int j = 0; j < 16; ++j)
-                acc[j] = __fadd_rn(acc[j], j < nt ? __ldcg(src + z * zs + (int64_t)j * p.Mw) : 0.f);
-            }
-#pragma unroll
-            for (int j = 0; j < 16; ++j)
-              if (j < nt) small_emit<kOut>(p, m, t0 + j, acc[j]);
           }
         }
         if (threadIdx.x == 64) p.tickets[tile] = 0u;

@@ -522,6 +522,55 @@ __global__ void __launch_bounds__(256) nf4_dequantize_kernel(
 }
 
 // ---------------------------------------------------------------------------
+// Block scales a'_b = fp32(fp32(E4M3(absmax_q_b) * scale2_j) + mean) of every
+// block, written once per GEMM call in the layout the dequantising GEMMs load
+// by TMA next to the codes (one tile of scales per K-step):
+//   transposed = 1: out[s * ld + n]  (block column s, row n: one K-step of the
+//                   forward reads consecutive rows)
+//   transposed = 0: out[n * ld + s]  (row n, block column s: one K-step of dX
+//                   reads consecutive block columns of 64 rows)
+// Threads of a 32 x 32 tile read the constants row by row and write through
+// shared memory, so both the loads and the stores are coalesced.  The CTAs of
+// the first tile row also zero `zero_n` words at `zero` (the completion
+// tickets of the few-token kernels that follow).
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) nf4_block_scales(const uint8_t* __restrict__ absmax_q,
+                                                        const float* __restrict__ scale2,
+                                                        const float* __restrict__ mean, int64_t d, int64_t kb,
+                                                        int transposed, int64_t ld, float* __restrict__ out,
+                                                        unsigned int* __restrict__ zero, int zero_n) {
+  __shared__ float tile[32][33];
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;       // 32 x 8 threads
+  const int64_t n0 = (int64_t)blockIdx.y * 32, s0 = (int64_t)blockIdx.x * 32;
+  const float mu = mean[0];
+  if (zero != nullptr && blockIdx.y == 0) {
+    for (int i = (int)(blockIdx.x * blockDim.x + threadIdx.x); i < zero_n; i += (int)(gridDim.x * blockDim.x))
+      zero[i] = 0u;
+  }
+  for (int j = ty; j < 32; j += 8) {
+    const int64_t n = n0 + j, sc = s0 + tx;
+    float a = 0.f;
+    if (n < d && sc < kb) {
+      const int64_t b = n * kb + sc;
+      a = __fadd_rn(__fmul_rn(e4m3_to_f32(absmax_q[b]), scale2[b / kBlock2]), mu);
+    }
+    tile[j][tx] = a;
+  }
+  __syncthreads();
+  if (transposed) {
+    for (int j = ty; j < 32; j += 8) {
+      const int64_t sc = s0 + j, n = n0 + tx;
+      if (sc < kb && n < d) out[sc * ld + n] = tile[tx][j];
+    }
+  } else {
+    for (int j = ty; j < 32; j += 8) {
+      const int64_t n = n0 + j, sc = s0 + tx;
+      if (n < d && sc < kb) out[n * ld + sc] = tile[j][tx];
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Small helpers for the rank-r operands.
 // ---------------------------------------------------------------------------
 // dst (rows x ld_dst, bf16) = src (rows x cols, bf16) with zero columns
@@ -583,6 +632,92 @@ __global__ void apply_keep_bf16(const uint4* __restrict__ X, const uint8_t* __re
     const uint32_t m2 = ((b & 16u) ? 0x0000FFFFu : 0u) | ((b & 32u) ? 0xFFFF0000u : 0u);
     const uint32_t m3 = ((b & 64u) ? 0x0000FFFFu : 0u) | ((b & 128u) ? 0xFFFF0000u : 0u);
     Xm[u] = make_uint4(x.x & m0, x.y & m1, x.z & m2, x.w & m3);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Several unmerged adapters in one batch: token t uses adapter idx[t] of a
+// stack (A_i r x k, B_i d x r, scale s_i).  Their rank-r operands are laid out
+// side by side, R = n r columns, each token's values in its adapter's block of
+// r columns and zeros elsewhere, so one GEMM with depth R computes every
+// token's own adapter term.
+// ---------------------------------------------------------------------------
+constexpr int kMaxAdapters = 64;
+struct AdapterScales {
+  float s[kMaxAdapters];
+};
+
+// Bcat[row][i r + j] = Bs[i][row][j]  (d x R, bf16)
+__global__ void cat_adapters_b(const uint16_t* __restrict__ Bs, int64_t d, int r, int n,
+                               uint16_t* __restrict__ Bcat) {
+  const int R = n * r;
+  const int64_t total = d * R;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += stride) {
+    const int64_t row = e / R;
+    const int c = (int)(e - row * R);
+    const int i = c / r, j = c - i * r;
+    Bcat[e] = Bs[((int64_t)i * d + row) * r + j];
+  }
+}
+
+// From U_all = X [A_0; ...; A_{n-1}]^T (T x R fp32): the token's own
+// U_save[t][j] = U_all[t][idx r + j], and sU[t][c] (T x ldo bf16) =
+// bf16(s_idx U_all[t][c]) inside the token's block, 0 elsewhere.  A token
+// whose index lies outside [0, n) has no block: its U_save row is 0.
+__global__ void scatter_adapter_u(const float* __restrict__ U_all, const int32_t* __restrict__ idx, int64_t T,
+                                  int r, int n, int ldo, const __grid_constant__ AdapterScales sc,
+                                  float* __restrict__ U_save, uint16_t* __restrict__ sU) {
+  const int R = n * r;
+  const int64_t total = T * ldo;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += stride) {
+    const int64_t t = e / ldo;
+    const int c = (int)(e - t * ldo);
+    const int a = idx[t];
+    const bool mine = c < R && c / r == a;
+    const float u = mine ? U_all[t * R + c] : 0.f;
+    const __nv_bfloat16 h = __float2bfloat16_rn(mine ? __fmul_rn(sc.s[a], u) : 0.f);
+    sU[e] = *reinterpret_cast<const uint16_t*>(&h);
+    if (mine) U_save[t * r + (c - a * r)] = u;
+    else if ((a < 0 || a >= n) && c < r) U_save[t * r + c] = 0.f;
+  }
+}
+
+// hi/lo pair of v = s_idx V (hi = bf16(v), lo = bf16(v - hi)) into the token's
+// block: out row t has hi in columns [0, half) and lo in [half, 2 half), zero
+// outside the block.  V is per token (T x r: the value of block column j is
+// V[t][j]) or over all blocks (T x R: V[t][c]).
+__global__ void scatter_adapter_hilo(const float* __restrict__ V, int per_token, const int32_t* __restrict__ idx,
+                                     int64_t T, int r, int n, int half, const __grid_constant__ AdapterScales sc,
+                                     uint16_t* __restrict__ out) {
+  const int R = n * r;
+  const int64_t total = T * half;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += stride) {
+    const int64_t t = e / half;
+    const int c = (int)(e - t * half);
+    const int a = idx[t];
+    const bool mine = c < R && c / r == a;
+    float v = 0.f;
+    if (mine) v = __fmul_rn(sc.s[a], per_token ? V[t * r + (c - a * r)] : V[t * R + c]);
+    const __nv_bfloat16 h = __float2bfloat16_rn(v);
+    const __nv_bfloat16 l = __float2bfloat16_rn(__fsub_rn(v, __bfloat162float(h)));
+    out[t * 2 * half + c] = *reinterpret_cast<const uint16_t*>(&h);
+    out[t * 2 * half + half + c] = *reinterpret_cast<const uint16_t*>(&l);
+  }
+}
+
+// dBs[i][row][j] = dBcat[row][i r + j]
+__global__ void uncat_adapters_db(const float* __restrict__ dBcat, int64_t d, int r, int n, float* __restrict__ dBs) {
+  const int R = n * r;
+  const int64_t total = d * R;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += stride) {
+    const int64_t row = e / R;
+    const int c = (int)(e - row * R);
+    const int i = c / r, j = c - i * r;
+    dBs[((int64_t)i * d + row) * r + j] = dBcat[e];
   }
 }
 

@@ -120,6 +120,19 @@ def test_argument_validation_without_device(lib):
     assert L.qlora_fwd_dropout(ctypes.byref(nf), 16, 16, 8, 16.0, 16, 16, 0.1, 16, 16, 16, 16,
                                64, None) == 4                                                  # workspace
     assert q4.qlora_fwd_dropout_workspace_bytes(256, 256, 8, 16) > q4.qlora_fwd_workspace_bytes(256, 256, 8, 16)
+    # several adapters: count, total rank and alphas are checked on the host
+    al = (ctypes.c_float * 4)(16.0, 16.0, 16.0, 16.0)
+    assert L.qlora_fwd_multi(ctypes.byref(nf), 0, 16, 16, 8, ctypes.addressof(al), 16, 16, 16, 16, 16,
+                             16, 1 << 20, None) == 1                                           # n = 0
+    assert L.qlora_fwd_multi(ctypes.byref(nf), 65, 16, 16, 1, ctypes.addressof(al), 16, 16, 16, 16, 16,
+                             16, 1 << 20, None) == 1                                           # n > 64
+    assert L.qlora_fwd_multi(ctypes.byref(nf), 4, 16, 16, 65, ctypes.addressof(al), 16, 16, 16, 16, 16,
+                             16, 1 << 20, None) == 2                                           # n r > 256
+    bad = (ctypes.c_float * 2)(16.0, -1.0)
+    assert L.qlora_fwd_multi(ctypes.byref(nf), 2, 16, 16, 8, ctypes.addressof(bad), 16, 16, 16, 16, 16,
+                             16, 1 << 20, None) == 1                                           # alpha <= 0
+    assert L.qlora_bwd_multi(ctypes.byref(nf), 2, 16, 16, 8, ctypes.addressof(al), 18, 16, 16, 16, 16, 16,
+                             16, 16, 16, 1 << 20, None) == 3                                   # misaligned idx
     # Adam: step, betas, lr and alignment are checked on the host; n = 0 is a no-op
     assert L.lora_adam_step(16, 16, 16, 16, 16, 8, 0, 1e-3, 0.9, 0.999, 1e-8, 0.0, None) == 1     # step 0
     assert L.lora_adam_step(16, 16, 16, 16, 16, 8, 1, 1e-3, 1.0, 0.999, 1e-8, 0.0, None) == 1     # beta1 = 1
