@@ -60,9 +60,9 @@ def algorithmic_bytes(T, d, k, r):
     return weights + adapters + acts
 
 
-def workload(config_index: int):
+def workload(config_index: int, tokens=None):
     cfg = synthetic.config(config_index)
-    T = cfg.tokens[0]
+    T = cfg.tokens[0] if tokens is None else tokens
     return cfg, T
 
 
@@ -199,7 +199,7 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    cfg, T = workload(args.config)
+    cfg, T = workload(args.config, args.tokens)
     flops_step = 0.0
     times = []
     for i in range(args.warmup + args.steps):
@@ -449,7 +449,7 @@ def run_ours(args):
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
     q4.lib()
-    cfg, T = workload(args.config)
+    cfg, T = workload(args.config, args.tokens)
 
     # ---- resident inputs (per rank: its own tokens, the same frozen weights)
     layers = []
@@ -797,6 +797,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", type=int, default=4)
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="tokens per GPU instead of the config's own (small profiling cases)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-configs", action="store_true",
                     help="skip the per-config block (configs 1, 2, 3, 5) of the JSON line")

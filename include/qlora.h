@@ -365,6 +365,17 @@ QLORA_API int qlora_profile_end(qlora_kernel_stat_t* out, int capacity, int* n_o
 /* Number of kernels this library has launched in this process (all devices). */
 QLORA_API int64_t qlora_launch_count(void);
 
+/*
+ * Selects the build of the NF4 base GEMM used above 64 tokens, for every
+ * later call in this process: 0 = default (CTA pairs where the device can
+ * hold clusters of two, else one CTA per tile), 1 = one CTA per 256 x 256
+ * tile, 2 = CTA pairs (two CTAs of a cluster run 256-row tensor-core MMAs
+ * over both SMs, each decoding half of every weight tile).  Both builds give
+ * bit-identical results; the choice only changes speed.  Returns
+ * QLORA_ERR_INVALID_ARG for any other mode.
+ */
+QLORA_API int qlora_set_nf4_gemm_mode(int mode);
+
 #ifdef __cplusplus
 }
 #endif

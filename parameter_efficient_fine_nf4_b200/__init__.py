@@ -89,6 +89,7 @@ _SIGNATURES = {
     "qlora_profile_begin": (_INT, []),
     "qlora_profile_end": (_INT, [ctypes.POINTER(KernelStat), _INT, ctypes.POINTER(_INT)]),
     "qlora_launch_count": (_I64, []),
+    "qlora_set_nf4_gemm_mode": (_INT, [_INT]),
 }
 
 EXPORTED = tuple(_SIGNATURES)
@@ -201,6 +202,11 @@ def lora_merge_workspace_bytes(d: int, k: int, r: int) -> int:
 
 def qlora_launch_count() -> int:
     return lib().qlora_launch_count()
+
+
+def qlora_set_nf4_gemm_mode(mode: int) -> None:
+    """0 = by shape, 1 = one CTA per tile, 2 = CTA pairs (same bits, other speed)."""
+    _check(lib().qlora_set_nf4_gemm_mode(mode), "qlora_set_nf4_gemm_mode")
 
 
 # ------------------------------------------------------------------- device calls

@@ -141,6 +141,10 @@ std::mutex g_init_mu;
 bool g_dev_ready[kMaxDevices] = {false};
 unsigned long long g_dev_ctx[kMaxDevices] = {0};
 int g_dev_sms[kMaxDevices] = {0};
+int g_dev_pair_clusters[kMaxDevices] = {0};
+// Which build of the NF4 base GEMM runs for more than 64 tokens: 0 = chosen by
+// shape, 1 = one CTA per tile, 2 = CTA pairs (both give the same bits).
+std::atomic<int> g_nf4_gemm_mode{0};
 
 // Unique id of the calling thread's current CUDA context, 0 if there is none
 // yet.  Ids are never reused within a process, so a device reset (which
@@ -186,14 +190,34 @@ cudaError_t set_gemm_attrs() {
                               GemmCfg<BN>::kSmemBytes);
 }
 
-template <bool kDx>
+template <bool kDx, bool kPair>
 cudaError_t set_nf4_gemm_attrs() {
-  const cudaError_t e = cudaFuncSetAttribute(gemm_nf4_kernel<kDx>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             kNf4SmemBytes);
+  using Cfg = Nf4Cfg<kPair>;
+  const cudaError_t e = cudaFuncSetAttribute(gemm_nf4_kernel<kDx, kPair>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, Cfg::kSmemBytes);
   if (e != cudaSuccess) return e;
   cudaFuncAttributes fa;
-  if (cudaFuncGetAttributes(&fa, gemm_nf4_kernel<kDx>) != cudaSuccess) return cudaErrorInvalidValue;
-  return fa.maxThreadsPerBlock >= kNf4Threads ? cudaSuccess : cudaErrorLaunchOutOfResources;
+  if (cudaFuncGetAttributes(&fa, gemm_nf4_kernel<kDx, kPair>) != cudaSuccess) return cudaErrorInvalidValue;
+  return fa.maxThreadsPerBlock >= Cfg::kThreads ? cudaSuccess : cudaErrorLaunchOutOfResources;
+}
+
+// Clusters of two CTAs of the paired NF4 GEMM that fit on the device at once.
+int pair_clusters_on_device() {
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3(2 * kSMs);
+  cfg.blockDim = dim3(Nf4Cfg<true>::kThreads);
+  cfg.dynamicSmemBytes = Nf4Cfg<true>::kSmemBytes;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = 2;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, gemm_nf4_kernel<false, true>, &cfg) != cudaSuccess) return 0;
+  return n;
 }
 
 template <int kSrc, int kOut, int TN>
@@ -254,9 +278,11 @@ int ensure_device() {
   if (set_gemm_attrs<64>() != cudaSuccess || set_gemm_attrs<128>() != cudaSuccess ||
       set_gemm_attrs<256>() != cudaSuccess || set_deploy_attrs<true, 1>() != cudaSuccess ||
       set_deploy_attrs<true, 2>() != cudaSuccess || set_deploy_attrs<false, 1>() != cudaSuccess ||
-      set_deploy_attrs<false, 2>() != cudaSuccess || set_nf4_gemm_attrs<false>() != cudaSuccess ||
-      set_nf4_gemm_attrs<true>() != cudaSuccess || set_small_attrs() != cudaSuccess)
+      set_deploy_attrs<false, 2>() != cudaSuccess || set_nf4_gemm_attrs<false, false>() != cudaSuccess ||
+      set_nf4_gemm_attrs<true, false>() != cudaSuccess || set_nf4_gemm_attrs<false, true>() != cudaSuccess ||
+      set_nf4_gemm_attrs<true, true>() != cudaSuccess || set_small_attrs() != cudaSuccess)
     return QLORA_ERR_CUDA;
+  g_dev_pair_clusters[dev] = pair_clusters_on_device();
   g_dev_ctx[dev] = current_ctx_id();
   g_dev_ready[dev] = true;
   return QLORA_OK;
@@ -726,6 +752,20 @@ int adapter_grad_gemm(const char* name, const uint16_t* big, int64_t M, int64_t 
   return QLORA_OK;
 }
 
+int pair_clusters() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
+  return g_dev_pair_clusters[dev];
+}
+
+// CTA pairs halve each SM's share of the decode at the same MMA work per SM;
+// measured faster than one CTA per tile at every shape from 65 to 16384
+// tokens, so they are the default wherever clusters of two fit.
+bool nf4_use_pair() {
+  const int mode = g_nf4_gemm_mode.load();
+  return mode != 1 && pair_clusters() > 0;
+}
+
 // Base GEMM on the NF4 weight with the rank-r extension (gemm_nf4_kernel):
 //   forward (dx = false): out = Y (T x d)  = [X | sU][W' | B]^T,  a1 = sU (T x r8, ld r8), b1 = B (d x r8)
 //   dX      (dx = true):  out = dX (T x k) = [dY | sG][W' ; A],    a1 = sG (T x r, ld a1_ld), b1 = A (r x k)
@@ -739,21 +779,28 @@ int launch_nf4_gemm(bool dx, const qlora_nf4_t* q, const float* scales, const ui
   a.N = (int)(dx ? k : d);
   a.K0 = (int)(dx ? d : k);
   a.K1 = r;
-  a.tiles_m = (int)cdiv(T, 256);
+  const bool pair = nf4_use_pair();
+  a.tiles_m = (int)cdiv(T, pair ? 512 : 256);
   a.tiles_n = (int)cdiv(a.N, 256);
-  a.group_m = 8;
+  a.group_m = pair ? 4 : 8;
   memcpy(a.levels, tables().levels, sizeof(a.levels));
   CUtensorMap mA0, mC, mS, mA1, mB1, mO;
+  // codes and scales: a pair's CTA loads the half of the weight tile it decodes
   if (dx) {
     if (!make_map_f32(&mS, scales, k / 64, d, scales_ld_dx(k), 4, 64)) return QLORA_ERR_CUDA;
   } else {
-    if (!make_map_f32(&mS, scales, d, k / 64, scales_ld_fwd(d), 256, 1)) return QLORA_ERR_CUDA;
+    if (!make_map_f32(&mS, scales, d, k / 64, scales_ld_fwd(d), pair ? 128 : 256, 1)) return QLORA_ERR_CUDA;
   }
   if (!make_map(&mA0, act, a.K0, T, a.K0, 128)) return QLORA_ERR_CUDA;
   if (dx) {
-    if (!make_map_u8(&mC, q->codes, k / 2, d, k / 2, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
+    if (pair) {
+      if (!make_map_u8(&mC, q->codes, k / 2, d, k / 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_64B)) return QLORA_ERR_CUDA;
+    } else {
+      if (!make_map_u8(&mC, q->codes, k / 2, d, k / 2, 128, 64, CU_TENSOR_MAP_SWIZZLE_128B)) return QLORA_ERR_CUDA;
+    }
   } else {
-    if (!make_map_u8(&mC, q->codes, k / 2, d, k / 2, 32, 256, CU_TENSOR_MAP_SWIZZLE_32B)) return QLORA_ERR_CUDA;
+    if (!make_map_u8(&mC, q->codes, k / 2, d, k / 2, 32, pair ? 128 : 256, CU_TENSOR_MAP_SWIZZLE_32B))
+      return QLORA_ERR_CUDA;
   }
   if (r == 0) {
     mA1 = mA0;
@@ -763,7 +810,8 @@ int launch_nf4_gemm(bool dx, const qlora_nf4_t* q, const float* scales, const ui
     if (dx) {
       if (!make_map(&mB1, b1, k, r, k, 64)) return QLORA_ERR_CUDA;        // A columns, MN-major
     } else {
-      if (!make_map(&mB1, b1, r8, d, r8, 256)) return QLORA_ERR_CUDA;     // B rows, K-major
+      // B rows, K-major (a pair's CTA loads its 128 of the tile's 256 rows)
+      if (!make_map(&mB1, b1, r8, d, r8, pair ? 128 : 256)) return QLORA_ERR_CUDA;
     }
   }
   mO = mA0;
@@ -774,15 +822,41 @@ int launch_nf4_gemm(bool dx, const qlora_nf4_t* q, const float* scales, const ui
     if (!make_map(&mO, out, a.N, T, a.N, 32)) return QLORA_ERR_CUDA;
     a.tma_store = 1;
   }
-  const int64_t units = (int64_t)a.tiles_m * a.tiles_n;
-  const dim3 grid((unsigned)std::min<int64_t>(units, current_sms()));
   const double flops = 2.0 * (double)T * a.N * ((double)a.K0 + r);
   const char* name = dx ? "gemm_nf4_dx" : "gemm_nf4_fwd";
+  const int64_t units = (int64_t)a.tiles_m * a.tiles_n;
+  if (!pair) {
+    const dim3 grid((unsigned)std::min<int64_t>(units, current_sms()));
+    return launch(name, flops, 0.0, st, [&] {
+      if (dx)
+        gemm_nf4_kernel<true, false>
+            <<<grid, Nf4Cfg<false>::kThreads, Nf4Cfg<false>::kSmemBytes, st>>>(mA0, mC, mS, mA1, mB1, mO, a);
+      else
+        gemm_nf4_kernel<false, false>
+            <<<grid, Nf4Cfg<false>::kThreads, Nf4Cfg<false>::kSmemBytes, st>>>(mA0, mC, mS, mA1, mB1, mO, a);
+    });
+  }
+  // CTA pairs: units of 512 rows, one cluster of two per unit, as many
+  // clusters as fit at once
+  const int64_t clusters = std::min<int64_t>(units, std::max(1, pair_clusters()));
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3((unsigned)(2 * clusters));
+  cfg.blockDim = dim3(Nf4Cfg<true>::kThreads);
+  cfg.dynamicSmemBytes = Nf4Cfg<true>::kSmemBytes;
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = 2;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
   return launch(name, flops, 0.0, st, [&] {
     if (dx)
-      gemm_nf4_kernel<true><<<grid, kNf4Threads, kNf4SmemBytes, st>>>(mA0, mC, mS, mA1, mB1, mO, a);
+      cudaLaunchKernelEx(&cfg, gemm_nf4_kernel<true, true>, mA0, mC, mS, mA1, mB1, mO, a);
     else
-      gemm_nf4_kernel<false><<<grid, kNf4Threads, kNf4SmemBytes, st>>>(mA0, mC, mS, mA1, mB1, mO, a);
+      cudaLaunchKernelEx(&cfg, gemm_nf4_kernel<false, true>, mA0, mC, mS, mA1, mB1, mO, a);
   });
 }
 
@@ -1233,6 +1307,12 @@ int qlora_nf4_levels(float* levels16, float* thresholds15) {
 }
 
 int64_t qlora_launch_count(void) { return g_launches.load(); }
+
+int qlora_set_nf4_gemm_mode(int mode) {
+  if (mode < 0 || mode > 2) return QLORA_ERR_INVALID_ARG;
+  g_nf4_gemm_mode.store(mode);
+  return QLORA_OK;
+}
 
 size_t qlora_quantize_workspace_bytes(int64_t d, int64_t k) {
   if (d < 1 || k < 1) return 0;

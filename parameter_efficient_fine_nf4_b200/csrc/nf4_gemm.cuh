@@ -125,31 +125,59 @@ struct Nf4GemmArgs {
   float levels[16];
 };
 
-constexpr int kNf4DqWarps = 8;
-constexpr int kNf4Threads = (6 + kNf4DqWarps) * 32;     // 448
-constexpr int kNf4SA = 3;          // activation stages: two 128 x 64 bf16 tiles (32 KB)
-constexpr int kNf4SB = 2;          // weight stages: 256 x 64 bf16 (32 KB), dequantised or (rank-r) TMA
-constexpr int kNf4SC = 3;          // code stages: 8 KB of codes + 1 KB of block scales
-constexpr int kNf4ABytes = 32768;
-constexpr int kNf4BBytes = 32768;
-constexpr int kNf4CodeBytes = 8192;
-constexpr int kNf4CBytes = kNf4CodeBytes + 1024;
-constexpr int kNf4StgBoxes = 2;                         // epilogue staging: 4 KB boxes per warp
-constexpr int kNf4Stage = 4 * kNf4StgBoxes * 4096;
-constexpr int kNf4SmemBytes =
-    kNf4SA * kNf4ABytes + kNf4SB * kNf4BBytes + kNf4SC * kNf4CBytes + kNf4Stage + 1024 /*align*/ + 512 /*bars*/;
+// Two builds of the kernel:
+//   kPair = false: one CTA per unit of 256 rows x 256 columns; it decodes the
+//                  whole 256-wide weight tile of each K-step (8 dequantising
+//                  warps) and runs two 128-row MMAs on it.
+//   kPair = true:  a cluster of two CTAs per unit of 512 rows x 256 columns,
+//                  running pair MMAs (tcgen05 cta_group::2, M = 256): each
+//                  CTA holds 128 rows of each of the unit's two 256-row A
+//                  tiles and decodes 128 of the weight tile's 256 rows into
+//                  its own shared memory, which the pair MMA reads from both
+//                  SMs.  Per SM the MMA work per K-step is the same as one
+//                  CTA's, the decode half of it.  Rank 0 issues the MMAs;
+//                  the operand-ready barriers live in rank 0, the stage-free
+//                  and accumulator-ready barriers in both CTAs (the MMA
+//                  completions are multicast to both).
+template <bool kPair>
+struct Nf4Cfg {
+  static constexpr int kDqWarps = kPair ? 4 : 8;
+  // warps: 0 activation / rank-r loads, 1 MMA, 2-5 epilogue, 6 code loads,
+  // 7.. dequantisation
+  static constexpr int kDqWarp0 = 7;
+  static constexpr int kThreads = (kDqWarp0 + kDqWarps) * 32;
+  static constexpr int SA = kPair ? 4 : 3;        // activation stages: two 128 x 64 bf16 tiles (32 KB)
+  static constexpr int SB = kPair ? 3 : 2;        // weight stages: this CTA's rows of the 256 x 64 tile
+  static constexpr int SC = 3;                    // code stages: codes + block scales
+  static constexpr int kABytes = 32768;
+  static constexpr int kBBytes = kPair ? 16384 : 32768;
+  static constexpr int kCodeBytes = kPair ? 4096 : 8192;   // this CTA's rows of codes
+  static constexpr int kCBytes = kCodeBytes + 1024;
+  static constexpr int kStgBoxes = 2;             // epilogue staging: 4 KB boxes per warp
+  static constexpr int kStage = 4 * kStgBoxes * 4096;
+  static constexpr int kSmemBytes = SA * kABytes + SB * kBBytes + SC * kCBytes + kStage + 1024 + 512;
+  // arrivals that complete a weight stage: every dequantising warp of the
+  // unit (a rank-r stage: the TMA thread's expect_tx plus the rest)
+  static constexpr int kBFull = kPair ? 2 * kDqWarps : kDqWarps;
+  // arrivals that free the accumulators: the epilogue warps of the unit
+  static constexpr int kAccEmpty = kPair ? 8 : 4;
+  static constexpr int kRowsPerUnit = kPair ? 512 : 256;
+};
+constexpr int kNf4Threads = Nf4Cfg<false>::kThreads;         // 480
+constexpr int kNf4PairThreads = Nf4Cfg<true>::kThreads;      // 352
 
 struct Nf4Unit {
   int m0, n0;
 };
-__device__ __forceinline__ Nf4Unit nf4_unit(const Nf4GemmArgs& p, int u) {
+// Unit u of the raster: tiles_m counts units of `rows` rows of M.
+__device__ __forceinline__ Nf4Unit nf4_unit(const Nf4GemmArgs& p, int u, int rows) {
   const int per_group = p.group_m * p.tiles_n;
   const int gidx = u / per_group;
   const int first_m = gidx * p.group_m;
   const int gsize = min(p.group_m, p.tiles_m - first_m);
   const int in_group = u - gidx * per_group;
   Nf4Unit r;
-  r.m0 = (first_m + in_group % gsize) * 256;
+  r.m0 = (first_m + in_group % gsize) * rows;
   r.n0 = (in_group / gsize) * 256;
   return r;
 }
@@ -163,32 +191,55 @@ __device__ __forceinline__ void mbar_wait_drain(uint32_t bar, uint32_t parity) {
   }
 }
 
+// Waits (bounded, no abort flag) for the last `n` ring uses before `g` of a
+// stage ring of S barriers to complete: used before exit so that no MMA
+// completion is still on its way to this CTA's barriers.
+template <int S>
+__device__ __forceinline__ void wait_ring_tail(const uint64_t* bars, int g, int n) {
+  for (int q = 0; q < n && g - 1 - q >= 0; ++q) {
+    const int last = g - 1 - q;
+    mbar_wait_bounded<true>(smem_u32(&bars[last % S]), (uint32_t)((last / S) & 1), nullptr);
+  }
+}
+
+// Loads one activation (or rank-r operand) tile: into this CTA, completing on
+// `bar` (a local barrier for one CTA; rank 0's, as a cluster address, in a pair).
+template <bool kPair>
+__device__ __forceinline__ void nf4_tile_load(uint32_t dst, const CUtensorMap* map, uint32_t bar, int x, int y) {
+  if constexpr (kPair)
+    tma_load_2d_pair(dst, map, bar, x, y);
+  else
+    tma_load_2d(dst, map, bar, x, y);
+}
+
 // kDx = false: forward (W' rows are N, K-major tiles); true: dX (W' rows are
 // K, MN-major tiles).
-template <bool kDx>
-__global__ void __launch_bounds__(kNf4Threads, 1)
+template <bool kDx, bool kPair>
+__global__ void __launch_bounds__(Nf4Cfg<kPair>::kThreads, 1)
     gemm_nf4_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmC,
                     const __grid_constant__ CUtensorMap tmS, const __grid_constant__ CUtensorMap tmA1,
                     const __grid_constant__ CUtensorMap tmB1, const __grid_constant__ CUtensorMap tmOut,
                     const __grid_constant__ Nf4GemmArgs p) {
+  using Cfg = Nf4Cfg<kPair>;
+  constexpr int SA = Cfg::SA, SB = Cfg::SB, SC = Cfg::SC;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_u32(smem_raw);
   const uint32_t pad = (1024u - (raw_addr & 1023u)) & 1023u;
   uint8_t* smem = smem_raw + pad;
   const uint32_t sbase = raw_addr + pad;
   const uint32_t sA = sbase;
-  const uint32_t sB = sA + kNf4SA * kNf4ABytes;
-  const uint32_t sC = sB + kNf4SB * kNf4BBytes;
-  const uint32_t sStg = sC + kNf4SC * kNf4CBytes;
+  const uint32_t sB = sA + SA * Cfg::kABytes;
+  const uint32_t sC = sB + SB * Cfg::kBBytes;
+  const uint32_t sStg = sC + SC * Cfg::kCBytes;
   uint8_t* stg_ptr = smem + (sStg - sbase);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (sStg - sbase) + kNf4Stage);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + (sStg - sbase) + Cfg::kStage);
   uint64_t* a_full = bars;
-  uint64_t* a_empty = a_full + kNf4SA;
-  uint64_t* b_full = a_empty + kNf4SA;
-  uint64_t* b_empty = b_full + kNf4SB;
-  uint64_t* c_full = b_empty + kNf4SB;
-  uint64_t* c_empty = c_full + kNf4SC;
-  uint64_t* acc_full = c_empty + kNf4SC;
+  uint64_t* a_empty = a_full + SA;
+  uint64_t* b_full = a_empty + SA;
+  uint64_t* b_empty = b_full + SB;
+  uint64_t* c_full = b_empty + SB;
+  uint64_t* c_empty = c_full + SC;
+  uint64_t* acc_full = c_empty + SC;
   uint64_t* acc_empty = acc_full + 1;
   uint64_t* drain_bar = acc_empty + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_bar + 1);
@@ -196,33 +247,53 @@ __global__ void __launch_bounds__(kNf4Threads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const uint32_t rank = kPair ? cluster_ctarank() : 0u;
+  const bool leader = rank == 0;
+  // a barrier that completes the unit's operands: this CTA's, or rank 0's in a pair
+  auto lead_bar = [&](const uint64_t* b) -> uint32_t {
+    return kPair ? mapa_shared(smem_u32(b), 0) : smem_u32(b);
+  };
+  const int unit0 = kPair ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+  const int ustride = kPair ? (int)(gridDim.x >> 1) : (int)gridDim.x;
   const int units = p.tiles_m * p.tiles_n;
   const int steps0 = (p.K0 + 63) / 64;
   const int steps1 = (p.K1 + 63) / 64;
   const int steps = steps0 + steps1;
+  // Rows of a unit held by this CTA: A tile t (t = 0, 1) starts at row
+  // m0 + t * tile_step + row_off of the unit starting at m0.
+  const int tile_step = kPair ? 256 : 128;
+  const int row_off = kPair ? 128 * (int)rank : 0;
+  // The unit's second tile (second 256 rows of a pair unit) is used only if
+  // it holds rows below M; both CTAs of a pair decide alike.
+  auto has_second = [&](int m0) -> bool { return m0 + tile_step < p.M; };
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kNf4SA; ++i) {
+    for (int i = 0; i < SA; ++i) {
       mbar_init(smem_u32(&a_full[i]), 1);
       mbar_init(smem_u32(&a_empty[i]), 1);
     }
-    for (int i = 0; i < kNf4SB; ++i) {
-      mbar_init(smem_u32(&b_full[i]), kNf4DqWarps);
+    for (int i = 0; i < SB; ++i) {
+      mbar_init(smem_u32(&b_full[i]), Cfg::kBFull);
       mbar_init(smem_u32(&b_empty[i]), 1);
     }
-    for (int i = 0; i < kNf4SC; ++i) {
+    for (int i = 0; i < SC; ++i) {
       mbar_init(smem_u32(&c_full[i]), 1);
-      mbar_init(smem_u32(&c_empty[i]), kNf4DqWarps);
+      mbar_init(smem_u32(&c_empty[i]), Cfg::kDqWarps);
     }
     mbar_init(smem_u32(acc_full), 1);
-    mbar_init(smem_u32(acc_empty), 4);
+    mbar_init(smem_u32(acc_empty), Cfg::kAccEmpty);
     mbar_init(smem_u32(drain_bar), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_slot), 512);
-    tmem_relinquish();
+    if constexpr (kPair) {
+      tmem_alloc_pair(smem_u32(tmem_slot), 512);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(smem_u32(tmem_slot), 512);
+      tmem_relinquish();
+    }
   }
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmA0);
@@ -237,171 +308,224 @@ __global__ void __launch_bounds__(kNf4Threads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // the peer's barriers are initialised before anyone signals them
+  if (kPair) cluster_sync();
   const uint32_t tmem_base = *tmem_slot;
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
+    // (activation tiles, and the rank-r weight tiles of the extension steps)
     if (lane == 0) {
-      int a_iss[kNf4SA], c_iss[kNf4SC];
-      int b_last[kNf4SB];              // ring use index of this warp's last weight-tile load per stage
-      for (int i = 0; i < kNf4SA; ++i) a_iss[i] = 0;
-      for (int i = 0; i < kNf4SC; ++i) c_iss[i] = 0;
-      for (int i = 0; i < kNf4SB; ++i) b_last[i] = -1;
-      int g = 0, gc = 0;
+      int a_iss[SA];
+      int b_last[SB];                  // ring use index of this warp's last weight-tile load per stage
+      for (int i = 0; i < SA; ++i) a_iss[i] = 0;
+      for (int i = 0; i < SB; ++i) b_last[i] = -1;
+      int g = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
-        const Nf4Unit c = nf4_unit(p, u);
-        const bool has2 = c.m0 + 128 < p.M;
+      for (int u = unit0; u < units && ok; u += ustride) {
+        const Nf4Unit c = nf4_unit(p, u, Cfg::kRowsPerUnit);
+        const bool has2 = has_second(c.m0);
+        const int mA = c.m0 + row_off;
         for (int step = 0; step < steps; ++step, ++g) {
-          const int sa = g % kNf4SA;
-          if (!mbar_wait_bounded(smem_u32(&a_empty[sa]), (uint32_t)(((g / kNf4SA) & 1) ^ 1), abort_flag)) {
+          const int sa = g % SA;
+          if (!mbar_wait_bounded<kPair>(smem_u32(&a_empty[sa]), (uint32_t)(((g / SA) & 1) ^ 1), abort_flag)) {
             ok = false;
             break;
           }
           const bool ext = step >= steps0;
           const int e = step - steps0;
-          const uint32_t fa = smem_u32(&a_full[sa]);
-          mbar_arrive_expect_tx(fa, has2 ? 2u * 16384u : 16384u);
+          const uint32_t fa = lead_bar(&a_full[sa]);
+          // rank 0 expects the tiles of both CTAs of a pair
+          if (leader)
+            mbar_arrive_expect_tx(smem_u32(&a_full[sa]), (uint32_t)((has2 ? 2 : 1) * 16384 * (kPair ? 2 : 1)));
           const CUtensorMap* ma = ext ? &tmA1 : &tmA0;
           const int x = ext ? e * 64 : step * 64;
-          tma_load_2d(sA + sa * kNf4ABytes, ma, fa, x, c.m0);
-          if (has2) tma_load_2d(sA + sa * kNf4ABytes + 16384, ma, fa, x, c.m0 + 128);
+          nf4_tile_load<kPair>(sA + sa * Cfg::kABytes, ma, fa, x, mA);
+          if (has2) nf4_tile_load<kPair>(sA + sa * Cfg::kABytes + 16384, ma, fa, x, mA + tile_step);
           a_iss[sa] += 1;
-          if (!ext) {
-            const int sc = gc % kNf4SC;
-            if (!mbar_wait_bounded(smem_u32(&c_empty[sc]), (uint32_t)(((gc / kNf4SC) & 1) ^ 1), abort_flag)) {
+          if (ext) {
+            // rank-r weight operand: B rows (forward) or A columns (dX) by
+            // TMA, this CTA's half of the tile in a pair
+            const int sb = g % SB;
+            if (!mbar_wait_bounded<kPair>(smem_u32(&b_empty[sb]), (uint32_t)(((g / SB) & 1) ^ 1), abort_flag)) {
               ok = false;
               break;
             }
-            const uint32_t fc = smem_u32(&c_full[sc]);
-            mbar_arrive_expect_tx(fc, (uint32_t)(kNf4CodeBytes + 1024));
+            const uint32_t fb = lead_bar(&b_full[sb]);
+            if (leader) {
+              mbar_arrive_expect_tx(smem_u32(&b_full[sb]), (uint32_t)(kPair ? 2 * Cfg::kBBytes : Cfg::kBBytes));
+              mbar_arrive_count(smem_u32(&b_full[sb]), Cfg::kBFull - 1);
+            }
+            const int nb = kPair ? 128 : 256;              // rows (forward) or MN columns (dX) loaded here
+            const int n1 = c.n0 + (kPair ? 128 * (int)rank : 0);
             if (kDx) {
-              tma_load_2d(sC + sc * kNf4CBytes, &tmC, fc, c.n0 / 2, step * 64);
-              // scales of the tile's 64 K-rows x 4 block columns
-              tma_load_2d(sC + sc * kNf4CBytes + kNf4CodeBytes, &tmS, fc, c.n0 / 64, step * 64);
+              for (int i = 0; i < nb / 64; ++i)
+                nf4_tile_load<kPair>(sB + sb * Cfg::kBBytes + i * 8192, &tmB1, fb, n1 + 64 * i, e * 64);
             } else {
-              tma_load_2d(sC + sc * kNf4CBytes, &tmC, fc, step * 32, c.n0);
-              // scales of the tile's 256 rows at block column `step`
-              tma_load_2d(sC + sc * kNf4CBytes + kNf4CodeBytes, &tmS, fc, c.n0, step);
+              nf4_tile_load<kPair>(sB + sb * Cfg::kBBytes, &tmB1, fb, e * 64, n1);
             }
-            c_iss[sc] += 1;
-            ++gc;
-          } else {
-            // rank-r weight operand: B rows (forward) or A columns (dX) by TMA
-            const int sb = g % kNf4SB;
-            if (!mbar_wait_bounded(smem_u32(&b_empty[sb]), (uint32_t)(((g / kNf4SB) & 1) ^ 1), abort_flag)) {
-              ok = false;
-              break;
-            }
-            const uint32_t fb = smem_u32(&b_full[sb]);
-            mbar_arrive_expect_tx(fb, (uint32_t)kNf4BBytes);
-            mbar_arrive_count(fb, kNf4DqWarps - 1);
-            if (kDx) {
-#pragma unroll
-              for (int i = 0; i < 4; ++i)
-                tma_load_2d(sB + sb * kNf4BBytes + i * 8192, &tmB1, fb, c.n0 + 64 * i, e * 64);
-            } else {
-              tma_load_2d(sB + sb * kNf4BBytes, &tmB1, fb, e * 64, c.n0);
-            }
-            b_last[sb] = g / kNf4SB;
+            b_last[sb] = g / SB;
           }
         }
       }
       if (*abort_flag) {
-        // let copies already in flight land before the CTA exits
-        for (int i = 0; i < kNf4SA; ++i)
-          if (a_iss[i] > 0) mbar_wait_drain(smem_u32(&a_full[i]), (uint32_t)((a_iss[i] - 1) & 1));
-        for (int i = 0; i < kNf4SC; ++i)
+        // let copies already in flight land before the CTA exits (a pair's
+        // operand loads complete on rank 0's barriers: rank 0 drains them)
+        if (leader) {
+          for (int i = 0; i < SA; ++i)
+            if (a_iss[i] > 0) mbar_wait_drain(smem_u32(&a_full[i]), (uint32_t)((a_iss[i] - 1) & 1));
+          for (int i = 0; i < SB; ++i)
+            if (b_last[i] >= 0) mbar_wait_drain(smem_u32(&b_full[i]), (uint32_t)(b_last[i] & 1));
+        }
+      } else if (kPair) {
+        // the last stage releases (rank 0's MMA completions) have reached this CTA
+        wait_ring_tail<SA>(a_empty, g, SA);
+      }
+    }
+  } else if (warp == 6) {
+    // ------------------------------------------------------------ code loads
+    // Codes and block scales of this CTA's rows of each main K-step's weight
+    // tile; they run ahead of the MMA by as many stages as the decode allows.
+    if (lane == 0) {
+      int c_iss[SC];
+      for (int i = 0; i < SC; ++i) c_iss[i] = 0;
+      int gc = 0;
+      bool ok = true;
+      for (int u = unit0; u < units && ok; u += ustride) {
+        const Nf4Unit c = nf4_unit(p, u, Cfg::kRowsPerUnit);
+        for (int step = 0; step < steps0; ++step, ++gc) {
+          const int sc = gc % SC;
+          if (!mbar_wait_bounded(smem_u32(&c_empty[sc]), (uint32_t)(((gc / SC) & 1) ^ 1), abort_flag)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fc = smem_u32(&c_full[sc]);
+          const uint32_t cdst = sC + sc * Cfg::kCBytes;
+          if (kDx) {
+            mbar_arrive_expect_tx(fc, (uint32_t)(Cfg::kCodeBytes + 1024));
+            // codes of 64 K-rows x this CTA's MN columns; scales of the
+            // tile's 4 block columns
+            tma_load_2d(cdst, &tmC, fc, c.n0 / 2 + (kPair ? 64 * (int)rank : 0), step * 64);
+            tma_load_2d(cdst + Cfg::kCodeBytes, &tmS, fc, c.n0 / 64, step * 64);
+          } else {
+            const int rows = kPair ? 128 : 256;
+            mbar_arrive_expect_tx(fc, (uint32_t)(Cfg::kCodeBytes + rows * 4));
+            // codes and scales of this CTA's rows at block column `step`
+            tma_load_2d(cdst, &tmC, fc, step * 32, c.n0 + (kPair ? 128 * (int)rank : 0));
+            tma_load_2d(cdst + Cfg::kCodeBytes, &tmS, fc, c.n0 + (kPair ? 128 * (int)rank : 0), step);
+          }
+          c_iss[sc] += 1;
+        }
+      }
+      if (*abort_flag) {
+        for (int i = 0; i < SC; ++i)
           if (c_iss[i] > 0) mbar_wait_drain(smem_u32(&c_full[i]), (uint32_t)((c_iss[i] - 1) & 1));
-        for (int i = 0; i < kNf4SB; ++i)
-          if (b_last[i] >= 0) mbar_wait_drain(smem_u32(&b_full[i]), (uint32_t)(b_last[i] & 1));
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    if (lane == 0 && leader) {
       const uint64_t adesc = smem_desc_sw128(sA, 16, 1024);
       const uint64_t bdesc = kDx ? smem_desc_sw128(sB, 8192, 1024) : smem_desc_sw128(sB, 16, 1024);
       const uint32_t bstep = kDx ? 128u : 2u;
-      const uint32_t idesc = idesc_bf16_f32(128, 256, 0, kDx ? 1 : 0);
+      const uint32_t idesc = idesc_bf16_f32(kPair ? 256 : 128, 256, 0, kDx ? 1 : 0);
       bool ok = true;
       int issued_any = 0;
       int g = 0, it = 0;
-      for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++it) {
-        const Nf4Unit c = nf4_unit(p, u);
-        const bool has2 = c.m0 + 128 < p.M;
-        if (!mbar_wait_bounded(smem_u32(acc_empty), (uint32_t)((it & 1) ^ 1), abort_flag)) {
+      for (int u = unit0; u < units && ok; u += ustride, ++it) {
+        const Nf4Unit c = nf4_unit(p, u, Cfg::kRowsPerUnit);
+        const bool has2 = has_second(c.m0);
+        if (!mbar_wait_bounded<kPair>(smem_u32(acc_empty), (uint32_t)((it & 1) ^ 1), abort_flag)) {
           ok = false;
           break;
         }
         tc_fence_after();
         for (int step = 0; step < steps; ++step, ++g) {
-          const int sa = g % kNf4SA;
-          const int sb = g % kNf4SB;
-          if (!mbar_wait_bounded(smem_u32(&a_full[sa]), (uint32_t)((g / kNf4SA) & 1), abort_flag) ||
-              !mbar_wait_bounded(smem_u32(&b_full[sb]), (uint32_t)((g / kNf4SB) & 1), abort_flag)) {
+          const int sa = g % SA;
+          const int sb = g % SB;
+          if (!mbar_wait_bounded<kPair>(smem_u32(&a_full[sa]), (uint32_t)((g / SA) & 1), abort_flag) ||
+              !mbar_wait_bounded<kPair>(smem_u32(&b_full[sb]), (uint32_t)((g / SB) & 1), abort_flag)) {
             ok = false;
             break;
           }
           tc_fence_after();
           const bool ext = step >= steps0;
           const int nsub = ext ? min(4, (p.K1 - (step - steps0) * 64 + 15) / 16) : 4;
-          const uint64_t a0 = adesc + (uint64_t)((sa * kNf4ABytes) >> 4);
-          const uint64_t b0 = bdesc + (uint64_t)((sb * kNf4BBytes) >> 4);
+          const uint64_t a0 = adesc + (uint64_t)((sa * Cfg::kABytes) >> 4);
+          const uint64_t b0 = bdesc + (uint64_t)((sb * Cfg::kBBytes) >> 4);
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             if (j < nsub) {
               const uint32_t acc = (step == 0 && j == 0) ? 0u : 1u;
-              umma_bf16(tmem_base, a0 + (uint64_t)(2 * j), b0 + (uint64_t)(j * bstep), idesc, acc);
-              if (has2)
-                umma_bf16(tmem_base + 256u, a0 + (uint64_t)(1024 + 2 * j), b0 + (uint64_t)(j * bstep), idesc,
-                          acc);
+              const uint64_t aj = a0 + (uint64_t)(2 * j), bj = b0 + (uint64_t)(j * bstep);
+              if constexpr (kPair) {
+                umma_bf16_pair(tmem_base, aj, bj, idesc, acc);
+                if (has2) umma_bf16_pair(tmem_base + 256u, aj + 1024u, bj, idesc, acc);
+              } else {
+                umma_bf16(tmem_base, aj, bj, idesc, acc);
+                if (has2) umma_bf16(tmem_base + 256u, aj + 1024u, bj, idesc, acc);
+              }
             }
           }
           issued_any = 1;
-          umma_commit(smem_u32(&a_empty[sa]));
-          umma_commit(smem_u32(&b_empty[sb]));
+          if constexpr (kPair) {
+            // both CTAs' stages are free once the pair MMA has read them
+            umma_commit_pair(smem_u32(&a_empty[sa]), (uint16_t)0x3);
+            umma_commit_pair(smem_u32(&b_empty[sb]), (uint16_t)0x3);
+          } else {
+            umma_commit(smem_u32(&a_empty[sa]));
+            umma_commit(smem_u32(&b_empty[sb]));
+          }
         }
-        if (ok) umma_commit(smem_u32(acc_full));
+        if (ok) {
+          if constexpr (kPair)
+            umma_commit_pair(smem_u32(acc_full), (uint16_t)0x3);
+          else
+            umma_commit(smem_u32(acc_full));
+        }
       }
       if (!ok && issued_any) {
-        umma_commit(smem_u32(drain_bar));
+        if constexpr (kPair)
+          umma_commit_pair(smem_u32(drain_bar), (uint16_t)0x1);
+        else
+          umma_commit(smem_u32(drain_bar));
         mbar_wait_bounded(smem_u32(drain_bar), 0, nullptr);
       }
     }
   } else if (warp < 6) {
     // ------------------------------------------------------------ epilogue
     const int quarter = warp & 3;
-    uint8_t* stg = stg_ptr + (warp - 2) * (kNf4StgBoxes * 4096);
-    const uint32_t stg_s = sStg + (uint32_t)((warp - 2) * (kNf4StgBoxes * 4096));
+    uint8_t* stg = stg_ptr + (warp - 2) * (Cfg::kStgBoxes * 4096);
+    const uint32_t stg_s = sStg + (uint32_t)((warp - 2) * (Cfg::kStgBoxes * 4096));
     int it = 0, nbox = 0;
-    for (int u = blockIdx.x; u < units; u += gridDim.x, ++it) {
-      const Nf4Unit c = nf4_unit(p, u);
-      const bool has2 = c.m0 + 128 < p.M;
-      const bool ok = mbar_wait_bounded(smem_u32(acc_full), (uint32_t)(it & 1), abort_flag);
+    for (int u = unit0; u < units; u += ustride, ++it) {
+      const Nf4Unit c = nf4_unit(p, u, Cfg::kRowsPerUnit);
+      const bool has2 = has_second(c.m0);
+      const bool ok = mbar_wait_bounded<kPair>(smem_u32(acc_full), (uint32_t)(it & 1), abort_flag);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
       for (int t = 0; t < (has2 ? 2 : 1); ++t) {
-        const int mrow0 = c.m0 + t * 128 + quarter * 32;
+        const int mrow0 = c.m0 + t * tile_step + row_off + quarter * 32;
         const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(t * 256);
         if (p.tma_store) {
 #pragma unroll 1
-          for (int b = 0; b < 4; ++b, ++nbox) {
+          for (int b = 0; b < 4; ++b) {
             uint32_t v0[32], v1[32];
             tmem_ld_32x32b_x32(taddr + (uint32_t)(b * 64), v0);
             tmem_ld_32x32b_x32(taddr + (uint32_t)(b * 64 + 32), v1);
             tmem_ld_wait();
-            if (nbox >= kNf4StgBoxes) {
+            if (mrow0 >= p.M) continue;          // rows of this warp lie beyond M
+            if (nbox >= Cfg::kStgBoxes) {
               // the store that used this buffer has read it
               if (lane == 0) {
-                if (kNf4StgBoxes == 2)
+                if (Cfg::kStgBoxes == 2)
                   bulk_wait_group_read1();
                 else
                   bulk_wait_group_read0();
               }
               __syncwarp();
             }
-            const int slot = nbox % kNf4StgBoxes;
+            const int slot = nbox % Cfg::kStgBoxes;
             uint8_t* box = stg + slot * 4096;
 #pragma unroll
             for (int q = 0; q < 8; ++q) {
@@ -420,6 +544,7 @@ __global__ void __launch_bounds__(kNf4Threads, 1)
               tma_store_2d(&tmOut, stg_s + (uint32_t)(slot * 4096), c.n0 + 64 * b, mrow0);
               bulk_commit_group();
             }
+            ++nbox;
           }
         } else {
           const int m = mrow0 + lane;
@@ -439,40 +564,57 @@ __global__ void __launch_bounds__(kNf4Threads, 1)
           }
         }
       }
-      // the accumulators may be overwritten once all four warps are done
+      // the accumulators may be overwritten once all epilogue warps of the
+      // unit (both CTAs of a pair) are done
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(acc_empty));
+      if (lane == 0) {
+        if (kPair && rank != 0)
+          mbar_arrive_remote(lead_bar(acc_empty));
+        else
+          mbar_arrive(smem_u32(acc_empty));
+      }
     }
     if (p.tma_store && lane == 0) bulk_wait_group0();
   } else {
     // ------------------------------------------------------------ dequantisation
     // Thread i of these warps owns one 64-weight block of each K-step's
-    // weight tile.  Forward: tile row i (W' row n0 + i, block column = the
-    // K-step).  dX: K-row kk = i % 64 (W' row 64 * step + kk) and MN chunk
-    // c = i / 64 (W' block column n0 / 64 + c).
-    const int i = threadIdx.x - 192;
-    const int kk = i & 63, cc = i >> 6;
+    // weight tile.  Forward: local tile row i (W' row n0 + i; in a pair, rank
+    // 1 holds rows n0 + 128 + i), block column = the K-step.  dX: K-row
+    // kk = i % 64 (W' row 64 * step + kk) and local chunk cl = i / 64 (W'
+    // block column n0 / 64 + cc, cc = cl, or 2 rank + cl in a pair).
+    const int i = threadIdx.x - Cfg::kDqWarp0 * 32;
+    const int kk = i & 63;
+    const int cl = i >> 6;
+    const int cc = kPair ? 2 * (int)rank + cl : cl;
     int g = 0, gc = 0;
-    for (int u = blockIdx.x; u < units; u += gridDim.x) {
-      bool live = true;
+    bool live = true;
+    for (int u = unit0; u < units && live; u += ustride) {
       for (int step = 0; step < steps0; ++step, ++g, ++gc) {
-        const int sc = gc % kNf4SC;
-        bool ok = mbar_wait_bounded(smem_u32(&c_full[sc]), (uint32_t)((gc / kNf4SC) & 1), abort_flag);
+        const int sc = gc % SC;
+        bool ok = mbar_wait_bounded(smem_u32(&c_full[sc]), (uint32_t)((gc / SC) & 1), abort_flag);
         if (!__all_sync(0xffffffffu, ok)) {
           live = false;
           break;
         }
         uint4 c0, c1;
-        const uint32_t cs = sC + sc * kNf4CBytes;
-        const float* scl = reinterpret_cast<const float*>(smem + (cs - sbase) + kNf4CodeBytes);
+        const uint32_t cs = sC + sc * Cfg::kCBytes;
+        const float* scl = reinterpret_cast<const float*>(smem + (cs - sbase) + Cfg::kCodeBytes);
         float a;
         if (kDx) {
-          // 128-byte rows (K-rows), 128B swizzle: 16-byte chunk j at (j ^ (row & 7))
-          const uint32_t row = cs + kk * 128;
-          const int sw = kk & 7;
-          c0 = ld_shared_v4(row + (((2 * cc) ^ sw) << 4));
-          c1 = ld_shared_v4(row + (((2 * cc + 1) ^ sw) << 4));
+          if (kPair) {
+            // 64-byte rows (this CTA's 128 MN columns), 64B swizzle: chunk j at (j ^ ((row >> 1) & 3))
+            const uint32_t row = cs + kk * 64;
+            const int sw = (kk >> 1) & 3;
+            c0 = ld_shared_v4(row + (((2 * cl) ^ sw) << 4));
+            c1 = ld_shared_v4(row + (((2 * cl + 1) ^ sw) << 4));
+          } else {
+            // 128-byte rows (K-rows), 128B swizzle: 16-byte chunk j at (j ^ (row & 7))
+            const uint32_t row = cs + kk * 128;
+            const int sw = kk & 7;
+            c0 = ld_shared_v4(row + (((2 * cc) ^ sw) << 4));
+            c1 = ld_shared_v4(row + (((2 * cc + 1) ^ sw) << 4));
+          }
           a = scl[kk * 4 + cc];
         } else {
           // 32-byte rows, 32B swizzle: chunk j at (j ^ ((row >> 2) & 1))
@@ -487,8 +629,8 @@ __global__ void __launch_bounds__(kNf4Threads, 1)
         // the codes and scales are consumed (the decode read them): release the stage
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&c_empty[sc]));
-        const int sb = g % kNf4SB;
-        ok = mbar_wait_bounded(smem_u32(&b_empty[sb]), (uint32_t)(((g / kNf4SB) & 1) ^ 1), abort_flag);
+        const int sb = g % SB;
+        ok = mbar_wait_bounded<kPair>(smem_u32(&b_empty[sb]), (uint32_t)(((g / SB) & 1) ^ 1), abort_flag);
         if (!__all_sync(0xffffffffu, ok)) {
           live = false;
           break;
@@ -496,25 +638,38 @@ __global__ void __launch_bounds__(kNf4Threads, 1)
         uint32_t dst;
         int sw;
         if (kDx) {
-          dst = sB + sb * kNf4BBytes + cc * 8192 + kk * 128;
+          dst = sB + sb * Cfg::kBBytes + cl * 8192 + kk * 128;
           sw = kk & 7;
         } else {
-          dst = sB + sb * kNf4BBytes + i * 128;
+          dst = sB + sb * Cfg::kBBytes + i * 128;
           sw = i & 7;
         }
 #pragma unroll
         for (int j = 0; j < 8; ++j) st_shared_v4(dst + ((j ^ sw) << 4), o[j]);
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&b_full[sb]));
+        if (lane == 0) {
+          if (kPair && rank != 0)
+            mbar_arrive_remote(lead_bar(&b_full[sb]));
+          else
+            mbar_arrive(smem_u32(&b_full[sb]));
+        }
       }
       if (!live) break;
       g += steps1;     // the rank-r weight tiles arrive by TMA
     }
+    // the last stage releases (rank 0's MMA completions) have reached this CTA
+    if (kPair && live) wait_ring_tail<SB>(b_empty, g, SB);
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) tmem_dealloc(tmem_base, 512);
+  if (kPair) cluster_sync();
+  if (warp == 1) {
+    if constexpr (kPair)
+      tmem_dealloc_pair(tmem_base, 512);
+    else
+      tmem_dealloc(tmem_base, 512);
+  }
 }
 
 // ===========================================================================

@@ -133,6 +133,9 @@ def test_argument_validation_without_device(lib):
                              16, 1 << 20, None) == 1                                           # alpha <= 0
     assert L.qlora_bwd_multi(ctypes.byref(nf), 2, 16, 16, 8, ctypes.addressof(al), 18, 16, 16, 16, 16, 16,
                              16, 16, 16, 1 << 20, None) == 3                                   # misaligned idx
+    # the NF4 GEMM build selector takes 0, 1 or 2
+    assert L.qlora_set_nf4_gemm_mode(3) == 1 and L.qlora_set_nf4_gemm_mode(-1) == 1
+    assert L.qlora_set_nf4_gemm_mode(2) == 0 and L.qlora_set_nf4_gemm_mode(0) == 0
     # Adam: step, betas, lr and alignment are checked on the host; n = 0 is a no-op
     assert L.lora_adam_step(16, 16, 16, 16, 16, 8, 0, 1e-3, 0.9, 0.999, 1e-8, 0.0, None) == 1     # step 0
     assert L.lora_adam_step(16, 16, 16, 16, 16, 8, 1, 1e-3, 1.0, 0.999, 1e-8, 0.0, None) == 1     # beta1 = 1

@@ -18,6 +18,16 @@ pytestmark = pytest.mark.gpu
 q4 = pytest.importorskip("parameter_efficient_fine_nf4_b200")
 
 
+# Both builds of the NF4 GEMM: one CTA per 256 x 256 tile (mode 1), and CTA
+# pairs that share the decode of each weight tile over 512-token units
+# (mode 2).  Both must give the plain-LoRA GEMM's bits.
+@pytest.fixture(params=[1, 2], ids=["one_cta", "cta_pair"])
+def gemm_mode(request):
+    q4.qlora_set_nf4_gemm_mode(request.param)
+    yield request.param
+    q4.qlora_set_nf4_gemm_mode(0)
+
+
 def _same_bits(lay, alpha):
     qw = q4.qlora_nf4_quantize(f32_dev(lay.W0))
     Wp = q4.qlora_nf4_dequantize(qw)
@@ -35,7 +45,9 @@ def _same_bits(lay, alpha):
 
 
 # (T > 64: the 256 x 256-tile kernel; fewer tokens take the split-depth
-# kernel, whose fp32 sums run in another order: see test_gpu_small_tokens.py)
+# kernel, whose fp32 sums run in another order: see test_gpu_small_tokens.py.
+# In a pair, the second CTA's 256 rows start at token 256 of the unit: the
+# shapes below leave it empty, one row, partial and full.)
 @pytest.mark.parametrize("d,k,r,T", [
     (256, 256, 8, 100),       # one tile, T < 128: the second M tile is absent
     (512, 384, 16, 300),      # two N tiles in the forward, ragged N tile (k = 384) in dX
@@ -45,19 +57,21 @@ def _same_bits(lay, alpha):
     (384, 256, 256, 72),      # maximum rank (four rank-r steps)
     (1024, 1024, 64, 1000),   # several units per CTA
     (200, 64, 16, 65),        # K = 64: one main step
+    (520, 320, 16, 513),      # one token past a 512-token unit
+    (256, 640, 32, 1536),     # three full 512-token units, ragged dX tile (k = 640)
 ])
-def test_fused_dequant_bit_identical(d, k, r, T):
+def test_fused_dequant_bit_identical(d, k, r, T, gemm_mode):
     lay = synthetic.custom_layer(seed=d * 31 + k * 3 + r + T, d=d, k=k, r=r, T=T, alpha=2.0 * r)
     _same_bits(lay, 2.0 * r)
 
 
 @pytest.mark.parametrize("ci", [2, 3])
-def test_fused_dequant_bit_identical_configs(ci):
+def test_fused_dequant_bit_identical_configs(ci, gemm_mode):
     cfg = synthetic.config(ci)
     _same_bits(synthetic.make_layer(cfg, T=512 if ci == 3 else None), cfg.alpha)
 
 
-def test_fused_dequant_large_shape_sampled():
+def test_fused_dequant_large_shape(gemm_mode):
     # the 8192 -> 22016 projection at 2048 tokens: long K loops, many units
     cfg = synthetic.config(4)
     lay = synthetic.make_layer(cfg, 0, T=2048)
