@@ -600,7 +600,8 @@ SmallPlan small_plan(int64_t Mw, int64_t K0, int64_t T) {
   sp.tn = T <= 16 ? 16 : (T <= 32 ? 32 : 64);
   sp.tiles_m = (int)cdiv(Mw, 128);
   const int steps0 = (int)cdiv(K0, 64);
-  const int want = (int)cdiv(3 * kSMs, sp.tiles_m);
+  // two CTAs of the few-token kernel fit on an SM; one wave of them
+  const int want = std::max(1, (int)(2 * kSMs / sp.tiles_m));
   const int splits = std::max(1, std::min(std::min(want, steps0 / 8), kSmMaxSplits));
   sp.sps = (int)cdiv(steps0, splits);
   sp.splits = (int)cdiv(steps0, sp.sps);
@@ -867,7 +868,6 @@ struct SmallJob {
   int src = SRC_NF4_ROWS, out = OUT_BF16;
   const char* name = "";
   const qlora_nf4_t* q = nullptr;                         // NF4 sources
-  const float* scales = nullptr;                          // their block scales (nf4_block_scales)
   const void* w = nullptr;                                // bf16 sources: the tensor tiles are cut from
   int64_t w_inner = 0, w_outer = 0, w_ld = 0;
   const uint16_t* act = nullptr;                          // T x K0 activations (row stride K0)
@@ -887,16 +887,16 @@ struct SmallJob {
 
 template <int kSrc, int kOut>
 void small_dispatch(int tn, dim3 grid, cudaStream_t st, const CUtensorMap& a, const CUtensorMap& w,
-                    const CUtensorMap& sc, const CUtensorMap& w1, const CUtensorMap& a1, const Nf4SmallArgs& p) {
+                    const CUtensorMap& w1, const CUtensorMap& a1, const Nf4SmallArgs& p) {
   switch (tn) {
     case 16:
-      gemm_nf4_small_kernel<kSrc, kOut, 16><<<grid, kSmThreads, SmallCfg<16>::kSmem, st>>>(a, w, sc, w1, a1, p);
+      gemm_nf4_small_kernel<kSrc, kOut, 16><<<grid, kSmThreads, SmallCfg<16>::kSmem, st>>>(a, w, w1, a1, p);
       break;
     case 32:
-      gemm_nf4_small_kernel<kSrc, kOut, 32><<<grid, kSmThreads, SmallCfg<32>::kSmem, st>>>(a, w, sc, w1, a1, p);
+      gemm_nf4_small_kernel<kSrc, kOut, 32><<<grid, kSmThreads, SmallCfg<32>::kSmem, st>>>(a, w, w1, a1, p);
       break;
     default:
-      gemm_nf4_small_kernel<kSrc, kOut, 64><<<grid, kSmThreads, SmallCfg<64>::kSmem, st>>>(a, w, sc, w1, a1, p);
+      gemm_nf4_small_kernel<kSrc, kOut, 64><<<grid, kSmThreads, SmallCfg<64>::kSmem, st>>>(a, w, w1, a1, p);
       break;
   }
 }
@@ -924,19 +924,20 @@ int launch_small(const SmallJob& j, int64_t T, cudaStream_t st) {
   a.scale = j.scale;
   a.f32_scale = j.f32_scale;
   memcpy(a.levels, tables().levels, sizeof(a.levels));
-  CUtensorMap mAct, mW, mS, mW1, mAct1;
+  CUtensorMap mAct, mW, mW1, mAct1;
   if (!make_map(&mAct, j.act, j.K0, T, j.K0, sp.tn)) return QLORA_ERR_CUDA;
-  mS = mAct;
   double bytes = 0.0;
   if (j.src == SRC_NF4_ROWS || j.src == SRC_NF4_COLS) {
     const int64_t d = j.q->d, k = j.q->k;
     bytes = (double)nf4_storage_bytes(d, k);
+    a.absmax_q = j.q->absmax_q;
+    a.scale2 = j.q->scale2;
+    a.mean = j.q->mean;
+    a.kb = (int)(k / 64);
     if (j.src == SRC_NF4_COLS) {
       if (!make_map_u8(&mW, j.q->codes, k / 2, d, k / 2, 64, 64, CU_TENSOR_MAP_SWIZZLE_64B)) return QLORA_ERR_CUDA;
-      if (!make_map_f32(&mS, j.scales, k / 64, d, scales_ld_dx(k), 4, 64)) return QLORA_ERR_CUDA;
     } else {
       if (!make_map_u8(&mW, j.q->codes, k / 2, d, k / 2, 32, 128, CU_TENSOR_MAP_SWIZZLE_32B)) return QLORA_ERR_CUDA;
-      if (!make_map_f32(&mS, j.scales, d, k / 64, scales_ld_fwd(d), 128, 1)) return QLORA_ERR_CUDA;
     }
     if (j.r == 0) {
       mW1 = mW;
@@ -959,14 +960,14 @@ int launch_small(const SmallJob& j, int64_t T, cudaStream_t st) {
   const double flops = 2.0 * (double)T * j.Mw * ((double)j.K0 + j.r);
   return launch(j.name, flops, bytes, st, [&] {
     switch (j.src) {
-      case SRC_NF4_ROWS: small_dispatch<SRC_NF4_ROWS, OUT_BF16>(sp.tn, grid, st, mAct, mW, mS, mW1, mAct1, a); break;
-      case SRC_NF4_COLS: small_dispatch<SRC_NF4_COLS, OUT_BF16>(sp.tn, grid, st, mAct, mW, mS, mW1, mAct1, a); break;
-      case SRC_TMA_K: small_dispatch<SRC_TMA_K, OUT_U>(sp.tn, grid, st, mAct, mW, mS, mW1, mAct1, a); break;
+      case SRC_NF4_ROWS: small_dispatch<SRC_NF4_ROWS, OUT_BF16>(sp.tn, grid, st, mAct, mW, mW1, mAct1, a); break;
+      case SRC_NF4_COLS: small_dispatch<SRC_NF4_COLS, OUT_BF16>(sp.tn, grid, st, mAct, mW, mW1, mAct1, a); break;
+      case SRC_TMA_K: small_dispatch<SRC_TMA_K, OUT_U>(sp.tn, grid, st, mAct, mW, mW1, mAct1, a); break;
       default:
         if (j.out == OUT_U)
-          small_dispatch<SRC_TMA_MN, OUT_U>(sp.tn, grid, st, mAct, mW, mS, mW1, mAct1, a);
+          small_dispatch<SRC_TMA_MN, OUT_U>(sp.tn, grid, st, mAct, mW, mW1, mAct1, a);
         else
-          small_dispatch<SRC_TMA_MN, OUT_HILO>(sp.tn, grid, st, mAct, mW, mS, mW1, mAct1, a);
+          small_dispatch<SRC_TMA_MN, OUT_HILO>(sp.tn, grid, st, mAct, mW, mW1, mAct1, a);
         break;
     }
   });
@@ -1022,11 +1023,13 @@ int fwd_core(const qlora_nf4_t* q, const uint16_t* W, int64_t d, int64_t k, cons
   const uint16_t* Bp = padded_B(B, d, r, r8, w.Bp, st, &pst);
   QLORA_TRY(pst);
 
-  if (q) {
-    // block scales for the dequantising GEMM (and the few-token tickets)
-    QLORA_TRY(block_scales(q, true, w.scales, T <= kSmallT ? w.tickets : nullptr, w.n_tickets, st));
-  } else if (T <= kSmallT) {
+  if (T <= kSmallT) {
+    // the few-token kernels read the block constants themselves; their
+    // completion tickets start at zero
     QLORA_TRY(zero_tickets(w.tickets, w.n_tickets, st));
+  } else if (q) {
+    // block scales for the dequantising GEMM
+    QLORA_TRY(block_scales(q, true, w.scales, nullptr, 0, st));
   }
   // U = X A^T (fp32 to U_save), sU = bf16(s U) (operand of the extension)
   if (T <= kSmallT) {
@@ -1059,7 +1062,7 @@ int fwd_core(const qlora_nf4_t* q, const uint16_t* W, int64_t d, int64_t k, cons
   if (q && T <= kSmallT) {
     SmallJob j;
     j.src = SRC_NF4_ROWS; j.out = OUT_BF16; j.name = "gemm_nf4_small_fwd";
-    j.q = q; j.scales = w.scales; j.act = X; j.K0 = k; j.Mw = d;
+    j.q = q; j.act = X; j.K0 = k; j.Mw = d;
     j.r = r; j.r8 = r8; j.a1 = w.sU; j.a1_inner = r8; j.a1_ld = r8; j.w1 = Bp;
     j.b16_out = Y; j.ldb = (int)d; j.nb = (int)d;
     j.part = w.part_y; j.tickets = w.tickets + w.tickets_y_off;
@@ -1111,10 +1114,10 @@ int bwd_core(const qlora_nf4_t* q, const uint16_t* W, int64_t d, int64_t k, cons
   const uint16_t* Bp = padded_B(B, d, r, r8, w.Bp, st, &pst);
   QLORA_TRY(pst);
   const int rp = w.rp;
-  if (q) {
-    QLORA_TRY(block_scales(q, false, w.scales, T <= kSmallT ? w.tickets : nullptr, w.n_tickets, st));
-  } else if (T <= kSmallT) {
+  if (T <= kSmallT) {
     QLORA_TRY(zero_tickets(w.tickets, w.n_tickets, st));
+  } else if (q) {
+    QLORA_TRY(block_scales(q, false, w.scales, nullptr, 0, st));
   }
   // Us2 = hi/lo of bf16(s U)
   if (ma) {
@@ -1198,7 +1201,7 @@ int bwd_dx_base(const qlora_nf4_t* q, const uint16_t* W, int64_t d, int64_t k, c
   if (q && T <= kSmallT) {
     SmallJob j;
     j.src = SRC_NF4_COLS; j.out = OUT_BF16; j.name = "gemm_nf4_small_dx";
-    j.q = q; j.scales = w.scales; j.act = dY; j.K0 = d; j.Mw = k;
+    j.q = q; j.act = dY; j.K0 = d; j.Mw = k;
     j.r = re; j.r8 = r8; j.a1 = w.Gs2; j.a1_inner = r; j.a1_ld = 2 * rp; j.w1 = A;
     j.b16_out = dX; j.ldb = (int)k; j.nb = (int)k;
     j.part = w.part_x; j.tickets = w.tickets + w.tickets_x_off;

@@ -114,6 +114,15 @@ __device__ __forceinline__ void nf4_decode_block(uint4 c0, uint4 c1, float a, co
   o[7] = nf4_decode8(c1.w, t);
 }
 
+// Half a block: the 32 codes of one uint4, with the block's table.
+__device__ __forceinline__ void nf4_decode_half(uint4 c, float a, const float (&lv)[16], uint4 (&o)[4]) {
+  const Nf4Lut t = nf4_block_lut(a, lv);
+  o[0] = nf4_decode8(c.x, t);
+  o[1] = nf4_decode8(c.y, t);
+  o[2] = nf4_decode8(c.z, t);
+  o[3] = nf4_decode8(c.w, t);
+}
+
 // ------------------------------------------------------------------ kernel
 struct Nf4GemmArgs {
   int M, N, K0, K1;           // M tokens, N output columns, K0 main depth, K1 = r
@@ -155,7 +164,10 @@ struct Nf4Cfg {
   static constexpr int kCBytes = kCodeBytes + 1024;
   static constexpr int kStgBoxes = 2;             // epilogue staging: 4 KB boxes per warp
   static constexpr int kStage = 4 * kStgBoxes * 4096;
+  // mbarriers of the rings, accumulator full / empty and drain, and three words
+  static constexpr int kBarBytes = (2 * (SA + SB + SC) + 3) * 8 + 16;
   static constexpr int kSmemBytes = SA * kABytes + SB * kBBytes + SC * kCBytes + kStage + 1024 + 512;
+  static_assert(kBarBytes <= 512, "barrier region");
   // arrivals that complete a weight stage: every dequantising warp of the
   // unit (a rank-r stage: the TMA thread's expect_tx plus the rest)
   static constexpr int kBFull = kPair ? 2 * kDqWarps : kDqWarps;
@@ -684,8 +696,10 @@ __global__ void __launch_bounds__(Nf4Cfg<kPair>::kThreads, 1)
 // weight), so the depth is split across CTAs to put every SM to work; each CTA
 // writes fp32 partials and the last CTA of a row tile (a completion ticket)
 // sums them in split order, so results are deterministic.
-// Warps: 0 TMA, 1 TMEM + MMA, 2-5 dequantisation (NF4 sources), then all four
-// run the epilogue.
+// Warps: 0 TMA, 1 TMEM + MMA, 2-9 dequantisation (NF4 sources: two threads
+// per 64-weight block, half a block each, which halves the latency of a
+// K-step's decode); warps 2-5 then read the accumulator, and all eight sum
+// the depth splits.
 // ===========================================================================
 enum SmallSrc : int {
   SRC_NF4_ROWS = 0,   // W' rows (forward), K-major tiles dequantised in the kernel
@@ -713,23 +727,34 @@ struct Nf4SmallArgs {
   int lo_off;                 // OUT_HILO
   float scale;                // OUT_U / OUT_HILO: bf16 output = bf16(scale v)
   float f32_scale;            // OUT_U: fp32 output = f32_scale v
+  // NF4 sources: the double-quantised block constants, read by the
+  // dequantising threads themselves (kb = 64-blocks per W' row)
+  const uint8_t* absmax_q;
+  const float* scale2;
+  const float* mean;
+  int kb;
   float levels[16];
 };
 
-constexpr int kSmDqWarps = 4;
-constexpr int kSmThreads = (2 + kSmDqWarps) * 32;       // 192
+constexpr int kSmDqWarps = 8;
+constexpr int kSmThreads = (2 + kSmDqWarps) * 32;       // 320
 constexpr int kSmMaxSplits = 16;                         // depth splits per row tile (host plan caps it)
 
 template <int TN>
 struct SmallCfg {
+  // The codes ring holds a whole split's codes (the tiny per-step MMA cannot
+  // hide a load latency per step) while two CTAs still fit on an SM.
   static constexpr int SA = 3;                 // weight tiles, 128 x 64 bf16
-  static constexpr int SC = 3;                 // codes (4 KB) + block scales (up to 1 KB)
+  static constexpr int SC = TN >= 64 ? 6 : 8;  // codes, 4 KB per K-step
   static constexpr int SB = 4;                 // activation tiles, TN x 64 bf16
   static constexpr int kABytes = 16384;
   static constexpr int kCodeBytes = 4096;
-  static constexpr int kCBytes = kCodeBytes + 1024;
+  static constexpr int kCBytes = kCodeBytes;
   static constexpr int kBBytes = TN * 128;
-  static constexpr int kSmem = SA * kABytes + SC * kCBytes + SB * kBBytes + 1024 + 256;
+  // mbarriers (full and empty of each ring, accumulator, drain) and three words
+  static constexpr int kBarBytes = (2 * (SA + SB + SC) + 2) * 8 + 16;
+  // 1024 of slack for aligning the rings to the 128-byte swizzle atom's 1 KB
+  static constexpr int kSmem = SA * kABytes + SC * kCBytes + SB * kBBytes + 1024 + kBarBytes;
   static constexpr int kTmemCols = TN < 32 ? 32 : TN;
 };
 
@@ -755,11 +780,12 @@ __device__ __forceinline__ void small_emit(const Nf4SmallArgs& p, int m, int t, 
 }
 
 template <int kSrc, int kOut, int TN>
-__global__ void __launch_bounds__(kSmThreads, 1)
+__global__ void __launch_bounds__(kSmThreads, 2)
     gemm_nf4_small_kernel(const __grid_constant__ CUtensorMap tmAct, const __grid_constant__ CUtensorMap tmW,
-                          const __grid_constant__ CUtensorMap tmS, const __grid_constant__ CUtensorMap tmW1,
-                          const __grid_constant__ CUtensorMap tmAct1, const __grid_constant__ Nf4SmallArgs p) {
+                          const __grid_constant__ CUtensorMap tmW1, const __grid_constant__ CUtensorMap tmAct1,
+                          const __grid_constant__ Nf4SmallArgs p) {
   using Cfg = SmallCfg<TN>;
+  static_assert(Cfg::kSmem <= 232448, "shared memory per CTA");
   constexpr bool kNf4 = kSrc == SRC_NF4_ROWS || kSrc == SRC_NF4_COLS;
   constexpr bool kMnA = kSrc == SRC_NF4_COLS || kSrc == SRC_TMA_MN;
   extern __shared__ uint8_t smem_raw[];
@@ -820,7 +846,6 @@ __global__ void __launch_bounds__(kSmThreads, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tmAct);
     tma_prefetch_desc(&tmW);
-    if (kNf4) tma_prefetch_desc(&tmS);
     if (steps1 > 0) {
       tma_prefetch_desc(&tmW1);
       tma_prefetch_desc(&tmAct1);
@@ -839,10 +864,31 @@ __global__ void __launch_bounds__(kSmThreads, 1)
       for (int i = 0; i < Cfg::SB; ++i) b_iss[i] = 0;
       for (int i = 0; i < Cfg::SC; ++i) c_iss[i] = 0;
       for (int i = 0; i < Cfg::SA; ++i) a_last[i] = -1;
-      for (int step = 0; step < steps; ++step) {
+      // codes run ahead of the activations by up to SC K-steps (issued in
+      // step order, each when the decode of the step SC before it is done)
+      int cnext = 0;
+      bool ok = true;
+      auto issue_codes = [&](int upto) -> bool {
+        for (; cnext < nmain && cnext < upto; ++cnext) {
+          const int sc = cnext % Cfg::SC;
+          if (!mbar_wait_bounded(smem_u32(&c_empty[sc]), (uint32_t)(((cnext / Cfg::SC) & 1) ^ 1), abort_flag))
+            return false;
+          const uint32_t fc = smem_u32(&c_full[sc]);
+          const int ks = s_begin + cnext;
+          mbar_arrive_expect_tx(fc, (uint32_t)Cfg::kCodeBytes);
+          if (kSrc == SRC_NF4_COLS)
+            tma_load_2d(sC + sc * Cfg::kCBytes, &tmW, fc, m0 / 2, ks * 64);
+          else
+            tma_load_2d(sC + sc * Cfg::kCBytes, &tmW, fc, ks * 32, m0);
+          c_iss[sc] += 1;
+        }
+        return true;
+      };
+      for (int step = 0; step < steps && ok; ++step) {
         const bool main = step < nmain;
         const int ks = s_begin + step;
         const int e = step - nmain;
+        if (kNf4 && !issue_codes(step + Cfg::SC)) break;
         const int sb = step % Cfg::SB;
         if (!mbar_wait_bounded(smem_u32(&b_empty[sb]), (uint32_t)(((step / Cfg::SB) & 1) ^ 1), abort_flag)) break;
         const uint32_t fb = smem_u32(&b_full[sb]);
@@ -852,25 +898,7 @@ __global__ void __launch_bounds__(kSmThreads, 1)
         else
           tma_load_2d(sB + sb * Cfg::kBBytes, &tmAct1, fb, e * 64, 0);
         b_iss[sb] += 1;
-        if (main && kNf4) {
-          const int sc = step % Cfg::SC;
-          if (!mbar_wait_bounded(smem_u32(&c_empty[sc]), (uint32_t)(((step / Cfg::SC) & 1) ^ 1), abort_flag))
-            break;
-          const uint32_t fc = smem_u32(&c_full[sc]);
-          if (kSrc == SRC_NF4_COLS) {
-            mbar_arrive_expect_tx(fc, (uint32_t)(Cfg::kCodeBytes + 1024));
-            tma_load_2d(sC + sc * Cfg::kCBytes, &tmW, fc, m0 / 2, ks * 64);
-            // scales of 64 K-rows x 4 block columns from a 16-byte aligned
-            // column (the tile's two columns sit at (m0 / 64) % 4)
-            tma_load_2d(sC + sc * Cfg::kCBytes + Cfg::kCodeBytes, &tmS, fc, (m0 >> 6) & ~3, ks * 64);
-          } else {
-            mbar_arrive_expect_tx(fc, (uint32_t)(Cfg::kCodeBytes + 512));
-            tma_load_2d(sC + sc * Cfg::kCBytes, &tmW, fc, ks * 32, m0);
-            // scales of the tile's 128 rows at block column ks
-            tma_load_2d(sC + sc * Cfg::kCBytes + Cfg::kCodeBytes, &tmS, fc, m0, ks);
-          }
-          c_iss[sc] += 1;
-        } else {
+        if (!(main && kNf4)) {
           // a bf16 weight-side tile by TMA: the main operand of U / G, or the
           // rank-r operand (B rows / A columns) of the NF4 products
           const int sa = step % Cfg::SA;
@@ -944,67 +972,100 @@ __global__ void __launch_bounds__(kSmThreads, 1)
       // Thread i owns one block per K-step.  Rows: tile row i (W' row m0 + i,
       // block column = the K-step).  Columns: K-row kk = i % 64 (W' row
       // 64 * ks + kk) and MN chunk cc = i / 64 (W' block column m0 / 64 + cc).
-      const int i = threadIdx.x - 64;
+      // The thread reads its blocks' constants itself, kAhead K-steps ahead
+      // (a register ring), and forms each block scale
+      // a' = fl(fl(absmax * scale2) + mean) exactly as the dequantiser does;
+      // blocks past the weight's edge get a' = 0.
+      const int h = (threadIdx.x - 64) >> 7;           // which half of the block
+      const int i = (threadIdx.x - 64) & 127;
       const int kk = i & 63, cc = i >> 6;
-      for (int step = 0; step < nmain; ++step) {
-        const int sc = step % Cfg::SC;
-        bool ok = mbar_wait_bounded(smem_u32(&c_full[sc]), (uint32_t)((step / Cfg::SC) & 1), abort_flag);
-        if (!__all_sync(0xffffffffu, ok)) {
-          live = false;
-          break;
-        }
-        uint4 c0, c1;
-        const uint32_t cs = sC + sc * Cfg::kCBytes;
-        const float* scl =
-            reinterpret_cast<const float*>(smem + (cs - sA) + Cfg::kCodeBytes);
-        float a;
+      const int Mrows = kSrc == SRC_NF4_COLS ? p.kb : p.Mw;   // forward: W' rows; dX: block columns
+      const float mu = *p.mean;
+      auto block_of = [&](int step, int64_t& b) -> bool {
+        const int ks = s_begin + step;
         if (kSrc == SRC_NF4_COLS) {
-          // 64-byte rows, 64B swizzle: chunk j at (j ^ ((row >> 1) & 3))
-          const uint32_t row = cs + kk * 64;
-          const int sw = (kk >> 1) & 3;
-          c0 = ld_shared_v4(row + (((2 * cc) ^ sw) << 4));
-          c1 = ld_shared_v4(row + (((2 * cc + 1) ^ sw) << 4));
-          a = scl[kk * 4 + ((m0 >> 6) & 3) + cc];
-        } else {
-          const uint32_t row = cs + i * 32;
-          const int sw = (i >> 2) & 1;
-          c0 = ld_shared_v4(row + ((0 ^ sw) << 4));
-          c1 = ld_shared_v4(row + ((1 ^ sw) << 4));
-          a = scl[i];
+          const int bc = (m0 >> 6) + cc;                 // block column
+          const int wr = ks * 64 + kk;                   // W' row
+          b = (int64_t)wr * p.kb + bc;
+          return bc < Mrows && wr < p.K0;
         }
-        uint4 o[8];
-        nf4_decode_block(c0, c1, a, p.levels, o);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&c_empty[sc]));
-        const int sa = step % Cfg::SA;
-        ok = mbar_wait_bounded(smem_u32(&a_empty[sa]), (uint32_t)(((step / Cfg::SA) & 1) ^ 1), abort_flag);
-        if (!__all_sync(0xffffffffu, ok)) {
-          live = false;
-          break;
-        }
-        uint32_t dst;
-        int sw;
-        if (kSrc == SRC_NF4_COLS) {
-          dst = sA + sa * Cfg::kABytes + cc * 8192 + kk * 128;
-          sw = kk & 7;
-        } else {
-          dst = sA + sa * Cfg::kABytes + i * 128;
-          sw = i & 7;
-        }
+        b = (int64_t)(m0 + i) * p.kb + ks;
+        return m0 + i < Mrows;
+      };
+      constexpr int kAhead = 4;
+      constexpr uint32_t kOutside = 0x100u;          // not a code byte: the block lies outside W'
+      uint32_t q_r[kAhead];
+      float s2_r[kAhead];
+      auto load_step = [&](int step, uint32_t& q, float& s2) {
+        int64_t b = 0;
+        const bool in = step < nmain && block_of(step, b);
+        q = in ? (uint32_t)__ldg(p.absmax_q + b) : kOutside;
+        s2 = in ? __ldg(p.scale2 + b / kBlock2) : 0.f;
+      };
 #pragma unroll
-        for (int j = 0; j < 8; ++j) st_shared_v4(dst + ((j ^ sw) << 4), o[j]);
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(smem_u32(&a_full[sa]));
+      for (int j = 0; j < kAhead; ++j) load_step(j, q_r[j], s2_r[j]);
+      for (int s0 = 0; s0 < nmain && live; s0 += kAhead) {
+#pragma unroll
+        for (int jw = 0; jw < kAhead; ++jw) {
+          const int step = s0 + jw;
+          if (step >= nmain) break;
+          const int sc = step % Cfg::SC;
+          bool ok = mbar_wait_bounded(smem_u32(&c_full[sc]), (uint32_t)((step / Cfg::SC) & 1), abort_flag);
+          if (!__all_sync(0xffffffffu, ok)) {
+            live = false;
+            break;
+          }
+          uint4 c;
+          const uint32_t cs = sC + sc * Cfg::kCBytes;
+          const float a =
+              q_r[jw] != kOutside ? __fadd_rn(__fmul_rn(e4m3_to_f32((uint8_t)q_r[jw]), s2_r[jw]), mu) : 0.f;
+          load_step(step + kAhead, q_r[jw], s2_r[jw]);
+          if (kSrc == SRC_NF4_COLS) {
+            // 64-byte rows, 64B swizzle: chunk j at (j ^ ((row >> 1) & 3))
+            const uint32_t row = cs + kk * 64;
+            const int sw = (kk >> 1) & 3;
+            c = ld_shared_v4(row + (((2 * cc + h) ^ sw) << 4));
+          } else {
+            const uint32_t row = cs + i * 32;
+            const int sw = (i >> 2) & 1;
+            c = ld_shared_v4(row + ((h ^ sw) << 4));
+          }
+          uint4 o[4];
+          nf4_decode_half(c, a, p.levels, o);
+          __syncwarp();
+          if (lane == 0) mbar_arrive(smem_u32(&c_empty[sc]));
+          const int sa = step % Cfg::SA;
+          ok = mbar_wait_bounded(smem_u32(&a_empty[sa]), (uint32_t)(((step / Cfg::SA) & 1) ^ 1), abort_flag);
+          if (!__all_sync(0xffffffffu, ok)) {
+            live = false;
+            break;
+          }
+          uint32_t dst;
+          int sw;
+          if (kSrc == SRC_NF4_COLS) {
+            dst = sA + sa * Cfg::kABytes + cc * 8192 + kk * 128;
+            sw = kk & 7;
+          } else {
+            dst = sA + sa * Cfg::kABytes + i * 128;
+            sw = i & 7;
+          }
+#pragma unroll
+          for (int j = 0; j < 4; ++j) st_shared_v4(dst + (((4 * h + j) ^ sw) << 4), o[j]);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(smem_u32(&a_full[sa]));
+        }
       }
     }
     // ---------------------------------------------------------- epilogue
-    // lane quarter of this warp: accumulator rows m0 + 32 q .. + 31
+    // warps 2-5 read the accumulator: lane quarter q = warp & 3 holds rows
+    // m0 + 32 q .. + 31
+    const bool acc_warp = warp < 6;
     const int quarter = warp & 3;
     const int m = m0 + quarter * 32 + lane;
     bool ok = live && mbar_wait_bounded(smem_u32(acc_full), 0u, abort_flag);
     ok = __all_sync(0xffffffffu, ok);
-    if (ok) {
+    if (ok && acc_warp) {
       tc_fence_after();
       const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16);
 #pragma unroll 1
@@ -1037,27 +1098,49 @@ __global__ void __launch_bounds__(kSmThreads, 1)
       named_bar_sync(1, kSmDqWarps * 32);
       if (*last_flag && ok) {
         __threadfence();
-        if (m < p.Mw) {
-          // four tokens at a time with every split's partial in flight
-          // (at most kSmMaxSplits), then summed in split order
-          const int64_t zs = (int64_t)p.T * p.Mw;
-          for (int t0 = 0; t0 < p.T; t0 += 4) {
-            const int nt = min(4, p.T - t0);
-            const float* src = p.part + (int64_t)t0 * p.Mw + m;
-            float v[kSmMaxSplits][4];
+        // all eight warps: each item is (token, features), with every split's
+        // partial in flight at once (at most kSmMaxSplits), summed in split order
+        const int tid = threadIdx.x - 64;
+        const int64_t zs = (int64_t)p.T * p.Mw;
+        if ((p.Mw & 3) == 0) {
+          for (int it = tid; it < p.T * 32; it += kSmDqWarps * 32) {
+            const int t = it >> 5;
+            const int mq = m0 + (it & 31) * 4;
+            if (mq >= p.Mw) continue;
+            const float4* src = reinterpret_cast<const float4*>(p.part + (int64_t)t * p.Mw + mq);
+            float4 v[kSmMaxSplits];
 #pragma unroll
             for (int z = 0; z < kSmMaxSplits; ++z)
+              v[z] = z < p.splits ? __ldcg(src + z * (zs >> 2)) : make_float4(0.f, 0.f, 0.f, 0.f);
+            float4 acc = v[0];
 #pragma unroll
-              for (int j = 0; j < 4; ++j)
-                v[z][j] = (z < p.splits && j < nt) ? __ldcg(src + z * zs + (int64_t)j * p.Mw) : 0.f;
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              float acc = v[0][j];
-#pragma unroll
-              for (int z = 1; z < kSmMaxSplits; ++z)
-                if (z < p.splits) acc = __fadd_rn(acc, v[z][j]);
-              if (j < nt) small_emit<kOut>(p, m, t0 + j, acc);
+            for (int z = 1; z < kSmMaxSplits; ++z) {
+              if (z < p.splits) {
+                acc.x = __fadd_rn(acc.x, v[z].x);
+                acc.y = __fadd_rn(acc.y, v[z].y);
+                acc.z = __fadd_rn(acc.z, v[z].z);
+                acc.w = __fadd_rn(acc.w, v[z].w);
+              }
             }
+            small_emit<kOut>(p, mq, t, acc.x);
+            small_emit<kOut>(p, mq + 1, t, acc.y);
+            small_emit<kOut>(p, mq + 2, t, acc.z);
+            small_emit<kOut>(p, mq + 3, t, acc.w);
+          }
+        } else {
+          for (int it = tid; it < p.T * 128; it += kSmDqWarps * 32) {
+            const int t = it >> 7;
+            const int mm = m0 + (it & 127);
+            if (mm >= p.Mw) continue;
+            const float* src = p.part + (int64_t)t * p.Mw + mm;
+            float v[kSmMaxSplits];
+#pragma unroll
+            for (int z = 0; z < kSmMaxSplits; ++z) v[z] = z < p.splits ? __ldcg(src + z * zs) : 0.f;
+            float acc = v[0];
+#pragma unroll
+            for (int z = 1; z < kSmMaxSplits; ++z)
+              if (z < p.splits) acc = __fadd_rn(acc, v[z]);
+            small_emit<kOut>(p, mm, t, acc);
           }
         }
         if (threadIdx.x == 64) p.tickets[tile] = 0u;
