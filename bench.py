@@ -19,6 +19,7 @@ from __future__ import annotations
 
 import argparse
 import hashlib
+import re
 import json
 import os
 import statistics
@@ -239,11 +240,19 @@ GEMM_SOURCES = ("parameter_efficient_fine_nf4_b200/csrc/nf4_gemm.cuh",
                 "include/qlora.h")
 
 
+def _code_only(text: str) -> str:
+    """Source text without comments and blank space, so that edits to comments
+    do not invalidate a recorded capture."""
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return " ".join(text.split())
+
+
 def kernel_source_hash():
     h = hashlib.sha256()
     for f in GEMM_SOURCES:
-        with open(os.path.join(ROOT, f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, f), "r", encoding="utf-8") as fh:
+            h.update(_code_only(fh.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -7,23 +7,28 @@
 //   backward dX = [dY | sG] [W' ; A]       (M = T, N = k, K = d (+ r))
 //
 // W' never exists in global memory.  Dequantising warps read the packed codes
-// of one K-step and the fp32 block scales a' of its blocks (both staged in
-// shared memory by TMA, the codes read back with 128-bit loads; the scales are
-// formed once per call by nf4_block_scales in a TMA-friendly layout), form per
-// 64-weight block the 16 products bf16(level[i] * a') once,
-// select each weight's value from them with byte permutes on registers, and
-// write the bf16 tile in exactly the 128B-swizzled layout a TMA load of W'
-// would have produced (K-major rows for the forward, MN-major for dX).  So the
-// MMA sees the same operand bytes as on a dequantised weight and the result
-// is bit-identical to the plain-LoRA GEMM on W'.
+// of one K-step (staged in shared memory by TMA and read back with 128-bit
+// loads) and the fp32 block scales a' of its blocks.  Above 64 tokens the
+// scales are formed once per call by nf4_block_scales in a TMA-friendly layout
+// and staged with the codes; the few-token kernels form them in the
+// dequantising threads from the stored constants.  Per 64-weight block the
+// 16 products bf16(level[i] * a') are formed once, each weight's value is
+// selected from them with byte permutes on registers, and the bf16 tile is
+// written in exactly the 128B-swizzled layout a TMA load of W' would have
+// produced (K-major rows for the forward, MN-major for dX).  So the MMA sees
+// the same operand bytes as on a dequantised weight and the result is
+// bit-identical to the plain-LoRA GEMM on W'.
 //
-// Tiles: one CTA per SM, each work unit is 256 rows of M (two 128-row MMA
-// tiles, two TMEM accumulators) by 256 columns of N, so one dequantised
-// weight tile feeds 256 x 256 x 64 of MMA work per K-step: the decode costs
-// 16 weights per MMA cycle-equivalent instead of 32.
+// Above 64 tokens (gemm_nf4_kernel), by default a cluster of two CTAs per SM
+// pair runs 256-row tcgen05 MMAs over both SMs (cta_group::2) on units of 512
+// tokens by 256 columns; each CTA decodes 128 of the 256 weight rows of a
+// K-step, so per SM the decode halves at the same MMA work.  A one-CTA build
+// (units of 256 tokens, the whole weight tile decoded per CTA) gives the same
+// bits.  Warps: 0 activation and rank-r tile loads, 1 TMEM + MMA issue (rank
+// 0 of a pair), 2-5 epilogue, 6 code and block-scale loads, 7.. dequantisation.
 //
-// Warps: 0 TMA (activations, codes, rank-r operands), 1 TMEM + MMA issue,
-// 2-5 epilogue, 6-13 dequantisation (thread i owns weight-tile row i).
+// At most 64 tokens (gemm_nf4_small_kernel) the products are computed with
+// the operands swapped and the depth split over CTAs; see its section below.
 #pragma once
 #include "gemm_tc.cuh"
 #include "nf4_kernels.cuh"
