@@ -668,6 +668,8 @@ struct BwdWs {
   uint16_t* Xm;            // LoRA dropout: the masked adapter input
   uint16_t* Bcat; float* Gall; float* dBcat;   // several adapters
   float* scales;           // fp32 block scales of the NF4 weight (dX layout)
+  float* sGf;              // T <= 64: s G in fp32 (T x r), operand of the CUDA-core dA
+  float* sUf;              // T <= 64, several adapters: s U scattered into the token's block (T x r)
   int rp, halves, splitsA, splitsB; size_t bytes;
 };
 // Backward workspace.  U and G enter the T-reductions (dB, dA) as two bf16
@@ -703,6 +705,8 @@ BwdWs carve_bwd(void* ws, int64_t d, int64_t k, int r, int64_t T, bool dropout =
     w.n_tickets = sg.tiles_m + sx.tiles_m;
     w.tickets = (unsigned int*)c.take((size_t)w.n_tickets * 4);
   }
+  w.sGf = (T >= 1 && T <= kSmallT) ? (float*)c.take((size_t)(T * r * 4)) : nullptr;
+  w.sUf = (T >= 1 && T <= kSmallT && multi) ? (float*)c.take((size_t)(T * r * 4)) : nullptr;
   w.Xm = dropout ? (uint16_t*)c.take((size_t)(Tm * k * 2)) : nullptr;
   w.Bcat = multi ? (uint16_t*)c.take((size_t)(d * r * 2)) : nullptr;
   w.Gall = multi ? (float*)c.take((size_t)(Tm * r * 4)) : nullptr;
@@ -990,6 +994,20 @@ int block_scales(const qlora_nf4_t* q, bool transposed, float* out, unsigned int
   });
 }
 
+// dA (r x k) and dB (d x r) of a few tokens on CUDA cores (adapter_grads_small).
+int grads_small(const uint16_t* X, const uint16_t* dY, const float* U, const float* sG, float s, int64_t T,
+                int64_t d, int64_t k, int r, float* dA, float* dB, cudaStream_t st) {
+  // four columns of dA / four rows of dB per thread (k % 64 == 0, d % 8 == 0)
+  const int kblk = (int)cdiv(k / 4, kGradThreads);
+  const int nb_a = r * kblk;
+  const int nb_b = (int)cdiv(d / 4, kGradThreads / r);
+  const double n = (double)r * k + (double)d * r;
+  return launch("adapter_grads_small", 2.0 * (double)T * n, n * 4, st, [&] {
+    adapter_grads_small<<<nb_a + nb_b, kGradThreads, 0, st>>>(X, dY, U, sG, s, (int)T, (int)d, (int)k, r, kblk,
+                                                              nb_a, dA, dB);
+  });
+}
+
 // Forward on a bf16 d x k weight W (plain LoRA: the caller's W) or, when `q`
 // is given, on the NF4 weight dequantised inside the GEMM (W unused).
 // A stack of n unmerged adapters of rank ra chosen per token (idx[t]); the
@@ -1118,6 +1136,51 @@ int bwd_core(const qlora_nf4_t* q, const uint16_t* W, int64_t d, int64_t k, cons
     QLORA_TRY(zero_tickets(w.tickets, w.n_tickets, st));
   } else if (q) {
     QLORA_TRY(block_scales(q, false, w.scales, nullptr, 0, st));
+  }
+  // Few tokens, several adapters, no dropout: G of every adapter in fp32, the
+  // token's s_i U and s_i G scattered into its block, then dA (the stack) and
+  // dB (side by side) in one CUDA-core kernel; the bf16 s G of the dX
+  // extension as before.  With one adapter this is the arithmetic of the
+  // single-adapter path below, so both give the same bits.
+  if (T <= kSmallT && ma && !keep) {
+    SmallJob j;
+    j.src = SRC_TMA_MN; j.out = OUT_U; j.name = "gemm_lora_g_small";
+    j.w = Bp; j.w_inner = r8; j.w_outer = d; j.w_ld = r8;
+    j.act = dY; j.K0 = d; j.Mw = rp;
+    j.f32_out = w.Gall; j.ldf = r; j.nf = r; j.nb = 0;
+    j.part = w.part_g; j.tickets = w.tickets;
+    QLORA_TRY(launch_small(j, T, st));
+    QLORA_TRY(launch("scatter_adapter_hilo", 0.0, 0.0, st, [&] {
+      scatter_adapter_hilo<<<grid_for(T * rp, 256), 256, 0, st>>>(w.Gall, 0, ma->idx, T, ma->ra, ma->n, rp,
+                                                                  ma->sc, w.Gs2);
+    }));
+    QLORA_TRY(launch("scatter_adapter_f32", 0.0, 0.0, st, [&] {
+      scatter_adapter_f32<<<grid_for(T * r, 256), 256, 0, st>>>(U_saved, 1, ma->idx, T, ma->ra, ma->n, ma->sc,
+                                                               w.sUf);
+    }));
+    QLORA_TRY(launch("scatter_adapter_f32", 0.0, 0.0, st, [&] {
+      scatter_adapter_f32<<<grid_for(T * r, 256), 256, 0, st>>>(w.Gall, 0, ma->idx, T, ma->ra, ma->n, ma->sc,
+                                                               w.sGf);
+    }));
+    QLORA_TRY(grads_small(X, dY, w.sUf, w.sGf, 1.0f, T, d, k, r, dA, w.dBcat, st));
+    QLORA_TRY(launch("uncat_adapters_db", 0.0, 0.0, st, [&] {
+      uncat_adapters_db<<<grid_for(d * r, 256), 256, 0, st>>>(w.dBcat, d, ma->ra, ma->n, dB);
+    }));
+    return bwd_dx_base(q, W, d, k, A, r, r8, rp, dY, T, dX, w, st, true);
+  }
+  // Few tokens, one adapter, no dropout: G gives s G in fp32 (and the bf16
+  // operand of the dX extension), then dA and dB in one CUDA-core kernel.
+  if (T <= kSmallT && !ma && !keep) {
+    SmallJob j;
+    j.src = SRC_TMA_MN; j.out = OUT_U; j.name = "gemm_lora_g_small";
+    j.w = Bp; j.w_inner = r8; j.w_outer = d; j.w_ld = r8;
+    j.act = dY; j.K0 = d; j.Mw = rp;
+    j.f32_out = w.sGf; j.ldf = r; j.nf = r; j.f32_scale = s;
+    j.b16_out = w.Gs2; j.ldb = 2 * rp; j.nb = rp; j.scale = s;
+    j.part = w.part_g; j.tickets = w.tickets;
+    QLORA_TRY(launch_small(j, T, st));
+    QLORA_TRY(grads_small(X, dY, U_saved, w.sGf, s, T, d, k, r, dA, dB, st));
+    return bwd_dx_base(q, W, d, k, A, r, r8, rp, dY, T, dX, w, st, true);
   }
   // Us2 = hi/lo of bf16(s U)
   if (ma) {

@@ -573,6 +573,91 @@ __global__ void __launch_bounds__(256) nf4_block_scales(const uint8_t* __restric
 // ---------------------------------------------------------------------------
 // Small helpers for the rank-r operands.
 // ---------------------------------------------------------------------------
+// Adapter gradients for a few tokens (T <= 64), in fp32 on CUDA cores: with
+// so few terms the T-reductions are a handful of FMAs per output, and the
+// outputs (r x k and d x r fp32) are what costs.  Each output is summed over
+// the tokens in order, so results are deterministic:
+//   dA[i][j] = sum_t sG[t][i] X[t][j]          (r x k; sG = s G, fp32)
+//   dB[i][j] = sum_t dY[t][i] fl(s U[t][j])    (d x r)
+// A thread forms four outputs from 8-byte loads: blocks [0, nb_a) take dA,
+// row i = block / kblk and four consecutive columns j per thread; the rest
+// take dB, four consecutive rows i (d % 8 == 0) for one column j, 256 / r
+// row quads of r columns per block (r <= 256).  Needs k % 4 == 0, d % 4 == 0
+// and 8-byte aligned X and dY rows.
+constexpr int kGradThreads = 256;
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+__global__ void __launch_bounds__(kGradThreads) adapter_grads_small(const uint16_t* __restrict__ X,
+                                                                    const uint16_t* __restrict__ dY,
+                                                                    const float* __restrict__ U,
+                                                                    const float* __restrict__ sG, float s, int T,
+                                                                    int d, int k, int r, int kblk, int nb_a,
+                                                                    float* __restrict__ dA, float* __restrict__ dB) {
+  const int b = (int)blockIdx.x;
+  float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
+  if (b < nb_a) {
+    const int i = b / kblk;
+    const int j = 4 * ((b - i * kblk) * kGradThreads + (int)threadIdx.x);
+    if (j >= k) return;
+    // the loads of 16 tokens are all issued before their FMAs
+    for (int t0 = 0; t0 < T; t0 += 16) {
+      float g[16];
+      uint2 x[16];
+#pragma unroll
+      for (int q = 0; q < 16; ++q) {
+        const int t = min(t0 + q, T - 1);
+        g[q] = __ldg(sG + t * r + i);
+        x[q] = __ldg(reinterpret_cast<const uint2*>(X + (int64_t)t * k + j));
+      }
+#pragma unroll
+      for (int q = 0; q < 16; ++q) {
+        if (t0 + q < T) {
+          a0 = __fmaf_rn(g[q], bf16_lo(x[q].x), a0);
+          a1 = __fmaf_rn(g[q], bf16_hi(x[q].x), a1);
+          a2 = __fmaf_rn(g[q], bf16_lo(x[q].y), a2);
+          a3 = __fmaf_rn(g[q], bf16_hi(x[q].y), a3);
+        }
+      }
+    }
+    float* o = dA + (int64_t)i * k + j;
+    o[0] = a0;
+    o[1] = a1;
+    o[2] = a2;
+    o[3] = a3;
+    return;
+  }
+  const int qpb = kGradThreads / r;                 // row quads of dB per block
+  const int tq = (int)threadIdx.x / r;
+  const int j = (int)threadIdx.x - tq * r;
+  const int i = 4 * ((b - nb_a) * qpb + tq);
+  if (tq >= qpb || i >= d) return;
+  for (int t0 = 0; t0 < T; t0 += 16) {
+    float u[16];
+    uint2 y[16];
+#pragma unroll
+    for (int q = 0; q < 16; ++q) {
+      const int t = min(t0 + q, T - 1);
+      u[q] = __ldg(U + t * r + j);
+      y[q] = __ldg(reinterpret_cast<const uint2*>(dY + (int64_t)t * d + i));
+    }
+#pragma unroll
+    for (int q = 0; q < 16; ++q) {
+      if (t0 + q < T) {
+        const float su = __fmul_rn(s, u[q]);
+        a0 = __fmaf_rn(bf16_lo(y[q].x), su, a0);
+        a1 = __fmaf_rn(bf16_hi(y[q].x), su, a1);
+        a2 = __fmaf_rn(bf16_lo(y[q].y), su, a2);
+        a3 = __fmaf_rn(bf16_hi(y[q].y), su, a3);
+      }
+    }
+  }
+  float* o = dB + (int64_t)i * r + j;
+  o[0] = a0;
+  o[r] = a1;
+  o[2 * r] = a2;
+  o[3 * r] = a3;
+}
+
 // dst (rows x ld_dst, bf16) = src (rows x cols, bf16) with zero columns
 // [cols, ld_dst).
 __global__ void pad_cols_bf16(const uint16_t* __restrict__ src, int64_t rows, int cols,
@@ -705,6 +790,24 @@ __global__ void scatter_adapter_hilo(const float* __restrict__ V, int per_token,
     const __nv_bfloat16 l = __float2bfloat16_rn(__fsub_rn(v, __bfloat162float(h)));
     out[t * 2 * half + c] = *reinterpret_cast<const uint16_t*>(&h);
     out[t * 2 * half + half + c] = *reinterpret_cast<const uint16_t*>(&l);
+  }
+}
+
+// fp32 v = s_idx V into the token's block of out (T x R), zero outside it
+// (the operands of the few-token CUDA-core adapter gradients).  V is per token
+// (T x r) or over all blocks (T x R), as for scatter_adapter_hilo.
+__global__ void scatter_adapter_f32(const float* __restrict__ V, int per_token, const int32_t* __restrict__ idx,
+                                    int64_t T, int r, int n, const __grid_constant__ AdapterScales sc,
+                                    float* __restrict__ out) {
+  const int R = n * r;
+  const int64_t total = T * R;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += stride) {
+    const int64_t t = e / R;
+    const int c = (int)(e - t * R);
+    const int a = idx[t];
+    const bool mine = c / r == a;
+    out[e] = mine ? __fmul_rn(sc.s[a], per_token ? V[t * r + (c - a * r)] : V[t * R + c]) : 0.f;
   }
 }
 
