@@ -602,7 +602,9 @@ SmallPlan small_plan(int64_t Mw, int64_t K0, int64_t T) {
   const int steps0 = (int)cdiv(K0, 64);
   // two CTAs of the few-token kernel fit on an SM; one wave of them
   const int want = std::max(1, (int)(2 * kSMs / sp.tiles_m));
-  const int splits = std::max(1, std::min(std::min(want, steps0 / 8), kSmMaxSplits));
+  // at least 4 K-steps per split (the single-tile U and G products get 16
+  // splits; the NF4 products are capped by their tile count first)
+  const int splits = std::max(1, std::min(std::min(want, steps0 / 4), kSmMaxSplits));
   sp.sps = (int)cdiv(steps0, splits);
   sp.splits = (int)cdiv(steps0, sp.sps);
   return sp;
