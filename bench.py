@@ -459,6 +459,8 @@ def run_ours(args):
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
     q4.lib()
     cfg, T = workload(args.config, args.tokens)
+    # the library's own communicator for the one exchange (sum of dA and dB)
+    comm = q4.communicator_from_process_group() if world > 1 else None
 
     # ---- resident inputs (per rank: its own tokens, the same frozen weights)
     layers = []
@@ -509,9 +511,8 @@ def run_ours(args):
             q4.qlora_fwd(L["qw"], L["A"], L["B"], cfg.alpha, X, Y=L["Y"], U_save=L["U"], ws=L["ws"])
             q4.qlora_bwd(L["qw"], L["A"], L["B"], cfg.alpha, X, L["U"], dY, dX=L["dX"],
                          dA=L["dA"], dB=L["dB"], ws=L["ws"])
-        if world > 1:
-            dist.all_reduce(L["dA"])
-            dist.all_reduce(L["dB"])
+        if comm is not None:
+            q4.qlora_grad_allreduce(comm, L["dA"], L["dB"])
         if not plain:
             q4.lora_merge(L["qw"], L["A"], L["B"], cfg.alpha, W_out=L["Wm"], ws=L["ws"])
             q4.lora_unmerge(L["Wm"], L["A"], L["B"], cfg.alpha, W0_out=L["W0u"], ws=L["ws"])
@@ -734,6 +735,8 @@ def run_ours(args):
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier(device_ids=[local])
+        torch.cuda.synchronize(dev)
+        comm.close()
         dist.destroy_process_group()
     return 0
 

@@ -45,7 +45,8 @@ typedef enum {
   QLORA_ERR_CUDA = 5,              /* a CUDA runtime/driver call or launch failed */
   QLORA_ERR_TIMEOUT = 6,           /* a device-side wait gave up (device status) */
   QLORA_ERR_NO_DEVICE = 7,         /* no sm_100 device is current */
-  QLORA_ERR_EXCEEDS_STATIC_SCRATCH = 8 /* too large for qlora_nf4_quantize_noalloc */
+  QLORA_ERR_EXCEEDS_STATIC_SCRATCH = 8, /* too large for qlora_nf4_quantize_noalloc */
+  QLORA_ERR_NCCL = 9               /* NCCL could not be loaded, or an NCCL call failed */
 } qlora_status_t;
 
 /* A cudaStream_t passed as an opaque pointer (NULL = legacy default stream). */
@@ -349,6 +350,43 @@ QLORA_API int qlora_get_device_status(qlora_stream_t stream, int* status);
  * qlora_get_device_status.  The wait limit of other kernels is unchanged.
  */
 QLORA_API int qlora_selftest_wait_timeout(int limit_us, qlora_stream_t stream);
+
+/* ------------------------------------------------------------ data parallel */
+
+/*
+ * The layer is data-parallel over tokens ([P1] "The update LoRA is allowed to
+ * learn": only A and B get gradients, the frozen weight needs no exchange).
+ * Each GPU keeps a replica of the NF4 weight, A and B, runs forward and
+ * backward on its own tokens, and the one exchange is the sum of dA and dB
+ * over the ranks.  The library makes that call through NCCL; the caller owns
+ * the communicator.  NCCL (libnccl.so.2) is loaded at the first of these
+ * calls, so the library itself loads without it; QLORA_ERR_NCCL when it is
+ * missing or a call fails.
+ */
+#define QLORA_NCCL_ID_BYTES 128
+
+/* Writes a new NCCL unique id (QLORA_NCCL_ID_BYTES bytes, host memory) for
+ * the caller to share with every rank before qlora_comm_init. */
+QLORA_API int qlora_comm_unique_id(uint8_t* id);
+
+/* Creates this rank's communicator on the current device (collective: every
+ * rank calls it with the same id and nranks, each with its own rank in
+ * [0, nranks)).  *comm receives an opaque handle. */
+QLORA_API int qlora_comm_init(const uint8_t* id, int nranks, int rank, void** comm);
+
+/* Releases a communicator made by qlora_comm_init (call it on every rank,
+ * after the last collective using it has completed). */
+QLORA_API int qlora_comm_destroy(void* comm);
+
+/*
+ * In place, on `stream`: dA (nA fp32) and dB (nB fp32, device memory) become
+ * their sums over the ranks of `comm`, as one group of two NCCL all-reduces.
+ * Either count may be 0.  Every rank must make the same call with the same
+ * counts.  Returns at once (stream-ordered); QLORA_ERR_INVALID_ARG for a null
+ * communicator, a negative count or a null pointer with a positive count.
+ */
+QLORA_API int qlora_grad_allreduce(void* comm, float* dA, int64_t nA, float* dB, int64_t nB,
+                                   qlora_stream_t stream);
 
 /* ---------------------------------------------------------------- profiling */
 

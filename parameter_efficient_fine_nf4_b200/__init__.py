@@ -90,6 +90,10 @@ _SIGNATURES = {
     "qlora_profile_end": (_INT, [ctypes.POINTER(KernelStat), _INT, ctypes.POINTER(_INT)]),
     "qlora_launch_count": (_I64, []),
     "qlora_set_nf4_gemm_mode": (_INT, [_INT]),
+    "qlora_comm_unique_id": (_INT, [_VP]),
+    "qlora_comm_init": (_INT, [_VP, _INT, _INT, ctypes.POINTER(_VP)]),
+    "qlora_comm_destroy": (_INT, [_VP]),
+    "qlora_grad_allreduce": (_INT, [_VP, _VP, _I64, _VP, _I64, _VP]),
 }
 
 EXPORTED = tuple(_SIGNATURES)
@@ -541,6 +545,56 @@ def qlora_get_device_status(stream=None) -> int:
 
 def qlora_selftest_wait_timeout(limit_us: int, stream=None) -> None:
     _check(lib().qlora_selftest_wait_timeout(int(limit_us), _stream(stream)), "qlora_selftest_wait_timeout")
+
+
+# ------------------------------------------------------------------ data parallel
+NCCL_ID_BYTES = 128
+
+
+def qlora_comm_unique_id() -> bytes:
+    """A new NCCL unique id for the caller to share with every rank."""
+    buf = (ctypes.c_uint8 * NCCL_ID_BYTES)()
+    _check(lib().qlora_comm_unique_id(ctypes.addressof(buf)), "qlora_comm_unique_id")
+    return bytes(buf)
+
+
+class Communicator:
+    """This rank's NCCL communicator for the adapter-gradient sum (owned by
+    the caller; release it with close() after its last collective)."""
+
+    def __init__(self, unique_id: bytes, nranks: int, rank: int):
+        if len(unique_id) != NCCL_ID_BYTES:
+            raise ValueError(f"unique_id must be {NCCL_ID_BYTES} bytes")
+        buf = (ctypes.c_uint8 * NCCL_ID_BYTES).from_buffer_copy(unique_id)
+        h = ctypes.c_void_p()
+        _check(lib().qlora_comm_init(ctypes.addressof(buf), int(nranks), int(rank), ctypes.byref(h)),
+               "qlora_comm_init")
+        self.handle = h.value
+        self.nranks, self.rank = nranks, rank
+
+    def close(self) -> None:
+        if self.handle:
+            _check(lib().qlora_comm_destroy(self.handle), "qlora_comm_destroy")
+            self.handle = None
+
+
+def communicator_from_process_group(group=None, make=Communicator):
+    """This rank's communicator over the ranks of a torch.distributed group:
+    rank 0 draws the NCCL id and the group broadcasts it (any backend)."""
+    import torch.distributed as dist
+    rank, n = dist.get_rank(group), dist.get_world_size(group)
+    box = [qlora_comm_unique_id() if rank == 0 else None]
+    dist.broadcast_object_list(box, src=dist.get_global_rank(group, 0) if group is not None else 0, group=group)
+    return make(box[0], n, rank)
+
+
+def qlora_grad_allreduce(comm: "Communicator", dA: torch.Tensor, dB: torch.Tensor, stream=None) -> None:
+    """dA and dB (fp32, device) become their sums over the ranks, in place."""
+    for name, t in (("dA", dA), ("dB", dB)):
+        if t.dtype != torch.float32 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous fp32 CUDA tensor")
+    _check(lib().qlora_grad_allreduce(comm.handle, _ptr(dA), dA.numel(), _ptr(dB), dB.numel(), _stream(stream)),
+           "qlora_grad_allreduce")
 
 
 def qlora_profile_begin() -> None:

@@ -14,6 +14,8 @@
 
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <dlfcn.h>
+#include <nccl.h>
 
 #include "../../include/qlora.h"
 #include "adam_kernels.cuh"
@@ -1347,6 +1349,38 @@ int noalloc_scratch(void** out) {
 // =====================================================================
 // C ABI
 // =====================================================================
+namespace {
+// NCCL entry points, resolved from libnccl.so.2 at the first use (a process
+// that already loaded NCCL, such as one running torch.distributed, gets that
+// copy).
+struct NcclApi {
+  bool ok = false;
+  decltype(&ncclGetUniqueId) get_unique_id = nullptr;
+  decltype(&ncclCommInitRank) comm_init_rank = nullptr;
+  decltype(&ncclCommDestroy) comm_destroy = nullptr;
+  decltype(&ncclAllReduce) all_reduce = nullptr;
+  decltype(&ncclGroupStart) group_start = nullptr;
+  decltype(&ncclGroupEnd) group_end = nullptr;
+};
+NcclApi load_nccl() {
+  NcclApi a;
+  void* h = dlopen("libnccl.so.2", RTLD_NOW | RTLD_GLOBAL);
+  if (h == nullptr) return a;
+  a.get_unique_id = reinterpret_cast<decltype(a.get_unique_id)>(dlsym(h, "ncclGetUniqueId"));
+  a.comm_init_rank = reinterpret_cast<decltype(a.comm_init_rank)>(dlsym(h, "ncclCommInitRank"));
+  a.comm_destroy = reinterpret_cast<decltype(a.comm_destroy)>(dlsym(h, "ncclCommDestroy"));
+  a.all_reduce = reinterpret_cast<decltype(a.all_reduce)>(dlsym(h, "ncclAllReduce"));
+  a.group_start = reinterpret_cast<decltype(a.group_start)>(dlsym(h, "ncclGroupStart"));
+  a.group_end = reinterpret_cast<decltype(a.group_end)>(dlsym(h, "ncclGroupEnd"));
+  a.ok = a.get_unique_id && a.comm_init_rank && a.comm_destroy && a.all_reduce && a.group_start && a.group_end;
+  return a;
+}
+const NcclApi& nccl_api() {
+  static const NcclApi api = load_nccl();
+  return api;
+}
+}  // namespace
+
 extern "C" {
 
 const char* qlora_strerror(int s) {
@@ -1361,11 +1395,60 @@ const char* qlora_strerror(int s) {
     case QLORA_ERR_NO_DEVICE: return "no sm_100 device is current";
     case QLORA_ERR_EXCEEDS_STATIC_SCRATCH:
       return "d*k exceeds the static scratch of qlora_nf4_quantize_noalloc (2^28 weights)";
+    case QLORA_ERR_NCCL: return "NCCL unavailable or an NCCL call failed";
     default: return "unknown status";
   }
 }
 
 int qlora_version(void) { return 100; }
+
+// ------------------------------------------------------------ data parallel
+
+int qlora_comm_unique_id(uint8_t* id) {
+  if (id == nullptr) return QLORA_ERR_INVALID_ARG;
+  const NcclApi& n = nccl_api();
+  if (!n.ok) return QLORA_ERR_NCCL;
+  ncclUniqueId u;
+  if (n.get_unique_id(&u) != ncclSuccess) return QLORA_ERR_NCCL;
+  static_assert(sizeof(u.internal) == QLORA_NCCL_ID_BYTES, "NCCL unique id size");
+  memcpy(id, u.internal, QLORA_NCCL_ID_BYTES);
+  return QLORA_OK;
+}
+
+int qlora_comm_init(const uint8_t* id, int nranks, int rank, void** comm) {
+  if (id == nullptr || comm == nullptr || nranks < 1 || rank < 0 || rank >= nranks) return QLORA_ERR_INVALID_ARG;
+  *comm = nullptr;
+  const NcclApi& n = nccl_api();
+  if (!n.ok) return QLORA_ERR_NCCL;
+  ncclUniqueId u;
+  memcpy(u.internal, id, QLORA_NCCL_ID_BYTES);
+  ncclComm_t c = nullptr;
+  if (n.comm_init_rank(&c, nranks, u, rank) != ncclSuccess) return QLORA_ERR_NCCL;
+  *comm = c;
+  return QLORA_OK;
+}
+
+int qlora_comm_destroy(void* comm) {
+  if (comm == nullptr) return QLORA_ERR_INVALID_ARG;
+  const NcclApi& n = nccl_api();
+  if (!n.ok) return QLORA_ERR_NCCL;
+  return n.comm_destroy(static_cast<ncclComm_t>(comm)) == ncclSuccess ? QLORA_OK : QLORA_ERR_NCCL;
+}
+
+int qlora_grad_allreduce(void* comm, float* dA, int64_t nA, float* dB, int64_t nB, qlora_stream_t stream) {
+  if (comm == nullptr || nA < 0 || nB < 0 || (nA > 0 && dA == nullptr) || (nB > 0 && dB == nullptr))
+    return QLORA_ERR_INVALID_ARG;
+  const NcclApi& n = nccl_api();
+  if (!n.ok) return QLORA_ERR_NCCL;
+  const ncclComm_t c = static_cast<ncclComm_t>(comm);
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (n.group_start() != ncclSuccess) return QLORA_ERR_NCCL;
+  ncclResult_t r = ncclSuccess;
+  if (nA > 0) r = n.all_reduce(dA, dA, (size_t)nA, ncclFloat32, ncclSum, c, st);
+  if (r == ncclSuccess && nB > 0) r = n.all_reduce(dB, dB, (size_t)nB, ncclFloat32, ncclSum, c, st);
+  const ncclResult_t e = n.group_end();
+  return (r == ncclSuccess && e == ncclSuccess) ? QLORA_OK : QLORA_ERR_NCCL;
+}
 
 int qlora_nf4_levels(float* levels16, float* thresholds15) {
   const auto& T = tables();

@@ -133,6 +133,14 @@ def test_argument_validation_without_device(lib):
                              16, 1 << 20, None) == 1                                           # alpha <= 0
     assert L.qlora_bwd_multi(ctypes.byref(nf), 2, 16, 16, 8, ctypes.addressof(al), 18, 16, 16, 16, 16, 16,
                              16, 16, 16, 1 << 20, None) == 3                                   # misaligned idx
+    # data parallel: communicator and gradient all-reduce arguments
+    assert L.qlora_grad_allreduce(None, 16, 4, 16, 4, None) == 1                 # no communicator
+    assert L.qlora_grad_allreduce(16, 16, -1, 16, 4, None) == 1                  # negative count
+    assert L.qlora_grad_allreduce(16, None, 4, 16, 4, None) == 1                 # null dA
+    assert L.qlora_comm_init(None, 2, 0, ctypes.byref(ctypes.c_void_p())) == 1
+    assert L.qlora_comm_init(16, 2, 2, ctypes.byref(ctypes.c_void_p())) == 1     # rank outside [0, nranks)
+    assert L.qlora_comm_destroy(None) == 1
+    assert q4.strerror(9) == "NCCL unavailable or an NCCL call failed"
     # the NF4 GEMM build selector takes 0, 1 or 2
     assert L.qlora_set_nf4_gemm_mode(3) == 1 and L.qlora_set_nf4_gemm_mode(-1) == 1
     assert L.qlora_set_nf4_gemm_mode(2) == 0 and L.qlora_set_nf4_gemm_mode(0) == 0

@@ -110,3 +110,31 @@ def test_two_rank_adam_keeps_replicas_identical(tmp_path):
     mp.start_processes(_adam_worker, args=(2, _free_port(), out), nprocs=2, join=True,
                        start_method="spawn")
     assert open(out).read() == "ok"
+
+
+def _id_worker(rank, world, port, out_dir):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        import parameter_efficient_fine_nf4_b200 as q4
+        # the library's communicator set-up without a GPU: rank 0 draws the
+        # NCCL id, the group shares it, every rank gets (id, nranks, rank)
+        got = q4.communicator_from_process_group(make=lambda uid, n, r: (uid, n, r))
+        with open(os.path.join(out_dir, f"rank{rank}.bin"), "wb") as f:
+            f.write(got[0] + bytes([got[1], got[2]]))
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_communicator_id_is_shared_by_all_ranks(tmp_path):
+    q4 = pytest.importorskip("parameter_efficient_fine_nf4_b200")
+    q4.lib()
+    mp.start_processes(_id_worker, args=(2, _free_port(), str(tmp_path)), nprocs=2, join=True,
+                       start_method="spawn")
+    r0 = open(tmp_path / "rank0.bin", "rb").read()
+    r1 = open(tmp_path / "rank1.bin", "rb").read()
+    assert len(r0) == len(r1) == q4.NCCL_ID_BYTES + 2
+    assert r0[:q4.NCCL_ID_BYTES] == r1[:q4.NCCL_ID_BYTES]          # one id for the group
+    assert (r0[-2], r0[-1]) == (2, 0) and (r1[-2], r1[-1]) == (2, 1)
