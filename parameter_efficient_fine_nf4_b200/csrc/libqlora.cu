@@ -613,13 +613,12 @@ SmallPlan small_plan(int64_t Mw, int64_t K0, int64_t T) {
 }
 
 // Forward workspace: bf16 s*U (the rank-r operand of the extension), B
-// padded to r8 columns, and for T <= 64 the split partials of the few-token
-// kernels (U and Y) with their completion tickets in one array.  No copy of
+// padded to r8 columns and the block scales of the dequantising GEMM (the
+// few-token kernels keep their split partials in shared memory).  No copy of
 // the weight: the QLoRA path dequantises inside the GEMM and plain LoRA reads
 // the caller's W.
 struct FwdWs {
   uint16_t* sU; uint16_t* Bp;
-  float* part_u; float* part_y; unsigned int* tickets; int n_tickets; int tickets_y_off;
   uint16_t* Xm;            // LoRA dropout: the masked adapter input
   uint16_t* Bcat; float* Uall;   // several adapters: B_0..B_{n-1} side by side, U of every adapter
   float* scales;           // fp32 block scales of the NF4 weight (forward layout)
@@ -632,19 +631,6 @@ FwdWs carve_fwd(void* ws, int64_t d, int64_t k, int r, int64_t T, bool dropout =
   FwdWs w;
   w.sU = (uint16_t*)c.take((size_t)(std::max<int64_t>(T, 1) * r8 * 2));
   w.Bp = (uint16_t*)c.take((size_t)(d * r8 * 2));
-  w.part_u = w.part_y = nullptr;
-  w.tickets = nullptr;
-  w.n_tickets = w.tickets_y_off = 0;
-  if (T >= 1 && T <= kSmallT) {
-    // U runs over r8 accumulator rows so that the padding columns of sU are
-    // written (as zeros)
-    const SmallPlan su = small_plan(r8, k, T), sy = small_plan(d, k, T);
-    w.part_u = (float*)c.take((size_t)(su.splits > 1 ? (int64_t)su.splits * T * r8 * 4 : 0));
-    w.part_y = (float*)c.take((size_t)(sy.splits > 1 ? (int64_t)sy.splits * T * d * 4 : 0));
-    w.tickets_y_off = su.tiles_m;
-    w.n_tickets = su.tiles_m + sy.tiles_m;
-    w.tickets = (unsigned int*)c.take((size_t)w.n_tickets * 4);
-  }
   w.Xm = dropout ? (uint16_t*)c.take((size_t)(std::max<int64_t>(T, 1) * k * 2)) : nullptr;
   w.Bcat = multi ? (uint16_t*)c.take((size_t)(d * r * 2)) : nullptr;
   w.Uall = multi ? (float*)c.take((size_t)(std::max<int64_t>(T, 1) * r * 4)) : nullptr;
@@ -668,7 +654,6 @@ int eff_splits(int64_t K, int splits) {
 
 struct BwdWs {
   uint16_t* Us2; uint16_t* Gs2; uint16_t* Bp; float* partA; float* partB;
-  float* part_g; float* part_x; unsigned int* tickets; int n_tickets; int tickets_x_off;
   uint16_t* Xm;            // LoRA dropout: the masked adapter input
   uint16_t* Bcat; float* Gall; float* dBcat;   // several adapters
   float* scales;           // fp32 block scales of the NF4 weight (dX layout)
@@ -696,19 +681,6 @@ BwdWs carve_bwd(void* ws, int64_t d, int64_t k, int r, int64_t T, bool dropout =
   const int64_t pa = (int64_t)w.splitsA * w.halves, pb = (int64_t)w.splitsB * w.halves;
   w.partA = (float*)c.take((size_t)(pa > 1 ? pa * r * k * 4 : 0));
   w.partB = (float*)c.take((size_t)(pb > 1 ? pb * d * r * 4 : 0));
-  w.part_g = w.part_x = nullptr;
-  w.tickets = nullptr;
-  w.n_tickets = w.tickets_x_off = 0;
-  if (T >= 1 && T <= kSmallT) {
-    // G runs over rp accumulator rows so that the padding columns of both
-    // halves of sG are written (as zeros)
-    const SmallPlan sg = small_plan(w.rp, d, T), sx = small_plan(k, d, T);
-    w.part_g = (float*)c.take((size_t)(sg.splits > 1 ? (int64_t)sg.splits * T * w.rp * 4 : 0));
-    w.part_x = (float*)c.take((size_t)(sx.splits > 1 ? (int64_t)sx.splits * T * k * 4 : 0));
-    w.tickets_x_off = sg.tiles_m;
-    w.n_tickets = sg.tiles_m + sx.tiles_m;
-    w.tickets = (unsigned int*)c.take((size_t)w.n_tickets * 4);
-  }
   w.sGf = (T >= 1 && T <= kSmallT) ? (float*)c.take((size_t)(T * r * 4)) : nullptr;
   w.sUf = (T >= 1 && T <= kSmallT && multi) ? (float*)c.take((size_t)(T * r * 4)) : nullptr;
   w.Xm = dropout ? (uint16_t*)c.take((size_t)(Tm * k * 2)) : nullptr;
@@ -889,23 +861,35 @@ struct SmallJob {
   uint16_t* b16_out = nullptr;
   int ldb = 0, nb = 0, lo_off = 0;
   float scale = 1.0f, f32_scale = 1.0f;
-  float* part = nullptr;
-  unsigned int* tickets = nullptr;
 };
 
+// One launch of the few-token kernel; the depth splits of a row tile form a
+// cluster (consecutive blocks) when there are several.
+template <int kSrc, int kOut, int TN>
+cudaError_t small_launch_tn(dim3 grid, int splits, cudaStream_t st, const CUtensorMap& a, const CUtensorMap& w,
+                            const CUtensorMap& w1, const CUtensorMap& a1, const Nf4SmallArgs& p) {
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(kSmThreads);
+  cfg.dynamicSmemBytes = SmallCfg<TN>::kSmem;
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = (unsigned)splits;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = splits > 1 ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, gemm_nf4_small_kernel<kSrc, kOut, TN>, a, w, w1, a1, p);
+}
 template <int kSrc, int kOut>
-void small_dispatch(int tn, dim3 grid, cudaStream_t st, const CUtensorMap& a, const CUtensorMap& w,
+void small_dispatch(int tn, dim3 grid, int splits, cudaStream_t st, const CUtensorMap& a, const CUtensorMap& w,
                     const CUtensorMap& w1, const CUtensorMap& a1, const Nf4SmallArgs& p) {
   switch (tn) {
-    case 16:
-      gemm_nf4_small_kernel<kSrc, kOut, 16><<<grid, kSmThreads, SmallCfg<16>::kSmem, st>>>(a, w, w1, a1, p);
-      break;
-    case 32:
-      gemm_nf4_small_kernel<kSrc, kOut, 32><<<grid, kSmThreads, SmallCfg<32>::kSmem, st>>>(a, w, w1, a1, p);
-      break;
-    default:
-      gemm_nf4_small_kernel<kSrc, kOut, 64><<<grid, kSmThreads, SmallCfg<64>::kSmem, st>>>(a, w, w1, a1, p);
-      break;
+    case 16: small_launch_tn<kSrc, kOut, 16>(grid, splits, st, a, w, w1, a1, p); break;
+    case 32: small_launch_tn<kSrc, kOut, 32>(grid, splits, st, a, w, w1, a1, p); break;
+    default: small_launch_tn<kSrc, kOut, 64>(grid, splits, st, a, w, w1, a1, p); break;
   }
 }
 
@@ -920,8 +904,6 @@ int launch_small(const SmallJob& j, int64_t T, cudaStream_t st) {
   a.tiles_m = sp.tiles_m;
   a.splits = sp.splits;
   a.steps_per_split = sp.sps;
-  a.part = j.part;
-  a.tickets = j.tickets;
   a.f32_out = j.f32_out;
   a.ldf = j.ldf;
   a.nf = j.nf;
@@ -968,33 +950,26 @@ int launch_small(const SmallJob& j, int64_t T, cudaStream_t st) {
   const double flops = 2.0 * (double)T * j.Mw * ((double)j.K0 + j.r);
   return launch(j.name, flops, bytes, st, [&] {
     switch (j.src) {
-      case SRC_NF4_ROWS: small_dispatch<SRC_NF4_ROWS, OUT_BF16>(sp.tn, grid, st, mAct, mW, mW1, mAct1, a); break;
-      case SRC_NF4_COLS: small_dispatch<SRC_NF4_COLS, OUT_BF16>(sp.tn, grid, st, mAct, mW, mW1, mAct1, a); break;
-      case SRC_TMA_K: small_dispatch<SRC_TMA_K, OUT_U>(sp.tn, grid, st, mAct, mW, mW1, mAct1, a); break;
+      case SRC_NF4_ROWS: small_dispatch<SRC_NF4_ROWS, OUT_BF16>(sp.tn, grid, sp.splits, st, mAct, mW, mW1, mAct1, a); break;
+      case SRC_NF4_COLS: small_dispatch<SRC_NF4_COLS, OUT_BF16>(sp.tn, grid, sp.splits, st, mAct, mW, mW1, mAct1, a); break;
+      case SRC_TMA_K: small_dispatch<SRC_TMA_K, OUT_U>(sp.tn, grid, sp.splits, st, mAct, mW, mW1, mAct1, a); break;
       default:
         if (j.out == OUT_U)
-          small_dispatch<SRC_TMA_MN, OUT_U>(sp.tn, grid, st, mAct, mW, mW1, mAct1, a);
+          small_dispatch<SRC_TMA_MN, OUT_U>(sp.tn, grid, sp.splits, st, mAct, mW, mW1, mAct1, a);
         else
-          small_dispatch<SRC_TMA_MN, OUT_HILO>(sp.tn, grid, st, mAct, mW, mW1, mAct1, a);
+          small_dispatch<SRC_TMA_MN, OUT_HILO>(sp.tn, grid, sp.splits, st, mAct, mW, mW1, mAct1, a);
         break;
     }
   });
 }
 
-int zero_tickets(unsigned int* t, int n, cudaStream_t st) {
-  return launch("memset", 0.0, 0.0, st, [&] { cudaMemsetAsync(t, 0, (size_t)n * sizeof(unsigned int), st); });
-}
-
-// a' of every block of q into `out`, transposed (forward) or row-major (dX),
-// and zero `tickets` (n words) on the way.
-int block_scales(const qlora_nf4_t* q, bool transposed, float* out, unsigned int* tickets, int n,
-                 cudaStream_t st) {
+// a' of every block of q into `out`, transposed (forward) or row-major (dX).
+int block_scales(const qlora_nf4_t* q, bool transposed, float* out, cudaStream_t st) {
   const int64_t d = q->d, kb = q->k / 64;
   const int64_t ld = transposed ? scales_ld_fwd(d) : scales_ld_dx(q->k);
   const dim3 grid((unsigned)cdiv(kb, 32), (unsigned)cdiv(d, 32));
   return launch("nf4_block_scales", 0.0, (double)d * kb * 5, st, [&] {
-    nf4_block_scales<<<grid, 256, 0, st>>>(q->absmax_q, q->scale2, q->mean, d, kb, transposed ? 1 : 0, ld, out,
-                                          tickets, tickets ? n : 0);
+    nf4_block_scales<<<grid, 256, 0, st>>>(q->absmax_q, q->scale2, q->mean, d, kb, transposed ? 1 : 0, ld, out);
   });
 }
 
@@ -1045,13 +1020,10 @@ int fwd_core(const qlora_nf4_t* q, const uint16_t* W, int64_t d, int64_t k, cons
   const uint16_t* Bp = padded_B(B, d, r, r8, w.Bp, st, &pst);
   QLORA_TRY(pst);
 
-  if (T <= kSmallT) {
-    // the few-token kernels read the block constants themselves; their
-    // completion tickets start at zero
-    QLORA_TRY(zero_tickets(w.tickets, w.n_tickets, st));
-  } else if (q) {
-    // block scales for the dequantising GEMM
-    QLORA_TRY(block_scales(q, true, w.scales, nullptr, 0, st));
+  if (T > kSmallT && q) {
+    // block scales for the dequantising GEMM (the few-token kernels form
+    // them from the stored constants themselves)
+    QLORA_TRY(block_scales(q, true, w.scales, st));
   }
   // U = X A^T (fp32 to U_save), sU = bf16(s U) (operand of the extension)
   if (T <= kSmallT) {
@@ -1061,7 +1033,6 @@ int fwd_core(const qlora_nf4_t* q, const uint16_t* W, int64_t d, int64_t k, cons
     j.act = Xa; j.K0 = k; j.Mw = r8;
     j.f32_out = ma ? w.Uall : U_save; j.ldf = r; j.nf = r; j.f32_scale = c;
     j.b16_out = w.sU; j.ldb = r8; j.nb = ma ? 0 : r8; j.scale = su;
-    j.part = w.part_u; j.tickets = w.tickets;
     QLORA_TRY(launch_small(j, T, st));
   } else {
     GemmPlan g;
@@ -1087,7 +1058,6 @@ int fwd_core(const qlora_nf4_t* q, const uint16_t* W, int64_t d, int64_t k, cons
     j.q = q; j.act = X; j.K0 = k; j.Mw = d;
     j.r = r; j.r8 = r8; j.a1 = w.sU; j.a1_inner = r8; j.a1_ld = r8; j.w1 = Bp;
     j.b16_out = Y; j.ldb = (int)d; j.nb = (int)d;
-    j.part = w.part_y; j.tickets = w.tickets + w.tickets_y_off;
     return launch_small(j, T, st);
   }
   if (q) return launch_nf4_gemm(false, q, w.scales, X, T, w.sU, r8, r8, Bp, r, r8, Y, st);
@@ -1136,11 +1106,7 @@ int bwd_core(const qlora_nf4_t* q, const uint16_t* W, int64_t d, int64_t k, cons
   const uint16_t* Bp = padded_B(B, d, r, r8, w.Bp, st, &pst);
   QLORA_TRY(pst);
   const int rp = w.rp;
-  if (T <= kSmallT) {
-    QLORA_TRY(zero_tickets(w.tickets, w.n_tickets, st));
-  } else if (q) {
-    QLORA_TRY(block_scales(q, false, w.scales, nullptr, 0, st));
-  }
+  if (T > kSmallT && q) QLORA_TRY(block_scales(q, false, w.scales, st));
   // Few tokens, several adapters, no dropout: G of every adapter in fp32, the
   // token's s_i U and s_i G scattered into its block, then dA (the stack) and
   // dB (side by side) in one CUDA-core kernel; the bf16 s G of the dX
@@ -1152,7 +1118,6 @@ int bwd_core(const qlora_nf4_t* q, const uint16_t* W, int64_t d, int64_t k, cons
     j.w = Bp; j.w_inner = r8; j.w_outer = d; j.w_ld = r8;
     j.act = dY; j.K0 = d; j.Mw = rp;
     j.f32_out = w.Gall; j.ldf = r; j.nf = r; j.nb = 0;
-    j.part = w.part_g; j.tickets = w.tickets;
     QLORA_TRY(launch_small(j, T, st));
     QLORA_TRY(launch("scatter_adapter_hilo", 0.0, 0.0, st, [&] {
       scatter_adapter_hilo<<<grid_for(T * rp, 256), 256, 0, st>>>(w.Gall, 0, ma->idx, T, ma->ra, ma->n, rp,
@@ -1181,7 +1146,6 @@ int bwd_core(const qlora_nf4_t* q, const uint16_t* W, int64_t d, int64_t k, cons
     j.act = dY; j.K0 = d; j.Mw = rp;
     j.f32_out = w.sGf; j.ldf = r; j.nf = r; j.f32_scale = s;
     j.b16_out = w.Gs2; j.ldb = 2 * rp; j.nb = rp; j.scale = s;
-    j.part = w.part_g; j.tickets = w.tickets;
     QLORA_TRY(launch_small(j, T, st));
     QLORA_TRY(grads_small(X, dY, U_saved, w.sGf, s, T, d, k, r, dA, dB, st));
     return bwd_dx_base(q, W, d, k, A, r, r8, rp, dY, T, dX, w, st, true);
@@ -1209,7 +1173,6 @@ int bwd_core(const qlora_nf4_t* q, const uint16_t* W, int64_t d, int64_t k, cons
       j.out = OUT_U; j.name = "gemm_lora_g_small";
       j.f32_out = w.Gall; j.ldf = r; j.nf = r; j.nb = 0; j.lo_off = 0;
     }
-    j.part = w.part_g; j.tickets = w.tickets;
     QLORA_TRY(launch_small(j, T, st));
   } else {
     GemmPlan g;
@@ -1271,7 +1234,6 @@ int bwd_dx_base(const qlora_nf4_t* q, const uint16_t* W, int64_t d, int64_t k, c
     j.q = q; j.act = dY; j.K0 = d; j.Mw = k;
     j.r = re; j.r8 = r8; j.a1 = w.Gs2; j.a1_inner = r; j.a1_ld = 2 * rp; j.w1 = A;
     j.b16_out = dX; j.ldb = (int)k; j.nb = (int)k;
-    j.part = w.part_x; j.tickets = w.tickets + w.tickets_x_off;
     return launch_small(j, T, st);
   }
   if (q) return launch_nf4_gemm(true, q, w.scales, dY, T, w.Gs2, r, 2 * rp, A, re, r8, dX, st);

@@ -698,9 +698,11 @@ __global__ void __launch_bounds__(Nf4Cfg<kPair>::kThreads, 1)
 //   U         U^T  = A X^T                     (M = r,  K = k)
 //   G         G^T  = B^T dY^T                  (M = r,  K = d)
 // With few tokens the layer is bound by the weight stream (0.52 bytes per NF4
-// weight), so the depth is split across CTAs to put every SM to work; each CTA
-// writes fp32 partials and the last CTA of a row tile (a completion ticket)
-// sums them in split order, so results are deterministic.
+// weight), so the depth is split across CTAs to put every SM to work.  The
+// splits of a row tile are one thread-block cluster: each CTA keeps its fp32
+// partial in its own shared memory and, after a cluster barrier, every CTA
+// sums a share of the tile over the ranks' shared memory in split order, so
+// results are deterministic and nothing round-trips through global memory.
 // Warps: 0 TMA, 1 TMEM + MMA, 2-9 dequantisation (NF4 sources: two threads
 // per 64-weight block, half a block each, which halves the latency of a
 // K-step's decode); warps 2-5 then read the accumulator, and all eight sum
@@ -723,8 +725,6 @@ struct Nf4SmallArgs {
   int Mw;                     // output features (rows of the accumulator)
   int K0, K1;                 // main depth and r (rank-r extension of the NF4 products)
   int tiles_m, splits, steps_per_split;
-  float* part;                // fp32 partials [splits][T][Mw] when splits > 1
-  unsigned int* tickets;      // one counter per row tile, zero at launch
   float* f32_out;             // OUT_U
   int ldf, nf;
   uint16_t* b16_out;
@@ -743,7 +743,7 @@ struct Nf4SmallArgs {
 
 constexpr int kSmDqWarps = 8;
 constexpr int kSmThreads = (2 + kSmDqWarps) * 32;       // 320
-constexpr int kSmMaxSplits = 16;                         // depth splits per row tile (host plan caps it)
+constexpr int kSmMaxSplits = 8;                          // depth splits per row tile: one portable cluster
 
 template <int TN>
 struct SmallCfg {
@@ -812,7 +812,6 @@ __global__ void __launch_bounds__(kSmThreads, 2)
   uint64_t* drain_bar = acc_full + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_bar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  int* last_flag = const_cast<int*>(abort_flag) + 1;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -841,7 +840,6 @@ __global__ void __launch_bounds__(kSmThreads, 2)
     mbar_init(smem_u32(acc_full), 1);
     mbar_init(smem_u32(drain_bar), 1);
     *abort_flag = 0;
-    *last_flag = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -1064,96 +1062,99 @@ __global__ void __launch_bounds__(kSmThreads, 2)
     }
     // ---------------------------------------------------------- epilogue
     // warps 2-5 read the accumulator: lane quarter q = warp & 3 holds rows
-    // m0 + 32 q .. + 31
+    // m0 + 32 q .. + 31.  One split: emit.  Several: the partial goes to
+    // P[t][row] at the start of this CTA's shared memory (the weight ring,
+    // whose readers, the MMAs, are done).
     const bool acc_warp = warp < 6;
     const int quarter = warp & 3;
-    const int m = m0 + quarter * 32 + lane;
+    const int mloc = quarter * 32 + lane;
+    const int m = m0 + mloc;
     bool ok = live && mbar_wait_bounded(smem_u32(acc_full), 0u, abort_flag);
     ok = __all_sync(0xffffffffu, ok);
     if (ok && acc_warp) {
       tc_fence_after();
+      fence_proxy_async_smem();
+      float* P = reinterpret_cast<float*>(smem);
       const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16);
 #pragma unroll 1
       for (int t0 = 0; t0 < TN; t0 += 16) {
         uint32_t v[16];
         tmem_ld_32x32b_x16(taddr + (uint32_t)t0, v);
         tmem_ld_wait();
-        if (m < p.Mw) {
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int t = t0 + j;
-            if (t < p.T) {
-              if (p.splits == 1)
-                small_emit<kOut>(p, m, t, __uint_as_float(v[j]));
-              else
-                p.part[((int64_t)split * p.T + t) * p.Mw + m] = __uint_as_float(v[j]);
+        for (int j = 0; j < 16; ++j) {
+          const int t = t0 + j;
+          if (t < p.T) {
+            if (p.splits == 1) {
+              if (m < p.Mw) small_emit<kOut>(p, m, t, __uint_as_float(v[j]));
+            } else {
+              P[t * 128 + mloc] = __uint_as_float(v[j]);
             }
           }
         }
-      }
-    }
-    if (p.splits > 1) {
-      // completion ticket: the last CTA of this row tile sums the partials
-      __threadfence();
-      named_bar_sync(1, kSmDqWarps * 32);
-      if (threadIdx.x == 64) {
-        const unsigned int prev = atomicAdd(p.tickets + tile, 1u);
-        *last_flag = (prev == (unsigned int)(p.splits - 1)) ? 1 : 0;
-      }
-      named_bar_sync(1, kSmDqWarps * 32);
-      if (*last_flag && ok) {
-        __threadfence();
-        // all eight warps: each item is (token, features), with every split's
-        // partial in flight at once (at most kSmMaxSplits), summed in split order
-        const int tid = threadIdx.x - 64;
-        const int64_t zs = (int64_t)p.T * p.Mw;
-        if ((p.Mw & 3) == 0) {
-          for (int it = tid; it < p.T * 32; it += kSmDqWarps * 32) {
-            const int t = it >> 5;
-            const int mq = m0 + (it & 31) * 4;
-            if (mq >= p.Mw) continue;
-            const float4* src = reinterpret_cast<const float4*>(p.part + (int64_t)t * p.Mw + mq);
-            float4 v[kSmMaxSplits];
-#pragma unroll
-            for (int z = 0; z < kSmMaxSplits; ++z)
-              v[z] = z < p.splits ? __ldcg(src + z * (zs >> 2)) : make_float4(0.f, 0.f, 0.f, 0.f);
-            float4 acc = v[0];
-#pragma unroll
-            for (int z = 1; z < kSmMaxSplits; ++z) {
-              if (z < p.splits) {
-                acc.x = __fadd_rn(acc.x, v[z].x);
-                acc.y = __fadd_rn(acc.y, v[z].y);
-                acc.z = __fadd_rn(acc.z, v[z].z);
-                acc.w = __fadd_rn(acc.w, v[z].w);
-              }
-            }
-            small_emit<kOut>(p, mq, t, acc.x);
-            small_emit<kOut>(p, mq + 1, t, acc.y);
-            small_emit<kOut>(p, mq + 2, t, acc.z);
-            small_emit<kOut>(p, mq + 3, t, acc.w);
-          }
-        } else {
-          for (int it = tid; it < p.T * 128; it += kSmDqWarps * 32) {
-            const int t = it >> 7;
-            const int mm = m0 + (it & 127);
-            if (mm >= p.Mw) continue;
-            const float* src = p.part + (int64_t)t * p.Mw + mm;
-            float v[kSmMaxSplits];
-#pragma unroll
-            for (int z = 0; z < kSmMaxSplits; ++z) v[z] = z < p.splits ? __ldcg(src + z * zs) : 0.f;
-            float acc = v[0];
-#pragma unroll
-            for (int z = 1; z < kSmMaxSplits; ++z)
-              if (z < p.splits) acc = __fadd_rn(acc, v[z]);
-            small_emit<kOut>(p, mm, t, acc);
-          }
-        }
-        if (threadIdx.x == 64) p.tickets[tile] = 0u;
       }
     }
   }
   tc_fence_before();
   __syncthreads();
+  if (p.splits > 1) {
+    // The depth splits of a row tile form one cluster (rank = split): once
+    // every partial is in its CTA's shared memory, the eight dequantising /
+    // epilogue warps of every CTA sum a share of the tile's outputs over the
+    // ranks' shared memory, in rank (= split) order, so the result does not
+    // depend on timing.
+    cluster_sync();
+    if (warp >= 2) {
+      const int z0 = (int)cluster_ctarank();
+      const int tid = threadIdx.x - 64;
+      const int nthr = kSmDqWarps * 32;
+      if ((p.Mw & 3) == 0) {
+        for (int it = z0 * nthr + tid; it < p.T * 32; it += p.splits * nthr) {
+          const int t = it >> 5;
+          const int q4 = (it & 31) * 4;
+          const int mq = m0 + q4;
+          if (mq >= p.Mw) continue;
+          const uint32_t a = sA + (uint32_t)((t * 128 + q4) * 4);
+          float4 v[kSmMaxSplits];
+#pragma unroll
+          for (int z = 0; z < kSmMaxSplits; ++z)
+            v[z] = z < p.splits ? ld_shared_cluster_f4(mapa_shared(a, (uint32_t)z)) : make_float4(0.f, 0.f, 0.f, 0.f);
+          float4 acc = v[0];
+#pragma unroll
+          for (int z = 1; z < kSmMaxSplits; ++z) {
+            if (z < p.splits) {
+              acc.x = __fadd_rn(acc.x, v[z].x);
+              acc.y = __fadd_rn(acc.y, v[z].y);
+              acc.z = __fadd_rn(acc.z, v[z].z);
+              acc.w = __fadd_rn(acc.w, v[z].w);
+            }
+          }
+          small_emit<kOut>(p, mq, t, acc.x);
+          small_emit<kOut>(p, mq + 1, t, acc.y);
+          small_emit<kOut>(p, mq + 2, t, acc.z);
+          small_emit<kOut>(p, mq + 3, t, acc.w);
+        }
+      } else {
+        for (int it = z0 * nthr + tid; it < p.T * 128; it += p.splits * nthr) {
+          const int t = it >> 7;
+          const int r0 = it & 127;
+          const int mm = m0 + r0;
+          if (mm >= p.Mw) continue;
+          const uint32_t a = sA + (uint32_t)((t * 128 + r0) * 4);
+          float v[kSmMaxSplits];
+#pragma unroll
+          for (int z = 0; z < kSmMaxSplits; ++z) v[z] = z < p.splits ? ld_shared_cluster_f32(mapa_shared(a, (uint32_t)z)) : 0.f;
+          float acc = v[0];
+#pragma unroll
+          for (int z = 1; z < kSmMaxSplits; ++z)
+            if (z < p.splits) acc = __fadd_rn(acc, v[z]);
+          small_emit<kOut>(p, mm, t, acc);
+        }
+      }
+    }
+    // no CTA leaves while a peer may still read its shared memory
+    cluster_sync();
+  }
   if (warp == 1) tmem_dealloc(tmem_base, Cfg::kTmemCols);
 }
 

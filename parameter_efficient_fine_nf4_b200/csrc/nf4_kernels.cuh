@@ -530,23 +530,16 @@ __global__ void __launch_bounds__(256) nf4_dequantize_kernel(
 //   transposed = 0: out[n * ld + s]  (row n, block column s: one K-step of dX
 //                   reads consecutive block columns of 64 rows)
 // Threads of a 32 x 32 tile read the constants row by row and write through
-// shared memory, so both the loads and the stores are coalesced.  The CTAs of
-// the first tile row also zero `zero_n` words at `zero` (the completion
-// tickets of the few-token kernels that follow).
+// shared memory, so both the loads and the stores are coalesced.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) nf4_block_scales(const uint8_t* __restrict__ absmax_q,
                                                         const float* __restrict__ scale2,
                                                         const float* __restrict__ mean, int64_t d, int64_t kb,
-                                                        int transposed, int64_t ld, float* __restrict__ out,
-                                                        unsigned int* __restrict__ zero, int zero_n) {
+                                                        int transposed, int64_t ld, float* __restrict__ out) {
   __shared__ float tile[32][33];
   const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;       // 32 x 8 threads
   const int64_t n0 = (int64_t)blockIdx.y * 32, s0 = (int64_t)blockIdx.x * 32;
   const float mu = mean[0];
-  if (zero != nullptr && blockIdx.y == 0) {
-    for (int i = (int)(blockIdx.x * blockDim.x + threadIdx.x); i < zero_n; i += (int)(gridDim.x * blockDim.x))
-      zero[i] = 0u;
-  }
   for (int j = ty; j < 32; j += 8) {
     const int64_t n = n0 + j, sc = s0 + tx;
     float a = 0.f;
