@@ -973,6 +973,37 @@ int block_scales(const qlora_nf4_t* q, bool transposed, float* out, cudaStream_t
   });
 }
 
+// A second stream of the calling thread on the current device, with two
+// events, for work that may run beside the main stream's (fork / join by
+// events, so that stream capture into a CUDA graph turns it into parallel
+// branches).  Per thread, so that concurrent callers never share it.
+struct SideStream {
+  cudaStream_t st = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+  unsigned long long ctx = 0;
+};
+SideStream* side_stream() {
+  thread_local SideStream side[kMaxDevices];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  SideStream& s = side[dev];
+  const unsigned long long ctx = current_ctx_id();
+  if (s.st == nullptr || s.ctx != ctx) {
+    // a new context (first use, or after a device reset): the old handles
+    // belonged to the old one
+    s.st = nullptr;
+    s.fork = s.join = nullptr;
+    if (cudaStreamCreateWithFlags(&s.st, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaEventCreateWithFlags(&s.fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&s.join, cudaEventDisableTiming) != cudaSuccess) {
+      s.st = nullptr;
+      return nullptr;
+    }
+    s.ctx = ctx;
+  }
+  return &s;
+}
+
 // dA (r x k) and dB (d x r) of a few tokens on CUDA cores (adapter_grads_small).
 int grads_small(const uint16_t* X, const uint16_t* dY, const float* U, const float* sG, float s, int64_t T,
                 int64_t d, int64_t k, int r, float* dA, float* dB, cudaStream_t st) {
@@ -1147,8 +1178,17 @@ int bwd_core(const qlora_nf4_t* q, const uint16_t* W, int64_t d, int64_t k, cons
     j.f32_out = w.sGf; j.ldf = r; j.nf = r; j.f32_scale = s;
     j.b16_out = w.Gs2; j.ldb = 2 * rp; j.nb = rp; j.scale = s;
     QLORA_TRY(launch_small(j, T, st));
-    QLORA_TRY(grads_small(X, dY, U_saved, w.sGf, s, T, d, k, r, dA, dB, st));
-    return bwd_dx_base(q, W, d, k, A, r, r8, rp, dY, T, dX, w, st, true);
+    // dA and dB (which need only G) on a side stream, beside dX
+    SideStream* side = side_stream();
+    if (side == nullptr) return QLORA_ERR_CUDA;
+    if (cudaEventRecord(side->fork, st) != cudaSuccess || cudaStreamWaitEvent(side->st, side->fork, 0) != cudaSuccess)
+      return QLORA_ERR_CUDA;
+    const int gst = grads_small(X, dY, U_saved, w.sGf, s, T, d, k, r, dA, dB, side->st);
+    const int xst = bwd_dx_base(q, W, d, k, A, r, r8, rp, dY, T, dX, w, st, true);
+    // join (always, so that a capture in progress stays well formed)
+    if (cudaEventRecord(side->join, side->st) != cudaSuccess || cudaStreamWaitEvent(st, side->join, 0) != cudaSuccess)
+      return QLORA_ERR_CUDA;
+    return gst != QLORA_OK ? gst : xst;
   }
   // Us2 = hi/lo of bf16(s U)
   if (ma) {
