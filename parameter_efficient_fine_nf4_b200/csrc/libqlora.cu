@@ -874,13 +874,18 @@ cudaError_t small_launch_tn(dim3 grid, int splits, cudaStream_t st, const CUtens
   cfg.blockDim = dim3(kSmThreads);
   cfg.dynamicSmemBytes = SmallCfg<TN>::kSmem;
   cfg.stream = st;
-  cudaLaunchAttribute at[1];
-  at[0].id = cudaLaunchAttributeClusterDimension;
-  at[0].val.clusterDim.x = (unsigned)splits;
-  at[0].val.clusterDim.y = 1;
-  at[0].val.clusterDim.z = 1;
+  // programmatic dependent launch: the kernel's prologue may overlap the
+  // previous kernel of the stream (the kernel waits for it before touching
+  // global memory)
+  cudaLaunchAttribute at[2];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  at[1].id = cudaLaunchAttributeClusterDimension;
+  at[1].val.clusterDim.x = (unsigned)splits;
+  at[1].val.clusterDim.y = 1;
+  at[1].val.clusterDim.z = 1;
   cfg.attrs = at;
-  cfg.numAttrs = splits > 1 ? 1 : 0;
+  cfg.numAttrs = splits > 1 ? 2 : 1;
   return cudaLaunchKernelEx(&cfg, gemm_nf4_small_kernel<kSrc, kOut, TN>, a, w, w1, a1, p);
 }
 template <int kSrc, int kOut>
@@ -1013,8 +1018,17 @@ int grads_small(const uint16_t* X, const uint16_t* dY, const float* U, const flo
   const int nb_b = (int)cdiv(d / 4, kGradThreads / r);
   const double n = (double)r * k + (double)d * r;
   return launch("adapter_grads_small", 2.0 * (double)T * n, n * 4, st, [&] {
-    adapter_grads_small<<<nb_a + nb_b, kGradThreads, 0, st>>>(X, dY, U, sG, s, (int)T, (int)d, (int)k, r, kblk,
-                                                              nb_a, dA, dB);
+    cudaLaunchConfig_t cfg;
+    memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3((unsigned)(nb_a + nb_b));
+    cfg.blockDim = dim3(kGradThreads);
+    cfg.stream = st;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    cudaLaunchKernelEx(&cfg, adapter_grads_small, X, dY, U, sG, s, (int)T, (int)d, (int)k, r, kblk, nb_a, dA, dB);
   });
 }
 

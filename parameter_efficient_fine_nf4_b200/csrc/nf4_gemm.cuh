@@ -858,6 +858,10 @@ __global__ void __launch_bounds__(kSmThreads, 2)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // the prologue above overlaps the previous kernel of the stream; no global
+  // memory is touched before that kernel has completed
+  griddep_launch_dependents();
+  griddep_wait();
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer

@@ -586,6 +586,8 @@ __global__ void __launch_bounds__(kGradThreads) adapter_grads_small(const uint16
                                                                     const float* __restrict__ sG, float s, int T,
                                                                     int d, int k, int r, int kblk, int nb_a,
                                                                     float* __restrict__ dA, float* __restrict__ dB) {
+  griddep_launch_dependents();
+  griddep_wait();
   const int b = (int)blockIdx.x;
   float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
   if (b < nb_a) {

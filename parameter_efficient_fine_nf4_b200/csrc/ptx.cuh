@@ -149,6 +149,18 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
   }
 }
 
+// ------------------------------------------------------------------ dependent launch
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialisation may start while the previous kernel of its stream finishes;
+// griddep_wait() blocks until that kernel has completed and its memory
+// operations are visible (a no-op for a kernel launched without the
+// attribute), and griddep_launch_dependents() lets the next such kernel be
+// scheduled before this one completes.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ------------------------------------------------------------------ clusters
 __device__ __forceinline__ uint32_t cluster_ctarank() {
   uint32_t r;
