@@ -144,6 +144,7 @@ bool g_dev_ready[kMaxDevices] = {false};
 unsigned long long g_dev_ctx[kMaxDevices] = {0};
 int g_dev_sms[kMaxDevices] = {0};
 int g_dev_pair_clusters[kMaxDevices] = {0};
+int g_dev_small_splits[kMaxDevices] = {0};     // largest few-token split cluster the device schedules
 // Which build of the NF4 base GEMM runs for more than 64 tokens: 0 = chosen by
 // shape, 1 = one CTA per tile, 2 = CTA pairs (both give the same bits).
 std::atomic<int> g_nf4_gemm_mode{0};
@@ -222,11 +223,39 @@ int pair_clusters_on_device() {
   return n;
 }
 
+// 16 if clusters of 16 few-token CTAs (the largest configuration, two per SM)
+// can be scheduled, else the portable 8.
+int small_splits_on_device() {
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3(16);
+  cfg.blockDim = dim3(kSmThreads);
+  cfg.dynamicSmemBytes = SmallCfg<64>::kSmem;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = 16;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, gemm_nf4_small_kernel<SRC_TMA_K, OUT_U, 64>, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    return 8;
+  }
+  return n >= 1 ? 16 : 8;
+}
+
 template <int kSrc, int kOut, int TN>
 cudaError_t set_small_attrs_one() {
   const cudaError_t e = cudaFuncSetAttribute(gemm_nf4_small_kernel<kSrc, kOut, TN>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, SmallCfg<TN>::kSmem);
   if (e != cudaSuccess) return e;
+  // clusters of up to 16 depth splits (beyond the portable 8) where the
+  // device schedules them (small_max_splits checks)
+  if (cudaFuncSetAttribute(gemm_nf4_small_kernel<kSrc, kOut, TN>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
+      cudaSuccess)
+    cudaGetLastError();
   cudaFuncAttributes fa;
   if (cudaFuncGetAttributes(&fa, gemm_nf4_small_kernel<kSrc, kOut, TN>) != cudaSuccess)
     return cudaErrorInvalidValue;
@@ -285,6 +314,7 @@ int ensure_device() {
       set_nf4_gemm_attrs<true, true>() != cudaSuccess || set_small_attrs() != cudaSuccess)
     return QLORA_ERR_CUDA;
   g_dev_pair_clusters[dev] = pair_clusters_on_device();
+  g_dev_small_splits[dev] = small_splits_on_device();
   g_dev_ctx[dev] = current_ctx_id();
   g_dev_ready[dev] = true;
   return QLORA_OK;
@@ -604,9 +634,15 @@ SmallPlan small_plan(int64_t Mw, int64_t K0, int64_t T) {
   const int steps0 = (int)cdiv(K0, 64);
   // two CTAs of the few-token kernel fit on an SM; one wave of them
   const int want = std::max(1, (int)(2 * kSMs / sp.tiles_m));
-  // at least 4 K-steps per split (the single-tile U and G products get 16
-  // splits; the NF4 products are capped by their tile count first)
-  const int splits = std::max(1, std::min(std::min(want, steps0 / 4), kSmMaxSplits));
+  // at least 4 K-steps per split
+  // clusters beyond the portable 8 only for single-tile products (U and G),
+  // where one cluster holds the whole grid
+  int dev = 0;
+  int cap = 8;
+  if (sp.tiles_m == 1 && cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < kMaxDevices &&
+      g_dev_small_splits[dev] > 0)
+    cap = std::min(g_dev_small_splits[dev], kSmMaxSplits);
+  const int splits = std::max(1, std::min(std::min(want, steps0 / 4), cap));
   sp.sps = (int)cdiv(steps0, splits);
   sp.splits = (int)cdiv(steps0, sp.sps);
   return sp;

@@ -743,7 +743,10 @@ struct Nf4SmallArgs {
 
 constexpr int kSmDqWarps = 8;
 constexpr int kSmThreads = (2 + kSmDqWarps) * 32;       // 320
-constexpr int kSmMaxSplits = 8;                          // depth splits per row tile: one portable cluster
+// depth splits per row tile (one cluster): 8 is the portable cluster size;
+// 16 where the device schedules non-portable clusters of that size
+constexpr int kSmMaxSplits = 16;
+constexpr int kSmSumBatch = 8;                           // partials in flight per step of the split sum
 
 template <int TN>
 struct SmallCfg {
@@ -1119,18 +1122,20 @@ __global__ void __launch_bounds__(kSmThreads, 2)
           const int mq = m0 + q4;
           if (mq >= p.Mw) continue;
           const uint32_t a = sA + (uint32_t)((t * 128 + q4) * 4);
-          float4 v[kSmMaxSplits];
+          float4 acc = ld_shared_cluster_f4(mapa_shared(a, 0u));
+          for (int z0 = 1; z0 < p.splits; z0 += kSmSumBatch) {
+            float4 v[kSmSumBatch];
 #pragma unroll
-          for (int z = 0; z < kSmMaxSplits; ++z)
-            v[z] = z < p.splits ? ld_shared_cluster_f4(mapa_shared(a, (uint32_t)z)) : make_float4(0.f, 0.f, 0.f, 0.f);
-          float4 acc = v[0];
+            for (int z = 0; z < kSmSumBatch; ++z)
+              if (z0 + z < p.splits) v[z] = ld_shared_cluster_f4(mapa_shared(a, (uint32_t)(z0 + z)));
 #pragma unroll
-          for (int z = 1; z < kSmMaxSplits; ++z) {
-            if (z < p.splits) {
-              acc.x = __fadd_rn(acc.x, v[z].x);
-              acc.y = __fadd_rn(acc.y, v[z].y);
-              acc.z = __fadd_rn(acc.z, v[z].z);
-              acc.w = __fadd_rn(acc.w, v[z].w);
+            for (int z = 0; z < kSmSumBatch; ++z) {
+              if (z0 + z < p.splits) {
+                acc.x = __fadd_rn(acc.x, v[z].x);
+                acc.y = __fadd_rn(acc.y, v[z].y);
+                acc.z = __fadd_rn(acc.z, v[z].z);
+                acc.w = __fadd_rn(acc.w, v[z].w);
+              }
             }
           }
           small_emit<kOut>(p, mq, t, acc.x);
@@ -1145,13 +1150,16 @@ __global__ void __launch_bounds__(kSmThreads, 2)
           const int mm = m0 + r0;
           if (mm >= p.Mw) continue;
           const uint32_t a = sA + (uint32_t)((t * 128 + r0) * 4);
-          float v[kSmMaxSplits];
+          float acc = ld_shared_cluster_f32(mapa_shared(a, 0u));
+          for (int z0 = 1; z0 < p.splits; z0 += kSmSumBatch) {
+            float v[kSmSumBatch];
 #pragma unroll
-          for (int z = 0; z < kSmMaxSplits; ++z) v[z] = z < p.splits ? ld_shared_cluster_f32(mapa_shared(a, (uint32_t)z)) : 0.f;
-          float acc = v[0];
+            for (int z = 0; z < kSmSumBatch; ++z)
+              if (z0 + z < p.splits) v[z] = ld_shared_cluster_f32(mapa_shared(a, (uint32_t)(z0 + z)));
 #pragma unroll
-          for (int z = 1; z < kSmMaxSplits; ++z)
-            if (z < p.splits) acc = __fadd_rn(acc, v[z]);
+            for (int z = 0; z < kSmSumBatch; ++z)
+              if (z0 + z < p.splits) acc = __fadd_rn(acc, v[z]);
+          }
           small_emit<kOut>(p, mm, t, acc);
         }
       }
