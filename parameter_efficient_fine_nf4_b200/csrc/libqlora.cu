@@ -144,7 +144,9 @@ bool g_dev_ready[kMaxDevices] = {false};
 unsigned long long g_dev_ctx[kMaxDevices] = {0};
 int g_dev_sms[kMaxDevices] = {0};
 int g_dev_pair_clusters[kMaxDevices] = {0};
-int g_dev_small_splits[kMaxDevices] = {0};     // largest few-token split cluster the device schedules
+// per device, for few-token clusters of 9..16 CTAs: how many the device
+// holds at once (0 where not known)
+int g_dev_cluster_fit[kMaxDevices][kSmMaxSplits + 1] = {};
 // Which build of the NF4 base GEMM runs for more than 64 tokens: 0 = chosen by
 // shape, 1 = one CTA per tile, 2 = CTA pairs (both give the same bits).
 std::atomic<int> g_nf4_gemm_mode{0};
@@ -223,27 +225,30 @@ int pair_clusters_on_device() {
   return n;
 }
 
-// 16 if clusters of 16 few-token CTAs (the largest configuration, two per SM)
-// can be scheduled, else the portable 8.
-int small_splits_on_device() {
-  cudaLaunchConfig_t cfg;
-  memset(&cfg, 0, sizeof(cfg));
-  cfg.gridDim = dim3(16);
-  cfg.blockDim = dim3(kSmThreads);
-  cfg.dynamicSmemBytes = SmallCfg<64>::kSmem;
-  cudaLaunchAttribute at[1];
-  at[0].id = cudaLaunchAttributeClusterDimension;
-  at[0].val.clusterDim.x = 16;
-  at[0].val.clusterDim.y = 1;
-  at[0].val.clusterDim.z = 1;
-  cfg.attrs = at;
-  cfg.numAttrs = 1;
-  int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, gemm_nf4_small_kernel<SRC_TMA_K, OUT_U, 64>, &cfg) != cudaSuccess) {
-    cudaGetLastError();
-    return 8;
+// How many clusters of s few-token CTAs (s = 9..16, the largest configuration,
+// two CTAs per SM) the device holds at once; 0 where the query fails.
+void small_cluster_fit(int (&fit)[kSmMaxSplits + 1]) {
+  for (int sz = 0; sz <= kSmMaxSplits; ++sz) fit[sz] = 0;
+  for (int sz = 9; sz <= kSmMaxSplits; ++sz) {
+    cudaLaunchConfig_t cfg;
+    memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3((unsigned)sz);
+    cfg.blockDim = dim3(kSmThreads);
+    cfg.dynamicSmemBytes = SmallCfg<64>::kSmem;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = (unsigned)sz;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, gemm_nf4_small_kernel<SRC_TMA_K, OUT_U, 64>, &cfg) != cudaSuccess) {
+      cudaGetLastError();
+      n = 0;
+    }
+    fit[sz] = n;
   }
-  return n >= 1 ? 16 : 8;
 }
 
 template <int kSrc, int kOut, int TN>
@@ -314,7 +319,7 @@ int ensure_device() {
       set_nf4_gemm_attrs<true, true>() != cudaSuccess || set_small_attrs() != cudaSuccess)
     return QLORA_ERR_CUDA;
   g_dev_pair_clusters[dev] = pair_clusters_on_device();
-  g_dev_small_splits[dev] = small_splits_on_device();
+  small_cluster_fit(g_dev_cluster_fit[dev]);
   g_dev_ctx[dev] = current_ctx_id();
   g_dev_ready[dev] = true;
   return QLORA_OK;
@@ -625,7 +630,7 @@ const uint16_t* padded_B(const uint16_t* B, int64_t d, int r, int r8, uint16_t* 
 // all of them in flight).
 constexpr int64_t kSmallT = 64;
 struct SmallPlan {
-  int tn = 16, tiles_m = 1, splits = 1, sps = 1;
+  int tn = 16, tiles_m = 1, splits = 1;
 };
 SmallPlan small_plan(int64_t Mw, int64_t K0, int64_t T) {
   SmallPlan sp;
@@ -634,17 +639,13 @@ SmallPlan small_plan(int64_t Mw, int64_t K0, int64_t T) {
   const int steps0 = (int)cdiv(K0, 64);
   // two CTAs of the few-token kernel fit on an SM; one wave of them
   const int want = std::max(1, (int)(2 * kSMs / sp.tiles_m));
-  // at least 4 K-steps per split
-  // clusters beyond the portable 8 only for single-tile products (U and G),
-  // where one cluster holds the whole grid
+  // at least 4 K-steps per split; more than the portable 8 splits only where
+  // the device holds every cluster of that size at once (checked per size)
+  int splits = std::max(1, std::min(std::min(want, steps0 / 4), kSmMaxSplits));
   int dev = 0;
-  int cap = 8;
-  if (sp.tiles_m == 1 && cudaGetDevice(&dev) == cudaSuccess && dev >= 0 && dev < kMaxDevices &&
-      g_dev_small_splits[dev] > 0)
-    cap = std::min(g_dev_small_splits[dev], kSmMaxSplits);
-  const int splits = std::max(1, std::min(std::min(want, steps0 / 4), cap));
-  sp.sps = (int)cdiv(steps0, splits);
-  sp.splits = (int)cdiv(steps0, sp.sps);
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) dev = -1;
+  while (splits > 8 && (dev < 0 || g_dev_cluster_fit[dev][splits] < sp.tiles_m)) --splits;
+  sp.splits = splits;
   return sp;
 }
 
@@ -944,7 +945,6 @@ int launch_small(const SmallJob& j, int64_t T, cudaStream_t st) {
   a.K1 = j.r;
   a.tiles_m = sp.tiles_m;
   a.splits = sp.splits;
-  a.steps_per_split = sp.sps;
   a.f32_out = j.f32_out;
   a.ldf = j.ldf;
   a.nf = j.nf;

@@ -724,7 +724,7 @@ struct Nf4SmallArgs {
   int T;                      // tokens (MMA N side, at most TN)
   int Mw;                     // output features (rows of the accumulator)
   int K0, K1;                 // main depth and r (rank-r extension of the NF4 products)
-  int tiles_m, splits, steps_per_split;
+  int tiles_m, splits;        // depth splits per row tile: K-steps split as evenly as possible
   float* f32_out;             // OUT_U
   int ldf, nf;
   uint16_t* b16_out;
@@ -822,8 +822,10 @@ __global__ void __launch_bounds__(kSmThreads, 2)
   const int split = blockIdx.x - tile * p.splits;
   const int m0 = tile * 128;
   const int steps0 = (p.K0 + 63) / 64;
-  const int s_begin = split * p.steps_per_split;
-  const int nmain = max(0, min(steps0, s_begin + p.steps_per_split) - s_begin);
+  // split z takes steps0 / splits K-steps, the first steps0 % splits one more
+  const int s_base = steps0 / p.splits, s_rem = steps0 - s_base * p.splits;
+  const int s_begin = split * s_base + min(split, s_rem);
+  const int nmain = s_base + (split < s_rem ? 1 : 0);
   const int steps1 = (kNf4 && split == 0) ? (p.K1 + 63) / 64 : 0;
   const int steps = nmain + steps1;
 
