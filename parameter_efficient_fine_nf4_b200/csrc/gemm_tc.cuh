@@ -64,16 +64,26 @@ struct GemmArgs {
   float levels[16];
 };
 
-template <int BN>
+// One stage holds KSUB sub-blocks of 64 K-columns of each operand, laid out
+// [A sub 0 | A sub 1 | ... | B sub 0 | B sub 1 | ...], each sub-block the same
+// 128B-swizzled tile a one-sub-block stage would hold.  Wider stages issue the
+// loads of several consecutive K-blocks of the same rows together, which keeps
+// the DRAM rows of a streamed activation open across them.
+template <int BN, int KSUB = 1>
 struct GemmCfg {
-  static constexpr int kStages = (BN >= 256) ? 4 : (BN >= 128 ? 5 : 6);
-  static constexpr int kABytes = kBM * kBK * 2;                 // 16 KB
-  static constexpr int kBBytes = BN * kBK * 2;
+  static constexpr int kSubA = kBM * kBK * 2;                    // 16 KB
+  static constexpr int kSubB = BN * kBK * 2;
+  static constexpr int kABytes = KSUB * kSubA;
+  static constexpr int kBBytes = KSUB * kSubB;
   static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kStages =
+      KSUB == 1 ? ((BN >= 256) ? 4 : (BN >= 128 ? 5 : 6)) : (200 * 1024) / kStageBytes;
   static constexpr int kTmemCols = 2 * BN;                       // two accumulators
   // bf16 output staging for TMA stores: 2 boxes of 32 x 64 per epilogue warp
   static constexpr int kStoreStage = (BN == 256) ? 4 * 2 * 4096 : 0;
   static constexpr int kSmemBytes = kStages * kStageBytes + kStoreStage + 1024 /*align*/ + 512 /*bars*/;
+  static_assert(kStages >= 2, "a stage ring needs two stages");
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
 };
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -320,10 +330,10 @@ __device__ __forceinline__ StageDescs make_stage_descs(const GemmArgs& p, uint32
   return d;
 }
 
-__device__ __forceinline__ void issue_kstep(uint32_t d_tmem, const StageDescs& d, int seg, uint32_t stage_off16,
-                                            int nsub, bool first) {
-  const uint64_t a = d.a[seg] + stage_off16;
-  const uint64_t b = d.b[seg] + stage_off16;
+__device__ __forceinline__ void issue_kstep(uint32_t d_tmem, const StageDescs& d, int seg, uint32_t a_off16,
+                                            uint32_t b_off16, int nsub, bool first) {
+  const uint64_t a = d.a[seg] + a_off16;
+  const uint64_t b = d.b[seg] + b_off16;
   const uint32_t as = d.astep[seg], bs = d.bstep[seg], id = d.idesc[seg];
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
@@ -338,13 +348,14 @@ __device__ __forceinline__ void issue_kstep(uint32_t d_tmem, const StageDescs& d
 // shared-memory ring runs continuously across units; two TMEM accumulators
 // (columns [0, BN) and [BN, 2 BN)) let the epilogue of one unit overlap the
 // mainloop of the next (acc_full / acc_empty barriers per accumulator).
-template <int BN>
+template <int BN, int KSUB>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmB0,
                    const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
                    const __grid_constant__ CUtensorMap tmOut, const __grid_constant__ GemmArgs p) {
-  using Cfg = GemmCfg<BN>;
+  using Cfg = GemmCfg<BN, KSUB>;
   constexpr int S = Cfg::kStages;
+  constexpr int kStepK = kBK * KSUB;      // K columns per stage
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte alignment for the 128B-swizzle atoms
   const uint32_t raw_addr = smem_u32(smem_raw);
@@ -364,7 +375,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int units = p.tiles_m * p.tiles_n * (int)((p.K0 + p.k_per_split - 1) / p.k_per_split);
-  const int steps1 = (p.K1 + kBK - 1) / kBK;
+  const int steps1 = (p.K1 + kStepK - 1) / kStepK;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < S; ++i) {
@@ -407,7 +418,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       for (int u = blockIdx.x; u < units && !*abort_flag; u += gridDim.x) {
         const Unit c = unit_coords(p, u, BN);
         const int k_begin = c.split * p.k_per_split;
-        const int steps0 = (min(p.K0 - k_begin, p.k_per_split) + kBK - 1) / kBK;
+        const int k_end0 = min(p.K0, k_begin + p.k_per_split);
+        const int steps0 = (k_end0 - k_begin + kStepK - 1) / kStepK;
         const int steps = steps0 + (c.split == 0 ? steps1 : 0);
         bool ok = true;
         for (int step = 0; step < steps; ++step, ++g) {
@@ -415,26 +427,31 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const uint32_t ph = (uint32_t)((g / S) & 1);
           if (!mbar_wait_bounded(smem_u32(&empty_bar[st]), ph ^ 1u, abort_flag)) { ok = false; break; }
           const uint32_t fb = smem_u32(&full_bar[st]);
-          mbar_arrive_expect_tx(fb, Cfg::kStageBytes);
-          const uint32_t sa = sbase + st * Cfg::kStageBytes;
-          const uint32_t sb = sa + Cfg::kABytes;
           const bool ext = step >= steps0;
-          const int kk = ext ? (step - steps0) * kBK : k_begin + step * kBK;
+          const int kk = ext ? (step - steps0) * kStepK : k_begin + step * kStepK;
+          const int nk = min(KSUB, ((ext ? p.K1 : k_end0) - kk + kBK - 1) / kBK);   // sub-blocks in range
+          mbar_arrive_expect_tx(fb, (uint32_t)(nk * (Cfg::kSubA + Cfg::kSubB)));
+          const uint32_t sa0 = sbase + st * Cfg::kStageBytes;
           const CUtensorMap* ma = ext ? &tmA1 : &tmA0;
           const CUtensorMap* mb = ext ? &tmB1 : &tmB0;
           const int a_mn = ext ? p.a1_mn : p.a0_mn;
           const int b_mn = ext ? p.b1_mn : p.b0_mn;
-          if (a_mn) {
-            tma_load_2d(sa, ma, fb, c.m0, kk);
-            tma_load_2d(sa + 8192, ma, fb, c.m0 + 64, kk);
-          } else {
-            tma_load_2d(sa, ma, fb, kk, c.m0);
-          }
-          if (b_mn) {
+          for (int j = 0; j < nk; ++j) {
+            const uint32_t sa = sa0 + j * Cfg::kSubA;
+            const uint32_t sb = sa0 + Cfg::kABytes + j * Cfg::kSubB;
+            const int kj = kk + j * kBK;
+            if (a_mn) {
+              tma_load_2d(sa, ma, fb, c.m0, kj);
+              tma_load_2d(sa + 8192, ma, fb, c.m0 + 64, kj);
+            } else {
+              tma_load_2d(sa, ma, fb, kj, c.m0);
+            }
+            if (b_mn) {
 #pragma unroll
-            for (int i = 0; i < BN / 64; ++i) tma_load_2d(sb + i * 8192, mb, fb, c.n0 + 64 * i, kk);
-          } else {
-            tma_load_2d(sb, mb, fb, kk, c.n0);
+              for (int i = 0; i < BN / 64; ++i) tma_load_2d(sb + i * 8192, mb, fb, c.n0 + 64 * i, kj);
+            } else {
+              tma_load_2d(sb, mb, fb, kj, c.n0);
+            }
           }
           issued[st] += 1;
         }
@@ -456,7 +473,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++it) {
         const Unit c = unit_coords(p, u, BN);
         const int k_begin = c.split * p.k_per_split;
-        const int steps0 = (min(p.K0 - k_begin, p.k_per_split) + kBK - 1) / kBK;
+        const int k_end0 = min(p.K0, k_begin + p.k_per_split);
+        const int steps0 = (k_end0 - k_begin + kStepK - 1) / kStepK;
         const int steps = steps0 + (c.split == 0 ? steps1 : 0);
         const int buf = it & 1;
         // the epilogue must have drained this accumulator (two units ago)
@@ -472,9 +490,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           if (!mbar_wait_bounded(smem_u32(&full_bar[st]), ph, abort_flag)) { ok = false; break; }
           tc_fence_after();
           const bool ext = step >= steps0;
-          int nsub = 4;
-          if (ext) nsub = min(4, (p.K1 - (step - steps0) * kBK + 15) / 16);
-          issue_kstep(d_tmem, dsc, ext ? 1 : 0, (uint32_t)(st * Cfg::kStageBytes) >> 4, nsub, step == 0);
+          const int kk = ext ? (step - steps0) * kStepK : k_begin + step * kStepK;
+          const int nk = min(KSUB, ((ext ? p.K1 : k_end0) - kk + kBK - 1) / kBK);
+          for (int j = 0; j < nk; ++j) {
+            int nsub = 4;
+            if (ext) nsub = min(4, (p.K1 - (kk + j * kBK) + 15) / 16);
+            issue_kstep(d_tmem, dsc, ext ? 1 : 0, (uint32_t)(st * Cfg::kStageBytes + j * Cfg::kSubA) >> 4,
+                        (uint32_t)(st * Cfg::kStageBytes + j * Cfg::kSubB) >> 4, nsub, step == 0 && j == 0);
+          }
           issued_any = 1;
           umma_commit(smem_u32(&empty_bar[st]));
         }

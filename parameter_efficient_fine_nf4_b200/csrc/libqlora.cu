@@ -189,10 +189,10 @@ int current_sms() {
   return g_dev_sms[dev];
 }
 
-template <int BN>
+template <int BN, int KSUB = 1>
 cudaError_t set_gemm_attrs() {
-  return cudaFuncSetAttribute(gemm_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              GemmCfg<BN>::kSmemBytes);
+  return cudaFuncSetAttribute(gemm_tc_kernel<BN, KSUB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              GemmCfg<BN, KSUB>::kSmemBytes);
 }
 
 template <bool kDx, bool kPair>
@@ -312,6 +312,8 @@ int ensure_device() {
   if (encode_fn() == nullptr) return QLORA_ERR_CUDA;
   if (!tables().enc_ok) return QLORA_ERR_CUDA;
   if (set_gemm_attrs<64>() != cudaSuccess || set_gemm_attrs<128>() != cudaSuccess ||
+      set_gemm_attrs<64, 2>() != cudaSuccess || set_gemm_attrs<64, 4>() != cudaSuccess ||
+      set_gemm_attrs<128, 2>() != cudaSuccess ||
       set_gemm_attrs<256>() != cudaSuccess || set_deploy_attrs<true, 1>() != cudaSuccess ||
       set_deploy_attrs<true, 2>() != cudaSuccess || set_deploy_attrs<false, 1>() != cudaSuccess ||
       set_deploy_attrs<false, 2>() != cudaSuccess || set_nf4_gemm_attrs<false, false>() != cudaSuccess ||
@@ -498,9 +500,10 @@ struct GemmPlan {
   Operand a0, b0, a1, b1;
   int splits = 1;
   int bn = 256;
+  int ksub = 1;      // 64-wide K sub-blocks per pipeline stage
 };
 
-template <int BN>
+template <int BN, int KSUB = 1>
 int launch_gemm_bn(const char* name, const GemmPlan& g, GemmArgs args, cudaStream_t st) {
   CUtensorMap m[4];
   memset(m, 0, sizeof(m));
@@ -537,7 +540,8 @@ int launch_gemm_bn(const char* name, const GemmPlan& g, GemmArgs args, cudaStrea
   dim3 grid((unsigned)std::min<int64_t>(units, current_sms()), 1, 1);
   const double flops = 2.0 * g.M * (double)g.N * (g.K0 + g.K1);
   return launch(name, flops, 0.0, st, [&] {
-    gemm_tc_kernel<BN><<<grid, kGemmThreads, GemmCfg<BN>::kSmemBytes, st>>>(m[0], m[1], m[2], m[3], mo, args);
+    gemm_tc_kernel<BN, KSUB><<<grid, kGemmThreads, GemmCfg<BN, KSUB>::kSmemBytes, st>>>(m[0], m[1], m[2], m[3], mo,
+                                                                                        args);
   });
 }
 
@@ -550,13 +554,26 @@ int launch_gemm(const char* name, const GemmPlan& g, const GemmArgs& args, cudaS
       if (!aligned16(o->ptr) || (o->ld * 2) % 16 != 0) return QLORA_ERR_MISALIGNED;
   }
   switch (g.bn) {
-    case 64: return launch_gemm_bn<64>(name, g, args, st);
-    case 128: return launch_gemm_bn<128>(name, g, args, st);
+    case 64:
+      if (g.ksub >= 4) return launch_gemm_bn<64, 4>(name, g, args, st);
+      if (g.ksub == 2) return launch_gemm_bn<64, 2>(name, g, args, st);
+      return launch_gemm_bn<64>(name, g, args, st);
+    case 128:
+      if (g.ksub >= 2) return launch_gemm_bn<128, 2>(name, g, args, st);
+      return launch_gemm_bn<128>(name, g, args, st);
     default: return launch_gemm_bn<256>(name, g, args, st);
   }
 }
 
 inline int bn_for_rank(int r) { return r <= 64 ? 64 : (r <= 128 ? 128 : 256); }
+
+// 64-wide K sub-blocks per pipeline stage of the adapter GEMMs.  These stream
+// a T x k (or T x d) activation against a rank-r operand and are bound by
+// HBM; wider stages fetch 256 (U, G) or 128 (dA, dB) contiguous columns of
+// every activation row at once: 13-15 % faster than one sub-block per stage
+// at the 8192 -> 22016 projection pair, 16384 tokens.
+constexpr int kAdapterKSub = 4;    // U = X A^T and G = dY B: K-major rows of X / dY
+constexpr int kGradKSub = 2;       // dA, dB: T-reductions over MN-major X / dY
 
 GemmArgs blank_args() {
   GemmArgs a;
@@ -739,7 +756,7 @@ int adapter_grad_gemm(const char* name, const uint16_t* big, int64_t M, int64_t 
   const int64_t plane = M * r;
   for (int h = 0; h < halves; ++h) {
     GemmPlan g;
-    g.M = (int)M; g.K0 = (int)T; g.splits = splits;
+    g.M = (int)M; g.K0 = (int)T; g.splits = splits; g.ksub = kGradKSub;
     g.a0 = mnmajor(big, M, T, M);
     GemmArgs a = blank_args();
     a.epi = transposed ? EPI_F32_T : EPI_F32;
@@ -1117,7 +1134,7 @@ int fwd_core(const qlora_nf4_t* q, const uint16_t* W, int64_t d, int64_t k, cons
     QLORA_TRY(launch_small(j, T, st));
   } else {
     GemmPlan g;
-    g.M = (int)T; g.N = r; g.K0 = (int)k; g.bn = bn_for_rank(r);
+    g.M = (int)T; g.N = r; g.K0 = (int)k; g.bn = bn_for_rank(r); g.ksub = kAdapterKSub;
     g.a0 = kmajor(Xa, k, T, k);
     g.b0 = kmajor(A, k, r, k);
     GemmArgs a = blank_args();
@@ -1266,7 +1283,7 @@ int bwd_core(const qlora_nf4_t* q, const uint16_t* W, int64_t d, int64_t k, cons
     QLORA_TRY(launch_small(j, T, st));
   } else {
     GemmPlan g;
-    g.M = (int)T; g.N = r; g.K0 = (int)d; g.bn = bnr;
+    g.M = (int)T; g.N = r; g.K0 = (int)d; g.bn = bnr; g.ksub = kAdapterKSub;
     g.a0 = kmajor(dY, d, T, d);
     g.b0 = mnmajor(Bp, r8, d, r8);
     GemmArgs a = blank_args();
