@@ -863,39 +863,46 @@ __global__ void __launch_bounds__(kSmThreads, 2)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  // the prologue above overlaps the previous kernel of the stream; no global
-  // memory is touched before that kernel has completed
+  // The prologue above overlaps the previous kernel of the stream.
   griddep_launch_dependents();
-  griddep_wait();
+  // codes run ahead of the activations by up to SC K-steps (issued by warp 0
+  // in step order, each when the decode of the step SC before it is done)
+  int c_iss[Cfg::SC];
+  for (int i = 0; i < Cfg::SC; ++i) c_iss[i] = 0;
+  int cnext = 0;
+  auto issue_codes = [&](int upto) -> bool {
+    for (; cnext < nmain && cnext < upto; ++cnext) {
+      const int sc = cnext % Cfg::SC;
+      if (!mbar_wait_bounded(smem_u32(&c_empty[sc]), (uint32_t)(((cnext / Cfg::SC) & 1) ^ 1), abort_flag))
+        return false;
+      const uint32_t fc = smem_u32(&c_full[sc]);
+      const int ks = s_begin + cnext;
+      mbar_arrive_expect_tx(fc, (uint32_t)Cfg::kCodeBytes);
+      if (kSrc == SRC_NF4_COLS)
+        tma_load_2d(sC + sc * Cfg::kCBytes, &tmW, fc, m0 / 2, ks * 64);
+      else
+        tma_load_2d(sC + sc * Cfg::kCBytes, &tmW, fc, ks * 32, m0);
+      c_iss[sc] += 1;
+    }
+    return true;
+  };
+  // The first SC code stages, and the dequantising threads' first block
+  // constants, load before waiting for that kernel: the NF4 codes and
+  // constants are written only by the quantiser, whose kernels let no
+  // dependent kernel start before they complete.  All other global memory
+  // (activations, the rank-r operands, the outputs) is touched only after
+  // the wait, which every thread executes.
+  const bool pre_ok = !(kNf4 && warp == 0 && lane == 0) || issue_codes(Cfg::SC);
+  if (!(kNf4 && warp >= 2)) griddep_wait();
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      int b_iss[Cfg::SB], c_iss[Cfg::SC];
+      int b_iss[Cfg::SB];
       int a_last[Cfg::SA];
       for (int i = 0; i < Cfg::SB; ++i) b_iss[i] = 0;
-      for (int i = 0; i < Cfg::SC; ++i) c_iss[i] = 0;
       for (int i = 0; i < Cfg::SA; ++i) a_last[i] = -1;
-      // codes run ahead of the activations by up to SC K-steps (issued in
-      // step order, each when the decode of the step SC before it is done)
-      int cnext = 0;
-      bool ok = true;
-      auto issue_codes = [&](int upto) -> bool {
-        for (; cnext < nmain && cnext < upto; ++cnext) {
-          const int sc = cnext % Cfg::SC;
-          if (!mbar_wait_bounded(smem_u32(&c_empty[sc]), (uint32_t)(((cnext / Cfg::SC) & 1) ^ 1), abort_flag))
-            return false;
-          const uint32_t fc = smem_u32(&c_full[sc]);
-          const int ks = s_begin + cnext;
-          mbar_arrive_expect_tx(fc, (uint32_t)Cfg::kCodeBytes);
-          if (kSrc == SRC_NF4_COLS)
-            tma_load_2d(sC + sc * Cfg::kCBytes, &tmW, fc, m0 / 2, ks * 64);
-          else
-            tma_load_2d(sC + sc * Cfg::kCBytes, &tmW, fc, ks * 32, m0);
-          c_iss[sc] += 1;
-        }
-        return true;
-      };
+      bool ok = pre_ok;
       for (int step = 0; step < steps && ok; ++step) {
         const bool main = step < nmain;
         const int ks = s_begin + step;
@@ -1016,6 +1023,7 @@ __global__ void __launch_bounds__(kSmThreads, 2)
       };
 #pragma unroll
       for (int j = 0; j < kAhead; ++j) load_step(j, q_r[j], s2_r[j]);
+      griddep_wait();
       for (int s0 = 0; s0 < nmain && live; s0 += kAhead) {
 #pragma unroll
         for (int jw = 0; jw < kAhead; ++jw) {
